@@ -1,0 +1,408 @@
+"""Pins for the fp64 CPU oracle (no GPU).
+
+Each pin checks the token-by-token oracle against something other than itself:
+hand-worked values, a finite-difference gradient, closed forms of special cases,
+a textbook formula, explicit transition-matrix products, and an independent
+chunkwise solve.  ``test_pins_catch_planted_mistakes`` rebuilds the oracle with
+plausible mistakes planted in its source and checks that the battery rejects
+every one of them.
+
+Sources: "DeltaTTT: Layerwise Optimization for Nonlinear Recurrent Memory",
+§2 Background (delta rule = serial gradient descent on a linear memory; fixed-
+base evaluation = additive linear attention; the update is affine in the
+preceding memory, hence chunkwise evaluation) and §4.1 (a gradient step on a
+linear-regression objective is a delta-rule update); "Delta-Rule Linear
+Attention" topic page, FG^2-GDN card (KDA: channel-wise decay); Gated
+DeltaNet-2 abstract on page 2607.07953 (GDN-2 reduces to KDA, KDA to GDN).
+"""
+import os
+import re
+import shutil
+import subprocess
+import tempfile
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import chunkwise_ref, gdr_fwd
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden",
+                      "delta_rule_hand_examples.txt")
+
+
+# ----------------------------------------------------------------- helpers
+def _rand_case(rng, B=2, T=11, H=2, dk=3, dv=4, gate="scalar", s0=True,
+               decay=(0.05, 0.6)):
+    q = rng.standard_normal((B, T, H, dk))
+    k = rng.standard_normal((B, T, H, dk))
+    q /= np.linalg.norm(q, axis=-1, keepdims=True)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, T, H, dv))
+    beta = 1 / (1 + np.exp(-rng.standard_normal((B, T, H))))
+    la = None
+    if gate == "scalar":
+        la = -rng.uniform(*decay, size=(B, T, H))
+    elif gate == "channel":
+        la = -rng.uniform(*decay, size=(B, T, H, dk))
+    S0 = rng.standard_normal((B, H, dk, dv)) * 0.5 if s0 else None
+    return dict(q=q, k=k, v=v, beta=beta, log_alpha=la, gate=gate,
+                initial_state=S0)
+
+
+def _parse_golden(path=GOLDEN):
+    blocks, cur = {}, None
+    for line in open(path):
+        line = line.split("#", 1)[0].strip()
+        if not line:
+            continue
+        m = re.match(r"\[(\w+)\]", line)
+        if m:
+            cur = blocks.setdefault(m.group(1), {})
+            continue
+        key, val = [s.strip() for s in line.split("=", 1)]
+        if key == "gate":
+            cur[key] = val
+        else:
+            cur[key] = np.array([[float(x) for x in row.split()]
+                                 for row in val.split(";")])
+    return blocks
+
+
+def _decay_mats(la, gate, dk):
+    if gate == "none":
+        return np.eye(dk)
+    if gate == "scalar":
+        return np.exp(la) * np.eye(dk)
+    return np.diag(np.exp(la))
+
+
+# ------------------------------------------------ the battery (any library)
+def pin_golden(lib):
+    for name, b in _parse_golden().items():
+        T = b["k"].shape[0]
+        shp = lambda x: x.reshape(1, T, 1, -1)  # noqa: E731
+        la = None
+        if b["gate"] == "scalar":
+            la = np.log(b["alpha"]).reshape(1, T, 1)
+        elif b["gate"] == "channel":
+            la = np.log(b["alpha"]).reshape(1, T, 1, -1)
+        out, sT, _ = gdr_fwd(shp(b["q"]), shp(b["k"]), shp(b["v"]),
+                             b["beta"].reshape(1, T, 1), la, gate=b["gate"],
+                             initial_state=b["S0"][None, None], lib=lib)
+        if not (np.allclose(out[0, :, 0, :], b["out"], atol=1e-12)
+                and np.allclose(sT[0, 0], b["S_final"], atol=1e-12)):
+            return f"golden example {name}"
+    return None
+
+
+def pin_gradient_step(lib, rng=None):
+    """One token with alpha=1 is one gradient step of 1/2||S^T k - v||^2 with
+    learning rate beta; with a decay the step is taken at D S0.  The gradient
+    is found by central differences (exact for a quadratic up to rounding)."""
+    rng = rng or np.random.default_rng(1)
+    dk, dv = 3, 5
+    for gate in ("none", "scalar", "channel"):
+        c = _rand_case(rng, B=1, T=1, H=1, dk=dk, dv=dv, gate=gate)
+        k, v = c["k"][0, 0, 0], c["v"][0, 0, 0]
+        b = c["beta"][0, 0, 0]
+        la = None if gate == "none" else c["log_alpha"][0, 0, 0]
+        S = _decay_mats(la, gate, dk) @ c["initial_state"][0, 0]
+
+        def loss(M):
+            r = M.T @ k - v
+            return 0.5 * float(r @ r)
+        grad = np.zeros_like(S)
+        h = 1e-3
+        for i in range(dk):
+            for j in range(dv):
+                E = np.zeros_like(S)
+                E[i, j] = h
+                grad[i, j] = (loss(S + E) - loss(S - E)) / (2 * h)
+        expect = S - b * grad
+        out, sT, _ = gdr_fwd(**c, lib=lib)
+        if not np.allclose(sT[0, 0], expect, atol=1e-9):
+            return f"gradient step ({gate})"
+        if not np.allclose(out[0, 0, 0], expect.T @ c["q"][0, 0, 0],
+                           atol=1e-9):
+            return f"gradient step read-out ({gate})"
+    return None
+
+
+def pin_beta_zero(lib, rng=None):
+    """beta = 0: S_T = Gamma_T S0 and o_t = (Gamma_t S0)^T q_t."""
+    rng = rng or np.random.default_rng(2)
+    for gate in ("none", "scalar", "channel"):
+        c = _rand_case(rng, B=1, T=9, H=2, dk=4, dv=3, gate=gate)
+        c["beta"] = np.zeros_like(c["beta"])
+        out, sT, _ = gdr_fwd(**c, lib=lib)
+        for h in range(2):
+            G = np.zeros(4) if gate == "none" else None
+            for t in range(9):
+                if gate == "scalar":
+                    G = np.full(4, c["log_alpha"][0, :t + 1, h].sum())
+                elif gate == "channel":
+                    G = c["log_alpha"][0, :t + 1, h].sum(axis=0)
+                St = np.exp(G)[:, None] * c["initial_state"][0, h]
+                if not np.allclose(out[0, t, h], St.T @ c["q"][0, t, h],
+                                   atol=1e-12):
+                    return f"beta=0 output ({gate})"
+            if not np.allclose(sT[0, h], St, atol=1e-12):
+                return f"beta=0 final state ({gate})"
+    return None
+
+
+def pin_orthonormal_recall(lib, rng=None):
+    """alpha = beta = 1 on orthonormal keys: after writing all of them,
+    querying k_i returns v_i, from any initial state."""
+    rng = rng or np.random.default_rng(3)
+    dk, dv = 6, 5
+    for n in (1, 4, 6):
+        Qm, _ = np.linalg.qr(rng.standard_normal((dk, dk)))
+        k = Qm[:, :n].T.reshape(1, n, 1, dk)
+        v = rng.standard_normal((1, n, 1, dv))
+        S0 = rng.standard_normal((1, 1, dk, dv))
+        _, sT, _ = gdr_fwd(k, k, v, np.ones((1, n, 1)), None, gate="none",
+                           initial_state=S0, lib=lib)
+        if not np.allclose(sT[0, 0].T @ k[0, :, 0].T, v[0, :, 0].T,
+                           atol=1e-12):
+            return f"orthonormal recall (n={n})"
+    return None
+
+
+def pin_linear_attention(lib, rng=None):
+    """Fixed-base variant (erase term dropped), alpha = 1, S0 = 0:
+    o_t = sum_{i<=t} beta_i (k_i . q_t) v_i, the causal linear attention sum."""
+    rng = rng or np.random.default_rng(4)
+    c = _rand_case(rng, B=1, T=13, H=1, dk=4, dv=3, gate="none", s0=False)
+    out, _, _ = gdr_fwd(**c, fixed_base=True, lib=lib)
+    q, k, v, b = c["q"][0, :, 0], c["k"][0, :, 0], c["v"][0, :, 0], \
+        c["beta"][0, :, 0]
+    for t in range(13):
+        o = sum(b[i] * (k[i] @ q[t]) * v[i] for i in range(t + 1))
+        if not np.allclose(out[0, t, 0], o, atol=1e-12):
+            return "fixed base = causal linear attention"
+    return None
+
+
+def pin_transition_products(lib, rng=None):
+    """Brute force on tiny inputs: with transition matrices
+    M_t = (I - beta_t k_t k_t^T) D_t (dk x dk), the state after t tokens is
+    M_t..M_1 S0 + sum_{i<=t} M_t..M_{i+1} beta_i k_i v_i^T.  dk != dv so a
+    transposed operand cannot pass."""
+    rng = rng or np.random.default_rng(5)
+    dk, dv, T = 3, 4, 7
+    for gate in ("none", "scalar", "channel"):
+        c = _rand_case(rng, B=1, T=T, H=1, dk=dk, dv=dv, gate=gate)
+        out, sT, _ = gdr_fwd(**c, lib=lib)
+        k, v, q = c["k"][0, :, 0], c["v"][0, :, 0], c["q"][0, :, 0]
+        b = c["beta"][0, :, 0]
+        M = []
+        for t in range(T):
+            la = None if gate == "none" else c["log_alpha"][0, t, 0]
+            M.append((np.eye(dk) - b[t] * np.outer(k[t], k[t]))
+                     @ _decay_mats(la, gate, dk))
+
+        def prod(lo, hi):  # M_hi ... M_lo (1-based, inclusive); I if empty
+            P = np.eye(dk)
+            for s in range(lo, hi + 1):
+                P = M[s - 1] @ P
+            return P
+        for t in range(1, T + 1):
+            St = prod(1, t) @ c["initial_state"][0, 0]
+            for i in range(1, t + 1):
+                St = St + prod(i + 1, t) @ (b[i - 1] * np.outer(k[i - 1],
+                                                               v[i - 1]))
+            if not np.allclose(out[0, t - 1, 0], St.T @ q[t - 1], atol=1e-12):
+                return f"transition products, output ({gate})"
+        if not np.allclose(sT[0, 0], St, atol=1e-12):
+            return f"transition products, state ({gate})"
+    return None
+
+
+def pin_chunkwise(lib, rng=None):
+    """The independent chunkwise solve equals the token loop for several chunk
+    sizes, ragged tails included."""
+    rng = rng or np.random.default_rng(6)
+    for gate in ("none", "scalar", "channel"):
+        c = _rand_case(rng, B=2, T=19, H=2, dk=5, dv=3, gate=gate)
+        out, sT, _ = gdr_fwd(**c, lib=lib)
+        for C in (1, 2, 4, 16):
+            o2, s2 = chunkwise_ref(**c, chunk=C)
+            scale = max(np.abs(out).max(), 1.0)
+            if not (np.abs(o2 - out).max() <= 1e-10 * scale
+                    and np.abs(s2 - sT).max() <= 1e-10 * max(
+                        np.abs(sT).max(), 1.0)):
+                return f"chunkwise (gate={gate}, C={C})"
+    return None
+
+
+BATTERY = [pin_golden, pin_gradient_step, pin_beta_zero,
+           pin_orthonormal_recall, pin_linear_attention,
+           pin_transition_products, pin_chunkwise]
+
+
+def run_battery(lib):
+    return [f for f in (p(lib) for p in BATTERY) if f]
+
+
+# ---------------------------------------------------------------- the tests
+@pytest.mark.parametrize("pin", BATTERY, ids=lambda p: p.__name__)
+def test_pin(oracle_lib, pin):
+    assert pin(oracle_lib) is None
+
+
+def test_gate_reductions(oracle_lib):
+    """KDA with equal channels = GDN; GDN with log alpha = 0 = DeltaNet."""
+    rng = np.random.default_rng(7)
+    c = _rand_case(rng, B=2, T=17, H=3, dk=4, dv=5, gate="scalar")
+    o_s, s_s, _ = gdr_fwd(**c)
+    cc = dict(c, gate="channel",
+              log_alpha=np.repeat(c["log_alpha"][..., None], 4, axis=-1))
+    o_c, s_c, _ = gdr_fwd(**cc)
+    assert np.allclose(o_s, o_c, atol=1e-13) and np.allclose(s_s, s_c,
+                                                             atol=1e-13)
+    cz = dict(c, log_alpha=np.zeros_like(c["log_alpha"]))
+    o_z, s_z, _ = gdr_fwd(**cz)
+    o_n, s_n, _ = gdr_fwd(**dict(c, gate="none", log_alpha=None))
+    assert np.array_equal(o_z, o_n) and np.array_equal(s_z, s_n)
+
+
+def test_state_carry_split(oracle_lib):
+    """Two calls chained through final_state -> initial_state = one call."""
+    rng = np.random.default_rng(8)
+    c = _rand_case(rng, B=2, T=20, H=2, dk=4, dv=4, gate="channel")
+    o, s, _ = gdr_fwd(**c)
+    cut = 7
+    a = {x: (c[x][:, :cut] if x in ("q", "k", "v", "beta", "log_alpha")
+             else c[x]) for x in c}
+    o1, s1, _ = gdr_fwd(**a)
+    b = {x: (c[x][:, cut:] if x in ("q", "k", "v", "beta", "log_alpha")
+             else c[x]) for x in c}
+    b["initial_state"] = s1
+    o2, s2, _ = gdr_fwd(**b)
+    assert np.allclose(np.concatenate([o1, o2], axis=1), o, atol=1e-13)
+    assert np.allclose(s2, s, atol=1e-13)
+
+
+def test_varlen_equals_separate(oracle_lib):
+    rng = np.random.default_rng(9)
+    lens = [5, 1, 12, 0, 9]
+    H, dk, dv = 2, 3, 4
+    cases = [_rand_case(rng, B=1, T=L, H=H, dk=dk, dv=dv, gate="scalar")
+             for L in lens]
+    cat = lambda x: np.concatenate([c[x] for c in cases], axis=1)  # noqa
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    S0 = np.concatenate([c["initial_state"] for c in cases], axis=0)
+    o, s, _ = gdr_fwd(cat("q"), cat("k"), cat("v"), cat("beta"),
+                      cat("log_alpha"), gate="scalar", initial_state=S0,
+                      cu_seqlens=cu)
+    for n, c in enumerate(cases):
+        on, sn, _ = gdr_fwd(**c)
+        assert np.array_equal(o[:, cu[n]:cu[n + 1]], on)
+        assert np.array_equal(s[n], sn[0])
+    # chunkwise reformulation handles the same packing
+    o2, s2 = chunkwise_ref(cat("q"), cat("k"), cat("v"), cat("beta"),
+                           cat("log_alpha"), gate="scalar", initial_state=S0,
+                           cu_seqlens=cu, chunk=4)
+    assert np.allclose(o2, o, atol=1e-11) and np.allclose(s2, s, atol=1e-11)
+
+
+def test_thread_count_does_not_change_bits(oracle_lib):
+    rng = np.random.default_rng(10)
+    c = _rand_case(rng, B=3, T=15, H=5, dk=4, dv=4, gate="channel")
+    o1, s1, n1 = gdr_fwd(**c, nthreads=1)
+    o8, s8, n8 = gdr_fwd(**c, nthreads=8)
+    assert n1 == 1 and n8 >= 1
+    assert np.array_equal(o1, o8) and np.array_equal(s1, s8)
+
+
+def test_zero_length_and_zero_state(oracle_lib):
+    rng = np.random.default_rng(11)
+    c = _rand_case(rng, B=1, T=6, H=1, dk=2, dv=2, gate="none", s0=False)
+    cu = np.array([0, 0, 6, 6])
+    o, s, _ = gdr_fwd(c["q"], c["k"], c["v"], c["beta"], None, gate="none",
+                      cu_seqlens=cu)
+    assert np.all(s[0] == 0) and np.all(s[2] == 0)
+    on, sn, _ = gdr_fwd(**c)
+    assert np.array_equal(o, on) and np.array_equal(s[1], sn[0])
+
+
+def test_bad_arguments_rejected(oracle_lib):
+    rng = np.random.default_rng(12)
+    c = _rand_case(rng, B=1, T=4, H=1, dk=2, dv=2, gate="none", s0=False)
+    with pytest.raises(ValueError):
+        gdr_fwd(c["q"], c["k"], c["v"], c["beta"], None, gate="scalar")
+    with pytest.raises(ValueError):
+        gdr_fwd(c["q"], c["k"], c["v"], c["beta"], None, gate="none",
+                cu_seqlens=[0, 3, 2])
+
+
+# ------------------------------------------- planted mistakes (mutation test)
+_MUTANTS = {
+    # sign of the residual
+    "residual_sign": ("bt * (vt[j] - acc)", "bt * (vt[j] + acc)"),
+    # beta applied to v only
+    "beta_on_v_only": ("bt * (vt[j] - acc)", "(bt * vt[j] - acc)"),
+    # write with q instead of k
+    "write_with_q": ("S[c * dv + j] += kt[c] * r[j];",
+                     "S[c * dv + j] += qt[c] * r[j];"),
+    # read out with k instead of q
+    "readout_with_k": ("acc += S[c * dv + j] * qt[c];",
+                       "acc += S[c * dv + j] * kt[c];"),
+    # decay with the wrong sign of the log
+    "decay_sign": ("a[c] = exp(J->log_alpha[(size_t)t * H + h]);",
+                   "a[c] = exp(-J->log_alpha[(size_t)t * H + h]);"),
+    # channel-wise decay with reversed channel index
+    "decay_channel_index": (
+        "a[c] = exp(J->log_alpha[((size_t)t * H + h) * dk + c]);",
+        "a[c] = exp(J->log_alpha[((size_t)t * H + h) * dk + (dk - 1 - c)]);"),
+    # the decay dropped entirely
+    "no_decay": ("S[c * dv + j] *= a[c];", "S[c * dv + j] *= 1.0;"),
+    # the initial state ignored
+    "ignore_s0": ("if (J->s0)\n", "if (0)\n"),
+}
+
+
+def _mutant_sources():
+    src = open(oracle._SRC).read()
+    out = {name: src.replace(a, b, 1) for name, (a, b) in _MUTANTS.items()}
+    # read-out before the write of the current token: move the output loop
+    # above the write loop
+    w0 = src.index("    /* write S += k u^T */")
+    o0 = src.index("    /* output o = S^T q */")
+    o1 = src.index("  }\n  if (J->sT)")
+    out["read_before_write"] = src[:w0] + src[o0:o1] + src[w0:o0] + src[o1:]
+    # decay applied after the erase and the write
+    d0 = src.index("    for (int c = 0; c < dk; ++c)\n      for (int j = 0; "
+                   "j < dv; ++j) S[c * dv + j] *= a[c];\n")
+    d1 = d0 + len("    for (int c = 0; c < dk; ++c)\n      for (int j = 0; "
+                  "j < dv; ++j) S[c * dv + j] *= a[c];\n")
+    moved = src[:d0] + src[d1:]
+    o0m = moved.index("    /* output o = S^T q */")
+    out["decay_after_write"] = moved[:o0m] + src[d0:d1] + moved[o0m:]
+    for name, s in out.items():
+        assert s != src, name
+    return out
+
+
+def test_pins_catch_planted_mistakes(oracle_lib):
+    assert run_battery(oracle_lib) == []
+    tmp = tempfile.mkdtemp(prefix="oracle_mutants_")
+    try:
+        for name, s in _mutant_sources().items():
+            c_path = os.path.join(tmp, f"{name}.c")
+            so_path = os.path.join(tmp, f"{name}.so")
+            open(c_path, "w").write(s)
+            oracle.build(force=True, src=c_path, out=so_path)
+            fails = run_battery(oracle.load(so_path))
+            assert fails, f"planted mistake '{name}' passed every pin"
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
+
+
+def test_oracle_builds_with_warnings_clean():
+    r = subprocess.run(["gcc", "-O2", "-Wall", "-Wextra", "-fsyntax-only",
+                        "-std=c11", oracle._SRC], capture_output=True,
+                       text=True)
+    assert r.returncode == 0 and "warning" not in r.stderr, r.stderr
