@@ -1,0 +1,440 @@
+"""Benchmark of libgdr's chunkwise gated-delta forward pass.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--algo auto|staged|fused_tc]
+
+One step = one gdr_chunk_fwd call over one batch of the workload (all four
+stages: log-decay cumsum, WY/UT transform, state passing, output), inputs
+resident in HBM.  Timing: W untimed warm-up steps, then K steps bracketed by a
+barrier and a device synchronise, timed with CUDA events on the launching
+stream; the max over ranks is reported.  The workload's inputs (>= 557 MB at
+the headline size) exceed the 126 MB L2, so no flush is done between steps.
+
+N > 1 (launched with torch.distributed.run): every rank runs its own full
+workload on its own GPU (independent sequences, weak scaling); the only
+collectives are the barrier and the max/gather of timings.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("tokens/s & TFLOP/s, chunked gated-delta fwd H16 d128 T4096 bf16; "
+          "% roofline")
+# nominal-figure fallback, used only without the measured file
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                  "bf16_tflops_sustained": 1400.0}
+
+
+def flops_per_token_head(C, dk, dv):
+    # six dense tile products per token-head: K K^T, T.K, Q K^T (2 C dk each),
+    # T.V, P.V_new (2 C dv each), W.S, K^T.V_new, Q.S (2 dk dv each)
+    return 6 * C * dk + 4 * C * dv + 6 * dk * dv
+
+
+def algorithmic_bytes(w, ntok, nseq):
+    """Bytes a step must move at least: q, k, v, out in the I/O dtype, beta
+    and log-alpha in fp32, initial and final state in fp32."""
+    esz = 4 if w.dtype == "fp32" else 2
+    per_th = esz * (2 * w.dk + 2 * w.dv) + 4
+    if w.gate == "scalar":
+        per_th += 4
+    elif w.gate == "channel":
+        per_th += 4 * w.dk
+    states = (2 if w.init_state else 1) * nseq * w.H * w.dk * w.dv * 4
+    return ntok * w.H * per_th + states
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(algo):
+    files = {"fused_tc": ["fused_tc.cu"],
+             "staged": ["staged.cu"]}.get(algo, [])
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "chunkwise_recurrence_b200", "csrc",
+                                   f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file, src_hash):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", kernel_file)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    m_t = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_h or not m_t or m_h.group(1) != src_hash:
+        return None
+    return float(m_t.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "samples": 0}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]),
+                             float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, x in enumerate(r[3])
+                          if x.lower() == "active"})
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(inp, nseq_sample):
+    """The first `nseq_sample` sequences of a fixed-length workload (all
+    heads), as oracle inputs."""
+    f = inp.f64()
+    for key in ("q", "k", "v", "beta", "log_alpha"):
+        if f[key] is not None:
+            f[key] = f[key][:nseq_sample]
+    if f["initial_state"] is not None:
+        f["initial_state"] = f["initial_state"][:nseq_sample]
+    return f
+
+
+def time_oracle(inp, nseq_sample):
+    import oracle
+    f = oracle_sample(inp, nseq_sample)
+    t0 = time.perf_counter()
+    _, _, threads = oracle.gdr_fwd(**f)
+    dt = time.perf_counter() - t0
+    tokens = nseq_sample * inp.w.T
+    return tokens / dt, threads, dt, tokens
+
+
+def run_reference(args, w):
+    """CPU oracle arm: rank 0 only, bounded sample per step."""
+    from chunkwise_recurrence_b200.inputs import generate
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    inp = generate(w, seed=0)
+    nsample = max(1, min(args.ref_seqs, len(inp.lengths)))
+    for _ in range(args.warmup):
+        time_oracle(inp, nsample)
+    vals, total_tok, total_t, threads = [], 0, 0.0, 1
+    for _ in range(args.steps):
+        v, threads, dt, tok = time_oracle(inp, nsample)
+        vals.append(v)
+        total_tok += tok
+        total_t += dt
+    value = total_tok / total_t
+    sample = (f"sequences 0..{nsample - 1} of {len(inp.lengths)} "
+              f"({nsample * w.T} tokens x {w.H} heads) per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value,
+        "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H,
+                   "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "gate": w.gate},
+        "cpu_baseline": {"value": value, "unit": "tokens/s",
+                         "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def launches_per_step(algo_used, w):
+    if algo_used == "fused_tc":
+        return 1
+    return 4 + (0 if w.gate == "none" else 1)
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import chunkwise_recurrence_b200 as gdr
+    from chunkwise_recurrence_b200.inputs import generate
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    inp = generate(w, seed=args.seed + rank)
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    beta = inp.beta.to(dev)
+    la = None if inp.log_alpha is None else inp.log_alpha.to(dev)
+    s0 = None if inp.s0 is None else inp.s0.to(dev)
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.to(dev)
+    out = torch.empty_like(v)
+    sT = torch.empty(inp.nseq, w.H, w.dk, w.dv, dtype=torch.float32,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gdr.chunk_fwd(q, k, v, beta, la, s0, chunk=w.chunk, gate=w.gate,
+                      cu_seqlens=cu, out=out, final_state=sT, algo=args.algo,
+                      stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if gdr.device_error() != 0:
+        raise RuntimeError("device-side error during warm-up")
+    algo_used = args.algo
+    if algo_used == "auto":
+        algo_used = ("fused_tc" if (w.dtype == "bf16" and w.dk == 128 and
+                                    w.dv == 128 and w.chunk == 64 and
+                                    gdr_fused_available())
+                     else "staged")
+
+    # ---- device-timed region (inputs resident in HBM)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_gpu_index(local)) as clocks:
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    if gdr.device_error() != 0:
+        raise RuntimeError("device-side error during timing")
+
+    # ---- end to end through the host-buffer entry point
+    pin = lambda t: None if t is None else t.pin_memory()  # noqa: E731
+    hq, hk, hv, hb = pin(inp.q), pin(inp.k), pin(inp.v), pin(inp.beta)
+    hla, hs0 = pin(inp.log_alpha), pin(inp.s0)
+    hcu = None if inp.cu_seqlens is None else inp.cu_seqlens
+    hout = torch.empty_like(inp.v).pin_memory()
+    hsT = torch.empty(inp.nseq, w.H, w.dk, w.dv).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in
+              (hq, hk, hv, hb, hla, hs0, hcu) if t is not None)
+    d2h = hout.numel() * hout.element_size() + hsT.numel() * 4
+
+    def e2e_step():
+        gdr.chunk_fwd_host(hq, hk, hv, hb, hla, hs0, out=hout,
+                           final_state=hsT, chunk=w.chunk, gate=w.gate,
+                           cu_seqlens=hcu, algo=args.algo, stream=stream)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(1, min(args.steps, 10))
+    ea, eb = (torch.cuda.Event(enable_timing=True),
+              torch.cuda.Event(enable_timing=True))
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ea.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    eb.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ea.elapsed_time(eb)
+
+    # ---- max over ranks
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    ntok = inp.ntok
+    tokens_per_step = ntok * ws
+    value = tokens_per_step * args.steps / (total_ms / 1e3)
+    e2e_value = tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+    ms = total_ms / args.steps
+    fl = flops_per_token_head(w.chunk, w.dk, w.dv) * ntok * w.H
+    by = algorithmic_bytes(w, ntok, inp.nseq)
+    peaks, peak_src = load_peaks()
+    kernel_ms = statistics.mean(per_step)
+    achieved_gbs = by / (kernel_ms / 1e3) / 1e9
+    src_hash = kernel_source_hash(algo_used)
+    traffic = recorded_traffic(f"{algo_used}_{w.name}.md", src_hash)
+    roofline = {
+        "bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
+        "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
+        "traffic": traffic,
+        "peak_source": peak_src,
+        "kernel": "gdr_fused_tc_kernel" if algo_used == "fused_tc"
+        else "staged path (5 kernels, whole call)",
+        "algorithmic_bytes_per_launch": by,
+        "tflops": fl / (kernel_ms / 1e3) / 1e12,
+        "tensor_frac": fl / (kernel_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+        "roofline_time_us": 1e6 * max(by / (peaks["hbm_gbs"] * 1e9),
+                                      fl / (peaks["bf16_tflops"] * 1e12)),
+    }
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H,
+                   "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "gate": w.gate,
+                   "global_batch": w.B * ws, "seq_len": w.T,
+                   "parallelism": f"dp{ws} (independent sequences)",
+                   "algo": algo_used,
+                   "l2": "inputs larger than L2 (no flush)"},
+        "tflops": fl * ws / (ms / 1e3) / 1e12,
+        "roofline": roofline,
+        "clocks": clocks.summary(),
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d * ws, "d2h_bytes_per_step": d2h * ws,
+                "entry": "gdr_chunk_fwd_host (pinned host buffers)"},
+        "gpu_launches": launches_per_step(algo_used, w) * args.steps,
+        "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        nsample = max(1, min(args.cpu_seqs, len(inp.lengths)))
+        val, threads, dt, tok = time_oracle(inp, nsample)
+        line["cpu_baseline"] = {
+            "value": val, "unit": "tokens/s", "cores": threads,
+            "kind": "oracle",
+            "sample": (f"sequences 0..{nsample - 1} of {len(inp.lengths)} "
+                       f"({tok} tokens x {w.H} heads), {dt:.1f} s wall")}
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def gdr_fused_available():
+    from chunkwise_recurrence_b200 import fused_tc_available
+    return fused_tc_available()
+
+
+def local_gpu_index(local):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x for x in vis.split(",") if x.strip()]
+        if local < len(ids):
+            return ids[local]
+    return local
+
+
+def main(argv=None):
+    from chunkwise_recurrence_b200.inputs import HEADLINE, WORKLOADS
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS))
+    ap.add_argument("--algo", default="auto",
+                    choices=["auto", "staged", "fused_tc"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seqs", type=int, default=4,
+                    help="sequences in the CPU-baseline sample")
+    ap.add_argument("--ref-seqs", type=int, default=2,
+                    help="sequences per step in the reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if w.varlen_nseq:
+        raise SystemExit("the benchmark times fixed-length workloads")
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,1 +1,174 @@
-"""libgdr binding placeholder (filled in with the C-ABI binding)."""
+"""chunkwise_recurrence_b200 -- Python binding of libgdr.
+
+libgdr computes the chunkwise-parallel forward pass of the gated delta rule
+(DeltaNet, Gated DeltaNet and KDA) on one B200.  This module only marshals
+arguments into the C ABI declared in ``include/gdr.h``; every step of the
+computation runs in the library's CUDA kernels.  PyTorch supplies device
+memory and streams.  There is no CPU fallback: if ``libgdr.so`` is missing the
+calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["chunk_fwd", "chunk_fwd_host", "device_error", "status_string",
+           "algo_applies", "fused_tc_available",
+           "GdrError", "load_library", "LIB_PATH", "GATES", "ALGOS",
+           "EXPORTED_SYMBOLS"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdr.so")
+
+GATES = {"none": 0, "scalar": 1, "channel": 2}
+ALGOS = {"auto": 0, "staged": 1, "fused_tc": 2}
+DTYPES = {torch.bfloat16: 0, torch.float32: 1}
+STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARGUMENT", 2: "GDR_ERR_UNSUPPORTED",
+          3: "GDR_ERR_CUDA", 4: "GDR_ERR_OUT_OF_MEMORY", 5: "GDR_ERR_TIMEOUT"}
+EXPORTED_SYMBOLS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_device_error",
+                    "gdr_algo_applies", "gdr_status_string")
+
+_lib = None
+
+
+class GdrError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+
+
+class _Opts(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("gate", ctypes.c_int),
+                ("cu_seqlens", ctypes.c_void_p), ("num_seqs", ctypes.c_int),
+                ("algo", ctypes.c_int)]
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libgdr (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with "
+            "`python -m chunkwise_recurrence_b200.build` (needs nvcc)")
+    lib = ctypes.CDLL(path)
+    vp, fp, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
+    for name in ("gdr_chunk_fwd", "gdr_chunk_fwd_host"):
+        f = getattr(lib, name)
+        f.restype = ctypes.c_int
+        f.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, vp,
+                      ctypes.POINTER(_Opts)]
+    lib.gdr_device_error.restype = ctypes.c_int
+    lib.gdr_device_error.argtypes = [vp, i]
+    lib.gdr_algo_applies.restype = ctypes.c_int
+    lib.gdr_algo_applies.argtypes = [i, i, i, i, i, i]
+    lib.gdr_status_string.restype = ctypes.c_char_p
+    lib.gdr_status_string.argtypes = [i]
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def algo_applies(algo: str, dtype: str, gate: str, dk: int, dv: int,
+                 chunk: int) -> bool:
+    """Whether `algo` can run this dtype ("bf16"/"fp32"), gate and shape."""
+    dt = {"bf16": 0, "fp32": 1}[dtype]
+    return bool(load_library().gdr_algo_applies(ALGOS[algo], dt, GATES[gate],
+                                                dk, dv, chunk))
+
+
+def fused_tc_available() -> bool:
+    """Whether the fused tensor-core kernel serves the headline shape."""
+    return algo_applies("fused_tc", "bf16", "scalar", 128, 128, 64)
+
+
+def status_string(code: int) -> str:
+    return load_library().gdr_status_string(int(code)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _shapes(q, v, cu_seqlens):
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, T, H, d]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    nseq = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
+    return B, T, H, dk, dv, nseq
+
+
+def _gate_of(log_alpha, gate):
+    if gate is not None:
+        return gate
+    if log_alpha is None:
+        return "none"
+    return "scalar" if log_alpha.dim() == 3 else "channel"
+
+
+def chunk_fwd(q, k, v, beta, log_alpha=None, initial_state=None, *,
+              chunk: int = 64, gate: str | None = None, cu_seqlens=None,
+              out=None, final_state=None, output_final_state: bool = True,
+              algo: str = "auto", stream=None):
+    """Run ``gdr_chunk_fwd`` on CUDA tensors (layouts as in include/gdr.h).
+
+    Returns (out, final_state); final_state is None if not requested.
+    """
+    lib = load_library()
+    B, T, H, dk, dv, nseq = _shapes(q, v, cu_seqlens)
+    if out is None:
+        out = torch.empty_like(v)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(nseq, H, dk, dv, dtype=torch.float32,
+                                  device=q.device)
+    g = _gate_of(log_alpha, gate)
+    opts = _Opts(DTYPES[q.dtype], GATES[g],
+                 None if cu_seqlens is None else cu_seqlens.data_ptr(),
+                 nseq if cu_seqlens is not None else 0, ALGOS[algo])
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    rc = lib.gdr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                           _ptr(beta), _ptr(initial_state), _ptr(out),
+                           _ptr(final_state), B, T, H, dk, dv, chunk,
+                           ctypes.c_void_p(stream.cuda_stream),
+                           ctypes.byref(opts))
+    if rc != 0:
+        raise GdrError(rc, "gdr_chunk_fwd")
+    return out, final_state
+
+
+def chunk_fwd_host(q, k, v, beta, log_alpha=None, initial_state=None, *,
+                   out, final_state=None, chunk: int = 64,
+                   gate: str | None = None, cu_seqlens=None,
+                   algo: str = "auto", stream=None):
+    """Run ``gdr_chunk_fwd_host`` on CPU tensors (pinned for async copies).
+    Outputs land in ``out`` / ``final_state`` once ``stream`` is synchronised."""
+    lib = load_library()
+    B, T, H, dk, dv, nseq = _shapes(q, v, cu_seqlens)
+    g = _gate_of(log_alpha, gate)
+    opts = _Opts(DTYPES[q.dtype], GATES[g],
+                 None if cu_seqlens is None else cu_seqlens.data_ptr(),
+                 nseq if cu_seqlens is not None else 0, ALGOS[algo])
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    rc = lib.gdr_chunk_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                _ptr(beta), _ptr(initial_state), _ptr(out),
+                                _ptr(final_state), B, T, H, dk, dv, chunk,
+                                ctypes.c_void_p(stream.cuda_stream),
+                                ctypes.byref(opts))
+    if rc != 0:
+        raise GdrError(rc, "gdr_chunk_fwd_host")
+    return out, final_state
+
+
+def device_error(stream=None, clear: bool = True) -> int:
+    """Synchronise ``stream`` and return the library's device error status."""
+    lib = load_library()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return lib.gdr_device_error(ctypes.c_void_p(stream.cuda_stream),
+                                int(clear))

@@ -1,0 +1,49 @@
+// Internal declarations shared by the host API and the kernel files of libgdr.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "gdr.h"
+
+namespace gdr {
+
+// One chunk of one sequence: tokens [tok0, tok0 + len), sequence `seq`.
+struct ChunkInfo {
+  int tok0;
+  int len;
+  int seq;
+  int pad;
+};
+
+// Problem description after host validation.  Token index tok runs over the
+// flattened [B*T] (fixed length) or packed [T] (varlen) token axis; element
+// (tok, h, c) of a [.., H, d] tensor sits at (tok * H + h) * d + c.
+struct Problem {
+  const void *q, *k, *v;
+  const float *log_alpha, *beta, *s0;
+  void *out;
+  float *sT;
+  const int32_t *cu;  // device, nseq+1 entries, or nullptr (fixed length)
+  int nseq;           // number of sequences (B, or num_seqs)
+  int T;              // per-sequence length (fixed) / packed total (varlen)
+  int ntok;           // total tokens
+  int H, dk, dv, chunk;
+  gdr_dtype dtype;
+  gdr_gate gate;
+  int max_chunks;     // upper bound on the number of chunks over all sequences
+};
+
+// Staged path: four kernels + a chunk-table kernel, fp32 CUDA-core math.
+size_t staged_workspace_bytes(const Problem &p);
+cudaError_t staged_run(const Problem &p, void *workspace, cudaStream_t s);
+
+// Fused tensor-core path.
+bool fused_tc_applies(const Problem &p);
+cudaError_t fused_tc_run(const Problem &p, cudaStream_t s);
+// Reads (and optionally clears) the fused kernel's sticky device error word.
+cudaError_t fused_tc_read_error(unsigned *word, bool clear);
+
+}  // namespace gdr

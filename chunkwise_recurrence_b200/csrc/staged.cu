@@ -1,0 +1,411 @@
+// Staged path of libgdr: the chunkwise gated delta rule as four kernels with
+// fp32 CUDA-core arithmetic and the intermediates in scratch memory.
+//
+//   (a) cumsum_kernel  : in-chunk cumulative log-decay g_r = sum_{s<=r} log a_s
+//   (b) wy_kernel      : A = strictly-lower beta_r k_r^T Gamma_r Gamma_i^-1 k_i,
+//                        T = (I + A)^-1 by forward substitution,
+//                        W = T diag(beta) (K . e^g),  U = T diag(beta) V
+//   (c) state_kernel   : sequential over the chunks of one (sequence, head,
+//                        dv tile): V_new = U - W S_n,
+//                        S_{n+1} = Gamma_C S_n + (K . e^{g_C - g})^T V_new
+//   (d) output_kernel  : O = (Q . e^g) S_n + mask_{i<=r}[(Q . e^g)(K . e^-g)^T] V_new
+//
+// The chunkwise form rests on the update being affine in the preceding memory
+// ("DeltaTTT: Layerwise Optimization for Nonlinear Recurrent Memory",
+// §2 Background) and on the WY form with the decay folded into the erase
+// factors (Gated DeltaNet-2 abstract, comparative-study page 2607.07953).
+// Decay ratios exp(g_r - g_i) are always formed as one exponential of a
+// difference with i <= r, so they never exceed 1 for log-decays <= 0.
+//
+// This path serves every supported shape and both dtypes; it is the fp32
+// path (tensor-core TF32 cannot hold a 1e-4 relative error) and the reference
+// layout for the fused tensor-core kernel.
+
+#include <cuda_bf16.h>
+
+#include "gdr_internal.h"
+
+namespace gdr {
+namespace {
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Builds the chunk table from the sequence boundaries.  Boundaries are
+// clamped to [previous end, ntok] so that the table never exceeds
+// ntok / C + nseq entries, whatever the device-side contents of cu.
+__global__ void chunk_table_kernel(const int32_t *cu, int nseq, int T,
+                                   int ntok, int C, ChunkInfo *table,
+                                   int *seq_first) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int j = 0, prev_end = 0;
+  for (int n = 0; n < nseq; ++n) {
+    int s0 = cu ? cu[n] : n * T;
+    int e0 = cu ? cu[n + 1] : (n + 1) * T;
+    s0 = min(max(s0, prev_end), ntok);
+    e0 = min(max(e0, s0), ntok);
+    prev_end = e0;
+    seq_first[n] = j;
+    for (int s = s0; s < e0; s += C) {
+      ChunkInfo ci;
+      ci.tok0 = s;
+      ci.len = min(C, e0 - s);
+      ci.seq = n;
+      ci.pad = 0;
+      table[j++] = ci;
+    }
+  }
+  seq_first[nseq] = j;
+}
+
+// (a) segmented cumulative log-decay, restarting at every chunk start.
+__global__ void cumsum_kernel(const float *__restrict__ log_alpha,
+                              float *__restrict__ g,
+                              const ChunkInfo *__restrict__ table,
+                              const int *__restrict__ nchunks, int H,
+                              int gdim) {
+  const int j = blockIdx.x, h = blockIdx.y;
+  if (j >= *nchunks) return;
+  const ChunkInfo ci = table[j];
+  for (int c = threadIdx.x; c < gdim; c += blockDim.x) {
+    float acc = 0.f;
+    for (int r = 0; r < ci.len; ++r) {
+      const size_t idx = ((size_t)(ci.tok0 + r) * H + h) * gdim + c;
+      acc += log_alpha[idx];
+      g[idx] = acc;
+    }
+  }
+}
+
+// Cumulative log-decay of row r, channel c (0 when there is no gate).
+__device__ __forceinline__ float gval(const float *Gs, int gdim, int r,
+                                      int c) {
+  if (gdim == 0) return 0.f;
+  return gdim == 1 ? Gs[r] : Gs[r * gdim + c];
+}
+
+// (b) intra-chunk WY/UT transform of one (chunk, head).
+template <typename Tin>
+__global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
+                          const float *__restrict__ beta,
+                          const float *__restrict__ g, float *__restrict__ W,
+                          float *__restrict__ U,
+                          const ChunkInfo *__restrict__ table,
+                          const int *__restrict__ nchunks, int H, int dk,
+                          int dv, int C, int gdim) {
+  const int j = blockIdx.x, h = blockIdx.y;
+  if (j >= *nchunks) return;
+  const ChunkInfo ci = table[j];
+  const int L = ci.len;
+  const int gd = gdim == 0 ? 1 : gdim;
+  extern __shared__ float sm[];
+  float *Ks = sm;                  // [C][dk]
+  float *Gs = Ks + C * dk;         // [C][gd]
+  float *As = Gs + C * gd;         // [C][C+1]
+  float *Ts = As + C * (C + 1);    // [C][C+1]
+  float *bs = Ts + C * (C + 1);    // [C]
+  const int tid = threadIdx.x, nt = blockDim.x;
+
+  for (int idx = tid; idx < L * dk; idx += nt) {
+    const int r = idx / dk, c = idx % dk;
+    Ks[r * dk + c] = to_f(k[((size_t)(ci.tok0 + r) * H + h) * dk + c]);
+  }
+  if (gdim)
+    for (int idx = tid; idx < L * gdim; idx += nt) {
+      const int r = idx / gdim, c = idx % gdim;
+      Gs[r * gdim + c] = g[((size_t)(ci.tok0 + r) * H + h) * gdim + c];
+    }
+  for (int r = tid; r < L; r += nt) bs[r] = beta[(size_t)(ci.tok0 + r) * H + h];
+  __syncthreads();
+
+  // A[r][i] = beta_r sum_c k_r[c] k_i[c] exp(g_r[c] - g_i[c]),  i < r
+  for (int idx = tid; idx < L * L; idx += nt) {
+    const int r = idx / L, i = idx % L;
+    float a = 0.f;
+    if (i < r) {
+      if (gdim <= 1) {
+        for (int c = 0; c < dk; ++c) a += Ks[r * dk + c] * Ks[i * dk + c];
+        if (gdim == 1) a *= __expf(Gs[r] - Gs[i]);
+      } else {
+        for (int c = 0; c < dk; ++c)
+          a += Ks[r * dk + c] * Ks[i * dk + c] *
+               __expf(Gs[r * gdim + c] - Gs[i * gdim + c]);
+      }
+      a *= bs[r];
+    }
+    As[r * (C + 1) + i] = a;
+    Ts[r * (C + 1) + i] = (r == i) ? 1.f : 0.f;
+  }
+  __syncthreads();
+
+  // T = (I + A)^-1, row by row: T[r][j] = -sum_{j<=i<r} A[r][i] T[i][j]
+  for (int r = 1; r < L; ++r) {
+    for (int jj = tid; jj < r; jj += nt) {
+      float acc = 0.f;
+      for (int i = jj; i < r; ++i) acc += As[r * (C + 1) + i] * Ts[i * (C + 1) + jj];
+      Ts[r * (C + 1) + jj] = -acc;
+    }
+    __syncthreads();
+  }
+
+  // W = T diag(beta) (K . e^g),  U = T diag(beta) V
+  for (int idx = tid; idx < L * dk; idx += nt) {
+    const int r = idx / dk, c = idx % dk;
+    float acc = 0.f;
+    for (int i = 0; i <= r; ++i)
+      acc += Ts[r * (C + 1) + i] * bs[i] * Ks[i * dk + c] *
+             __expf(gval(Gs, gdim, i, c));
+    W[((size_t)(ci.tok0 + r) * H + h) * dk + c] = acc;
+  }
+  for (int idx = tid; idx < L * dv; idx += nt) {
+    const int r = idx / dv, c = idx % dv;
+    float acc = 0.f;
+    for (int i = 0; i <= r; ++i)
+      acc += Ts[r * (C + 1) + i] * bs[i] *
+             to_f(v[((size_t)(ci.tok0 + i) * H + h) * dv + c]);
+    U[((size_t)(ci.tok0 + r) * H + h) * dv + c] = acc;
+  }
+}
+
+// (c) sequential state passing for one (sequence, head, dv tile).
+template <typename Tin>
+__global__ void state_kernel(const Tin *__restrict__ k,
+                             const float *__restrict__ g,
+                             const float *__restrict__ W,
+                             const float *__restrict__ U,
+                             const float *__restrict__ s0,
+                             float *__restrict__ sT, float *__restrict__ Sbuf,
+                             float *__restrict__ Vn,
+                             const ChunkInfo *__restrict__ table,
+                             const int *__restrict__ seq_first, int H, int dk,
+                             int dv, int C, int gdim, int DVT) {
+  const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * DVT;
+  extern __shared__ float sm[];
+  float *S = sm;              // [dk][DVT]
+  float *V = S + dk * DVT;    // [C][DVT]
+  float *gl = V + C * DVT;    // [dk]
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const size_t sbase = ((size_t)n * H + h) * dk * dv;
+
+  for (int idx = tid; idx < dk * DVT; idx += nt) {
+    const int c = idx / DVT, jj = idx % DVT;
+    S[idx] = s0 ? s0[sbase + (size_t)c * dv + j0 + jj] : 0.f;
+  }
+  __syncthreads();
+
+  const int jb = seq_first[n], je = seq_first[n + 1];
+  for (int j = jb; j < je; ++j) {
+    const ChunkInfo ci = table[j];
+    const int L = ci.len;
+    float *Sn = Sbuf + ((size_t)j * H + h) * dk * dv;
+    for (int idx = tid; idx < dk * DVT; idx += nt) {
+      const int c = idx / DVT, jj = idx % DVT;
+      Sn[(size_t)c * dv + j0 + jj] = S[idx];
+    }
+    // V_new = U - W S
+    for (int idx = tid; idx < L * DVT; idx += nt) {
+      const int r = idx / DVT, jj = idx % DVT;
+      const size_t row = (size_t)(ci.tok0 + r) * H + h;
+      float acc = U[row * dv + j0 + jj];
+      for (int c = 0; c < dk; ++c) acc -= W[row * dk + c] * S[c * DVT + jj];
+      V[r * DVT + jj] = acc;
+      Vn[row * dv + j0 + jj] = acc;
+    }
+    for (int c = tid; c < dk; c += nt)
+      gl[c] = gdim == 0 ? 0.f
+                        : g[((size_t)(ci.tok0 + L - 1) * H + h) * gdim +
+                            (gdim == 1 ? 0 : c)];
+    __syncthreads();
+    // S <- Gamma_C S + (K . e^{g_C - g})^T V_new
+    for (int idx = tid; idx < dk * DVT; idx += nt) {
+      const int c = idx / DVT, jj = idx % DVT;
+      float acc = __expf(gl[c]) * S[idx];
+      for (int r = 0; r < L; ++r) {
+        const size_t row = (size_t)(ci.tok0 + r) * H + h;
+        const float gr =
+            gdim == 0 ? 0.f : g[row * gdim + (gdim == 1 ? 0 : c)];
+        acc += to_f(k[row * dk + c]) * __expf(gl[c] - gr) * V[r * DVT + jj];
+      }
+      S[idx] = acc;
+    }
+    __syncthreads();
+  }
+  if (sT)
+    for (int idx = tid; idx < dk * DVT; idx += nt) {
+      const int c = idx / DVT, jj = idx % DVT;
+      sT[sbase + (size_t)c * dv + j0 + jj] = S[idx];
+    }
+}
+
+// (d) chunk output for one (chunk, head).
+template <typename Tin>
+__global__ void output_kernel(const Tin *__restrict__ q,
+                              const Tin *__restrict__ k,
+                              const float *__restrict__ g,
+                              const float *__restrict__ Sbuf,
+                              const float *__restrict__ Vn,
+                              Tin *__restrict__ out,
+                              const ChunkInfo *__restrict__ table,
+                              const int *__restrict__ nchunks, int H, int dk,
+                              int dv, int C, int gdim) {
+  const int j = blockIdx.x, h = blockIdx.y;
+  if (j >= *nchunks) return;
+  const ChunkInfo ci = table[j];
+  const int L = ci.len;
+  const int gd = gdim == 0 ? 1 : gdim;
+  extern __shared__ float sm[];
+  float *Qs = sm;               // [C][dk]
+  float *Ks = Qs + C * dk;      // [C][dk]
+  float *Gs = Ks + C * dk;      // [C][gd]
+  float *Ps = Gs + C * gd;      // [C][C+1]
+  const int tid = threadIdx.x, nt = blockDim.x;
+  for (int idx = tid; idx < L * dk; idx += nt) {
+    const int r = idx / dk, c = idx % dk;
+    const size_t off = ((size_t)(ci.tok0 + r) * H + h) * dk + c;
+    Qs[r * dk + c] = to_f(q[off]);
+    Ks[r * dk + c] = to_f(k[off]);
+  }
+  if (gdim)
+    for (int idx = tid; idx < L * gdim; idx += nt) {
+      const int r = idx / gdim, c = idx % gdim;
+      Gs[r * gdim + c] = g[((size_t)(ci.tok0 + r) * H + h) * gdim + c];
+    }
+  __syncthreads();
+  // P[r][i] = sum_c q_r[c] k_i[c] exp(g_r[c] - g_i[c]),  i <= r
+  for (int idx = tid; idx < L * L; idx += nt) {
+    const int r = idx / L, i = idx % L;
+    float a = 0.f;
+    if (i <= r) {
+      if (gdim <= 1) {
+        for (int c = 0; c < dk; ++c) a += Qs[r * dk + c] * Ks[i * dk + c];
+        if (gdim == 1) a *= __expf(Gs[r] - Gs[i]);
+      } else {
+        for (int c = 0; c < dk; ++c)
+          a += Qs[r * dk + c] * Ks[i * dk + c] *
+               __expf(Gs[r * gdim + c] - Gs[i * gdim + c]);
+      }
+    }
+    Ps[r * (C + 1) + i] = a;
+  }
+  __syncthreads();
+  const float *Sn = Sbuf + ((size_t)j * H + h) * dk * dv;
+  for (int idx = tid; idx < L * dv; idx += nt) {
+    const int r = idx / dv, c = idx % dv;
+    float acc = 0.f;
+    for (int e = 0; e < dk; ++e)
+      acc += Qs[r * dk + e] * __expf(gval(Gs, gdim, r, e)) *
+             Sn[(size_t)e * dv + c];
+    for (int i = 0; i <= r; ++i)
+      acc += Ps[r * (C + 1) + i] *
+             Vn[((size_t)(ci.tok0 + i) * H + h) * dv + c];
+    out[((size_t)(ci.tok0 + r) * H + h) * dv + c] = from_f<Tin>(acc);
+  }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct StagedLayout {
+  size_t table, seq_first, g, W, U, Vn, Sbuf, total;
+};
+
+StagedLayout layout(const Problem &p) {
+  const int gdim = p.gate == GDR_GATE_NONE ? 0
+                   : p.gate == GDR_GATE_SCALAR ? 1
+                                               : p.dk;
+  const size_t th = (size_t)p.ntok * p.H;
+  StagedLayout L;
+  size_t o = 0;
+  L.table = o;     o += align256(sizeof(ChunkInfo) * (size_t)p.max_chunks);
+  L.seq_first = o; o += align256(sizeof(int) * ((size_t)p.nseq + 1));
+  L.g = o;         o += align256(sizeof(float) * th * (size_t)gdim);
+  L.W = o;         o += align256(sizeof(float) * th * p.dk);
+  L.U = o;         o += align256(sizeof(float) * th * p.dv);
+  L.Vn = o;        o += align256(sizeof(float) * th * p.dv);
+  L.Sbuf = o;
+  o += align256(sizeof(float) * (size_t)p.max_chunks * p.H * p.dk * p.dv);
+  L.total = o;
+  return L;
+}
+
+template <typename Tin>
+cudaError_t run_typed(const Problem &p, char *ws, cudaStream_t s) {
+  const StagedLayout L = layout(p);
+  const int gdim = p.gate == GDR_GATE_NONE ? 0
+                   : p.gate == GDR_GATE_SCALAR ? 1
+                                               : p.dk;
+  const int gd = gdim == 0 ? 1 : gdim;
+  const int C = p.chunk;
+  ChunkInfo *table = reinterpret_cast<ChunkInfo *>(ws + L.table);
+  int *seq_first = reinterpret_cast<int *>(ws + L.seq_first);
+  int *nchunks = seq_first + p.nseq;
+  float *g = gdim ? reinterpret_cast<float *>(ws + L.g) : nullptr;
+  float *W = reinterpret_cast<float *>(ws + L.W);
+  float *U = reinterpret_cast<float *>(ws + L.U);
+  float *Vn = reinterpret_cast<float *>(ws + L.Vn);
+  float *Sbuf = reinterpret_cast<float *>(ws + L.Sbuf);
+  const Tin *q = static_cast<const Tin *>(p.q);
+  const Tin *k = static_cast<const Tin *>(p.k);
+  const Tin *v = static_cast<const Tin *>(p.v);
+  Tin *out = static_cast<Tin *>(p.out);
+
+  chunk_table_kernel<<<1, 32, 0, s>>>(p.cu, p.nseq, p.T, p.ntok, C, table,
+                                      seq_first);
+  if (p.max_chunks > 0) {
+    const dim3 grid(p.max_chunks, p.H);
+    if (gdim)
+      cumsum_kernel<<<grid, 128, 0, s>>>(p.log_alpha, g, table, nchunks, p.H,
+                                         gdim);
+    const size_t wy_smem =
+        sizeof(float) * ((size_t)C * p.dk + (size_t)C * gd +
+                         2 * (size_t)C * (C + 1) + C);
+    cudaError_t e = cudaFuncSetAttribute(
+        wy_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)wy_smem);
+    if (e != cudaSuccess) return e;
+    wy_kernel<Tin><<<grid, 256, wy_smem, s>>>(k, v, p.beta, g, W, U, table,
+                                             nchunks, p.H, p.dk, p.dv, C,
+                                             gdim);
+  }
+  const int DVT = p.dv < 32 ? p.dv : 32;
+  const size_t st_smem =
+      sizeof(float) * ((size_t)p.dk * DVT + (size_t)C * DVT + p.dk);
+  state_kernel<Tin><<<dim3(p.nseq, p.H, p.dv / DVT), 256, st_smem, s>>>(
+      k, g, W, U, p.s0, p.sT, Sbuf, Vn, table, seq_first, p.H, p.dk, p.dv, C,
+      gdim, DVT);
+  if (p.max_chunks > 0) {
+    const size_t o_smem =
+        sizeof(float) * (2 * (size_t)C * p.dk + (size_t)C * gd +
+                         (size_t)C * (C + 1));
+    cudaError_t e = cudaFuncSetAttribute(
+        output_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)o_smem);
+    if (e != cudaSuccess) return e;
+    output_kernel<Tin><<<dim3(p.max_chunks, p.H), 256, o_smem, s>>>(
+        q, k, g, Sbuf, Vn, out, table, nchunks, p.H, p.dk, p.dv, C, gdim);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t staged_workspace_bytes(const Problem &p) { return layout(p).total; }
+
+cudaError_t staged_run(const Problem &p, void *workspace, cudaStream_t s) {
+  char *ws = static_cast<char *>(workspace);
+  if (p.dtype == GDR_FP32) return run_typed<float>(p, ws, s);
+  return run_typed<__nv_bfloat16>(p, ws, s);
+}
+
+}  // namespace gdr

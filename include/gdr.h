@@ -1,0 +1,184 @@
+/*
+ * gdr.h -- C ABI of libgdr: the chunkwise-parallel forward pass of the gated
+ * delta rule on one NVIDIA B200 (sm_100a).
+ *
+ * The operation (per sequence and head; tokens t in order; state S is dk x dv):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) D_t S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * with D_t = I (DeltaNet), alpha_t I (Gated DeltaNet, one scalar per token and
+ * head) or diag(alpha_t) (KDA, one factor per key channel).
+ *
+ * Sources:
+ *  - "DeltaTTT: Layerwise Optimization for Nonlinear Recurrent Memory",
+ *    §2 Background: the delta rule is serial gradient descent on a linear
+ *    memory; the update is affine in the preceding memory, which is what allows
+ *    chunkwise-parallel evaluation while keeping token-level corrections.
+ *    §4.1: a gradient step on a linear-regression objective in the memory
+ *    matrix is a delta-rule update.  App. B: keys are normalised.
+ *  - "Delta-Rule Linear Attention" topic page, FG^2-GDN card: KDA refines the
+ *    head-wise decay of Gated DeltaNet into a channel-wise decay.
+ *  - Gated DeltaNet-2 abstract, comparative-study page (2607.07953): a
+ *    chunkwise WY algorithm with channel-wise decay absorbed into the erase
+ *    factors; GDN-2 reduces to KDA and then to Gated DeltaNet.
+ *
+ * Readings taken where the pages are silent (the pages print no equation):
+ *  - decay is applied before the erase: (I - beta k k^T) D S, the order that
+ *    type-checks for dk != dv; it only matters for the channel-wise gate;
+ *  - o_t reads the state after token t's write (the intra-chunk causal mask
+ *    includes the diagonal);
+ *  - no query scaling; keys and queries are used as given (callers normalise);
+ *  - log_alpha is the natural log of the decay and is expected to be <= 0.
+ *
+ * Conventions shared by every entry point:
+ *  - Every call returns a gdr_status; nothing throws, aborts or traps.
+ *  - Argument checks happen on the host before any CUDA call, so a rejected
+ *    call has no side effect.
+ *  - Compute calls are asynchronous on `stream`; results are valid once the
+ *    stream has been synchronised.  Inputs are never modified.
+ *  - Scratch memory is allocated and released stream-ordered on `stream`
+ *    (cudaMallocAsync / cudaFreeAsync), so calls on different streams do not
+ *    share scratch.
+ */
+#ifndef GDR_H_
+#define GDR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define GDR_API __attribute__((visibility("default")))
+#else
+#define GDR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDR_OK = 0,
+  GDR_ERR_INVALID_ARGUMENT = 1, /* null/misaligned pointer, bad size, ...   */
+  GDR_ERR_UNSUPPORTED = 2,      /* valid but not implemented (shape, dtype) */
+  GDR_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed      */
+  GDR_ERR_OUT_OF_MEMORY = 4,    /* scratch allocation failed                 */
+  GDR_ERR_TIMEOUT = 5           /* a bounded device-side wait expired        */
+} gdr_status;
+
+/* Element type of q, k, v and out.  beta, log_alpha and the states are always
+ * fp32; arithmetic is fp32 (bf16 only as tensor-core operands). */
+typedef enum { GDR_BF16 = 0, GDR_FP32 = 1 } gdr_dtype;
+
+typedef enum {
+  GDR_GATE_NONE = 0,    /* alpha = 1 (DeltaNet); log_alpha must be NULL      */
+  GDR_GATE_SCALAR = 1,  /* Gated DeltaNet: log_alpha [ntok][H]               */
+  GDR_GATE_CHANNEL = 2  /* KDA: log_alpha [ntok][H][dk]                      */
+} gdr_gate;
+
+/* Which kernels run.  AUTO takes FUSED_TC where it applies and STAGED
+ * otherwise; naming one explicitly returns GDR_ERR_UNSUPPORTED where it does
+ * not apply. */
+typedef enum {
+  GDR_ALGO_AUTO = 0,
+  /* four kernels -- (a) segmented log-decay cumsum, (b) intra-chunk WY/UT
+   * transform, (c) sequential inter-chunk state passing, (d) chunk output --
+   * fp32 CUDA-core arithmetic, intermediates in scratch.  Any supported
+   * shape, fp32 or bf16. */
+  GDR_ALGO_STAGED = 1,
+  /* one persistent kernel per (sequence, head) that runs the same four steps
+   * chunk after chunk with every intermediate on chip; chunk products on
+   * tcgen05 tensor cores (bf16 operands, fp32 accumulation in tensor memory).
+   * bf16, dk = dv = 128, chunk = 64. */
+  GDR_ALGO_FUSED_TC = 2
+} gdr_algo;
+
+typedef struct {
+  gdr_dtype dtype;
+  gdr_gate gate;
+  /* Packed variable-length batch: device pointer to num_seqs+1 int32 token
+   * offsets (0 = first, non-decreasing, last = T), or NULL for fixed-length
+   * sequences.  With cu_seqlens, B must be 1 and T is the packed total. */
+  const int32_t *cu_seqlens;
+  int num_seqs;
+  gdr_algo algo;
+} gdr_opts;
+
+/*
+ * gdr_chunk_fwd -- forward pass over a batch, chunk by chunk.
+ *
+ * Device pointers, row-major and contiguous, 16-byte aligned:
+ *   q, k          [B][T][H][dk]   dtype
+ *   v             [B][T][H][dv]   dtype
+ *   log_alpha     NULL (GDR_GATE_NONE), [B][T][H] (SCALAR) or
+ *                 [B][T][H][dk] (CHANNEL), fp32
+ *   beta          [B][T][H] fp32
+ *   initial_state [N][H][dk][dv] fp32, or NULL for a zero state
+ *   out           [B][T][H][dv]   dtype (written)
+ *   final_state   [N][H][dk][dv] fp32 (written), or NULL to skip
+ * where N = B for fixed length, or num_seqs with cu_seqlens.
+ * The caller owns every buffer; out and final_state must not overlap inputs.
+ *
+ * Sizes: B, T, H >= 0 (an empty batch is a no-op returning GDR_OK);
+ * dk, dv in {16, 32, 64, 128}; chunk in {16, 32, 64} (chunk <= 64 and a
+ * multiple of 16).  A sequence length need not be a multiple of chunk: its
+ * last chunk is simply shorter.
+ *
+ * opts may be NULL: bf16, scalar gate, fixed length, AUTO.
+ * Returns GDR_ERR_INVALID_ARGUMENT for null or misaligned pointers and
+ * inconsistent sizes, GDR_ERR_UNSUPPORTED for shapes outside the list above,
+ * GDR_ERR_OUT_OF_MEMORY if scratch cannot be allocated, GDR_ERR_CUDA if a
+ * launch fails.  Device-side waits are bounded; an expired one is reported by
+ * gdr_device_error().
+ */
+GDR_API gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v,
+                         const float *log_alpha, const float *beta,
+                         const float *initial_state, void *out,
+                         float *final_state, int B, int T, int H, int dk,
+                         int dv, int chunk, cudaStream_t stream,
+                         const gdr_opts *opts);
+
+/*
+ * gdr_chunk_fwd_host -- the same computation on HOST buffers.
+ *
+ * Every tensor pointer (and opts->cu_seqlens) is a host pointer with the
+ * layouts above.  The call allocates device buffers stream-ordered, enqueues
+ * one host-to-device copy per input, the computation, one device-to-host copy
+ * per output and the release of the device buffers, all on `stream`, and
+ * returns.  Host buffers must stay valid until `stream` is synchronised.  With
+ * page-locked (pinned) host memory the copies are asynchronous; with pageable
+ * memory the CUDA runtime makes them synchronous to the host.
+ */
+GDR_API gdr_status gdr_chunk_fwd_host(const void *q, const void *k, const void *v,
+                              const float *log_alpha, const float *beta,
+                              const float *initial_state, void *out,
+                              float *final_state, int B, int T, int H, int dk,
+                              int dv, int chunk, cudaStream_t stream,
+                              const gdr_opts *opts);
+
+/*
+ * gdr_device_error -- synchronise `stream`, then read (and clear if `clear`)
+ * the library's sticky device-side error word for the current device.
+ * Returns GDR_OK if no kernel has reported an error, GDR_ERR_TIMEOUT if a
+ * bounded wait expired, GDR_ERR_CUDA if synchronisation itself failed.
+ */
+GDR_API gdr_status gdr_device_error(cudaStream_t stream, int clear);
+
+/*
+ * gdr_algo_applies -- 1 if `algo` can run a problem of this dtype, gate and
+ * shape (AUTO and STAGED: any supported shape; FUSED_TC: bf16, dk = dv = 128,
+ * chunk = 64, any gate), else 0.  Host-only; makes no CUDA call.
+ */
+GDR_API int gdr_algo_applies(gdr_algo algo, gdr_dtype dtype, gdr_gate gate,
+                             int dk, int dv, int chunk);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+GDR_API const char *gdr_status_string(gdr_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H_ */

@@ -1,0 +1,123 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol,
+and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import chunkwise_recurrence_b200 as gdr
+from chunkwise_recurrence_b200 import build as gdr_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, INVALID, UNSUPPORTED, CUDA, OOM, TIMEOUT = range(6)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    gdr_build.build()
+    return gdr.load_library()
+
+
+def _declared_symbols():
+    syms = []
+    for name in os.listdir(os.path.join(ROOT, "include")):
+        if name.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", name)).read()
+            syms += re.findall(r"^GDR_API[^(]*?\b(\w+)\s*\(", text, re.M)
+    return syms
+
+
+def test_exports_every_declared_symbol(lib):
+    syms = _declared_symbols()
+    assert set(gdr.EXPORTED_SYMBOLS) <= set(syms)
+    for s in syms:
+        assert hasattr(lib, s), s
+
+
+def test_status_strings(lib):
+    for code, name in gdr.STATUS.items():
+        assert gdr.status_string(code) == name
+    assert gdr.status_string(99) == "GDR_ERR_UNKNOWN"
+
+
+A = 0x10000       # a 16-byte-aligned fake device address (never dereferenced)
+
+
+def call(lib, *, q=A, k=A, v=A, la=A, beta=A, s0=None, out=A, sT=None, B=1,
+         T=64, H=1, dk=128, dv=128, chunk=64, dtype=0, gate=1, cu=None,
+         nseq=0, algo=0, host=False):
+    opts = gdr._Opts(dtype, gate, cu, nseq, algo)
+    f = lib.gdr_chunk_fwd_host if host else lib.gdr_chunk_fwd
+    return f(q, k, v, la, beta, s0, out, sT, B, T, H, dk, dv, chunk, None,
+             ctypes.byref(opts))
+
+
+@pytest.mark.parametrize("host", [False, True])
+def test_rejects_bad_arguments(lib, host):
+    c = lambda **kw: call(lib, host=host, **kw)  # noqa: E731
+    assert c(q=None) == INVALID
+    assert c(out=None) == INVALID
+    assert c(beta=None) == INVALID
+    assert c(k=A + 8) == INVALID                   # misaligned
+    assert c(s0=A + 4) == INVALID
+    assert c(la=None) == INVALID                   # scalar gate needs alpha
+    assert c(gate=0) == INVALID                    # no gate forbids alpha
+    assert c(gate=7) == INVALID
+    assert c(dtype=5) == INVALID
+    assert c(algo=9) == INVALID
+    assert c(T=-1) == INVALID
+    assert c(B=-2) == INVALID
+    assert c(dk=48) == UNSUPPORTED
+    assert c(dv=256) == UNSUPPORTED
+    assert c(dk=8) == UNSUPPORTED
+    assert c(chunk=128) == UNSUPPORTED
+    assert c(chunk=8) == UNSUPPORTED
+    assert c(chunk=48) == UNSUPPORTED
+    assert c(B=2, cu=A, nseq=1) == INVALID         # varlen needs B == 1
+    assert c(cu=A, nseq=-1) == INVALID
+    assert c(nseq=3) == INVALID                    # num_seqs without cu
+    assert c(B=1 << 20, T=1 << 12) == UNSUPPORTED  # too many tokens
+    assert c(H=70000) == UNSUPPORTED
+
+
+@pytest.mark.parametrize("host", [False, True])
+def test_empty_batch_is_a_noop(lib, host):
+    # no pointer is touched and no CUDA call is made
+    assert call(lib, q=None, k=None, v=None, la=None, beta=None, out=None, gate=0,
+                B=0, host=host) == OK
+    assert call(lib, q=None, k=None, v=None, la=None, beta=None, out=None, gate=0,
+                H=0, host=host) == OK
+    assert call(lib, q=None, k=None, v=None, la=None, beta=None, out=None, gate=0,
+                cu=A, nseq=0, host=host) == OK
+
+
+@pytest.mark.parametrize("host", [False, True])
+def test_scratch_allocation_failure_is_reported(lib, host, monkeypatch):
+    monkeypatch.setenv("GDR_FAULT_INJECT_ALLOC", "1")
+    assert call(lib, algo=1, host=host) == OOM
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="missing"):
+        gdr.load_library(str(tmp_path / "libgdr.so"))
+
+
+def test_product_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "chunkwise_recurrence_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".h", ".cuh", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle", text,
+                                     re.M), f
+                assert "gdr_oracle" not in text and "liboracle" not in text, f
+
+
+def test_algo_applies(lib):
+    assert gdr.algo_applies("staged", "fp32", "none", 16, 16, 16)
+    assert gdr.algo_applies("auto", "bf16", "channel", 128, 64, 32)
+    assert not gdr.algo_applies("staged", "bf16", "scalar", 48, 128, 64)
+    assert not gdr.algo_applies("fused_tc", "fp32", "scalar", 128, 128, 64)
+    assert not gdr.algo_applies("fused_tc", "bf16", "scalar", 64, 128, 64)

@@ -1,0 +1,229 @@
+"""GPU parity: libgdr (through its C ABI) against the fp64 CPU oracle.
+
+Tolerance (the parity bar): max |gpu - oracle| / RMS(oracle) over the whole
+tensor, for `out` and `final_state` separately: <= 1e-4 for fp32 inputs,
+<= 2e-2 for bf16 inputs.  The oracle runs on the device-rounded inputs, so
+only the GPU's arithmetic is measured.
+
+Small cases span several chunks and a ragged tail and are compared element by
+element; the full-size workloads run on the GPU in full and are compared on
+sampled heads (every (sequence, head) chain is independent, so a sampled head
+is an exact sub-problem for the oracle).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import chunkwise_recurrence_b200 as gdr
+from chunkwise_recurrence_b200.inputs import (WORKLOADS, generate, head_slice,
+                                              rel_err)
+from oracle import gdr_fwd
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"fp32": 1e-4, "bf16": 2e-2}
+
+
+def _dev(t):
+    return None if t is None else t.cuda()
+
+
+def run_gpu(inp, algo="auto", chunk=None):
+    w = inp.w
+    out, sT = gdr.chunk_fwd(_dev(inp.q), _dev(inp.k), _dev(inp.v),
+                            _dev(inp.beta), _dev(inp.log_alpha),
+                            _dev(inp.s0), chunk=chunk or w.chunk, gate=w.gate,
+                            cu_seqlens=_dev(inp.cu_seqlens), algo=algo)
+    assert gdr.device_error() == 0
+    return out.float().cpu().numpy(), sT.cpu().numpy()
+
+
+def run_oracle(inp):
+    out, sT, _ = gdr_fwd(**inp.f64())
+    return out, sT
+
+
+def check(inp, algo="auto", chunk=None):
+    o, s = run_gpu(inp, algo, chunk)
+    ro, rs = run_oracle(inp)
+    tol = TOL[inp.w.dtype]
+    eo, es = rel_err(o, ro), rel_err(s, rs)
+    assert np.isfinite(o).all() and np.isfinite(s).all()
+    assert eo <= tol and es <= tol, (eo, es)
+    return eo, es
+
+
+def algos_for(w):
+    """Every kernel path that serves this workload's dtype, gate and shape."""
+    return [a for a in ("staged", "fused_tc")
+            if gdr.algo_applies(a, w.dtype, w.gate, w.dk, w.dv, w.chunk)]
+
+
+# ---- small versions of every workload (same distributions), several chunks
+# ---- plus a ragged tail
+SMALL = {
+    "deltanet_b1_h1_t256_d16_fp32": dict(),                    # full size
+    "gdn_b4_h8_t2048_d128_bf16": dict(B=2, T=3 * 64 + 37, H=3),
+    "gdn_b8_h16_t4096_d128_bf16": dict(B=2, T=5 * 64 + 1, H=2),
+    "kda_b4_h16_t4096_d128_bf16": dict(B=2, T=4 * 64 + 63, H=2),
+    "gdn_varlen8_h16_d128_bf16": dict(H=2, varlen_nseq=5, varlen_lo=1,
+                                      varlen_hi=300),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_workloads(name):
+    w = WORKLOADS[name].with_(**SMALL[name])
+    inp = generate(w, seed=0)
+    for algo in algos_for(w):
+        check(inp, algo)
+
+
+@pytest.mark.parametrize("gate", ["none", "scalar", "channel"])
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("d", [16, 32, 64, 128])
+def test_shapes_and_gates(gate, dtype, d):
+    chunk = 16 if d == 16 else 64
+    w = WORKLOADS["gdn_b4_h8_t2048_d128_bf16"].with_(
+        B=1, T=2 * chunk + 5, H=2, dk=d, dv=d, chunk=chunk, dtype=dtype,
+        gate=gate, decay_lo=0.005, decay_hi=0.05, init_state=True)
+    for algo in algos_for(w):
+        check(generate(w, seed=1), algo)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 128), (128, 32), (16, 64)])
+def test_rectangular_state(dk, dv):
+    w = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(
+        B=1, T=150, H=2, dk=dk, dv=dv, init_state=True)
+    check(generate(w, seed=2), "staged")
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_chunk_size_does_not_change_the_result(chunk):
+    w = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=1, T=200, H=2,
+                                                       chunk=chunk)
+    check(generate(w, seed=3), "staged", chunk=chunk)
+
+
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 128])
+def test_short_and_boundary_lengths(T):
+    w = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=2, T=T, H=2)
+    inp = generate(w, seed=4)
+    for algo in algos_for(w):
+        check(inp, algo)
+
+
+def time_slice(inp, a, b):
+    """Tokens [a, b) of a fixed-length batch, same heads and initial state."""
+    cut = lambda t: None if t is None else t[:, a:b].contiguous()  # noqa
+    return dataclasses.replace(inp, w=inp.w.with_(T=b - a), q=cut(inp.q),
+                               k=cut(inp.k), v=cut(inp.v),
+                               beta=cut(inp.beta),
+                               log_alpha=cut(inp.log_alpha),
+                               lengths=[b - a] * len(inp.lengths))
+
+
+def test_zero_length_sequences_pass_state_through():
+    lens = [0, 70, 0, 1, 130, 0]
+    ntok = sum(lens)
+    w = WORKLOADS["gdn_varlen8_h16_d128_bf16"].with_(
+        B=1, T=ntok, H=2, varlen_nseq=0, init_state=False)
+    inp = generate(w, seed=5)
+    cu = torch.zeros(len(lens) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lens), 0).to(torch.int32)
+    g = torch.Generator().manual_seed(6)
+    inp = dataclasses.replace(
+        inp, w=inp.w.with_(varlen_nseq=len(lens)), cu_seqlens=cu,
+        lengths=lens,
+        s0=torch.randn(len(lens), 2, 128, 128, generator=g) * 0.02)
+    for algo in algos_for(inp.w):
+        o, s = run_gpu(inp, algo)
+        ro, rs = run_oracle(inp)
+        assert rel_err(o, ro) <= 2e-2 and rel_err(s, rs) <= 2e-2
+        # an empty sequence returns its initial state unchanged
+        for n in (0, 2, 5):
+            assert np.array_equal(s[n], inp.s0[n].numpy())
+
+
+def test_state_carry_across_calls():
+    w = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=2, T=300, H=2)
+    inp = generate(w, seed=8)
+    cut = 130          # not a chunk multiple
+    for algo in algos_for(w):
+        o, s = run_gpu(inp, algo)
+        o1, s1 = run_gpu(time_slice(inp, 0, cut), algo)
+        second = dataclasses.replace(time_slice(inp, cut, 300),
+                                     s0=torch.from_numpy(s1))
+        o2, s2 = run_gpu(second, algo)
+        oo = np.concatenate([o1, o2], axis=1)
+        assert rel_err(oo, o) <= 2e-2 and rel_err(s2, s) <= 2e-2
+
+
+def test_final_state_optional_and_no_out_of_bounds_writes():
+    w = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=2, T=77, H=2)
+    inp = generate(w, seed=9)
+    for algo in algos_for(w):
+        guard = 4096
+        buf = torch.full((2 * 77 * 2 * 128 + 2 * guard,), 7.0,
+                         dtype=torch.bfloat16, device="cuda")
+        out = buf[guard:guard + 2 * 77 * 2 * 128].view(2, 77, 2, 128)
+        gdr.chunk_fwd(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(),
+                      inp.beta.cuda(), inp.log_alpha.cuda(), inp.s0.cuda(),
+                      out=out, output_final_state=False, algo=algo)
+        torch.cuda.synchronize()
+        assert torch.all(buf[:guard] == 7.0) and torch.all(
+            buf[-guard:] == 7.0)
+        ro, _ = run_oracle(inp)
+        assert rel_err(out.float().cpu().numpy(), ro) <= 2e-2
+
+
+def test_host_entry_matches_device_entry():
+    w = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(B=2, T=150, H=2,
+                                                       init_state=True)
+    inp = generate(w, seed=10)
+    for algo in algos_for(w):
+        o, s = run_gpu(inp, algo)
+        pin = lambda t: None if t is None else t.pin_memory()  # noqa: E731
+        out = torch.empty_like(inp.v).pin_memory()
+        sT = torch.empty(2, 2, 128, 128).pin_memory()
+        gdr.chunk_fwd_host(pin(inp.q), pin(inp.k), pin(inp.v), pin(inp.beta),
+                           pin(inp.log_alpha), pin(inp.s0), out=out,
+                           final_state=sT, algo=algo)
+        torch.cuda.synchronize()
+        assert np.array_equal(out.float().numpy(), o)
+        assert np.array_equal(sT.numpy(), s)
+
+
+def test_deterministic():
+    w = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=2, T=200, H=2)
+    inp = generate(w, seed=11)
+    for algo in algos_for(w):
+        o1, s1 = run_gpu(inp, algo)
+        o2, s2 = run_gpu(inp, algo)
+        assert np.array_equal(o1, o2) and np.array_equal(s1, s2)
+
+
+# ---- full-size workloads, sampled heads
+FULL_SAMPLE_HEADS = {
+    "deltanet_b1_h1_t256_d16_fp32": [0],
+    "gdn_b4_h8_t2048_d128_bf16": [0, 5],
+    "gdn_b8_h16_t4096_d128_bf16": [3, 12],
+    "kda_b4_h16_t4096_d128_bf16": [7],
+    "gdn_varlen8_h16_d128_bf16": [1, 14],
+}
+
+
+@pytest.mark.parametrize("name", list(FULL_SAMPLE_HEADS))
+def test_full_size_workloads_sampled_heads(name):
+    w = WORKLOADS[name]
+    inp = generate(w, seed=0)
+    heads = FULL_SAMPLE_HEADS[name]
+    sub = head_slice(inp, heads)
+    ro, rs = run_oracle(sub)
+    for algo in ["auto"] + algos_for(w):
+        o, s = run_gpu(inp, algo)
+        o, s = o[:, :, heads], s[:, heads]
+        tol = TOL[w.dtype]
+        assert rel_err(o, ro) <= tol and rel_err(s, rs) <= tol, algo
