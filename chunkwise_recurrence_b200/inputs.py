@@ -159,6 +159,13 @@ def head_slice(inp: Inputs, heads) -> Inputs:
                   cu_seqlens=inp.cu_seqlens, lengths=inp.lengths)
 
 
+def round_to_dtype(x, dtype: str):
+    """An fp64 array rounded (nearest-even) to the output dtype and back:
+    the closest result a kernel writing that dtype can return."""
+    t = torch.from_numpy(np.ascontiguousarray(np.asarray(x, np.float64)))
+    return t.to(TORCH_DTYPE[dtype]).to(torch.float64).numpy()
+
+
 def rel_err(x, ref) -> float:
     """max |x - ref| / RMS(ref) over the whole tensor (the parity metric)."""
     x = np.asarray(x, np.float64)

@@ -3,7 +3,11 @@
 Tolerance (the parity bar): max |gpu - oracle| / RMS(oracle) over the whole
 tensor, for `out` and `final_state` separately: <= 1e-4 for fp32 inputs,
 <= 2e-2 for bf16 inputs.  The oracle runs on the device-rounded inputs, so
-only the GPU's arithmetic is measured.
+only the GPU's arithmetic is measured.  `out` is written in the input dtype,
+so its reference is the oracle's output rounded to that dtype (for bf16 the
+rounding alone is up to 2^-8 max|o|, which exceeds 2e-2 RMS once max|o| > 5.1
+RMS, as on the 1.3B-layer workload); `final_state` is fp32 and compared with
+the unrounded oracle.
 
 Small cases span several chunks and a ragged tail and are compared element by
 element; the full-size workloads run on the GPU in full and are compared on
@@ -18,7 +22,7 @@ import torch
 
 import chunkwise_recurrence_b200 as gdr
 from chunkwise_recurrence_b200.inputs import (WORKLOADS, generate, head_slice,
-                                              rel_err)
+                                              rel_err, round_to_dtype)
 from oracle import gdr_fwd
 
 pytestmark = pytest.mark.gpu
@@ -41,8 +45,9 @@ def run_gpu(inp, algo="auto", chunk=None):
 
 
 def run_oracle(inp):
+    """Oracle result with `out` rounded to the output dtype (see above)."""
     out, sT, _ = gdr_fwd(**inp.f64())
-    return out, sT
+    return round_to_dtype(out, inp.w.dtype), sT
 
 
 def check(inp, algo="auto", chunk=None):
