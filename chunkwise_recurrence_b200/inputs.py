@@ -159,11 +159,27 @@ def head_slice(inp: Inputs, heads) -> Inputs:
                   cu_seqlens=inp.cu_seqlens, lengths=inp.lengths)
 
 
-def round_to_dtype(x, dtype: str):
-    """An fp64 array rounded (nearest-even) to the output dtype and back:
-    the closest result a kernel writing that dtype can return."""
-    t = torch.from_numpy(np.ascontiguousarray(np.asarray(x, np.float64)))
-    return t.to(TORCH_DTYPE[dtype]).to(torch.float64).numpy()
+def half_ulp(x, dtype: str):
+    """Half a unit in the last place of |x| in `dtype` ("bf16": 8 significant
+    bits, "fp32": 24): the rounding error of a correctly rounded result."""
+    bits = {"bf16": 8, "fp32": 24}[dtype]
+    _, e = np.frexp(np.abs(np.asarray(x, np.float64)))
+    return np.ldexp(1.0, (e - 1 - bits).astype(np.int64))
+
+
+def out_err(x, ref, dtype: str) -> float:
+    """Parity metric of an output stored in `dtype`: max over elements of
+    max(0, |x - ref| - u) / RMS(ref), u = half an ulp (in `dtype`) of the
+    larger of |x| and |ref|.  The stored output must round its value; this
+    discounts exactly that rounding, so the budget measures the arithmetic."""
+    x = np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    if not x.size:
+        return 0.0
+    u = half_ulp(np.maximum(np.abs(x), np.abs(ref)), dtype)
+    d = np.maximum(np.abs(x - ref) - u, 0.0)
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    return float(d.max()) / rms if rms else float(d.max())
 
 
 def rel_err(x, ref) -> float:

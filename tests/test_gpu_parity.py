@@ -3,11 +3,11 @@
 Tolerance (the parity bar): max |gpu - oracle| / RMS(oracle) over the whole
 tensor, for `out` and `final_state` separately: <= 1e-4 for fp32 inputs,
 <= 2e-2 for bf16 inputs.  The oracle runs on the device-rounded inputs, so
-only the GPU's arithmetic is measured.  `out` is written in the input dtype,
-so its reference is the oracle's output rounded to that dtype (for bf16 the
-rounding alone is up to 2^-8 max|o|, which exceeds 2e-2 RMS once max|o| > 5.1
-RMS, as on the 1.3B-layer workload); `final_state` is fp32 and compared with
-the unrounded oracle.
+only the GPU's arithmetic is measured.  `out` is written in the input dtype and
+must be rounded to it: for bf16 that rounding alone is up to 2^-8 max|o|, above
+2e-2 RMS once max|o| > 5.1 RMS (the 1.3B-layer workload has max|o| = 7.6 RMS).
+So the metric of `out` discounts, per element, half an ulp of the output dtype
+(`out_err`); `final_state` is fp32 and uses the plain metric.
 
 Small cases span several chunks and a ragged tail and are compared element by
 element; the full-size workloads run on the GPU in full and are compared on
@@ -22,7 +22,7 @@ import torch
 
 import chunkwise_recurrence_b200 as gdr
 from chunkwise_recurrence_b200.inputs import (WORKLOADS, generate, head_slice,
-                                              rel_err, round_to_dtype)
+                                              out_err, rel_err)
 from oracle import gdr_fwd
 
 pytestmark = pytest.mark.gpu
@@ -45,16 +45,15 @@ def run_gpu(inp, algo="auto", chunk=None):
 
 
 def run_oracle(inp):
-    """Oracle result with `out` rounded to the output dtype (see above)."""
     out, sT, _ = gdr_fwd(**inp.f64())
-    return round_to_dtype(out, inp.w.dtype), sT
+    return out, sT
 
 
 def check(inp, algo="auto", chunk=None):
     o, s = run_gpu(inp, algo, chunk)
     ro, rs = run_oracle(inp)
     tol = TOL[inp.w.dtype]
-    eo, es = rel_err(o, ro), rel_err(s, rs)
+    eo, es = out_err(o, ro, inp.w.dtype), rel_err(s, rs)
     assert np.isfinite(o).all() and np.isfinite(s).all()
     assert eo <= tol and es <= tol, (eo, es)
     return eo, es
@@ -146,7 +145,7 @@ def test_zero_length_sequences_pass_state_through():
     for algo in algos_for(inp.w):
         o, s = run_gpu(inp, algo)
         ro, rs = run_oracle(inp)
-        assert rel_err(o, ro) <= 2e-2 and rel_err(s, rs) <= 2e-2
+        assert out_err(o, ro, "bf16") <= 2e-2 and rel_err(s, rs) <= 2e-2
         # an empty sequence returns its initial state unchanged
         for n in (0, 2, 5):
             assert np.array_equal(s[n], inp.s0[n].numpy())
@@ -163,7 +162,7 @@ def test_state_carry_across_calls():
                                      s0=torch.from_numpy(s1))
         o2, s2 = run_gpu(second, algo)
         oo = np.concatenate([o1, o2], axis=1)
-        assert rel_err(oo, o) <= 2e-2 and rel_err(s2, s) <= 2e-2
+        assert out_err(oo, o, "bf16") <= 2e-2 and rel_err(s2, s) <= 2e-2
 
 
 def test_final_state_optional_and_no_out_of_bounds_writes():
@@ -181,7 +180,7 @@ def test_final_state_optional_and_no_out_of_bounds_writes():
         assert torch.all(buf[:guard] == 7.0) and torch.all(
             buf[-guard:] == 7.0)
         ro, _ = run_oracle(inp)
-        assert rel_err(out.float().cpu().numpy(), ro) <= 2e-2
+        assert out_err(out.float().cpu().numpy(), ro, "bf16") <= 2e-2
 
 
 def test_host_entry_matches_device_entry():
@@ -231,4 +230,4 @@ def test_full_size_workloads_sampled_heads(name):
         o, s = run_gpu(inp, algo)
         o, s = o[:, :, heads], s[:, heads]
         tol = TOL[w.dtype]
-        assert rel_err(o, ro) <= tol and rel_err(s, rs) <= tol, algo
+        assert out_err(o, ro, w.dtype) <= tol and rel_err(s, rs) <= tol, algo
