@@ -14,7 +14,8 @@ import os
 
 import torch
 
-__all__ = ["chunk_fwd", "chunk_fwd_host", "device_error", "status_string",
+__all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_noalloc",
+           "device_error", "status_string",
            "algo_applies", "fused_tc_available",
            "GdrError", "load_library", "LIB_PATH", "GATES", "ALGOS",
            "EXPORTED_SYMBOLS"]
@@ -28,7 +29,10 @@ DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARGUMENT", 2: "GDR_ERR_UNSUPPORTED",
           3: "GDR_ERR_CUDA", 4: "GDR_ERR_OUT_OF_MEMORY", 5: "GDR_ERR_TIMEOUT"}
 EXPORTED_SYMBOLS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_device_error",
-                    "gdr_algo_applies", "gdr_status_string")
+                    "gdr_algo_applies", "gdr_status_string",
+                    "gdr_chunk_fwd_noalloc")
+# size of the static scratch array behind gdr_chunk_fwd_noalloc
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
 
@@ -56,7 +60,8 @@ def load_library(path: str = LIB_PATH):
             "`python -m chunkwise_recurrence_b200.build` (needs nvcc)")
     lib = ctypes.CDLL(path)
     vp, fp, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
-    for name in ("gdr_chunk_fwd", "gdr_chunk_fwd_host"):
+    for name in ("gdr_chunk_fwd", "gdr_chunk_fwd_host",
+                 "gdr_chunk_fwd_noalloc"):
         f = getattr(lib, name)
         f.restype = ctypes.c_int
         f.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, vp,
@@ -138,6 +143,33 @@ def chunk_fwd(q, k, v, beta, log_alpha=None, initial_state=None, *,
                            ctypes.byref(opts))
     if rc != 0:
         raise GdrError(rc, "gdr_chunk_fwd")
+    return out, final_state
+
+
+def chunk_fwd_noalloc(q, k, v, beta, log_alpha=None, initial_state=None, *,
+                      out, final_state=None, chunk: int = 64,
+                      gate: str | None = None, cu_seqlens=None,
+                      algo: str = "auto", stream=None):
+    """Run ``gdr_chunk_fwd_noalloc``: like ``chunk_fwd`` but the library
+    allocates nothing (its scratch is a static device array shared by every
+    call on a device, so calls must not overlap on the GPU).  The caller
+    passes preallocated ``out`` (and ``final_state`` if wanted)."""
+    lib = load_library()
+    B, T, H, dk, dv, nseq = _shapes(q, v, cu_seqlens)
+    g = _gate_of(log_alpha, gate)
+    opts = _Opts(DTYPES[q.dtype], GATES[g],
+                 None if cu_seqlens is None else cu_seqlens.data_ptr(),
+                 nseq if cu_seqlens is not None else 0, ALGOS[algo])
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    rc = lib.gdr_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v),
+                                   _ptr(log_alpha), _ptr(beta),
+                                   _ptr(initial_state), _ptr(out),
+                                   _ptr(final_state), B, T, H, dk, dv, chunk,
+                                   ctypes.c_void_p(stream.cuda_stream),
+                                   ctypes.byref(opts))
+    if rc != 0:
+        raise GdrError(rc, "gdr_chunk_fwd_noalloc")
     return out, final_state
 
 

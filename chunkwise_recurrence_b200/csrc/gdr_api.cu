@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "gdr_internal.h"
 
@@ -231,6 +232,59 @@ extern "C" gdr_status gdr_chunk_fwd_host(const void *q, const void *k,
   if (cudaFreeAsync(block, stream) != cudaSuccess && st == GDR_OK)
     st = GDR_ERR_CUDA;
   return st;
+}
+
+// ---------------------------------------------------------------------------
+// No-allocation entry: the staged kernels with their scratch in a static
+// device array instead of a stream-ordered allocation.  Host code cannot use
+// the array's name as a device address (in host code it names a host-side
+// stand-in), so each device's address is looked up once with
+// cudaGetSymbolAddress while that device is current, and cached.
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[GDR_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices];
+
+gdr_status noalloc_scratch(void **ptr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GDR_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return GDR_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+      return GDR_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return GDR_OK;
+}
+
+}  // namespace
+
+extern "C" gdr_status gdr_chunk_fwd_noalloc(
+    const void *q, const void *k, const void *v, const float *log_alpha,
+    const float *beta, const float *initial_state, void *out,
+    float *final_state, int B, int T, int H, int dk, int dv, int chunk,
+    cudaStream_t stream, const gdr_opts *opts) {
+  const gdr_opts o = opts ? *opts : default_opts();
+  Problem p;
+  gdr_status st = validate(q, k, v, log_alpha, beta, initial_state, out,
+                           final_state, B, T, H, dk, dv, chunk, o, &p);
+  if (st != GDR_OK) return st;
+  if (o.algo == GDR_ALGO_FUSED_TC) return GDR_ERR_UNSUPPORTED;
+  if (p.nseq == 0 || p.H == 0) return GDR_OK;
+  if (gdr::staged_workspace_bytes(p) > GDR_NOALLOC_SCRATCH_BYTES)
+    return GDR_ERR_UNSUPPORTED;
+  void *scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != GDR_OK) return st;
+  return gdr::staged_run(p, scratch, stream) == cudaSuccess ? GDR_OK
+                                                            : GDR_ERR_CUDA;
 }
 
 extern "C" gdr_status gdr_device_error(cudaStream_t stream, int clear) {

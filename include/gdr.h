@@ -159,6 +159,47 @@ GDR_API gdr_status gdr_chunk_fwd_host(const void *q, const void *k, const void *
                               const gdr_opts *opts);
 
 /*
+ * gdr_chunk_fwd_noalloc -- gdr_chunk_fwd without any device allocation.
+ *
+ * The pages have no counterpart to this entry point: it exists for callers
+ * that cannot allocate device memory at call time.  Examples are processes
+ * whose device memory is reserved up front by another allocator (a serving
+ * runtime whose caching pool already holds all free memory, so a new
+ * cudaMalloc / cudaMallocAsync fails), and code that must not allocate during
+ * steady-state operation (fixed memory budget, no allocator latency).
+ *
+ * It runs the STAGED kernels with their scratch in one statically sized
+ * device array that lives in this library (GDR_NOALLOC_SCRATCH_BYTES, 64 MiB;
+ * every GPU that loads the library holds it until the process exits).  The
+ * caller still passes all inputs and outputs, as for gdr_chunk_fwd; the same
+ * layouts, sizes and status codes apply, plus:
+ *  - opts->algo must be GDR_ALGO_AUTO or GDR_ALGO_STAGED (FUSED_TC returns
+ *    GDR_ERR_UNSUPPORTED: it does not use this scratch);
+ *  - a problem whose staged scratch would exceed GDR_NOALLOC_SCRATCH_BYTES is
+ *    rejected with GDR_ERR_UNSUPPORTED before any CUDA call;
+ *  - the current device must be the device of `stream`.  The first call on
+ *    each device looks up that device's address of the array
+ *    (cudaGetSymbolAddress, once per device, cached); make that first call
+ *    before any stream capture;
+ *  - every call on a device shares the one array, which keeps the last call's
+ *    contents (nothing in it needs to start at zero: every scratch word is
+ *    written before it is read).  Calls whose execution overlaps on the GPU
+ *    (different streams, or different host threads, without ordering between
+ *    them) race on the array and give undefined results: serialise them.
+ * No cudaMalloc, cudaFree or other allocating routine is called.
+ */
+#define GDR_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+GDR_API gdr_status gdr_chunk_fwd_noalloc(const void *q, const void *k,
+                                         const void *v, const float *log_alpha,
+                                         const float *beta,
+                                         const float *initial_state, void *out,
+                                         float *final_state, int B, int T,
+                                         int H, int dk, int dv, int chunk,
+                                         cudaStream_t stream,
+                                         const gdr_opts *opts);
+
+/*
  * gdr_device_error -- synchronise `stream`, then read (and clear if `clear`)
  * the library's sticky device-side error word for the current device.
  * Returns GDR_OK if no kernel has reported an error, GDR_ERR_TIMEOUT if a
