@@ -27,7 +27,8 @@ GATES = {"none": 0, "scalar": 1, "channel": 2}
 ALGOS = {"auto": 0, "staged": 1, "fused_tc": 2}
 DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARGUMENT", 2: "GDR_ERR_UNSUPPORTED",
-          3: "GDR_ERR_CUDA", 4: "GDR_ERR_OUT_OF_MEMORY", 5: "GDR_ERR_TIMEOUT"}
+          3: "GDR_ERR_CUDA", 4: "GDR_ERR_OUT_OF_MEMORY", 5: "GDR_ERR_TIMEOUT",
+          6: "GDR_ERR_RANGE"}
 EXPORTED_SYMBOLS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_device_error",
                     "gdr_algo_applies", "gdr_status_string",
                     "gdr_chunk_fwd_noalloc")

@@ -1,17 +1,931 @@
-// Fused tensor-core path (placeholder until the tcgen05 kernel lands).
+// Fused tensor-core path of libgdr: one persistent CTA per (sequence, head)
+// runs the whole chunkwise gated delta rule chunk after chunk, with every
+// intermediate on chip, on sm_100a tcgen05 tensor cores.
+//
+// Per chunk of C = 64 tokens (dk = dv = 128), with g the in-chunk cumulative
+// log-decay (per key channel for KDA), S the state at the chunk start:
+//   A  = strictly-lower beta_r k_r^T Gamma_r Gamma_i^-1 k_i      (K K^T on TC)
+//   T  = (I + A)^-1                          (blocked forward substitution)
+//   W  = T diag(beta) (K . e^g),  U = T diag(beta) V              (TC)
+//   V_new = U - W S                                               (TC)
+//   O  = (Q . e^g) S + mask_{i<=r}[(Q . e^g)(K . e^-g)^T] V_new   (TC)
+//   S <- Gamma_C S + (K . e^{g_C - g})^T V_new                    (TC)
+// This is the WY form of the delta rule with the decay absorbed into the
+// erase factors (Gated DeltaNet-2 abstract, comparative-study page
+// 2607.07953), which rests on the update being affine in the preceding memory
+// ("DeltaTTT: Layerwise Optimization for Nonlinear Recurrent Memory",
+// §2 Background).
+//
+// Everything that does not depend on S (A, T, W, U, the output mask P) for
+// chunk n+1 is computed while the S-dependent chain of chunk n runs:
+//   warp 0      TMA producer: Q, K (two stages) and V tiles, 128-B swizzle
+//   warp 1      tensor-memory allocation and the single MMA-issuing thread
+//   warps 2..5  "state" warps: S -> bf16 operand and decay, V_new -> bf16
+//               operand, output tile -> global (thread = tensor-memory lane
+//               = one value channel)
+//   warps 6..9  "prep" warps: gates and cumsum, A and P from K K^T / Q K^T,
+//               T = (I+A)^-1, T-factor operands, -W operand, in-place
+//               Q . e^g and K . e^{g_C - g}
+// All state lives in tensor memory as S^T (lane = value channel, column =
+// key channel) in fp32; bf16 is used only for tensor-core operands.
+//
+// Tensor memory (512 columns x 128 lanes, fp32):
+//   [0,128) S^T   [128,256) V_new^T x2   [256,384) O^T x2
+//   [384,448) [K;Q] K^T   [448,512) W^T
+//
+// Every mbarrier wait is bounded; on expiry the kernel raises a sticky error
+// word (read by gdr_device_error) and every role winds down.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <mutex>
+
 #include "gdr_internal.h"
+#include "sm100.cuh"
 
 namespace gdr {
+namespace {
 
-bool fused_tc_applies(const Problem &) { return false; }
+using namespace sm100;
 
-cudaError_t fused_tc_run(const Problem &, cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int kC = 64;         // chunk length
+constexpr int kD = 128;        // dk = dv
+constexpr int kThreads = 320;  // 10 warps
+
+// ---- shared memory layout (bytes from a 1024-aligned base) ----------------
+// A stage holds one chunk's K and Q as four 8 KB [64 rows][64 cols] blocks:
+// [K cols 0..63 | Q cols 0..63 | K cols 64..127 | Q cols 64..127], so that
+// rows 0..63 (K) and 64..127 (Q) of a 16 KB block form one M=128 operand.
+constexpr uint32_t kStageBytes = 32768;
+constexpr uint32_t OFF_STAGE = 0;                        // 2 stages
+constexpr uint32_t OFF_V = OFF_STAGE + 2 * kStageBytes;  // [2][64][64] bf16
+constexpr uint32_t OFF_ST = OFF_V + 16384;               // S^T [2][128][64]
+constexpr uint32_t OFF_NW = OFF_ST + 32768;              // -W^T [128][64]
+constexpr uint32_t OFF_VN = OFF_NW + 16384;              // V_new^T [128][64]
+constexpr uint32_t OFF_P = OFF_VN + 16384;               // P [2][64][64]
+constexpr uint32_t OFF_TPG = OFF_P + 16384;              // T diag(b e^g)
+constexpr uint32_t OFF_TPB = OFF_TPG + 8192;             // T diag(b)
+constexpr uint32_t OFF_KN = OFF_TPB + 8192;              // K e^-g (KDA)
+template <int GATE>
+struct Layout {
+  static constexpr uint32_t KN = (GATE == 2) ? 16384 : 0;
+  static constexpr uint32_t AC = OFF_KN + KN;     // A blocks fp32 [10][16][16]
+  static constexpr uint32_t TC = AC + 10240;      // T blocks fp32 [10][16][16]
+  static constexpr uint32_t YS = TC + 10240;      // per-warp 16x16 scratch x4
+  static constexpr uint32_t GS = YS + 4096;       // g [2][64]
+  static constexpr uint32_t BS = GS + 512;        // beta [2][64]
+  static constexpr uint32_t GC = BS + 512;        // g_C [2][128]
+  static constexpr uint32_t GM = GC + 1024;       // g at row 31 [128] (KDA)
+  static constexpr uint32_t MISC = GM + 512;      // barriers, tmem base, flags
+  static constexpr uint32_t BYTES = MISC + 256;
+  static_assert(BYTES + 1024 <= 232448, "shared memory budget");
+};
+
+// tensor-memory columns
+constexpr uint32_t ACC_S = 0, ACC_V = 128, ACC_O = 256, ACC_KK = 384,
+                   ACC_W = 448;
+
+// mbarrier indices
+enum {
+  B_FULL0, B_FULL1, B_EMPTY0, B_EMPTY1, B_VFREE, B_KKREADY, B_KKDONE,
+  B_TREADY, B_WDONE, B_WREADY, B_SREADY, B_XDONE, B_VNREADY, B_SDONE,
+  B_ODONE, B_DRAIN, B_COUNT
+};
+
+// Instruction descriptors (M = 128 everywhere).  Operands are fp16 (11-bit
+// significand: 8x finer than bf16 at the same tensor-core rate), except the
+// channel-gate K K^T product, whose e^{+-(g - g_m)} factors need bf16's range.
+constexpr uint32_t ID_KK_H = idesc_f16kind(128, 64, false, false, false);
+constexpr uint32_t ID_KK_B = idesc_f16kind(128, 64, false, false, true);
+constexpr uint32_t ID_UW = idesc_f16kind(128, 64, true, false, false);
+constexpr uint32_t ID_XV = idesc_f16kind(128, 64, false, true, false);
+constexpr uint32_t ID_XO = idesc_f16kind(128, 64, false, false, false);
+constexpr uint32_t ID_SU = idesc_f16kind(128, 128, false, true, false);
+constexpr uint32_t ID_OI = idesc_f16kind(128, 64, false, false, false);
+
+// error word bits: 0..15 = the mbarrier whose wait expired; range errors
+constexpr unsigned kErrRange = 1u << 24;      // input beyond fp16 range
+constexpr unsigned kErrNonFinite = 1u << 25;  // non-finite final state
+constexpr float kF16Max = 65504.f;
+
+constexpr long long kWaitCycles = 1ll << 32;   // ~2 s: a wait never lasts this
+
+__device__ unsigned g_fused_error;
+
+struct Params {
+  const float *beta;
+  const float *log_alpha;
+  const float *s0;
+  __nv_bfloat16 *out;
+  float *sT;
+  const int32_t *cu;
+  int nseq, T, ntok, H;
+};
+
+struct Ctx {
+  uint64_t *bar;
+  volatile int *abort_flag;
+};
+
+// Bounded wait: true when the phase completed, false on abort or timeout.
+__device__ __forceinline__ bool wait_bar(const Ctx &cx, int b,
+                                         uint32_t parity) {
+  if (mbar_try_wait(&cx.bar[b], parity)) return true;
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait(&cx.bar[b], parity)) return true;
+    if (*cx.abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *cx.abort_flag = 1;
+      atomicOr(&g_fused_error, 1u << b);
+      return false;
+    }
+  }
 }
 
-cudaError_t fused_tc_read_error(unsigned *word, bool) {
-  *word = 0;
-  return cudaSuccess;
+// AND of `pred` over the 128 threads of named barrier `id` (also a barrier):
+// a role group takes every wait decision together, so no thread is left
+// behind at a later named barrier when another one gives up.
+__device__ __forceinline__ bool group_all(bool pred, int id) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ void unpack_bf16(uint32_t w, float &lo, float &hi) {
+  __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162 *>(&w);
+  float2 f = __bfloat1622float2(v);
+  lo = f.x;
+  hi = f.y;
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ void unpack_f16(uint32_t w, float &lo, float &hi) {
+  __half2 v = *reinterpret_cast<__half2 *>(&w);
+  float2 f = __half22float2(v);
+  lo = f.x;
+  hi = f.y;
+}
+__device__ __forceinline__ void st_smem_v4(uint8_t *p, uint32_t a, uint32_t b,
+                                           uint32_t c, uint32_t d) {
+  *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, d);
+}
+
+// index of the 16x16 block (rb, cb), cb <= rb, in the compact lower storage
+__device__ __forceinline__ int blk(int rb, int cb) {
+  return rb * (rb + 1) / 2 + cb;
+}
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// acc (2 n-tiles of m16n8 C fragments) += X (16x16) * Z (16x16), both
+// row-major fp32 in shared memory, on mma.sync m16n8k8 tf32.
+__device__ __forceinline__ void mma16(const float *X, const float *Z,
+                                      float acc[8], int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    const uint32_t a0 = to_tf32(X[g * 16 + 8 * ks + t]);
+    const uint32_t a1 = to_tf32(X[(g + 8) * 16 + 8 * ks + t]);
+    const uint32_t a2 = to_tf32(X[g * 16 + 8 * ks + t + 4]);
+    const uint32_t a3 = to_tf32(X[(g + 8) * 16 + 8 * ks + t + 4]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const uint32_t b0 = to_tf32(Z[(8 * ks + t) * 16 + 8 * nt + g]);
+      const uint32_t b1 = to_tf32(Z[(8 * ks + t + 4) * 16 + 8 * nt + g]);
+      float *c = acc + 4 * nt;
+      asm volatile(
+          "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+          "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+          "{%0, %1, %2, %3};"
+          : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+          : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+  }
+}
+
+// store C fragments (scaled by s) to a row-major 16x16 fp32 block
+__device__ __forceinline__ void store16(float *Y, const float acc[8], float s,
+                                        int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    Y[g * 16 + 8 * nt + 2 * t] = s * acc[4 * nt + 0];
+    Y[g * 16 + 8 * nt + 2 * t + 1] = s * acc[4 * nt + 1];
+    Y[(g + 8) * 16 + 8 * nt + 2 * t] = s * acc[4 * nt + 2];
+    Y[(g + 8) * 16 + 8 * nt + 2 * t + 1] = s * acc[4 * nt + 3];
+  }
+}
+
+template <int GATE>
+__global__ void __launch_bounds__(kThreads, 1)
+    gdr_fused_tc_kernel(const __grid_constant__ CUtensorMap tmq,
+                        const __grid_constant__ CUtensorMap tmk,
+                        const __grid_constant__ CUtensorMap tmv, Params p) {
+  using Lay = Layout<GATE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + Lay::MISC);
+  uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(sm + Lay::MISC + 8 * B_COUNT);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Lay::MISC + 8 * B_COUNT + 4);
+  float *scan_tmp = reinterpret_cast<float *>(sm + Lay::MISC + 8 * B_COUNT + 8);
+  float *AC = reinterpret_cast<float *>(sm + Lay::AC);
+  float *TC = reinterpret_cast<float *>(sm + Lay::TC);
+  const Ctx cx{bar, abort_flag};
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = blockIdx.x / p.H, h = blockIdx.x % p.H;
+  int start = p.cu ? p.cu[n] : n * p.T;
+  int end = p.cu ? p.cu[n + 1] : (n + 1) * p.T;
+  start = min(max(start, 0), p.ntok);
+  end = min(max(end, start), p.ntok);
+  const int NC = (end - start + kC - 1) / kC;
+  const size_t sbase = ((size_t)n * p.H + h) * kD * kD;
+
+  if (threadIdx.x == 0) {
+    const uint32_t counts[B_COUNT] = {1, 1, 1, 1, 1, 128, 1, 128, 1, 128,
+                                      128, 1, 128, 1, 1, 1};
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], counts[i]);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_map(&tmq);
+      tma_prefetch_map(&tmk);
+      tma_prefetch_map(&tmv);
+      int issued = 0;
+      for (int m = 0; m < NC; ++m) {
+        const int s = m & 1;
+        if (m >= 2 && !wait_bar(cx, B_EMPTY0 + s, ((m - 2) >> 1) & 1)) break;
+        const int tok0 = start + m * kC;
+        uint8_t *stg = sm + OFF_STAGE + s * kStageBytes;
+        mbar_arrive_expect_tx(&bar[B_FULL0 + s], 6 * 8192);
+        for (int kb = 0; kb < 2; ++kb) {
+          tma_load_3d(stg + kb * 16384, &tmk, &bar[B_FULL0 + s], kb * 64, h,
+                      tok0);
+          tma_load_3d(stg + kb * 16384 + 8192, &tmq, &bar[B_FULL0 + s],
+                      kb * 64, h, tok0);
+        }
+        issued = m + 1;
+        if (m >= 1 && !wait_bar(cx, B_VFREE, (m - 1) & 1)) break;
+        for (int kb = 0; kb < 2; ++kb)
+          tma_load_3d(sm + OFF_V + kb * 8192, &tmv, &bar[B_FULL0 + s],
+                      kb * 64, h, tok0);
+      }
+      if (*abort_flag) {
+        // let in-flight copies land before the CTA exits (bounded)
+        for (int m = max(0, issued - 2); m < issued; ++m) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(&bar[B_FULL0 + (m & 1)], (m >> 1) & 1) &&
+                 clock64() - t0 < (1ll << 28)) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t st = smem_u32(sm + OFF_ST), nw = smem_u32(sm + OFF_NW),
+                     vn = smem_u32(sm + OFF_VN), vt = smem_u32(sm + OFF_V),
+                     tpg = smem_u32(sm + OFF_TPG),
+                     tpb = smem_u32(sm + OFF_TPB),
+                     kn = smem_u32(sm + OFF_KN);
+      auto stage = [&](int m) {
+        return smem_u32(sm + OFF_STAGE + (m & 1) * kStageBytes);
+      };
+      auto issue_kk = [&](int m) {
+        const uint32_t base = stage(m);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+          const uint64_t a = sdesc_sw128(base + koff, 16, 1024);
+          const uint64_t b =
+              GATE == 2
+                  ? sdesc_sw128(kn + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024)
+                  : sdesc_sw128(base + koff, 16, 1024);
+          mma_f16kind(tmem + ACC_KK, a, b, GATE == 2 ? ID_KK_B : ID_KK_H, ks > 0);
+        }
+        mma_commit(&bar[B_KKDONE]);
+      };
+      auto issue_uw = [&](int m) {
+        const uint32_t base = stage(m);
+        const uint32_t accv = tmem + ACC_V + (m & 1) * 64;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_f16kind(accv, sdesc_sw128(vt + ks * 2048, 8192, 1024),
+                   sdesc_sw128(tpb + ks * 32, 16, 1024), ID_UW, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_f16kind(tmem + ACC_W, sdesc_sw128(base + ks * 2048, 16384, 1024),
+                   sdesc_sw128((GATE == 2 ? tpb : tpg) + ks * 32, 16, 1024),
+                   ID_UW, ks > 0);
+        mma_commit(&bar[B_WDONE]);
+        mma_commit(&bar[B_VFREE]);
+      };
+      bool ok = true;
+      if (NC > 0) {
+        ok = wait_bar(cx, B_KKREADY, 0);
+        if (ok) {
+          tc_fence_after();
+          issue_kk(0);
+          ok = wait_bar(cx, B_TREADY, 0);
+        }
+        if (ok) {
+          tc_fence_after();
+          issue_uw(0);
+        }
+      }
+      for (int m = 0; m < NC && ok; ++m) {
+        const uint32_t base = stage(m);
+        // X(m): V_new^T = U^T + S^T (-W)^T ; O^T = S^T (Q e^g)^T
+        if (!wait_bar(cx, B_SREADY, m & 1) || !wait_bar(cx, B_WREADY, m & 1))
+          break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_f16kind(tmem + ACC_V + (m & 1) * 64,
+                   sdesc_sw128(st + (ks >> 2) * 16384 + (ks & 3) * 32, 16,
+                               1024),
+                   sdesc_sw128(nw + ks * 2048, 8192, 1024), ID_XV, 1);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_f16kind(tmem + ACC_O + (m & 1) * 64,
+                   sdesc_sw128(st + (ks >> 2) * 16384 + (ks & 3) * 32, 16,
+                               1024),
+                   sdesc_sw128(base + 8192 + (ks >> 2) * 16384 + (ks & 3) * 32,
+                               16, 1024),
+                   ID_XO, ks > 0);
+        mma_commit(&bar[B_XDONE]);
+        // KK(m+1) while the state warps turn V_new into an operand
+        if (m + 1 < NC) {
+          if (!wait_bar(cx, B_KKREADY, (m + 1) & 1)) break;
+          tc_fence_after();
+          issue_kk(m + 1);
+        }
+        // S update and intra-chunk output
+        if (!wait_bar(cx, B_VNREADY, m & 1)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_f16kind(tmem + ACC_S, sdesc_sw128(vn + ks * 32, 16, 1024),
+                   sdesc_sw128(base + ks * 2048, 16384, 1024), ID_SU, 1);
+        mma_commit(&bar[B_SDONE]);
+        const uint32_t pt = smem_u32(sm + OFF_P + (m & 1) * 8192);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_f16kind(tmem + ACC_O + (m & 1) * 64,
+                   sdesc_sw128(vn + ks * 32, 16, 1024),
+                   sdesc_sw128(pt + ks * 32, 16, 1024), ID_OI, 1);
+        mma_commit(&bar[B_ODONE]);
+        mma_commit(&bar[B_EMPTY0 + (m & 1)]);
+        // U, W of chunk m+1
+        if (m + 1 < NC) {
+          if (!wait_bar(cx, B_TREADY, (m + 1) & 1)) break;
+          tc_fence_after();
+          issue_uw(m + 1);
+        }
+      }
+      // every MMA issued has completed before tensor memory is released
+      mma_commit(&bar[B_DRAIN]);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&bar[B_DRAIN], 0) && clock64() - t0 < kWaitCycles) {
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------ state warps
+    const int q4 = warp & 3;
+    const int l = q4 * 32 + lane;                  // value channel
+    const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
+    float v[32];
+    // initial state -> S^T in tensor memory
+    for (int c0 = 0; c0 < kD; c0 += 32) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        v[j] = p.s0 ? p.s0[sbase + (size_t)(c0 + j) * kD + l] : 0.f;
+      tmem_st32(trow + ACC_S + c0, v);
+    }
+    tmem_wait_st();
+    bool ok = true;
+    auto store_output = [&](int m) {
+      const int tok0 = start + m * kC, L = min(kC, end - tok0);
+      uint8_t *stg = sm + OFF_VN;               // [64 rows][128 dv] bf16
+      for (int c0 = 0; c0 < kC; c0 += 32) {
+        tmem_ld32(trow + ACC_O + (m & 1) * 64 + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float send = (l & 1) ? v[j] : v[j + 1];
+          const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+          const int r = c0 + j + (l & 1);
+          const float lo = (l & 1) ? recv : v[j];
+          const float hi = (l & 1) ? v[j + 1] : recv;
+          *reinterpret_cast<uint32_t *>(stg + r * 256 + (l & ~1) * 2) =
+              pack_bf16(lo, hi);
+        }
+      }
+      named_bar_sync(1, 128);
+      for (int i = l; i < kC * 16; i += 128) {
+        const int r = i >> 4, ch = i & 15;
+        if (r < L) {
+          const uint4 x = *reinterpret_cast<const uint4 *>(stg + r * 256 + ch * 16);
+          *reinterpret_cast<uint4 *>(p.out + ((size_t)(tok0 + r) * p.H + h) * kD +
+                                     ch * 8) = x;
+        }
+      }
+      named_bar_sync(1, 128);
+    };
+    float *gC = reinterpret_cast<float *>(sm + Lay::GC);
+    for (int m = 0; m < NC; ++m) {
+      // S (chunk start) -> bf16 operand; decayed S back to tensor memory
+      if (m > 0 && !(ok = group_all(wait_bar(cx, B_SDONE, (m - 1) & 1), 1)))
+        break;
+      if (!(ok = group_all(wait_bar(cx, B_TREADY, m & 1), 1))) break;
+      tc_fence_after();
+      const float *gcm = gC + (m & 1) * 128;
+      const float dscal = GATE == 1 ? __expf(gcm[0]) : 1.f;
+      for (int c0 = 0; c0 < kD; c0 += 32) {
+        tmem_ld32(trow + ACC_S + c0, v);
+        tmem_wait_ld();
+        uint8_t *dst = sm + OFF_ST + (c0 >> 6) * 16384;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+          st_smem_v4(dst + sw128_chunk(l, ((c0 & 63) >> 3) + ch),
+                     pack_f16(v[8 * ch + 0], v[8 * ch + 1]),
+                     pack_f16(v[8 * ch + 2], v[8 * ch + 3]),
+                     pack_f16(v[8 * ch + 4], v[8 * ch + 5]),
+                     pack_f16(v[8 * ch + 6], v[8 * ch + 7]));
+        if (GATE != 0) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            v[j] *= (GATE == 1) ? dscal : __expf(gcm[c0 + j]);
+          tmem_st32(trow + ACC_S + c0, v);
+        }
+      }
+      if (GATE != 0) tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bar[B_SREADY]);
+      // output of the previous chunk while X(m) runs
+      if (m > 0) {
+        if (!(ok = group_all(wait_bar(cx, B_ODONE, (m - 1) & 1), 1))) break;
+        tc_fence_after();
+        store_output(m - 1);
+      }
+      // V_new^T -> bf16 operand
+      if (!(ok = group_all(wait_bar(cx, B_XDONE, m & 1), 1))) break;
+      tc_fence_after();
+      for (int c0 = 0; c0 < kC; c0 += 32) {
+        tmem_ld32(trow + ACC_V + (m & 1) * 64 + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+          st_smem_v4(sm + OFF_VN + sw128_chunk(l, (c0 >> 3) + ch),
+                     pack_f16(v[8 * ch + 0], v[8 * ch + 1]),
+                     pack_f16(v[8 * ch + 2], v[8 * ch + 3]),
+                     pack_f16(v[8 * ch + 4], v[8 * ch + 5]),
+                     pack_f16(v[8 * ch + 6], v[8 * ch + 7]));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bar[B_VNREADY]);
+    }
+    if (ok && NC > 0) {
+      ok = group_all(wait_bar(cx, B_ODONE, (NC - 1) & 1), 1);
+      if (ok) {
+        tc_fence_after();
+        store_output(NC - 1);
+        ok = group_all(wait_bar(cx, B_SDONE, (NC - 1) & 1), 1);
+      }
+    }
+    if (ok) {
+      tc_fence_after();
+      bool finite = true;
+      for (int c0 = 0; c0 < kD; c0 += 32) {
+        tmem_ld32(trow + ACC_S + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          finite = finite && isfinite(v[j]);
+          if (p.sT) p.sT[sbase + (size_t)(c0 + j) * kD + l] = v[j];
+        }
+      }
+      if (!finite) atomicOr(&g_fused_error, kErrNonFinite);
+    }
+  } else {
+    // ------------------------------------------------------ prep warps
+    const int q4 = warp & 3;
+    const int l = q4 * 32 + lane;                  // lane of tensor memory
+    const int pw = warp - 6;                       // 0..3
+    const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
+    float *gS = reinterpret_cast<float *>(sm + Lay::GS);
+    float *bS = reinterpret_cast<float *>(sm + Lay::BS);
+    float *gC = reinterpret_cast<float *>(sm + Lay::GC);
+    float *gM = reinterpret_cast<float *>(sm + Lay::GM);
+    float *YS = reinterpret_cast<float *>(sm + Lay::YS) + pw * 256;
+    float v[32];
+    for (int m = 0; m < NC; ++m) {
+      const int s = m & 1, tok0 = start + m * kC, L = min(kC, end - tok0);
+      uint8_t *stg = sm + OFF_STAGE + s * kStageBytes;
+      float *g = gS + s * 64, *b = bS + s * 64, *gc = gC + s * 128;
+      // ---- P1: gates (beta, in-chunk cumulative log-decay)
+      if (GATE != 2) {
+        float x = 0.f, bb = 0.f;
+        if (l < L) {
+          bb = p.beta[(size_t)(tok0 + l) * p.H + h];
+          if (GATE == 1) x = p.log_alpha[(size_t)(tok0 + l) * p.H + h];
+        }
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, x, off);
+          if (lane >= off) x += y;
+        }
+        if (l == 31) *scan_tmp = x;
+        named_bar_sync(2, 128);
+        if (l >= 32 && l < 64) x += *scan_tmp;
+        if (l < 64) {
+          g[l] = x;
+          b[l] = bb;
+        }
+        if (l == L - 1) gc[0] = x;
+      } else if (l < 64) {
+        b[l] = (l < L) ? p.beta[(size_t)(tok0 + l) * p.H + h] : 0.f;
+      }
+      // ---- P2: operand tiles.  V -> fp16 in place.  Scalar / no gate:
+      // Q, K -> fp16 in place.  Channel gate: thread l owns key channel l and
+      // forms, with g_m = g at row 31, Q e^{g-g_m}, K e^{g-g_m} and
+      // K e^{g_m-g} in bf16 (the exponent range of these factors needs bf16).
+      if (!group_all(wait_bar(cx, B_FULL0 + s, (m >> 1) & 1), 2)) break;
+      float amax = 0.f;
+      {
+        const int n16 = (GATE == 2) ? 1024 : 3072;  // 16-byte words
+        for (int i = l; i < n16; i += 128) {
+          uint8_t *ptr = (GATE == 2 || i >= 2048)
+                             ? sm + OFF_V + (i - (GATE == 2 ? 0 : 2048)) * 16
+                             : stg + i * 16;
+          uint4 x = *reinterpret_cast<uint4 *>(ptr);
+          uint32_t *w = reinterpret_cast<uint32_t *>(&x);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float a0, a1;
+            unpack_bf16(w[e], a0, a1);
+            amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
+            w[e] = pack_f16(a0, a1);
+          }
+          *reinterpret_cast<uint4 *>(ptr) = x;
+        }
+      }
+      if (GATE == 2) {
+        const float *la = p.log_alpha + ((size_t)tok0 * p.H + h) * kD + l;
+        const size_t rs = (size_t)p.H * kD;
+        float gr[kC];
+        float gg = 0.f;
+#pragma unroll
+        for (int r = 0; r < kC; ++r) {
+          gg += (r < L) ? la[r * rs] : 0.f;
+          gr[r] = gg;
+        }
+        const float gm = gr[31];
+        gM[l] = gm;
+        gc[l] = gg;
+        uint8_t *kt = stg + (l >> 6) * 16384, *qt = kt + 8192;
+        uint8_t *knt = sm + OFF_KN + (l >> 6) * 8192;
+#pragma unroll
+        for (int r = 0; r < kC; ++r) {
+          const float ep = __expf(gr[r] - gm), en = __expf(gm - gr[r]);
+          const uint32_t off = sw128_off(r, l & 63);
+          __nv_bfloat16 *qe = reinterpret_cast<__nv_bfloat16 *>(qt + off);
+          __nv_bfloat16 *ke = reinterpret_cast<__nv_bfloat16 *>(kt + off);
+          const float qv = __bfloat162float(*qe), kv = __bfloat162float(*ke);
+          amax = fmaxf(amax, fmaxf(fabsf(qv), fabsf(kv)));
+          *qe = __float2bfloat16_rn(qv * ep);
+          *ke = __float2bfloat16_rn(kv * ep);
+          *reinterpret_cast<__nv_bfloat16 *>(knt + off) =
+              __float2bfloat16_rn(kv * en);
+        }
+      }
+      if (!(amax <= kF16Max)) atomicOr(&g_fused_error, kErrRange);
+      fence_proxy_async_smem();
+      mbar_arrive(&bar[B_KKREADY]);
+      // ---- P3: A (strictly lower, fp32 blocks) and P (lower, fp16 operand)
+      if (!group_all(wait_bar(cx, B_KKDONE, m & 1), 2)) break;
+      tc_fence_after();
+      for (int c0 = 0; c0 < kC; c0 += 32) {
+        tmem_ld32(trow + ACC_KK + c0, v);
+        tmem_wait_ld();
+        if (l < 64) {
+          const int r = l;
+          const float gr = g[r], br = (r < L) ? b[r] : 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int i = c0 + j;
+            float a = 0.f;
+            if (i < r) {
+              a = br * v[j];
+              if (GATE == 1) a *= __expf(gr - g[i]);
+            }
+            v[j] = a;
+          }
+          // write the blocks (r/16, i/16) with i/16 <= r/16
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int cb = (c0 >> 4) + half;
+            if (cb <= (r >> 4)) {
+              float4 *dst = reinterpret_cast<float4 *>(
+                  AC + blk(r >> 4, cb) * 256 + (r & 15) * 16);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                dst[e] = make_float4(v[16 * half + 4 * e], v[16 * half + 4 * e + 1],
+                                     v[16 * half + 4 * e + 2], v[16 * half + 4 * e + 3]);
+            }
+          }
+        } else {
+          const int r = l - 64;
+          const float gr = g[r];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int i = c0 + j;
+            float pv = 0.f;
+            if (i <= r) {
+              pv = v[j];
+              if (GATE == 1) pv *= __expf(gr - g[i]);
+            }
+            v[j] = pv;
+          }
+          uint8_t *pt = sm + OFF_P + s * 8192;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch)
+            st_smem_v4(pt + sw128_chunk(r, (c0 >> 3) + ch),
+                       pack_f16(v[8 * ch + 0], v[8 * ch + 1]),
+                       pack_f16(v[8 * ch + 2], v[8 * ch + 3]),
+                       pack_f16(v[8 * ch + 4], v[8 * ch + 5]),
+                       pack_f16(v[8 * ch + 6], v[8 * ch + 7]));
+        }
+      }
+      if (GATE == 2) {
+        // Q e^{g-g_m}, K e^{g-g_m} (bf16) -> Q e^g, K e^g (fp16), in place
+        for (int idx = l; idx < kC * 16; idx += 128) {
+          const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
+          const uint32_t off = kb * 16384 + sw128_chunk(r, cc & 7);
+          const int c0 = kb * 64 + (cc & 7) * 8;
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+            uint4 *ptr = reinterpret_cast<uint4 *>(stg + off + part * 8192);
+            uint4 x = *ptr;
+            uint32_t *w = reinterpret_cast<uint32_t *>(&x);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float a0, a1;
+              unpack_bf16(w[e], a0, a1);
+              w[e] = pack_f16(a0 * __expf(gM[c0 + 2 * e]),
+                              a1 * __expf(gM[c0 + 2 * e + 1]));
+            }
+            *ptr = x;
+          }
+        }
+      }
+      named_bar_sync(2, 128);
+      // ---- P4: T = (I + A)^-1.  Diagonal 16x16 blocks by forward
+      // substitution (one thread per column), then the off-diagonal blocks
+      // T_bc = -D_b sum_{c<=e<b} A_be T_ec on mma.sync (tf32), level by level.
+      if (l < 64) {
+        const int bb = l >> 4, j = l & 15;
+        const float *Ab = AC + blk(bb, bb) * 256;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          float acc = (r == j) ? 1.f : 0.f;
+#pragma unroll
+          for (int i = 0; i < r; ++i) acc -= Ab[r * 16 + i] * x[i];
+          x[r] = acc;
+        }
+        float *Tb = TC + blk(bb, bb) * 256;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tb[r * 16 + j] = x[r];
+      }
+      named_bar_sync(2, 128);
+#pragma unroll 1
+      for (int lev = 1; lev <= 3; ++lev) {
+        if (pw <= 3 - lev) {
+          const int c = pw, bb = pw + lev;
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          for (int e = c; e < bb; ++e)
+            mma16(AC + blk(bb, e) * 256, TC + blk(e, c) * 256, acc, lane);
+          store16(YS, acc, 1.f, lane);
+          __syncwarp();
+          float acc2[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          mma16(TC + blk(bb, bb) * 256, YS, acc2, lane);
+          __syncwarp();
+          store16(TC + blk(bb, c) * 256, acc2, -1.f, lane);
+        }
+        named_bar_sync(2, 128);
+      }
+      // ---- T-factor operands (fp16): rows 0..63 -> T diag(beta e^g),
+      //      rows 64..127 -> T diag(beta)
+      {
+        const int r = l & 63;
+        const bool with_g = (l < 64);
+        uint8_t *dst = sm + (with_g ? OFF_TPG : OFF_TPB);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          float t8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int i = 8 * ch + e;
+            const int cb = i >> 4, rb = r >> 4;
+            float t = (cb <= rb) ? TC[blk(rb, cb) * 256 + (r & 15) * 16 + (i & 15)] : 0.f;
+            float f = (i < L) ? b[i] : 0.f;
+            if (with_g && GATE == 1) f *= __expf(g[i]);
+            t8[e] = t * f;
+          }
+          st_smem_v4(dst + sw128_chunk(r, ch), pack_f16(t8[0], t8[1]),
+                     pack_f16(t8[2], t8[3]), pack_f16(t8[4], t8[5]),
+                     pack_f16(t8[6], t8[7]));
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bar[B_TREADY]);
+      // ---- P5: -W^T operand; Q e^g and K e^{g_C - g} in place (fp16)
+      if (!group_all(wait_bar(cx, B_WDONE, m & 1), 2)) break;
+      tc_fence_after();
+      for (int c0 = 0; c0 < kC; c0 += 32) {
+        tmem_ld32(trow + ACC_W + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+          st_smem_v4(sm + OFF_NW + sw128_chunk(l, (c0 >> 3) + ch),
+                     pack_f16(-v[8 * ch + 0], -v[8 * ch + 1]),
+                     pack_f16(-v[8 * ch + 2], -v[8 * ch + 3]),
+                     pack_f16(-v[8 * ch + 4], -v[8 * ch + 5]),
+                     pack_f16(-v[8 * ch + 6], -v[8 * ch + 7]));
+      }
+      if (GATE != 0) {
+        for (int idx = l; idx < kC * 16; idx += 128) {
+          const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
+          const uint32_t off = kb * 16384 + sw128_chunk(r, cc & 7);
+          uint4 *kp = reinterpret_cast<uint4 *>(stg + off);
+          uint4 kv;
+          if (GATE == 1) {
+            uint4 *qp = reinterpret_cast<uint4 *>(stg + off + 8192);
+            const float eq = __expf(g[r]), ek = __expf(gc[0] - g[r]);
+            uint4 qv = *qp;
+            kv = *kp;
+            uint32_t *qw = reinterpret_cast<uint32_t *>(&qv);
+            uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float a0, a1;
+              unpack_f16(qw[e], a0, a1);
+              qw[e] = pack_f16(a0 * eq, a1 * eq);
+              unpack_f16(kw[e], a0, a1);
+              kw[e] = pack_f16(a0 * ek, a1 * ek);
+            }
+            *qp = qv;
+          } else {
+            // K~ = (K e^{g_m-g}) e^{g_C-g_m}, per channel
+            kv = *reinterpret_cast<const uint4 *>(sm + OFF_KN + kb * 8192 +
+                                                  sw128_chunk(r, cc & 7));
+            uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
+            const int c0 = kb * 64 + (cc & 7) * 8;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float a0, a1;
+              unpack_bf16(kw[e], a0, a1);
+              kw[e] = pack_f16(a0 * __expf(gc[c0 + 2 * e] - gM[c0 + 2 * e]),
+                               a1 * __expf(gc[c0 + 2 * e + 1] - gM[c0 + 2 * e + 1]));
+            }
+          }
+          *kp = kv;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bar[B_WREADY]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType,
+                                  cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr,
+                                cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [ntok][H][128] bf16, box of 64 channels x 1 head x 64 tokens, 128-B swizzle
+bool make_map(CUtensorMap *map, const void *base, int ntok, int H) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H,
+                              (cuuint64_t)(ntok > 0 ? ntok : 1)};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2};
+  const cuuint32_t box[3] = {64, 1, (cuuint32_t)kC};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base),
+             dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int GATE>
+cudaError_t launch(const Problem &pr, cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, pr.q, pr.ntok, pr.H) || !make_map(&mk, pr.k, pr.ntok, pr.H) ||
+      !make_map(&mv, pr.v, pr.ntok, pr.H))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.beta = pr.beta;
+  p.log_alpha = pr.log_alpha;
+  p.s0 = pr.s0;
+  p.out = static_cast<__nv_bfloat16 *>(pr.out);
+  p.sT = pr.sT;
+  p.cu = pr.cu;
+  p.nseq = pr.nseq;
+  p.T = pr.T;
+  p.ntok = pr.ntok;
+  p.H = pr.H;
+  const int smem = Layout<GATE>::BYTES + 1024;
+  cudaError_t e = cudaFuncSetAttribute(
+      gdr_fused_tc_kernel<GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      smem);
+  if (e != cudaSuccess) return e;
+  gdr_fused_tc_kernel<GATE><<<pr.nseq * pr.H, kThreads, smem, s>>>(mq, mk, mv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool fused_tc_applies(const Problem &p) {
+  return p.dtype == GDR_BF16 && p.dk == kD && p.dv == kD && p.chunk == kC &&
+         (long long)p.nseq * p.H < (1ll << 31);
+}
+
+cudaError_t fused_tc_run(const Problem &p, cudaStream_t s) {
+  switch (p.gate) {
+    case GDR_GATE_NONE: return launch<0>(p, s);
+    case GDR_GATE_SCALAR: return launch<1>(p, s);
+    default: return launch<2>(p, s);
+  }
+}
+
+cudaError_t fused_tc_read_error(unsigned *word, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(word, g_fused_error, sizeof(unsigned));
+  if (e != cudaSuccess) return e;
+  if (clear && *word) {
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_fused_error, &zero, sizeof(unsigned));
+  }
+  return e;
 }
 
 }  // namespace gdr

@@ -292,7 +292,8 @@ extern "C" gdr_status gdr_device_error(cudaStream_t stream, int clear) {
   unsigned word = 0;
   if (gdr::fused_tc_read_error(&word, clear != 0) != cudaSuccess)
     return GDR_ERR_CUDA;
-  return word ? GDR_ERR_TIMEOUT : GDR_OK;
+  if (word & 0xFFFFu) return GDR_ERR_TIMEOUT;   // an mbarrier wait expired
+  return word ? GDR_ERR_RANGE : GDR_OK;
 }
 
 extern "C" int gdr_algo_applies(gdr_algo algo, gdr_dtype dtype,
@@ -324,6 +325,7 @@ extern "C" const char *gdr_status_string(gdr_status s) {
     case GDR_ERR_CUDA: return "GDR_ERR_CUDA";
     case GDR_ERR_OUT_OF_MEMORY: return "GDR_ERR_OUT_OF_MEMORY";
     case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT";
+    case GDR_ERR_RANGE: return "GDR_ERR_RANGE";
   }
   return "GDR_ERR_UNKNOWN";
 }

@@ -65,7 +65,10 @@ typedef enum {
   GDR_ERR_UNSUPPORTED = 2,      /* valid but not implemented (shape, dtype) */
   GDR_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed      */
   GDR_ERR_OUT_OF_MEMORY = 4,    /* scratch allocation failed                 */
-  GDR_ERR_TIMEOUT = 5           /* a bounded device-side wait expired        */
+  GDR_ERR_TIMEOUT = 5,          /* a bounded device-side wait expired        */
+  GDR_ERR_RANGE = 6             /* an input (or the final state) fell outside
+                                   the fused path's fp16 operand range; the
+                                   STAGED path has no such limit             */
 } gdr_status;
 
 /* Element type of q, k, v and out.  beta, log_alpha and the states are always
@@ -90,8 +93,12 @@ typedef enum {
   GDR_ALGO_STAGED = 1,
   /* one persistent kernel per (sequence, head) that runs the same four steps
    * chunk after chunk with every intermediate on chip; chunk products on
-   * tcgen05 tensor cores (bf16 operands, fp32 accumulation in tensor memory).
-   * bf16, dk = dv = 128, chunk = 64. */
+   * tcgen05 tensor cores: fp16 operands (inputs converted on chip), fp32
+   * accumulation in tensor memory, fp32 state.  bf16 I/O, dk = dv = 128,
+   * chunk = 64.  Inputs must lie within fp16 range (|x| <= 65504); for the
+   * channel gate, each key channel's log-decay must move by at most ~88
+   * between a chunk's row 31 and its first or last row.  Violations are
+   * reported by gdr_device_error as GDR_ERR_RANGE. */
   GDR_ALGO_FUSED_TC = 2
 } gdr_algo;
 
@@ -203,7 +210,9 @@ GDR_API gdr_status gdr_chunk_fwd_noalloc(const void *q, const void *k,
  * gdr_device_error -- synchronise `stream`, then read (and clear if `clear`)
  * the library's sticky device-side error word for the current device.
  * Returns GDR_OK if no kernel has reported an error, GDR_ERR_TIMEOUT if a
- * bounded wait expired, GDR_ERR_CUDA if synchronisation itself failed.
+ * bounded wait expired, GDR_ERR_RANGE if the fused kernel met an input of
+ * magnitude above 65504 (or NaN) or produced a non-finite final state,
+ * GDR_ERR_CUDA if synchronisation itself failed.
  */
 GDR_API gdr_status gdr_device_error(cudaStream_t stream, int clear);
 
