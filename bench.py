@@ -157,6 +157,27 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+def max_over_ranks(values, ws, device=None):
+    """Element-wise max of a list of floats over all ranks (the timing
+    reduction: a job is as slow as its slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_throughput(tokens_per_rank_step, ws, steps, max_ms):
+    """Whole-job tokens/s: every rank processes its own batch each step."""
+    return tokens_per_rank_step * ws * steps / (max_ms / 1e3)
+
+
+def rank_seed(seed, rank):
+    """Each rank draws its own independent batch."""
+    return seed + rank
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -250,7 +271,7 @@ def run_ours(args, w):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
-    inp = generate(w, seed=args.seed + rank)
+    inp = generate(w, seed=rank_seed(args.seed, rank))
     q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
     beta = inp.beta.to(dev)
     la = None if inp.log_alpha is None else inp.log_alpha.to(dev)
@@ -329,15 +350,11 @@ def run_ours(args, w):
     e2e_ms = ea.elapsed_time(eb)
 
     # ---- max over ranks
-    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], ws, device=dev)
 
     ntok = inp.ntok
-    tokens_per_step = ntok * ws
-    value = tokens_per_step * args.steps / (total_ms / 1e3)
-    e2e_value = tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+    value = job_throughput(ntok, ws, args.steps, total_ms)
+    e2e_value = job_throughput(ntok, ws, e2e_steps, e2e_ms)
     ms = total_ms / args.steps
     fl = flops_per_token_head(w.chunk, w.dk, w.dv) * ntok * w.H
     by = algorithmic_bytes(w, ntok, inp.nseq)

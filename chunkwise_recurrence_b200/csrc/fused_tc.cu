@@ -23,9 +23,10 @@
 //   warps 2..5  "state" warps: S -> bf16 operand and decay, V_new -> bf16
 //               operand, output tile -> global (thread = tensor-memory lane
 //               = one value channel)
-//   warps 6..9  "prep" warps: gates and cumsum, A and P from K K^T / Q K^T,
-//               T = (I+A)^-1, T-factor operands, -W operand, in-place
-//               Q . e^g and K . e^{g_C - g}
+//   warps 6..13 "prep" warps (two per scheduler): gates, cumsum and per-row
+//               decay factors, A and P from K K^T / Q K^T, T = (I+A)^-1,
+//               T-factor operands, -W operand, in-place Q . e^g and
+//               K . e^{g_C - g}
 // All state lives in tensor memory as S^T (lane = value channel, column =
 // key channel) in fp32; bf16 is used only for tensor-core operands.
 //
@@ -52,7 +53,8 @@ using namespace sm100;
 
 constexpr int kC = 64;         // chunk length
 constexpr int kD = 128;        // dk = dv
-constexpr int kThreads = 320;  // 10 warps
+constexpr int kThreads = 448;  // 14 warps
+constexpr int kPrep = 256;     // prep threads (warps 6..13)
 
 // ---- shared memory layout (bytes from a 1024-aligned base) ----------------
 // A stage holds one chunk's K and Q as four 8 KB [64 rows][64 cols] blocks:
@@ -65,23 +67,30 @@ constexpr uint32_t OFF_ST = OFF_V + 16384;               // S^T [2][128][64]
 constexpr uint32_t OFF_NW = OFF_ST + 32768;              // -W^T [128][64]
 constexpr uint32_t OFF_VN = OFF_NW + 16384;              // V_new^T [128][64]
 constexpr uint32_t OFF_P = OFF_VN + 16384;               // P [2][64][64]
-constexpr uint32_t OFF_TPG = OFF_P + 16384;              // T diag(b e^g)
-constexpr uint32_t OFF_TPB = OFF_TPG + 8192;             // T diag(b)
-constexpr uint32_t OFF_KN = OFF_TPB + 8192;              // K e^-g (KDA)
+constexpr uint32_t OFF_TP = OFF_P + 16384;               // T-factor tiles
 template <int GATE>
 struct Layout {
-  static constexpr uint32_t KN = (GATE == 2) ? 16384 : 0;
-  static constexpr uint32_t AC = OFF_KN + KN;     // A blocks fp32 [10][16][16]
+  // scalar / no gate: T diag(b e^g) and T diag(b), each as a bf16 hi + lo
+  // pair (16 significant bits against raw bf16 K and V); channel gate: one
+  // fp16 T diag(b) tile, plus K e^{g_m - g} in bf16.
+  static constexpr uint32_t TP_BYTES = (GATE == 2) ? 8192 : 32768;
+  static constexpr uint32_t TPG_HI = OFF_TP, TPG_LO = OFF_TP + 8192,
+                            TPB_HI = OFF_TP + 16384, TPB_LO = OFF_TP + 24576;
+  static constexpr uint32_t KN = OFF_TP + TP_BYTES;
+  static constexpr uint32_t KN_BYTES = (GATE == 2) ? 16384 : 0;
+  static constexpr uint32_t AC = KN + KN_BYTES;   // A blocks fp32 [10][16][16]
   static constexpr uint32_t TC = AC + 10240;      // T blocks fp32 [10][16][16]
   static constexpr uint32_t YS = TC + 10240;      // per-warp 16x16 scratch x4
   static constexpr uint32_t GS = YS + 4096;       // g [2][64]
-  static constexpr uint32_t BS = GS + 512;        // beta [2][64]
-  static constexpr uint32_t GC = BS + 512;        // g_C [2][128]
+  static constexpr uint32_t FT = GS + 512;        // row factors [2][6][64]
+  static constexpr uint32_t GC = FT + 3072;       // g_C [2][128]
   static constexpr uint32_t GM = GC + 1024;       // g at row 31 [128] (KDA)
   static constexpr uint32_t MISC = GM + 512;      // barriers, tmem base, flags
   static constexpr uint32_t BYTES = MISC + 256;
   static_assert(BYTES + 1024 <= 232448, "shared memory budget");
 };
+// per-row factor arrays inside FT (each [64] fp32), for one chunk buffer
+enum { F_B, F_BG, F_E, F_F, F_EG, F_EK, F_COUNT };
 
 // tensor-memory columns
 constexpr uint32_t ACC_S = 0, ACC_V = 128, ACC_O = 256, ACC_KK = 384,
@@ -91,15 +100,18 @@ constexpr uint32_t ACC_S = 0, ACC_V = 128, ACC_O = 256, ACC_KK = 384,
 enum {
   B_FULL0, B_FULL1, B_EMPTY0, B_EMPTY1, B_VFREE, B_KKREADY, B_KKDONE,
   B_TREADY, B_WDONE, B_WREADY, B_SREADY, B_XDONE, B_VNREADY, B_SDONE,
-  B_ODONE, B_DRAIN, B_COUNT
+  B_ODONE, B_DRAIN, B_FULLV, B_COUNT
 };
 
-// Instruction descriptors (M = 128 everywhere).  Operands are fp16 (11-bit
-// significand: 8x finer than bf16 at the same tensor-core rate), except the
-// channel-gate K K^T product, whose e^{+-(g - g_m)} factors need bf16's range.
-constexpr uint32_t ID_KK_H = idesc_f16kind(128, 64, false, false, false);
+// Instruction descriptors (M = 128 everywhere).  Operands built on chip are
+// fp16 (11-bit significand: 8x finer than bf16 at the same tensor-core rate).
+// Products that read the raw bf16 inputs stay bf16: K K^T (exact inputs), and
+// for the scalar / no gate U and W, whose T factor is split into bf16 hi + lo.
+// The channel-gate K K^T reads e^{+-(g - g_m)}-scaled keys, which need bf16's
+// exponent range.
 constexpr uint32_t ID_KK_B = idesc_f16kind(128, 64, false, false, true);
-constexpr uint32_t ID_UW = idesc_f16kind(128, 64, true, false, false);
+constexpr uint32_t ID_UW_H = idesc_f16kind(128, 64, true, false, false);
+constexpr uint32_t ID_UW_B = idesc_f16kind(128, 64, true, false, true);
 constexpr uint32_t ID_XV = idesc_f16kind(128, 64, false, true, false);
 constexpr uint32_t ID_XO = idesc_f16kind(128, 64, false, false, false);
 constexpr uint32_t ID_SU = idesc_f16kind(128, 128, false, true, false);
@@ -111,6 +123,7 @@ constexpr unsigned kErrNonFinite = 1u << 25;  // non-finite final state
 constexpr float kF16Max = 65504.f;
 
 constexpr long long kWaitCycles = 1ll << 32;   // ~2 s: a wait never lasts this
+constexpr uint32_t kSleepNs = 20000;           // suspend hint per try (20 us)
 
 __device__ unsigned g_fused_error;
 
@@ -135,7 +148,7 @@ __device__ __forceinline__ bool wait_bar(const Ctx &cx, int b,
   if (mbar_try_wait(&cx.bar[b], parity)) return true;
   const long long t0 = clock64();
   for (;;) {
-    if (mbar_try_wait(&cx.bar[b], parity)) return true;
+    if (mbar_try_wait_sleep(&cx.bar[b], parity, kSleepNs)) return true;
     if (*cx.abort_flag) return false;
     if (clock64() - t0 > kWaitCycles) {
       *cx.abort_flag = 1;
@@ -145,18 +158,18 @@ __device__ __forceinline__ bool wait_bar(const Ctx &cx, int b,
   }
 }
 
-// AND of `pred` over the 128 threads of named barrier `id` (also a barrier):
+// AND of `pred` over the `count` threads of named barrier `id` (a barrier):
 // a role group takes every wait decision together, so no thread is left
 // behind at a later named barrier when another one gives up.
-__device__ __forceinline__ bool group_all(bool pred, int id) {
+__device__ __forceinline__ bool group_all(bool pred, int id, int count) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}\n"
       : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id)
+      : "r"((uint32_t)pred), "r"(id), "r"(count)
       : "memory");
   return r != 0;
 }
@@ -174,12 +187,6 @@ __device__ __forceinline__ void unpack_bf16(uint32_t w, float &lo, float &hi) {
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
-}
-__device__ __forceinline__ void unpack_f16(uint32_t w, float &lo, float &hi) {
-  __half2 v = *reinterpret_cast<__half2 *>(&w);
-  float2 f = __half22float2(v);
-  lo = f.x;
-  hi = f.y;
 }
 __device__ __forceinline__ void st_smem_v4(uint8_t *p, uint32_t a, uint32_t b,
                                            uint32_t c, uint32_t d) {
@@ -223,6 +230,35 @@ __device__ __forceinline__ void mma16(const float *X, const float *Z,
   }
 }
 
+// acc (one m16n8 C fragment: columns 8 nt .. 8 nt + 7) += X * Z
+__device__ __forceinline__ void mma16_nt(const float *X, const float *Z,
+                                         float acc[4], int lane, int nt) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    const uint32_t a0 = to_tf32(X[g * 16 + 8 * ks + t]);
+    const uint32_t a1 = to_tf32(X[(g + 8) * 16 + 8 * ks + t]);
+    const uint32_t a2 = to_tf32(X[g * 16 + 8 * ks + t + 4]);
+    const uint32_t a3 = to_tf32(X[(g + 8) * 16 + 8 * ks + t + 4]);
+    const uint32_t b0 = to_tf32(Z[(8 * ks + t) * 16 + 8 * nt + g]);
+    const uint32_t b1 = to_tf32(Z[(8 * ks + t + 4) * 16 + 8 * nt + g]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+}
+__device__ __forceinline__ void store16_nt(float *Y, const float acc[4],
+                                           float s, int lane, int nt) {
+  const int g = lane >> 2, t = lane & 3;
+  Y[g * 16 + 8 * nt + 2 * t] = s * acc[0];
+  Y[g * 16 + 8 * nt + 2 * t + 1] = s * acc[1];
+  Y[(g + 8) * 16 + 8 * nt + 2 * t] = s * acc[2];
+  Y[(g + 8) * 16 + 8 * nt + 2 * t + 1] = s * acc[3];
+}
+
 // store C fragments (scaled by s) to a row-major 16x16 fp32 block
 __device__ __forceinline__ void store16(float *Y, const float acc[8], float s,
                                         int lane) {
@@ -243,8 +279,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmv, Params p) {
   using Lay = Layout<GATE>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-aligned base, derived by pointer arithmetic on the shared array so
+  // that the compiler keeps every access in the shared address space
+  uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + Lay::MISC);
   uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(sm + Lay::MISC + 8 * B_COUNT);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Lay::MISC + 8 * B_COUNT + 4);
@@ -263,8 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const size_t sbase = ((size_t)n * p.H + h) * kD * kD;
 
   if (threadIdx.x == 0) {
-    const uint32_t counts[B_COUNT] = {1, 1, 1, 1, 1, 128, 1, 128, 1, 128,
-                                      128, 1, 128, 1, 1, 1};
+    const uint32_t counts[B_COUNT] = {1, 1, 1, 1, 1, kPrep, 1, kPrep, 1, kPrep,
+                                      128, 1, 128, 1, 1, 1, 1};
     for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], counts[i]);
     *abort_flag = 0;
     fence_mbar_init();
@@ -284,13 +321,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_map(&tmq);
       tma_prefetch_map(&tmk);
       tma_prefetch_map(&tmv);
-      int issued = 0;
+      int issued = 0, issued_v = 0;
       for (int m = 0; m < NC; ++m) {
         const int s = m & 1;
         if (m >= 2 && !wait_bar(cx, B_EMPTY0 + s, ((m - 2) >> 1) & 1)) break;
         const int tok0 = start + m * kC;
         uint8_t *stg = sm + OFF_STAGE + s * kStageBytes;
-        mbar_arrive_expect_tx(&bar[B_FULL0 + s], 6 * 8192);
+        // Q, K of chunk m -> stage m % 2 (full[s]); V -> its one buffer
+        // (fullv) once U of chunk m-1 has read the previous V
+        mbar_arrive_expect_tx(&bar[B_FULL0 + s], 4 * 8192);
         for (int kb = 0; kb < 2; ++kb) {
           tma_load_3d(stg + kb * 16384, &tmk, &bar[B_FULL0 + s], kb * 64, h,
                       tok0);
@@ -299,15 +338,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         issued = m + 1;
         if (m >= 1 && !wait_bar(cx, B_VFREE, (m - 1) & 1)) break;
+        mbar_arrive_expect_tx(&bar[B_FULLV], 2 * 8192);
         for (int kb = 0; kb < 2; ++kb)
-          tma_load_3d(sm + OFF_V + kb * 8192, &tmv, &bar[B_FULL0 + s],
-                      kb * 64, h, tok0);
+          tma_load_3d(sm + OFF_V + kb * 8192, &tmv, &bar[B_FULLV], kb * 64, h,
+                      tok0);
+        issued_v = m + 1;
       }
       if (*abort_flag) {
         // let in-flight copies land before the CTA exits (bounded)
         for (int m = max(0, issued - 2); m < issued; ++m) {
           const long long t0 = clock64();
           while (!mbar_try_wait(&bar[B_FULL0 + (m & 1)], (m >> 1) & 1) &&
+                 clock64() - t0 < (1ll << 28)) {
+          }
+        }
+        if (issued_v > 0) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(&bar[B_FULLV], (issued_v - 1) & 1) &&
                  clock64() - t0 < (1ll << 28)) {
           }
         }
@@ -318,11 +365,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t st = smem_u32(sm + OFF_ST), nw = smem_u32(sm + OFF_NW),
                      vn = smem_u32(sm + OFF_VN), vt = smem_u32(sm + OFF_V),
-                     tpg = smem_u32(sm + OFF_TPG),
-                     tpb = smem_u32(sm + OFF_TPB),
-                     kn = smem_u32(sm + OFF_KN);
+                     tp = smem_u32(sm + OFF_TP),
+                     kn = smem_u32(sm + Lay::KN);
       auto stage = [&](int m) {
         return smem_u32(sm + OFF_STAGE + (m & 1) * kStageBytes);
+      };
+      // channel gate: the prep warps rescale Q, K in place first (kk_ready);
+      // otherwise K K^T runs straight on the landed bf16 tiles
+      auto kk_inputs_ready = [&](int m) {
+        return GATE == 2 ? wait_bar(cx, B_KKREADY, m & 1)
+                         : wait_bar(cx, B_FULL0 + (m & 1), (m >> 1) & 1);
       };
       auto issue_kk = [&](int m) {
         const uint32_t base = stage(m);
@@ -334,36 +386,75 @@ __global__ void __launch_bounds__(kThreads, 1)
               GATE == 2
                   ? sdesc_sw128(kn + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024)
                   : sdesc_sw128(base + koff, 16, 1024);
-          mma_f16kind(tmem + ACC_KK, a, b, GATE == 2 ? ID_KK_B : ID_KK_H, ks > 0);
+          mma_f16kind(tmem + ACC_KK, a, b, ID_KK_B, ks > 0);
         }
         mma_commit(&bar[B_KKDONE]);
       };
+      // U^T = V^T (T diag b)^T and W^T = (K e^g)^T (T diag(b e^g))^T
       auto issue_uw = [&](int m) {
+        if (!wait_bar(cx, B_FULLV, m & 1)) return false;
+        tc_fence_after();
         const uint32_t base = stage(m);
         const uint32_t accv = tmem + ACC_V + (m & 1) * 64;
+        if (GATE == 2) {
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_f16kind(accv, sdesc_sw128(vt + ks * 2048, 8192, 1024),
-                   sdesc_sw128(tpb + ks * 32, 16, 1024), ID_UW, ks > 0);
+          for (int ks = 0; ks < 4; ++ks)
+            mma_f16kind(accv, sdesc_sw128(vt + ks * 2048, 8192, 1024),
+                        sdesc_sw128(tp + ks * 32, 16, 1024), ID_UW_H, ks > 0);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_f16kind(tmem + ACC_W, sdesc_sw128(base + ks * 2048, 16384, 1024),
-                   sdesc_sw128((GATE == 2 ? tpb : tpg) + ks * 32, 16, 1024),
-                   ID_UW, ks > 0);
+          for (int ks = 0; ks < 4; ++ks)
+            mma_f16kind(tmem + ACC_W,
+                        sdesc_sw128(base + ks * 2048, 16384, 1024),
+                        sdesc_sw128(tp + ks * 32, 16, 1024), ID_UW_H, ks > 0);
+        } else {
+          // hi and lo halves of the T factor accumulate into one result
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_f16kind(accv, sdesc_sw128(vt + (ks & 3) * 2048, 8192, 1024),
+                        sdesc_sw128(tp + 16384 + (ks >> 2) * 8192 + (ks & 3) * 32,
+                                    16, 1024),
+                        ID_UW_B, ks > 0);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_f16kind(tmem + ACC_W,
+                        sdesc_sw128(base + (ks & 3) * 2048, 16384, 1024),
+                        sdesc_sw128(tp + (ks >> 2) * 8192 + (ks & 3) * 32, 16,
+                                    1024),
+                        ID_UW_B, ks > 0);
+        }
         mma_commit(&bar[B_WDONE]);
         mma_commit(&bar[B_VFREE]);
+        return true;
+      };
+      // K K^T of chunk j may run as soon as its tiles are in and the prep
+      // warps have read K K^T of chunk j-1 (t_ready(j-1)); after each U/W
+      // issue the next one is tried without blocking, else it is issued at
+      // its place in the loop below
+      int kk_next = 0;
+      auto try_kk_early = [&](int j) {
+        if (kk_next != j || j >= NC) return;
+        const bool ready =
+            GATE == 2 ? mbar_try_wait(&bar[B_KKREADY], j & 1)
+                      : mbar_try_wait(&bar[B_FULL0 + (j & 1)], (j >> 1) & 1);
+        if (ready) {
+          tc_fence_after();
+          issue_kk(j);
+          ++kk_next;
+        }
       };
       bool ok = true;
       if (NC > 0) {
-        ok = wait_bar(cx, B_KKREADY, 0);
+        ok = kk_inputs_ready(0);
         if (ok) {
           tc_fence_after();
           issue_kk(0);
+          kk_next = 1;
           ok = wait_bar(cx, B_TREADY, 0);
         }
         if (ok) {
           tc_fence_after();
-          issue_uw(0);
+          ok = issue_uw(0);
+          try_kk_early(1);
         }
       }
       for (int m = 0; m < NC && ok; ++m) {
@@ -387,11 +478,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                16, 1024),
                    ID_XO, ks > 0);
         mma_commit(&bar[B_XDONE]);
-        // KK(m+1) while the state warps turn V_new into an operand
-        if (m + 1 < NC) {
-          if (!wait_bar(cx, B_KKREADY, (m + 1) & 1)) break;
+        // K K^T of chunk m+1 while the state warps turn V_new into an operand
+        if (m + 1 < NC && kk_next == m + 1) {
+          if (!kk_inputs_ready(m + 1)) break;
           tc_fence_after();
           issue_kk(m + 1);
+          ++kk_next;
         }
         // S update and intra-chunk output
         if (!wait_bar(cx, B_VNREADY, m & 1)) break;
@@ -413,7 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (m + 1 < NC) {
           if (!wait_bar(cx, B_TREADY, (m + 1) & 1)) break;
           tc_fence_after();
-          issue_uw(m + 1);
+          if (!issue_uw(m + 1)) break;
+          try_kk_early(m + 2);
         }
       }
       // every MMA issued has completed before tensor memory is released
@@ -437,9 +530,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tmem_wait_st();
     bool ok = true;
+    // O^T of chunk m (lane = value channel, column = row) -> out rows, via
+    // a [64 rows][128 channels] bf16 staging tile in the V_new^T tile, which
+    // is free between O(m) done and the V_new^T write of chunk m+1.
+    // Neighbouring lanes swap values so each writes two adjacent channels.
     auto store_output = [&](int m) {
       const int tok0 = start + m * kC, L = min(kC, end - tok0);
-      uint8_t *stg = sm + OFF_VN;               // [64 rows][128 dv] bf16
+      uint8_t *stg = sm + OFF_VN;
       for (int c0 = 0; c0 < kC; c0 += 32) {
         tmem_ld32(trow + ACC_O + (m & 1) * 64 + c0, v);
         tmem_wait_ld();
@@ -468,9 +565,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *gC = reinterpret_cast<float *>(sm + Lay::GC);
     for (int m = 0; m < NC; ++m) {
       // S (chunk start) -> bf16 operand; decayed S back to tensor memory
-      if (m > 0 && !(ok = group_all(wait_bar(cx, B_SDONE, (m - 1) & 1), 1)))
+      if (m > 0 && !(ok = group_all(wait_bar(cx, B_SDONE, (m - 1) & 1), 1, 128)))
         break;
-      if (!(ok = group_all(wait_bar(cx, B_TREADY, m & 1), 1))) break;
+      if (!(ok = group_all(wait_bar(cx, B_TREADY, m & 1), 1, 128))) break;
       tc_fence_after();
       const float *gcm = gC + (m & 1) * 128;
       const float dscal = GATE == 1 ? __expf(gcm[0]) : 1.f;
@@ -498,12 +595,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bar[B_SREADY]);
       // output of the previous chunk while X(m) runs
       if (m > 0) {
-        if (!(ok = group_all(wait_bar(cx, B_ODONE, (m - 1) & 1), 1))) break;
+        if (!(ok = group_all(wait_bar(cx, B_ODONE, (m - 1) & 1), 1, 128))) break;
         tc_fence_after();
         store_output(m - 1);
       }
-      // V_new^T -> bf16 operand
-      if (!(ok = group_all(wait_bar(cx, B_XDONE, m & 1), 1))) break;
+      // V_new^T -> fp16 operand
+      if (!(ok = group_all(wait_bar(cx, B_XDONE, m & 1), 1, 128))) break;
       tc_fence_after();
       for (int c0 = 0; c0 < kC; c0 += 32) {
         tmem_ld32(trow + ACC_V + (m & 1) * 64 + c0, v);
@@ -521,11 +618,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bar[B_VNREADY]);
     }
     if (ok && NC > 0) {
-      ok = group_all(wait_bar(cx, B_ODONE, (NC - 1) & 1), 1);
+      ok = group_all(wait_bar(cx, B_ODONE, (NC - 1) & 1), 1, 128);
       if (ok) {
         tc_fence_after();
         store_output(NC - 1);
-        ok = group_all(wait_bar(cx, B_SDONE, (NC - 1) & 1), 1);
+        ok = group_all(wait_bar(cx, B_SDONE, (NC - 1) & 1), 1, 128);
       }
     }
     if (ok) {
@@ -544,86 +641,99 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------ prep warps
+    // 8 warps, two per scheduler.  pt = 0..255; TMEM lane l (two threads per
+    // lane: hf selects which 32 of a 64-column accumulator each one reads).
+    const int pt = threadIdx.x - 6 * 32;
     const int q4 = warp & 3;
-    const int l = q4 * 32 + lane;                  // lane of tensor memory
-    const int pw = warp - 6;                       // 0..3
+    const int l = q4 * 32 + lane;
+    const int hf = (warp - 6) >> 2;
+    const int pw = warp - 6;                       // 0..7
     const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
     float *gS = reinterpret_cast<float *>(sm + Lay::GS);
-    float *bS = reinterpret_cast<float *>(sm + Lay::BS);
+    float *FT = reinterpret_cast<float *>(sm + Lay::FT);
     float *gC = reinterpret_cast<float *>(sm + Lay::GC);
     float *gM = reinterpret_cast<float *>(sm + Lay::GM);
-    float *YS = reinterpret_cast<float *>(sm + Lay::YS) + pw * 256;
     float v[32];
+    // gates of the next chunk are loaded one chunk ahead (threads pt < 64)
+    float nb = 0.f, na = 0.f;
+    auto load_gates = [&](int m) {
+      nb = 0.f;
+      na = 0.f;
+      const int tok0 = start + m * kC, L = min(kC, end - tok0);
+      if (m < NC && pt < L) {
+        nb = p.beta[(size_t)(tok0 + pt) * p.H + h];
+        if (GATE == 1) na = p.log_alpha[(size_t)(tok0 + pt) * p.H + h];
+      }
+    };
+    if (pt < 64) load_gates(0);
     for (int m = 0; m < NC; ++m) {
       const int s = m & 1, tok0 = start + m * kC, L = min(kC, end - tok0);
       uint8_t *stg = sm + OFF_STAGE + s * kStageBytes;
-      float *g = gS + s * 64, *b = bS + s * 64, *gc = gC + s * 128;
-      // ---- P1: gates (beta, in-chunk cumulative log-decay)
+      float *g = gS + s * 64, *gc = gC + s * 128;
+      float *F = FT + s * (F_COUNT * 64);
+      // ---- P1: beta, in-chunk cumulative log-decay, per-row factors
+      float x = na, bb = nb;
+      if (pt < 64) load_gates(m + 1);
       if (GATE != 2) {
-        float x = 0.f, bb = 0.f;
-        if (l < L) {
-          bb = p.beta[(size_t)(tok0 + l) * p.H + h];
-          if (GATE == 1) x = p.log_alpha[(size_t)(tok0 + l) * p.H + h];
-        }
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
           const float y = __shfl_up_sync(0xffffffffu, x, off);
           if (lane >= off) x += y;
         }
-        if (l == 31) *scan_tmp = x;
-        named_bar_sync(2, 128);
-        if (l >= 32 && l < 64) x += *scan_tmp;
-        if (l < 64) {
-          g[l] = x;
-          b[l] = bb;
-        }
-        if (l == L - 1) gc[0] = x;
-      } else if (l < 64) {
-        b[l] = (l < L) ? p.beta[(size_t)(tok0 + l) * p.H + h] : 0.f;
+        if (pt == 31) *scan_tmp = x;
       }
-      // ---- P2: operand tiles.  V -> fp16 in place.  Scalar / no gate:
-      // Q, K -> fp16 in place.  Channel gate: thread l owns key channel l and
-      // forms, with g_m = g at row 31, Q e^{g-g_m}, K e^{g-g_m} and
-      // K e^{g_m-g} in bf16 (the exponent range of these factors needs bf16).
-      if (!group_all(wait_bar(cx, B_FULL0 + s, (m >> 1) & 1), 2)) break;
+      named_bar_sync(2, kPrep);
+      if (pt < 64) {
+        if (GATE != 2 && pt >= 32) x += *scan_tmp;
+        if (GATE != 2) g[pt] = x;
+        F[F_B * 64 + pt] = bb;
+      }
+      if (GATE != 2 && pt == 63) gc[0] = x;
+      named_bar_sync(2, kPrep);
+      // factors: E_r = e^{g_r - g_31}, F_r = e^{g_31 - g_r} (so that
+      // e^{g_r - g_i} = E_r F_i without a per-element exponential; used
+      // when the chunk's decay range keeps both within fp32), b e^g, e^g,
+      // e^{g_C - g}
+      if (GATE != 2 && pt < 64) {
+        const float gr = x, gref = g[31], gcv = g[63];
+        F[F_BG * 64 + pt] = bb * __expf(gr);
+        F[F_E * 64 + pt] = __expf(gr - gref);
+        F[F_F * 64 + pt] = __expf(gref - gr);
+        F[F_EG * 64 + pt] = __expf(gr);
+        F[F_EK * 64 + pt] = __expf(gcv - gr);
+      }
+      // ---- P2 (channel gate only): per key channel c, with g_m = g at row
+      // 31: Q e^{g-g_m}, K e^{g-g_m}, K e^{g_m-g} (bf16)
       float amax = 0.f;
-      {
-        const int n16 = (GATE == 2) ? 1024 : 3072;  // 16-byte words
-        for (int i = l; i < n16; i += 128) {
-          uint8_t *ptr = (GATE == 2 || i >= 2048)
-                             ? sm + OFF_V + (i - (GATE == 2 ? 0 : 2048)) * 16
-                             : stg + i * 16;
-          uint4 x = *reinterpret_cast<uint4 *>(ptr);
-          uint32_t *w = reinterpret_cast<uint32_t *>(&x);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float a0, a1;
-            unpack_bf16(w[e], a0, a1);
-            amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
-            w[e] = pack_f16(a0, a1);
-          }
-          *reinterpret_cast<uint4 *>(ptr) = x;
-        }
-      }
       if (GATE == 2) {
-        const float *la = p.log_alpha + ((size_t)tok0 * p.H + h) * kD + l;
+        if (!group_all(wait_bar(cx, B_FULL0 + s, (m >> 1) & 1), 2, kPrep))
+          break;
+        const int c = pt & 127, half = pt >> 7;
+        const float *la = p.log_alpha + ((size_t)tok0 * p.H + h) * kD + c;
         const size_t rs = (size_t)p.H * kD;
-        float gr[kC];
-        float gg = 0.f;
+        float lv[32];
 #pragma unroll
-        for (int r = 0; r < kC; ++r) {
-          gg += (r < L) ? la[r * rs] : 0.f;
-          gr[r] = gg;
+        for (int j = 0; j < 32; ++j) {
+          const int r = half * 32 + j;
+          lv[j] = (r < L) ? la[r * rs] : 0.f;
         }
-        const float gm = gr[31];
-        gM[l] = gm;
-        gc[l] = gg;
-        uint8_t *kt = stg + (l >> 6) * 16384, *qt = kt + 8192;
-        uint8_t *knt = sm + OFF_KN + (l >> 6) * 8192;
+        float gm = 0.f;
+        if (half == 0) {
 #pragma unroll
-        for (int r = 0; r < kC; ++r) {
-          const float ep = __expf(gr[r] - gm), en = __expf(gm - gr[r]);
-          const uint32_t off = sw128_off(r, l & 63);
+          for (int j = 0; j < 32; ++j) gm += lv[j];
+        } else {
+#pragma unroll
+          for (int r = 0; r < 32; ++r) gm += (r < L) ? la[r * rs] : 0.f;
+        }
+        float gg = half ? gm : 0.f;
+        uint8_t *kt = stg + (c >> 6) * 16384, *qt = kt + 8192;
+        uint8_t *knt = sm + Lay::KN + (c >> 6) * 8192;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int r = half * 32 + j;
+          gg += lv[j];
+          const float ep = __expf(gg - gm), en = __expf(gm - gg);
+          const uint32_t off = sw128_off(r, c & 63);
           __nv_bfloat16 *qe = reinterpret_cast<__nv_bfloat16 *>(qt + off);
           __nv_bfloat16 *ke = reinterpret_cast<__nv_bfloat16 *>(kt + off);
           const float qv = __bfloat162float(*qe), kv = __bfloat162float(*ke);
@@ -633,59 +743,68 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<__nv_bfloat16 *>(knt + off) =
               __float2bfloat16_rn(kv * en);
         }
+        if (half == 0) gM[c] = gm;
+        else gc[c] = gg;
+        fence_proxy_async_smem();
+        mbar_arrive(&bar[B_KKREADY]);
       }
-      if (!(amax <= kF16Max)) atomicOr(&g_fused_error, kErrRange);
-      fence_proxy_async_smem();
-      mbar_arrive(&bar[B_KKREADY]);
       // ---- P3: A (strictly lower, fp32 blocks) and P (lower, fp16 operand)
-      if (!group_all(wait_bar(cx, B_KKDONE, m & 1), 2)) break;
+      if (!group_all(wait_bar(cx, B_KKDONE, m & 1), 2, kPrep)) break;
       tc_fence_after();
-      for (int c0 = 0; c0 < kC; c0 += 32) {
+      const bool fact = (GATE != 1) || (g[0] - g[63] < 80.f);
+      {
+        const int c0 = hf * 32;
         tmem_ld32(trow + ACC_KK + c0, v);
         tmem_wait_ld();
-        if (l < 64) {
-          const int r = l;
-          const float gr = g[r], br = (r < L) ? b[r] : 0.f;
+        const bool arow = (l < 64);
+        const int r = arow ? l : l - 64;
+        // A row: beta_r e^{g_r - g_i} (K K^T)_ri, i < r;
+        // P row: e^{g_r - g_i} (Q K^T)_ri, i <= r
+        const float br = arow ? ((r < L) ? F[F_B * 64 + r] : 0.f) : 1.f;
+        const float gr = (GATE == 1) ? g[r] : 0.f;
+        const bool use_f = (GATE == 1) && fact;
+        const float sc = use_f ? br * F[F_E * 64 + r] : br;
+        if (GATE == 1 && !fact) {
+          // decay range too wide to factor: one exponential per element
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int i = c0 + j;
-            float a = 0.f;
-            if (i < r) {
-              a = br * v[j];
-              if (GATE == 1) a *= __expf(gr - g[i]);
-            }
-            v[j] = a;
+            const bool keep = arow ? (i < r) : (i <= r);
+            v[j] = keep ? v[j] * __expf(gr - g[i]) * sc : 0.f;
           }
-          // write the blocks (r/16, i/16) with i/16 <= r/16
+        } else {
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int cb = (c0 >> 4) + half;
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 f4 = use_f
+                ? *reinterpret_cast<const float4 *>(F + F_F * 64 + c0 + 4 * j4)
+                : make_float4(1.f, 1.f, 1.f, 1.f);
+            const float fi[4] = {f4.x, f4.y, f4.z, f4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = 4 * j4 + e, i = c0 + j;
+              const bool keep = arow ? (i < r) : (i <= r);
+              v[j] = keep ? v[j] * fi[e] * sc : 0.f;
+            }
+          }
+        }
+        if (arow) {
+#pragma unroll
+          for (int half2 = 0; half2 < 2; ++half2) {
+            const int cb = (c0 >> 4) + half2;
             if (cb <= (r >> 4)) {
               float4 *dst = reinterpret_cast<float4 *>(
                   AC + blk(r >> 4, cb) * 256 + (r & 15) * 16);
 #pragma unroll
               for (int e = 0; e < 4; ++e)
-                dst[e] = make_float4(v[16 * half + 4 * e], v[16 * half + 4 * e + 1],
-                                     v[16 * half + 4 * e + 2], v[16 * half + 4 * e + 3]);
+                dst[e] = make_float4(v[16 * half2 + 4 * e], v[16 * half2 + 4 * e + 1],
+                                     v[16 * half2 + 4 * e + 2], v[16 * half2 + 4 * e + 3]);
             }
           }
         } else {
-          const int r = l - 64;
-          const float gr = g[r];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int i = c0 + j;
-            float pv = 0.f;
-            if (i <= r) {
-              pv = v[j];
-              if (GATE == 1) pv *= __expf(gr - g[i]);
-            }
-            v[j] = pv;
-          }
-          uint8_t *pt = sm + OFF_P + s * 8192;
+          uint8_t *ptl = sm + OFF_P + s * 8192;
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch)
-            st_smem_v4(pt + sw128_chunk(r, (c0 >> 3) + ch),
+            st_smem_v4(ptl + sw128_chunk(r, (c0 >> 3) + ch),
                        pack_f16(v[8 * ch + 0], v[8 * ch + 1]),
                        pack_f16(v[8 * ch + 2], v[8 * ch + 3]),
                        pack_f16(v[8 * ch + 4], v[8 * ch + 5]),
@@ -694,91 +813,143 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (GATE == 2) {
         // Q e^{g-g_m}, K e^{g-g_m} (bf16) -> Q e^g, K e^g (fp16), in place
-        for (int idx = l; idx < kC * 16; idx += 128) {
+        for (int idx = pt; idx < kC * 16; idx += kPrep) {
           const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
           const uint32_t off = kb * 16384 + sw128_chunk(r, cc & 7);
-          const int c0 = kb * 64 + (cc & 7) * 8;
+          const int cbase = kb * 64 + (cc & 7) * 8;
 #pragma unroll
           for (int part = 0; part < 2; ++part) {
             uint4 *ptr = reinterpret_cast<uint4 *>(stg + off + part * 8192);
-            uint4 x = *ptr;
-            uint32_t *w = reinterpret_cast<uint32_t *>(&x);
+            uint4 xv = *ptr;
+            uint32_t *w = reinterpret_cast<uint32_t *>(&xv);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               float a0, a1;
               unpack_bf16(w[e], a0, a1);
-              w[e] = pack_f16(a0 * __expf(gM[c0 + 2 * e]),
-                              a1 * __expf(gM[c0 + 2 * e + 1]));
+              w[e] = pack_f16(a0 * __expf(gM[cbase + 2 * e]),
+                              a1 * __expf(gM[cbase + 2 * e + 1]));
             }
-            *ptr = x;
+            *ptr = xv;
           }
         }
       }
-      named_bar_sync(2, 128);
+      named_bar_sync(2, kPrep);
       // ---- P4: T = (I + A)^-1.  Diagonal 16x16 blocks by forward
       // substitution (one thread per column), then the off-diagonal blocks
       // T_bc = -D_b sum_{c<=e<b} A_be T_ec on mma.sync (tf32), level by level.
-      if (l < 64) {
-        const int bb = l >> 4, j = l & 15;
+      if (pt < 64) {
+        const int bb = pt >> 4, j = pt & 15;
         const float *Ab = AC + blk(bb, bb) * 256;
-        float x[16];
+        float xs[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-          float acc = (r == j) ? 1.f : 0.f;
+          float acc0 = (r == j) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-          for (int i = 0; i < r; ++i) acc -= Ab[r * 16 + i] * x[i];
-          x[r] = acc;
+          for (int i = 0; i < r; ++i) {
+            if (i & 1) acc1 -= Ab[r * 16 + i] * xs[i];
+            else acc0 -= Ab[r * 16 + i] * xs[i];
+          }
+          xs[r] = acc0 + acc1;
         }
         float *Tb = TC + blk(bb, bb) * 256;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Tb[r * 16 + j] = x[r];
+        for (int r = 0; r < 16; ++r) Tb[r * 16 + j] = xs[r];
       }
-      named_bar_sync(2, 128);
+      named_bar_sync(2, kPrep);
+      // M_be = D_b A_be for the six blocks below the diagonal, in place
+      if (pw < 6) {
+        const int bb = (pw < 1) ? 1 : (pw < 3) ? 2 : 3;
+        const int e = (pw < 1) ? 0 : (pw < 3) ? pw - 1 : pw - 3;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        mma16(TC + blk(bb, bb) * 256, AC + blk(bb, e) * 256, acc, lane);
+        __syncwarp();
+        store16(AC + blk(bb, e) * 256, acc, 1.f, lane);
+      }
+      named_bar_sync(2, kPrep);
+      // T_bc = -sum_{c<=e<b} M_be T_ec (T_cc = D_c), level b - c at a time;
+      // one warp per 8-column half of each block of the level
 #pragma unroll 1
       for (int lev = 1; lev <= 3; ++lev) {
-        if (pw <= 3 - lev) {
-          const int c = pw, bb = pw + lev;
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (pw < 2 * (4 - lev)) {
+          const int c = pw >> 1, nt = pw & 1, bb = c + lev;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
           for (int e = c; e < bb; ++e)
-            mma16(AC + blk(bb, e) * 256, TC + blk(e, c) * 256, acc, lane);
-          store16(YS, acc, 1.f, lane);
-          __syncwarp();
-          float acc2[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          mma16(TC + blk(bb, bb) * 256, YS, acc2, lane);
-          __syncwarp();
-          store16(TC + blk(bb, c) * 256, acc2, -1.f, lane);
+            mma16_nt(AC + blk(bb, e) * 256, TC + blk(e, c) * 256, acc, lane, nt);
+          store16_nt(TC + blk(bb, c) * 256, acc, -1.f, lane, nt);
         }
-        named_bar_sync(2, 128);
+        named_bar_sync(2, kPrep);
       }
-      // ---- T-factor operands (fp16): rows 0..63 -> T diag(beta e^g),
-      //      rows 64..127 -> T diag(beta)
-      {
-        const int r = l & 63;
-        const bool with_g = (l < 64);
-        uint8_t *dst = sm + (with_g ? OFF_TPG : OFF_TPB);
+      // channel gate: V -> fp16 in place for U = (T diag b) V
+      if (GATE == 2) {
+        if (!group_all(wait_bar(cx, B_FULLV, m & 1), 2, kPrep)) break;
+        for (int i = pt; i < 1024; i += kPrep) {
+          uint8_t *ptr = sm + OFF_V + i * 16;
+          uint4 xv = *reinterpret_cast<uint4 *>(ptr);
+          uint32_t *w = reinterpret_cast<uint32_t *>(&xv);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          float t8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int i = 8 * ch + e;
-            const int cb = i >> 4, rb = r >> 4;
-            float t = (cb <= rb) ? TC[blk(rb, cb) * 256 + (r & 15) * 16 + (i & 15)] : 0.f;
-            float f = (i < L) ? b[i] : 0.f;
-            if (with_g && GATE == 1) f *= __expf(g[i]);
-            t8[e] = t * f;
+          for (int e = 0; e < 4; ++e) {
+            float a0, a1;
+            unpack_bf16(w[e], a0, a1);
+            amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
+            w[e] = pack_f16(a0, a1);
           }
-          st_smem_v4(dst + sw128_chunk(r, ch), pack_f16(t8[0], t8[1]),
-                     pack_f16(t8[2], t8[3]), pack_f16(t8[4], t8[5]),
-                     pack_f16(t8[6], t8[7]));
+          *reinterpret_cast<uint4 *>(ptr) = xv;
+        }
+      }
+      // ---- T-factor operands.  Scalar / no gate: T diag(b e^g) and
+      // T diag(b) as bf16 hi + lo pairs.  Channel gate: T diag(b) in fp16.
+      {
+        const int r = pt & 63, rb = r >> 4;
+        const int which = (GATE == 2) ? 1 : ((pt >> 6) & 1);   // 0: b e^g, 1: b
+        const int chs = (GATE == 2) ? 0 : ((pt >> 7) * 4);     // chunk range
+        const int che = (GATE == 2) ? 8 : chs + 4;
+        const float *fac = F + (which == 0 ? F_BG : F_B) * 64;
+        if (GATE != 2 || pt < 64) {
+          for (int ch = chs; ch < che; ++ch) {
+            const int cb = (8 * ch) >> 4;
+            float t8[8];
+            if (cb <= rb) {
+              const float4 *tsrc = reinterpret_cast<const float4 *>(
+                  TC + blk(rb, cb) * 256 + (r & 15) * 16 + ((8 * ch) & 15));
+              const float4 t0 = tsrc[0], t1 = tsrc[1];
+              const float4 f0 = *reinterpret_cast<const float4 *>(fac + 8 * ch);
+              const float4 f1 = *reinterpret_cast<const float4 *>(fac + 8 * ch + 4);
+              t8[0] = t0.x * f0.x; t8[1] = t0.y * f0.y; t8[2] = t0.z * f0.z;
+              t8[3] = t0.w * f0.w; t8[4] = t1.x * f1.x; t8[5] = t1.y * f1.y;
+              t8[6] = t1.z * f1.z; t8[7] = t1.w * f1.w;
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) t8[e] = 0.f;
+            }
+            if (GATE == 2) {
+              st_smem_v4(sm + OFF_TP + sw128_chunk(r, ch),
+                         pack_f16(t8[0], t8[1]), pack_f16(t8[2], t8[3]),
+                         pack_f16(t8[4], t8[5]), pack_f16(t8[6], t8[7]));
+            } else {
+              uint32_t hw[4], lw[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat16 h0 = __float2bfloat16_rn(t8[2 * e]);
+                const __nv_bfloat16 h1 = __float2bfloat16_rn(t8[2 * e + 1]);
+                hw[e] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
+                lw[e] = pack_bf16(t8[2 * e] - __bfloat162float(h0),
+                                  t8[2 * e + 1] - __bfloat162float(h1));
+              }
+              const uint32_t hi = which == 0 ? Lay::TPG_HI : Lay::TPB_HI;
+              const uint32_t lo = which == 0 ? Lay::TPG_LO : Lay::TPB_LO;
+              st_smem_v4(sm + hi + sw128_chunk(r, ch), hw[0], hw[1], hw[2], hw[3]);
+              st_smem_v4(sm + lo + sw128_chunk(r, ch), lw[0], lw[1], lw[2], lw[3]);
+            }
+          }
         }
       }
       fence_proxy_async_smem();
       mbar_arrive(&bar[B_TREADY]);
       // ---- P5: -W^T operand; Q e^g and K e^{g_C - g} in place (fp16)
-      if (!group_all(wait_bar(cx, B_WDONE, m & 1), 2)) break;
+      if (!group_all(wait_bar(cx, B_WDONE, m & 1), 2, kPrep)) break;
       tc_fence_after();
-      for (int c0 = 0; c0 < kC; c0 += 32) {
+      {
+        const int c0 = hf * 32;
         tmem_ld32(trow + ACC_W + c0, v);
         tmem_wait_ld();
 #pragma unroll
@@ -789,45 +960,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                      pack_f16(-v[8 * ch + 4], -v[8 * ch + 5]),
                      pack_f16(-v[8 * ch + 6], -v[8 * ch + 7]));
       }
-      if (GATE != 0) {
-        for (int idx = l; idx < kC * 16; idx += 128) {
-          const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
-          const uint32_t off = kb * 16384 + sw128_chunk(r, cc & 7);
-          uint4 *kp = reinterpret_cast<uint4 *>(stg + off);
-          uint4 kv;
-          if (GATE == 1) {
-            uint4 *qp = reinterpret_cast<uint4 *>(stg + off + 8192);
-            const float eq = __expf(g[r]), ek = __expf(gc[0] - g[r]);
-            uint4 qv = *qp;
-            kv = *kp;
-            uint32_t *qw = reinterpret_cast<uint32_t *>(&qv);
-            uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
+      for (int idx = pt; idx < kC * 16; idx += kPrep) {
+        const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
+        const uint32_t off = kb * 16384 + sw128_chunk(r, cc & 7);
+        uint4 *kp = reinterpret_cast<uint4 *>(stg + off);
+        uint4 kv;
+        uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
+        if (GATE != 2) {
+          // raw bf16 -> fp16, scaled by e^g (Q) and e^{g_C - g} (K)
+          uint4 *qp = reinterpret_cast<uint4 *>(stg + off + 8192);
+          const float eq = (GATE == 1) ? F[F_EG * 64 + r] : 1.f;
+          const float ek = (GATE == 1) ? F[F_EK * 64 + r] : 1.f;
+          uint4 qv = *qp;
+          kv = *kp;
+          uint32_t *qw = reinterpret_cast<uint32_t *>(&qv);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float a0, a1;
-              unpack_f16(qw[e], a0, a1);
-              qw[e] = pack_f16(a0 * eq, a1 * eq);
-              unpack_f16(kw[e], a0, a1);
-              kw[e] = pack_f16(a0 * ek, a1 * ek);
-            }
-            *qp = qv;
-          } else {
-            // K~ = (K e^{g_m-g}) e^{g_C-g_m}, per channel
-            kv = *reinterpret_cast<const uint4 *>(sm + OFF_KN + kb * 8192 +
-                                                  sw128_chunk(r, cc & 7));
-            uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
-            const int c0 = kb * 64 + (cc & 7) * 8;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float a0, a1;
-              unpack_bf16(kw[e], a0, a1);
-              kw[e] = pack_f16(a0 * __expf(gc[c0 + 2 * e] - gM[c0 + 2 * e]),
-                               a1 * __expf(gc[c0 + 2 * e + 1] - gM[c0 + 2 * e + 1]));
-            }
+          for (int e = 0; e < 4; ++e) {
+            float a0, a1;
+            unpack_bf16(qw[e], a0, a1);
+            amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
+            qw[e] = pack_f16(a0 * eq, a1 * eq);
+            unpack_bf16(kw[e], a0, a1);
+            amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
+            kw[e] = pack_f16(a0 * ek, a1 * ek);
           }
-          *kp = kv;
+          *qp = qv;
+        } else {
+          // K~ = (K e^{g_m-g}) e^{g_C-g_m}, per channel
+          kv = *reinterpret_cast<const uint4 *>(sm + Lay::KN + kb * 8192 +
+                                                sw128_chunk(r, cc & 7));
+          const int cbase = kb * 64 + (cc & 7) * 8;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float a0, a1;
+            unpack_bf16(kw[e], a0, a1);
+            kw[e] = pack_f16(a0 * __expf(gc[cbase + 2 * e] - gM[cbase + 2 * e]),
+                             a1 * __expf(gc[cbase + 2 * e + 1] - gM[cbase + 2 * e + 1]));
+          }
         }
+        *kp = kv;
       }
+      if (!(amax <= kF16Max)) atomicOr(&g_fused_error, kErrRange);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bar[B_WREADY]);
