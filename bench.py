@@ -193,25 +193,42 @@ def cpu_cores():
 
 
 def oracle_sample(inp, nseq_sample):
-    """The first `nseq_sample` sequences of a fixed-length workload (all
-    heads), as oracle inputs."""
+    """The first `nseq_sample` sequences of the workload (all heads), as
+    oracle inputs, and their token count."""
     f = inp.f64()
-    for key in ("q", "k", "v", "beta", "log_alpha"):
-        if f[key] is not None:
-            f[key] = f[key][:nseq_sample]
+    if f["cu_seqlens"] is None:
+        for key in ("q", "k", "v", "beta", "log_alpha"):
+            if f[key] is not None:
+                f[key] = f[key][:nseq_sample]
+        tokens = nseq_sample * inp.w.T
+    else:
+        tokens = int(f["cu_seqlens"][nseq_sample])
+        for key in ("q", "k", "v", "beta", "log_alpha"):
+            if f[key] is not None:
+                f[key] = f[key][:, :tokens]
+        f["cu_seqlens"] = f["cu_seqlens"][:nseq_sample + 1]
     if f["initial_state"] is not None:
         f["initial_state"] = f["initial_state"][:nseq_sample]
-    return f
+    return f, tokens
 
 
 def time_oracle(inp, nseq_sample):
     import oracle
-    f = oracle_sample(inp, nseq_sample)
+    f, tokens = oracle_sample(inp, nseq_sample)
     t0 = time.perf_counter()
     _, _, threads = oracle.gdr_fwd(**f)
     dt = time.perf_counter() - t0
-    tokens = nseq_sample * inp.w.T
     return tokens / dt, threads, dt, tokens
+
+
+def workload_config(w, inp):
+    """The `config` object of a bench line: the workload and its sizes."""
+    cfg = {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk,
+           "dv": w.dv, "chunk": w.chunk, "gate": w.gate}
+    if w.varlen_nseq:
+        cfg.update(B=inp.nseq, T=None, total_tokens=inp.ntok,
+                   lengths=list(inp.lengths))
+    return cfg
 
 
 def run_reference(args, w):
@@ -231,16 +248,16 @@ def run_reference(args, w):
         total_tok += tok
         total_t += dt
     value = total_tok / total_t
+    _, tok = oracle_sample(inp, nsample)
     sample = (f"sequences 0..{nsample - 1} of {len(inp.lengths)} "
-              f"({nsample * w.T} tokens x {w.H} heads) per step")
+              f"({tok} tokens x {w.H} heads) per step")
     line = {
         "impl": "reference", "metric": METRIC, "value": value,
         "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H,
-                   "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "gate": w.gate},
+        "config": workload_config(w, inp),
         "cpu_baseline": {"value": value, "unit": "tokens/s",
                          "cores": threads, "kind": "oracle",
                          "sample": sample},
@@ -321,7 +338,7 @@ def run_ours(args, w):
     pin = lambda t: None if t is None else t.pin_memory()  # noqa: E731
     hq, hk, hv, hb = pin(inp.q), pin(inp.k), pin(inp.v), pin(inp.beta)
     hla, hs0 = pin(inp.log_alpha), pin(inp.s0)
-    hcu = None if inp.cu_seqlens is None else inp.cu_seqlens
+    hcu = pin(inp.cu_seqlens)
     hout = torch.empty_like(inp.v).pin_memory()
     hsT = torch.empty(inp.nseq, w.H, w.dk, w.dv).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in
@@ -381,9 +398,9 @@ def run_ours(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H,
-                   "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "gate": w.gate,
-                   "global_batch": w.B * ws, "seq_len": w.T,
+        "config": {**workload_config(w, inp),
+                   "global_batch": inp.nseq * ws,
+                   "seq_len": None if w.varlen_nseq else w.T,
                    "parallelism": f"dp{ws} (independent sequences)",
                    "algo": algo_used,
                    "l2": "inputs larger than L2 (no flush)"},
@@ -446,8 +463,6 @@ def main(argv=None):
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
-    if w.varlen_nseq:
-        raise SystemExit("the benchmark times fixed-length workloads")
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -20,15 +20,15 @@
 // chunk n+1 is computed while the S-dependent chain of chunk n runs:
 //   warp 0      TMA producer: Q, K (two stages) and V tiles, 128-B swizzle
 //   warp 1      tensor-memory allocation and the single MMA-issuing thread
-//   warps 2..5  "state" warps: S -> bf16 operand and decay, V_new -> bf16
+//   warps 2..5  "state" warps: S -> fp16 operand and decay, V_new -> fp16
 //               operand, output tile -> global (thread = tensor-memory lane
 //               = one value channel)
 //   warps 6..13 "prep" warps (two per scheduler): gates, cumsum and per-row
 //               decay factors, A and P from K K^T / Q K^T, T = (I+A)^-1,
-//               T-factor operands, -W operand, in-place Q . e^g and
-//               K . e^{g_C - g}
+//               T-factor operands (bf16 hi + lo), -W operand, in-place
+//               Q . e^g and K . e^{g_C - g} (fp16)
 // All state lives in tensor memory as S^T (lane = value channel, column =
-// key channel) in fp32; bf16 is used only for tensor-core operands.
+// key channel) in fp32; fp16 / bf16 appear only as tensor-core operands.
 //
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [0,128) S^T   [128,256) V_new^T x2   [256,384) O^T x2
@@ -117,9 +117,9 @@ constexpr uint32_t ID_XO = idesc_f16kind(128, 64, false, false, false);
 constexpr uint32_t ID_SU = idesc_f16kind(128, 128, false, true, false);
 constexpr uint32_t ID_OI = idesc_f16kind(128, 64, false, false, false);
 
-// error word bits: 0..15 = the mbarrier whose wait expired; range errors
+// error word bits: 0..23 = the mbarrier whose wait expired; range errors
 constexpr unsigned kErrRange = 1u << 24;      // input beyond fp16 range
-constexpr unsigned kErrNonFinite = 1u << 25;  // non-finite final state
+constexpr unsigned kErrNonFinite = 1u << 25;  // non-finite output or state
 constexpr float kF16Max = 65504.f;
 
 constexpr long long kWaitCycles = 1ll << 32;   // ~2 s: a wait never lasts this
@@ -198,11 +198,9 @@ __device__ __forceinline__ int blk(int rb, int cb) {
   return rb * (rb + 1) / 2 + cb;
 }
 
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
+// tf32 operand: the fp32 bit pattern as is (the tensor core reads the top
+// 19 bits, i.e. truncates; a rounding cvt would cost an ALU op per operand)
+__device__ __forceinline__ uint32_t to_tf32(float x) { return __float_as_uint(x); }
 
 // acc (2 n-tiles of m16n8 C fragments) += X (16x16) * Z (16x16), both
 // row-major fp32 in shared memory, on mma.sync m16n8k8 tf32.
@@ -537,9 +535,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto store_output = [&](int m) {
       const int tok0 = start + m * kC, L = min(kC, end - tok0);
       uint8_t *stg = sm + OFF_VN;
+      float osum = 0.f;   // a non-finite output shows up in this sum
       for (int c0 = 0; c0 < kC; c0 += 32) {
         tmem_ld32(trow + ACC_O + (m & 1) * 64 + c0, v);
         tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) osum += (c0 + j < L) ? v[j] : 0.f;
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const float send = (l & 1) ? v[j] : v[j + 1];
@@ -551,6 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               pack_bf16(lo, hi);
         }
       }
+      if (!isfinite(osum)) atomicOr(&g_fused_error, kErrNonFinite);
       named_bar_sync(1, 128);
       for (int i = l; i < kC * 16; i += 128) {
         const int r = i >> 4, ch = i & 15;
@@ -782,8 +784,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int j = 4 * j4 + e, i = c0 + j;
-              const bool keep = arow ? (i < r) : (i <= r);
-              v[j] = keep ? v[j] * fi[e] * sc : 0.f;
+              // A rows are used below the diagonal only (the inverse never
+              // reads i >= r), so only the P rows need the causal mask
+              v[j] = (arow || i <= r) ? v[j] * fi[e] * sc : 0.f;
             }
           }
         }
@@ -978,10 +981,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 4; ++e) {
             float a0, a1;
             unpack_bf16(qw[e], a0, a1);
-            amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
             qw[e] = pack_f16(a0 * eq, a1 * eq);
             unpack_bf16(kw[e], a0, a1);
-            amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
             kw[e] = pack_f16(a0 * ek, a1 * ek);
           }
           *qp = qv;

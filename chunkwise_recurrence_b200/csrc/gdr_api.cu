@@ -99,10 +99,14 @@ gdr_status validate(const void *q, const void *k, const void *v,
 // Scratch allocation with a host-side failure hook: GDR_FAULT_INJECT_ALLOC=1
 // in the environment makes every scratch allocation fail before any CUDA
 // call (used by the failure-handling tests).
+bool alloc_fault_injected() {
+  const char *inj = std::getenv("GDR_FAULT_INJECT_ALLOC");
+  return inj && inj[0] == '1';
+}
+
 gdr_status scratch_alloc(void **ptr, size_t bytes, cudaStream_t s) {
   *ptr = nullptr;
-  const char *inj = std::getenv("GDR_FAULT_INJECT_ALLOC");
-  if (inj && inj[0] == '1') return GDR_ERR_OUT_OF_MEMORY;
+  if (alloc_fault_injected()) return GDR_ERR_OUT_OF_MEMORY;
   if (bytes == 0) return GDR_OK;
   cudaError_t e = cudaMallocAsync(ptr, bytes, s);
   if (e == cudaErrorMemoryAllocation) {
@@ -147,6 +151,88 @@ extern "C" gdr_status gdr_chunk_fwd(const void *q, const void *k,
   return run(p, o.algo, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Host-buffer entry.  The batch is cut into up to kHostPieces pieces of whole
+// sequences; each piece is an independent sub-problem with its own device
+// buffers.  Three streams overlap the pieces: the host-to-device copies of
+// piece i+1 (upload stream) run while piece i computes (the caller's stream)
+// and the results of piece i-1 come back (download stream), so the host link
+// carries both directions at once and the kernels hide behind the copies.
+namespace {
+
+constexpr int kHostPieces = 8;
+
+// Per-device resources of the host entry, created on first use and kept for
+// the life of the process: a memory pool that keeps its memory between calls
+// (repeated calls then reuse it instead of mapping and unmapping device
+// memory every time), and the two copy streams.
+struct HostCtx {
+  cudaMemPool_t pool = nullptr;
+  cudaStream_t up = nullptr, down = nullptr;
+};
+constexpr int kMaxHostDevices = 64;
+std::mutex g_host_mu;
+HostCtx g_host_ctx[kMaxHostDevices];
+
+gdr_status host_ctx(HostCtx *out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GDR_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxHostDevices) return GDR_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  HostCtx &c = g_host_ctx[dev];
+  if (!c.pool) {
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return GDR_ERR_CUDA;
+    uint64_t keep = UINT64_MAX;
+    cudaStream_t up = nullptr, down = nullptr;
+    if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold,
+                                &keep) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&up, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&down, cudaStreamNonBlocking) !=
+            cudaSuccess) {
+      if (up) cudaStreamDestroy(up);
+      cudaMemPoolDestroy(pool);
+      return GDR_ERR_CUDA;
+    }
+    c.pool = pool;
+    c.up = up;
+    c.down = down;
+  }
+  *out = c;
+  return GDR_OK;
+}
+
+// Token offsets of one piece, relative to its first sequence.
+__global__ void rebase_offsets_kernel(const int32_t *src, int32_t *dst,
+                                      int nseq) {
+  const int32_t base = src[0];
+  for (int j = threadIdx.x; j <= nseq; j += blockDim.x) dst[j] = src[j] - base;
+}
+
+// Events of one call, destroyed when the call returns (a destroyed event
+// that is still pending is released by the runtime once it completes).
+struct EventSet {
+  cudaEvent_t ev[2 * kHostPieces + 3] = {};
+  int n = 0;
+  cudaEvent_t make() {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+    ev[n++] = e;
+    return e;
+  }
+  ~EventSet() {
+    for (int i = 0; i < n; ++i) cudaEventDestroy(ev[i]);
+  }
+};
+
+}  // namespace
+
 extern "C" gdr_status gdr_chunk_fwd_host(const void *q, const void *k,
                                          const void *v, const float *log_alpha,
                                          const float *beta,
@@ -162,76 +248,171 @@ extern "C" gdr_status gdr_chunk_fwd_host(const void *q, const void *k,
   if (st != GDR_OK) return st;
   if (p.nseq == 0 || p.H == 0) return GDR_OK;
 
+  // host offsets are read here, so that every piece is exact
+  const bool varlen = o.cu_seqlens != nullptr;
+  const int32_t *hcu = o.cu_seqlens;
+  if (varlen) {
+    if (hcu[0] != 0 || hcu[p.nseq] != p.ntok) return GDR_ERR_INVALID_ARGUMENT;
+    for (int n = 0; n < p.nseq; ++n)
+      if (hcu[n + 1] < hcu[n]) return GDR_ERR_INVALID_ARGUMENT;
+  }
+  auto first_token = [&](int n) -> long long {
+    return varlen ? hcu[n] : (long long)n * p.T;
+  };
+
+  // pieces: sequence boundaries sb[], about ntok / P tokens each, at least
+  // one sequence each
+  const int P = p.nseq < kHostPieces ? p.nseq : kHostPieces;
+  int sb[kHostPieces + 1];
+  sb[0] = 0;
+  sb[P] = p.nseq;
+  for (int i = 1; i < P; ++i) {
+    const long long target = (long long)p.ntok * i / P;
+    int n = sb[i - 1] + 1;
+    while (n < p.nseq - (P - i) && first_token(n) < target) ++n;
+    sb[i] = n;
+  }
+
+  // device layout: the caller's offsets (varlen), then per piece its inputs
+  // and outputs, every buffer 256-byte aligned
   const size_t esz = o.dtype == GDR_FP32 ? 4 : 2;
-  const size_t th = (size_t)p.ntok * p.H;
   const size_t gdim = o.gate == GDR_GATE_NONE     ? 0
                       : o.gate == GDR_GATE_SCALAR ? 1
                                                   : (size_t)dk;
-  const size_t state = (size_t)p.nseq * H * dk * dv * sizeof(float);
-  struct Buf {
-    const void *host;
-    void *dev;
-    size_t bytes;
-    bool in, out;
-  } bufs[] = {
-      {q, nullptr, th * dk * esz, true, false},
-      {k, nullptr, th * dk * esz, true, false},
-      {v, nullptr, th * dv * esz, true, false},
-      {log_alpha, nullptr, log_alpha ? th * gdim * sizeof(float) : 0, true,
-       false},
-      {beta, nullptr, th * sizeof(float), true, false},
-      {initial_state, nullptr, initial_state ? state : 0, true, false},
-      {o.cu_seqlens, nullptr,
-       o.cu_seqlens ? ((size_t)p.nseq + 1) * sizeof(int32_t) : 0, true,
-       false},
-      {out, nullptr, th * dv * esz, false, true},
-      {final_state, nullptr, final_state ? state : 0, false, true},
-  };
-  const int nb = sizeof(bufs) / sizeof(bufs[0]);
-  size_t total = 0, offs[nb];
-  for (int i = 0; i < nb; ++i) {
-    offs[i] = total;
-    total += (bufs[i].bytes + 255) & ~size_t(255);
+  const size_t state1 = (size_t)H * dk * dv * sizeof(float);
+  // per-token bytes of each tensor, in the order q k v log_alpha beta out
+  const size_t tok_bytes[6] = {
+      (size_t)H * dk * esz, (size_t)H * dk * esz, (size_t)H * dv * esz,
+      log_alpha ? (size_t)H * gdim * sizeof(float) : 0,
+      (size_t)H * sizeof(float), (size_t)H * dv * esz};
+  const void *host_in[5] = {q, k, v, log_alpha, beta};
+  auto up256 = [](size_t x) { return (x + 255) & ~size_t(255); };
+  enum { BQ, BK, BV, BLA, BB, BOUT, BS0, BST, BCU, NBUF };
+  size_t off[kHostPieces][NBUF];
+  size_t total = varlen ? up256(((size_t)p.nseq + 1) * sizeof(int32_t)) : 0;
+  for (int i = 0; i < P; ++i) {
+    const size_t nt = first_token(sb[i + 1]) - first_token(sb[i]);
+    const size_t ns = sb[i + 1] - sb[i];
+    const size_t bytes[NBUF] = {
+        nt * tok_bytes[0], nt * tok_bytes[1], nt * tok_bytes[2],
+        nt * tok_bytes[3], nt * tok_bytes[4], nt * tok_bytes[5],
+        initial_state ? ns * state1 : 0, final_state ? ns * state1 : 0,
+        varlen ? (ns + 1) * sizeof(int32_t) : 0};
+    for (int b = 0; b < NBUF; ++b) {
+      off[i][b] = total;
+      total += up256(bytes[b]);
+    }
   }
-  void *block = nullptr;
-  st = scratch_alloc(&block, total, stream);
+
+  if (alloc_fault_injected()) return GDR_ERR_OUT_OF_MEMORY;
+  HostCtx hc;
+  st = host_ctx(&hc);
   if (st != GDR_OK) return st;
+  EventSet evs;
+  cudaEvent_t ev_start = evs.make(), ev_up_end = evs.make(),
+              ev_down_end = evs.make();
+  cudaEvent_t ev_in[kHostPieces], ev_run[kHostPieces];
+  for (int i = 0; i < P; ++i) {
+    ev_in[i] = evs.make();
+    ev_run[i] = evs.make();
+  }
+  if (evs.n != 3 + 2 * P) return GDR_ERR_CUDA;
+  void *block = nullptr;
+  {
+    cudaError_t e = cudaMallocFromPoolAsync(&block, total, hc.pool, stream);
+    if (e == cudaErrorMemoryAllocation) {
+      (void)cudaGetLastError();
+      return GDR_ERR_OUT_OF_MEMORY;
+    }
+    if (e != cudaSuccess) return GDR_ERR_CUDA;
+  }
   char *base = static_cast<char *>(block);
-  for (int i = 0; i < nb; ++i) {
-    if (!bufs[i].host || bufs[i].bytes == 0) continue;
-    bufs[i].dev = base + offs[i];
-    if (bufs[i].in &&
-        cudaMemcpyAsync(bufs[i].dev, bufs[i].host, bufs[i].bytes,
-                        cudaMemcpyHostToDevice, stream) != cudaSuccess) {
-      cudaFreeAsync(block, stream);
-      return GDR_ERR_CUDA;
+  auto ok = [&](cudaError_t e) {
+    if (e != cudaSuccess && st == GDR_OK) st = GDR_ERR_CUDA;
+    return st == GDR_OK;
+  };
+
+  // the upload stream starts after the caller's earlier work (and the
+  // allocation) on `stream`
+  ok(cudaEventRecord(ev_start, stream));
+  ok(cudaStreamWaitEvent(hc.up, ev_start, 0));
+  if (varlen)
+    ok(cudaMemcpyAsync(base, hcu, ((size_t)p.nseq + 1) * sizeof(int32_t),
+                       cudaMemcpyHostToDevice, hc.up));
+  for (int i = 0; i < P && st == GDR_OK; ++i) {
+    const long long t0 = first_token(sb[i]), t1 = first_token(sb[i + 1]);
+    const int s0 = sb[i], ns = sb[i + 1] - sb[i];
+    char *pb[NBUF];
+    for (int b = 0; b < NBUF; ++b) pb[b] = base + off[i][b];
+    // inputs of piece i
+    for (int b = BQ; b <= BB; ++b)
+      if (host_in[b] && tok_bytes[b])
+        ok(cudaMemcpyAsync(pb[b],
+                           static_cast<const char *>(host_in[b]) +
+                               t0 * tok_bytes[b],
+                           (t1 - t0) * tok_bytes[b], cudaMemcpyHostToDevice,
+                           hc.up));
+    if (initial_state)
+      ok(cudaMemcpyAsync(pb[BS0],
+                         reinterpret_cast<const char *>(initial_state) +
+                             s0 * state1,
+                         ns * state1, cudaMemcpyHostToDevice, hc.up));
+    ok(cudaEventRecord(ev_in[i], hc.up));
+    if (st != GDR_OK) break;
+    // compute on the caller's stream
+    ok(cudaStreamWaitEvent(stream, ev_in[i], 0));
+    Problem pp = p;
+    pp.q = pb[BQ];
+    pp.k = pb[BK];
+    pp.v = pb[BV];
+    pp.log_alpha = log_alpha ? reinterpret_cast<const float *>(pb[BLA])
+                             : nullptr;
+    pp.beta = reinterpret_cast<const float *>(pb[BB]);
+    pp.s0 = initial_state ? reinterpret_cast<const float *>(pb[BS0]) : nullptr;
+    pp.out = pb[BOUT];
+    pp.sT = final_state ? reinterpret_cast<float *>(pb[BST]) : nullptr;
+    pp.nseq = ns;
+    pp.ntok = (int)(t1 - t0);
+    if (varlen) {
+      int32_t *cu = reinterpret_cast<int32_t *>(pb[BCU]);
+      rebase_offsets_kernel<<<1, 256, 0, stream>>>(
+          reinterpret_cast<const int32_t *>(base) + s0, cu, ns);
+      if (!ok(cudaGetLastError())) break;
+      pp.cu = cu;
+      pp.T = pp.ntok;
+      pp.max_chunks = pp.ntok / p.chunk + ns;
+    } else {
+      pp.cu = nullptr;
+      pp.max_chunks = ns * ((p.T + p.chunk - 1) / p.chunk);
     }
-  }
-  Problem pd = p;
-  pd.q = bufs[0].dev;
-  pd.k = bufs[1].dev;
-  pd.v = bufs[2].dev;
-  pd.log_alpha = static_cast<const float *>(bufs[3].dev);
-  pd.beta = static_cast<const float *>(bufs[4].dev);
-  pd.s0 = static_cast<const float *>(bufs[5].dev);
-  pd.cu = static_cast<const int32_t *>(bufs[6].dev);
-  pd.out = bufs[7].dev;
-  pd.sT = static_cast<float *>(bufs[8].dev);
-  st = run(pd, o.algo, stream);
-  if (st == GDR_OK) {
-    for (int i = 0; i < nb; ++i) {
-      if (!bufs[i].out || !bufs[i].dev) continue;
-      if (cudaMemcpyAsync(const_cast<void *>(bufs[i].host), bufs[i].dev,
-                          bufs[i].bytes, cudaMemcpyDeviceToHost,
-                          stream) != cudaSuccess) {
-        st = GDR_ERR_CUDA;
-        break;
-      }
+    const gdr_status rs = run(pp, o.algo, stream);
+    if (rs != GDR_OK) {
+      st = rs;
+      break;
     }
+    ok(cudaEventRecord(ev_run[i], stream));
+    // results of piece i
+    ok(cudaStreamWaitEvent(hc.down, ev_run[i], 0));
+    ok(cudaMemcpyAsync(static_cast<char *>(out) + t0 * tok_bytes[BOUT],
+                       pb[BOUT], (t1 - t0) * tok_bytes[BOUT],
+                       cudaMemcpyDeviceToHost, hc.down));
+    if (final_state)
+      ok(cudaMemcpyAsync(reinterpret_cast<char *>(final_state) + s0 * state1,
+                         pb[BST], ns * state1, cudaMemcpyDeviceToHost,
+                         hc.down));
   }
-  if (cudaFreeAsync(block, stream) != cudaSuccess && st == GDR_OK)
-    st = GDR_ERR_CUDA;
-  return st;
+  // the caller's stream waits for both copy streams, then releases the
+  // block; this runs on every path once the allocation has succeeded
+  gdr_status fin = GDR_OK;
+  auto fin_ok = [&](cudaError_t e) {
+    if (e != cudaSuccess) fin = GDR_ERR_CUDA;
+  };
+  fin_ok(cudaEventRecord(ev_up_end, hc.up));
+  fin_ok(cudaEventRecord(ev_down_end, hc.down));
+  fin_ok(cudaStreamWaitEvent(stream, ev_up_end, 0));
+  fin_ok(cudaStreamWaitEvent(stream, ev_down_end, 0));
+  fin_ok(cudaFreeAsync(block, stream));
+  return st != GDR_OK ? st : fin;
 }
 
 // ---------------------------------------------------------------------------
@@ -292,7 +473,7 @@ extern "C" gdr_status gdr_device_error(cudaStream_t stream, int clear) {
   unsigned word = 0;
   if (gdr::fused_tc_read_error(&word, clear != 0) != cudaSuccess)
     return GDR_ERR_CUDA;
-  if (word & 0xFFFFu) return GDR_ERR_TIMEOUT;   // an mbarrier wait expired
+  if (word & 0xFFFFFFu) return GDR_ERR_TIMEOUT;  // an mbarrier wait expired
   return word ? GDR_ERR_RANGE : GDR_OK;
 }
 

@@ -66,9 +66,9 @@ typedef enum {
   GDR_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed      */
   GDR_ERR_OUT_OF_MEMORY = 4,    /* scratch allocation failed                 */
   GDR_ERR_TIMEOUT = 5,          /* a bounded device-side wait expired        */
-  GDR_ERR_RANGE = 6             /* an input (or the final state) fell outside
-                                   the fused path's fp16 operand range; the
-                                   STAGED path has no such limit             */
+  GDR_ERR_RANGE = 6             /* a value fell outside the fused path's fp16
+                                   operand range (non-finite output/state);
+                                   the STAGED path has no such limit         */
 } gdr_status;
 
 /* Element type of q, k, v and out.  beta, log_alpha and the states are always
@@ -95,10 +95,11 @@ typedef enum {
    * chunk after chunk with every intermediate on chip; chunk products on
    * tcgen05 tensor cores: fp16 operands (inputs converted on chip), fp32
    * accumulation in tensor memory, fp32 state.  bf16 I/O, dk = dv = 128,
-   * chunk = 64.  Inputs must lie within fp16 range (|x| <= 65504); for the
-   * channel gate, each key channel's log-decay must move by at most ~88
-   * between a chunk's row 31 and its first or last row.  Violations are
-   * reported by gdr_device_error as GDR_ERR_RANGE. */
+   * chunk = 64.  Inputs and on-chip intermediates must lie within fp16
+   * range (|x| <= 65504); for the channel gate, each key channel's
+   * log-decay must move by at most ~88 between a chunk's row 31 and its
+   * first or last row.  A violation shows as a non-finite output or state
+   * and is reported by gdr_device_error as GDR_ERR_RANGE. */
   GDR_ALGO_FUSED_TC = 2
 } gdr_algo;
 
@@ -151,10 +152,21 @@ GDR_API gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v,
  * gdr_chunk_fwd_host -- the same computation on HOST buffers.
  *
  * Every tensor pointer (and opts->cu_seqlens) is a host pointer with the
- * layouts above.  The call allocates device buffers stream-ordered, enqueues
- * one host-to-device copy per input, the computation, one device-to-host copy
- * per output and the release of the device buffers, all on `stream`, and
- * returns.  Host buffers must stay valid until `stream` is synchronised.  With
+ * layouts above; with cu_seqlens the offsets are checked on the host (first
+ * 0, non-decreasing, last T), else GDR_ERR_INVALID_ARGUMENT.
+ *
+ * The batch is cut into up to 8 pieces of whole sequences, each computed as
+ * an independent sub-problem.  The call enqueues, and returns without
+ * waiting: per piece, the host-to-device copies of its inputs on an upload
+ * stream, its computation on `stream`, and the device-to-host copies of its
+ * results on a download stream, so that the copies of neighbouring pieces
+ * overlap each other and the computation; then `stream` waits for both copy
+ * streams and the device buffers are released.  Work enqueued on `stream`
+ * after the call sees every result.  The upload and download streams are
+ * created per device on first use and kept, as is a device memory pool that
+ * holds the largest call's buffers between calls.
+ *
+ * Host buffers must stay valid until `stream` is synchronised.  With
  * page-locked (pinned) host memory the copies are asynchronous; with pageable
  * memory the CUDA runtime makes them synchronous to the host.
  */
@@ -210,8 +222,10 @@ GDR_API gdr_status gdr_chunk_fwd_noalloc(const void *q, const void *k,
  * gdr_device_error -- synchronise `stream`, then read (and clear if `clear`)
  * the library's sticky device-side error word for the current device.
  * Returns GDR_OK if no kernel has reported an error, GDR_ERR_TIMEOUT if a
- * bounded wait expired, GDR_ERR_RANGE if the fused kernel met an input of
- * magnitude above 65504 (or NaN) or produced a non-finite final state,
+ * bounded wait expired, GDR_ERR_RANGE if the fused kernel produced a
+ * non-finite output or final state (an input or intermediate beyond the
+ * fp16 operand range, |x| > 65504, or a NaN input) or, for the channel gate,
+ * met such an input,
  * GDR_ERR_CUDA if synchronisation itself failed.
  */
 GDR_API gdr_status gdr_device_error(cudaStream_t stream, int clear);

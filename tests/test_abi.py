@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import chunkwise_recurrence_b200 as gdr
@@ -80,6 +81,19 @@ def test_rejects_bad_arguments(lib, host):
     assert c(nseq=3) == INVALID                    # num_seqs without cu
     assert c(B=1 << 20, T=1 << 12) == UNSUPPORTED  # too many tokens
     assert c(H=70000) == UNSUPPORTED
+
+
+@pytest.mark.parametrize("cu", [[1, 10, 64], [0, 40, 30, 64], [0, 10, 63],
+                                [0, 10, 65]])
+def test_host_entry_checks_sequence_offsets(lib, cu):
+    # the host entry reads cu_seqlens on the host: first 0, non-decreasing,
+    # last T; the tensor pointers are never touched on rejection
+    arr = np.zeros(len(cu) + 4, dtype=np.int32)
+    base = (-arr.ctypes.data // 4) % 4          # a 16-byte-aligned start
+    view = arr[base:base + len(cu)]
+    view[:] = cu
+    assert call(lib, host=True, cu=view.ctypes.data, nseq=len(cu) - 1,
+                T=64) == INVALID
 
 
 @pytest.mark.parametrize("host", [False, True])

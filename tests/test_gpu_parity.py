@@ -200,6 +200,55 @@ def test_host_entry_matches_device_entry():
         assert np.array_equal(sT.numpy(), s)
 
 
+def run_host(inp, algo, final_state=True):
+    """The host-buffer entry on pinned copies of the inputs."""
+    pin = lambda t: None if t is None else t.pin_memory()  # noqa: E731
+    out = torch.empty_like(inp.v).pin_memory()
+    sT = (torch.full((inp.nseq, inp.w.H, inp.w.dk, inp.w.dv), 7.0).pin_memory()
+          if final_state else None)
+    gdr.chunk_fwd_host(pin(inp.q), pin(inp.k), pin(inp.v), pin(inp.beta),
+                       pin(inp.log_alpha), pin(inp.s0), out=out,
+                       final_state=sT, chunk=inp.w.chunk, gate=inp.w.gate,
+                       cu_seqlens=pin(inp.cu_seqlens), algo=algo)
+    torch.cuda.synchronize()
+    assert gdr.device_error() == 0
+    return out.float().numpy(), None if sT is None else sT.numpy()
+
+
+def test_host_entry_pieces_varlen():
+    # 11 sequences, four of them empty: the host entry cuts them into 8
+    # pieces of uneven size, each computed as its own sub-problem; the result
+    # is the device entry's, bit for bit
+    lens = [0, 70, 0, 1, 130, 0, 64, 200, 5, 0, 90]
+    w = WORKLOADS["gdn_varlen8_h16_d128_bf16"].with_(
+        B=1, T=sum(lens), H=2, varlen_nseq=0, init_state=False)
+    inp = generate(w, seed=21)
+    cu = torch.zeros(len(lens) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lens), 0).to(torch.int32)
+    g = torch.Generator().manual_seed(22)
+    inp = dataclasses.replace(
+        inp, w=inp.w.with_(varlen_nseq=len(lens)), cu_seqlens=cu,
+        lengths=lens,
+        s0=torch.randn(len(lens), 2, 128, 128, generator=g) * 0.02)
+    for algo in algos_for(inp.w):
+        o, s = run_gpu(inp, algo)
+        ho, hs = run_host(inp, algo)
+        assert np.array_equal(ho, o) and np.array_equal(hs, s)
+
+
+def test_host_entry_pieces_fixed_length():
+    # 10 sequences -> 8 pieces (two of two sequences); no initial state, and
+    # no final state requested
+    w = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(B=10, T=100, H=3)
+    inp = generate(w, seed=23)
+    for algo in algos_for(w):
+        o, _ = run_gpu(inp, algo)
+        ho, hs = run_host(inp, algo, final_state=False)
+        assert hs is None and np.array_equal(ho, o)
+        ro, _ = run_oracle(inp)
+        assert out_err(ho, ro, "bf16") <= 2e-2
+
+
 def test_deterministic():
     w = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=2, T=200, H=2)
     inp = generate(w, seed=11)
