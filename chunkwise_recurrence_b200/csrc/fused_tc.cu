@@ -63,10 +63,9 @@ constexpr int kPrep = 256;     // prep threads (warps 6..13)
 constexpr uint32_t kStageBytes = 32768;
 constexpr uint32_t OFF_STAGE = 0;                        // 2 stages
 constexpr uint32_t OFF_V = OFF_STAGE + 2 * kStageBytes;  // [2][64][64] bf16
-constexpr uint32_t OFF_ST = OFF_V + 16384;               // S^T [2][128][64]
-constexpr uint32_t OFF_NW = OFF_ST + 32768;              // -W^T [128][64]
-constexpr uint32_t OFF_VN = OFF_NW + 16384;              // V_new^T [128][64]
-constexpr uint32_t OFF_P = OFF_VN + 16384;               // P [2][64][64]
+constexpr uint32_t OFF_NW = OFF_V + 16384;               // -W^T [128][64]
+constexpr uint32_t OFF_OS = OFF_NW + 16384;              // output staging
+constexpr uint32_t OFF_P = OFF_OS + 16384;               // P [2][64][64]
 constexpr uint32_t OFF_TP = OFF_P + 16384;               // T-factor tiles
 template <int GATE>
 struct Layout {
@@ -361,8 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t st = smem_u32(sm + OFF_ST), nw = smem_u32(sm + OFF_NW),
-                     vn = smem_u32(sm + OFF_VN), vt = smem_u32(sm + OFF_V),
+      const uint32_t nw = smem_u32(sm + OFF_NW), vt = smem_u32(sm + OFF_V),
                      tp = smem_u32(sm + OFF_TP),
                      kn = smem_u32(sm + Lay::KN);
       auto stage = [&](int m) {
@@ -461,20 +459,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_bar(cx, B_SREADY, m & 1) || !wait_bar(cx, B_WREADY, m & 1))
           break;
         tc_fence_after();
+        // A = S^T, fp16 pairs in tensor memory (8 columns per K step)
+        const uint32_t st_op = tmem + ACC_V + ((m + 1) & 1) * 64;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_f16kind(tmem + ACC_V + (m & 1) * 64,
-                   sdesc_sw128(st + (ks >> 2) * 16384 + (ks & 3) * 32, 16,
-                               1024),
-                   sdesc_sw128(nw + ks * 2048, 8192, 1024), ID_XV, 1);
+          mma_f16kind_ts(tmem + ACC_V + (m & 1) * 64, st_op + 8 * ks,
+                         sdesc_sw128(nw + ks * 2048, 8192, 1024), ID_XV, 1);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_f16kind(tmem + ACC_O + (m & 1) * 64,
-                   sdesc_sw128(st + (ks >> 2) * 16384 + (ks & 3) * 32, 16,
-                               1024),
-                   sdesc_sw128(base + 8192 + (ks >> 2) * 16384 + (ks & 3) * 32,
-                               16, 1024),
-                   ID_XO, ks > 0);
+          mma_f16kind_ts(tmem + ACC_O + (m & 1) * 64, st_op + 8 * ks,
+                         sdesc_sw128(base + 8192 + (ks >> 2) * 16384 +
+                                         (ks & 3) * 32,
+                                     16, 1024),
+                         ID_XO, ks > 0);
         mma_commit(&bar[B_XDONE]);
         // K K^T of chunk m+1 while the state warps turn V_new into an operand
         if (m + 1 < NC && kk_next == m + 1) {
@@ -486,17 +483,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         // S update and intra-chunk output
         if (!wait_bar(cx, B_VNREADY, m & 1)) break;
         tc_fence_after();
+        // A = V_new^T, fp16 pairs in tensor memory
+        const uint32_t vn_op = tmem + ACC_V + (m & 1) * 64;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_f16kind(tmem + ACC_S, sdesc_sw128(vn + ks * 32, 16, 1024),
-                   sdesc_sw128(base + ks * 2048, 16384, 1024), ID_SU, 1);
-        mma_commit(&bar[B_SDONE]);
+          mma_f16kind_ts(tmem + ACC_S, vn_op + 8 * ks,
+                         sdesc_sw128(base + ks * 2048, 16384, 1024), ID_SU, 1);
         const uint32_t pt = smem_u32(sm + OFF_P + (m & 1) * 8192);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_f16kind(tmem + ACC_O + (m & 1) * 64,
-                   sdesc_sw128(vn + ks * 32, 16, 1024),
-                   sdesc_sw128(pt + ks * 32, 16, 1024), ID_OI, 1);
+          mma_f16kind_ts(tmem + ACC_O + (m & 1) * 64, vn_op + 8 * ks,
+                         sdesc_sw128(pt + ks * 32, 16, 1024), ID_OI, 1);
+        // S done also covers the intra-chunk output: both read V_new(m),
+        // whose columns S^T(m+1) reuses
+        mma_commit(&bar[B_SDONE]);
         mma_commit(&bar[B_ODONE]);
         mma_commit(&bar[B_EMPTY0 + (m & 1)]);
         // U, W of chunk m+1
@@ -529,12 +529,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_wait_st();
     bool ok = true;
     // O^T of chunk m (lane = value channel, column = row) -> out rows, via
-    // a [64 rows][128 channels] bf16 staging tile in the V_new^T tile, which
-    // is free between O(m) done and the V_new^T write of chunk m+1.
+    // a [64 rows][128 channels] bf16 staging tile in shared memory.
     // Neighbouring lanes swap values so each writes two adjacent channels.
     auto store_output = [&](int m) {
       const int tok0 = start + m * kC, L = min(kC, end - tok0);
-      uint8_t *stg = sm + OFF_VN;
+      uint8_t *stg = sm + OFF_OS;
       float osum = 0.f;   // a non-finite output shows up in this sum
       for (int c0 = 0; c0 < kC; c0 += 32) {
         tmem_ld32(trow + ACC_O + (m & 1) * 64 + c0, v);
@@ -566,24 +565,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     float *gC = reinterpret_cast<float *>(sm + Lay::GC);
     for (int m = 0; m < NC; ++m) {
-      // S (chunk start) -> bf16 operand; decayed S back to tensor memory
+      // S (chunk start) -> fp16 operand; decayed S back to tensor memory
       if (m > 0 && !(ok = group_all(wait_bar(cx, B_SDONE, (m - 1) & 1), 1, 128)))
         break;
       if (!(ok = group_all(wait_bar(cx, B_TREADY, m & 1), 1, 128))) break;
       tc_fence_after();
       const float *gcm = gC + (m & 1) * 128;
       const float dscal = GATE == 1 ? __expf(gcm[0]) : 1.f;
+      // S^T as fp16 pairs (key channels 2j, 2j+1 in column j) into the
+      // V_new^T region of the other chunk parity, free from S done(m-1)
+      // (whose commit follows the last reader of V_new(m-1)) until U(m+1)
+      const uint32_t st_op = trow + ACC_V + ((m + 1) & 1) * 64;
       for (int c0 = 0; c0 < kD; c0 += 32) {
         tmem_ld32(trow + ACC_S + c0, v);
         tmem_wait_ld();
-        uint8_t *dst = sm + OFF_ST + (c0 >> 6) * 16384;
+        uint32_t pk[16];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-          st_smem_v4(dst + sw128_chunk(l, ((c0 & 63) >> 3) + ch),
-                     pack_f16(v[8 * ch + 0], v[8 * ch + 1]),
-                     pack_f16(v[8 * ch + 2], v[8 * ch + 3]),
-                     pack_f16(v[8 * ch + 4], v[8 * ch + 5]),
-                     pack_f16(v[8 * ch + 6], v[8 * ch + 7]));
+        for (int j = 0; j < 16; ++j) pk[j] = pack_f16(v[2 * j], v[2 * j + 1]);
+        tmem_st16(st_op + (c0 >> 1), pk);
         if (GATE != 0) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -591,8 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(trow + ACC_S + c0, v);
         }
       }
-      if (GATE != 0) tmem_wait_st();
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar[B_SREADY]);
       // output of the previous chunk while X(m) runs
@@ -601,21 +599,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         store_output(m - 1);
       }
-      // V_new^T -> fp16 operand
+      // V_new^T -> fp16 pairs (tokens 2j, 2j+1 in column j) in place, in
+      // the first 32 columns of its own region
       if (!(ok = group_all(wait_bar(cx, B_XDONE, m & 1), 1, 128))) break;
       tc_fence_after();
-      for (int c0 = 0; c0 < kC; c0 += 32) {
-        tmem_ld32(trow + ACC_V + (m & 1) * 64 + c0, v);
+      {
+        // both halves are loaded before the first store overwrites
+        // columns 0..15
+        const uint32_t vreg = trow + ACC_V + (m & 1) * 64;
+        uint32_t pk[16];
+        tmem_ld32(vreg, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-          st_smem_v4(sm + OFF_VN + sw128_chunk(l, (c0 >> 3) + ch),
-                     pack_f16(v[8 * ch + 0], v[8 * ch + 1]),
-                     pack_f16(v[8 * ch + 2], v[8 * ch + 3]),
-                     pack_f16(v[8 * ch + 4], v[8 * ch + 5]),
-                     pack_f16(v[8 * ch + 6], v[8 * ch + 7]));
+        for (int j = 0; j < 16; ++j) pk[j] = pack_f16(v[2 * j], v[2 * j + 1]);
+        tmem_ld32(vreg + 32, v);
+        tmem_wait_ld();
+        tmem_st16(vreg, pk);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pk[j] = pack_f16(v[2 * j], v[2 * j + 1]);
+        tmem_st16(vreg + 16, pk);
+        tmem_wait_st();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bar[B_VNREADY]);
     }
