@@ -55,6 +55,12 @@ constexpr int kC = 64;         // chunk length
 constexpr int kD = 128;        // dk = dv
 constexpr int kThreads = 448;  // 14 warps
 constexpr int kPrep = 256;     // prep threads (warps 6..13)
+// fp32 16x16 blocks: rows kRS floats apart, blocks kBS floats apart.  The
+// padding spreads eight consecutive rows (16-byte accesses) and the tf32
+// fragment rows over distinct banks, and puts neighbouring blocks on
+// opposite bank halves.
+constexpr int kRS = 20;
+constexpr int kBS = 16 * kRS + 16;
 
 // ---- shared memory layout (bytes from a 1024-aligned base) ----------------
 // A stage holds one chunk's K and Q as four 8 KB [64 rows][64 cols] blocks:
@@ -77,10 +83,9 @@ struct Layout {
                             TPB_HI = OFF_TP + 16384, TPB_LO = OFF_TP + 24576;
   static constexpr uint32_t KN = OFF_TP + TP_BYTES;
   static constexpr uint32_t KN_BYTES = (GATE == 2) ? 16384 : 0;
-  static constexpr uint32_t AC = KN + KN_BYTES;   // A blocks fp32 [10][16][16]
-  static constexpr uint32_t TC = AC + 10240;      // T blocks fp32 [10][16][16]
-  static constexpr uint32_t YS = TC + 10240;      // per-warp 16x16 scratch x4
-  static constexpr uint32_t GS = YS + 4096;       // g [2][64]
+  static constexpr uint32_t AC = KN + KN_BYTES;   // A blocks fp32 [10][kBS]
+  static constexpr uint32_t TC = AC + 40 * kBS;   // T blocks fp32 [10][kBS]
+  static constexpr uint32_t GS = TC + 40 * kBS;   // g [2][64]
   static constexpr uint32_t FT = GS + 512;        // row factors [2][6][64]
   static constexpr uint32_t GC = FT + 3072;       // g_C [2][128]
   static constexpr uint32_t GM = GC + 1024;       // g at row 31 [128] (KDA)
@@ -208,14 +213,14 @@ __device__ __forceinline__ void mma16(const float *X, const float *Z,
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int ks = 0; ks < 2; ++ks) {
-    const uint32_t a0 = to_tf32(X[g * 16 + 8 * ks + t]);
-    const uint32_t a1 = to_tf32(X[(g + 8) * 16 + 8 * ks + t]);
-    const uint32_t a2 = to_tf32(X[g * 16 + 8 * ks + t + 4]);
-    const uint32_t a3 = to_tf32(X[(g + 8) * 16 + 8 * ks + t + 4]);
+    const uint32_t a0 = to_tf32(X[g * kRS + 8 * ks + t]);
+    const uint32_t a1 = to_tf32(X[(g + 8) * kRS + 8 * ks + t]);
+    const uint32_t a2 = to_tf32(X[g * kRS + 8 * ks + t + 4]);
+    const uint32_t a3 = to_tf32(X[(g + 8) * kRS + 8 * ks + t + 4]);
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-      const uint32_t b0 = to_tf32(Z[(8 * ks + t) * 16 + 8 * nt + g]);
-      const uint32_t b1 = to_tf32(Z[(8 * ks + t + 4) * 16 + 8 * nt + g]);
+      const uint32_t b0 = to_tf32(Z[(8 * ks + t) * kRS + 8 * nt + g]);
+      const uint32_t b1 = to_tf32(Z[(8 * ks + t + 4) * kRS + 8 * nt + g]);
       float *c = acc + 4 * nt;
       asm volatile(
           "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
@@ -233,12 +238,12 @@ __device__ __forceinline__ void mma16_nt(const float *X, const float *Z,
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int ks = 0; ks < 2; ++ks) {
-    const uint32_t a0 = to_tf32(X[g * 16 + 8 * ks + t]);
-    const uint32_t a1 = to_tf32(X[(g + 8) * 16 + 8 * ks + t]);
-    const uint32_t a2 = to_tf32(X[g * 16 + 8 * ks + t + 4]);
-    const uint32_t a3 = to_tf32(X[(g + 8) * 16 + 8 * ks + t + 4]);
-    const uint32_t b0 = to_tf32(Z[(8 * ks + t) * 16 + 8 * nt + g]);
-    const uint32_t b1 = to_tf32(Z[(8 * ks + t + 4) * 16 + 8 * nt + g]);
+    const uint32_t a0 = to_tf32(X[g * kRS + 8 * ks + t]);
+    const uint32_t a1 = to_tf32(X[(g + 8) * kRS + 8 * ks + t]);
+    const uint32_t a2 = to_tf32(X[g * kRS + 8 * ks + t + 4]);
+    const uint32_t a3 = to_tf32(X[(g + 8) * kRS + 8 * ks + t + 4]);
+    const uint32_t b0 = to_tf32(Z[(8 * ks + t) * kRS + 8 * nt + g]);
+    const uint32_t b1 = to_tf32(Z[(8 * ks + t + 4) * kRS + 8 * nt + g]);
     asm volatile(
         "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
         "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
@@ -250,10 +255,10 @@ __device__ __forceinline__ void mma16_nt(const float *X, const float *Z,
 __device__ __forceinline__ void store16_nt(float *Y, const float acc[4],
                                            float s, int lane, int nt) {
   const int g = lane >> 2, t = lane & 3;
-  Y[g * 16 + 8 * nt + 2 * t] = s * acc[0];
-  Y[g * 16 + 8 * nt + 2 * t + 1] = s * acc[1];
-  Y[(g + 8) * 16 + 8 * nt + 2 * t] = s * acc[2];
-  Y[(g + 8) * 16 + 8 * nt + 2 * t + 1] = s * acc[3];
+  Y[g * kRS + 8 * nt + 2 * t] = s * acc[0];
+  Y[g * kRS + 8 * nt + 2 * t + 1] = s * acc[1];
+  Y[(g + 8) * kRS + 8 * nt + 2 * t] = s * acc[2];
+  Y[(g + 8) * kRS + 8 * nt + 2 * t + 1] = s * acc[3];
 }
 
 // store C fragments (scaled by s) to a row-major 16x16 fp32 block
@@ -262,10 +267,10 @@ __device__ __forceinline__ void store16(float *Y, const float acc[8], float s,
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
-    Y[g * 16 + 8 * nt + 2 * t] = s * acc[4 * nt + 0];
-    Y[g * 16 + 8 * nt + 2 * t + 1] = s * acc[4 * nt + 1];
-    Y[(g + 8) * 16 + 8 * nt + 2 * t] = s * acc[4 * nt + 2];
-    Y[(g + 8) * 16 + 8 * nt + 2 * t + 1] = s * acc[4 * nt + 3];
+    Y[g * kRS + 8 * nt + 2 * t] = s * acc[4 * nt + 0];
+    Y[g * kRS + 8 * nt + 2 * t + 1] = s * acc[4 * nt + 1];
+    Y[(g + 8) * kRS + 8 * nt + 2 * t] = s * acc[4 * nt + 2];
+    Y[(g + 8) * kRS + 8 * nt + 2 * t + 1] = s * acc[4 * nt + 3];
   }
 }
 
@@ -800,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int cb = (c0 >> 4) + half2;
             if (cb <= (r >> 4)) {
               float4 *dst = reinterpret_cast<float4 *>(
-                  AC + blk(r >> 4, cb) * 256 + (r & 15) * 16);
+                  AC + blk(r >> 4, cb) * kBS + (r & 15) * kRS);
 #pragma unroll
               for (int e = 0; e < 4; ++e)
                 dst[e] = make_float4(v[16 * half2 + 4 * e], v[16 * half2 + 4 * e + 1],
@@ -846,21 +851,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // T_bc = -D_b sum_{c<=e<b} A_be T_ec on mma.sync (tf32), level by level.
       if (pt < 64) {
         const int bb = pt >> 4, j = pt & 15;
-        const float *Ab = AC + blk(bb, bb) * 256;
+        const float *Ab = AC + blk(bb, bb) * kBS;
         float xs[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
           float acc0 = (r == j) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
           for (int i = 0; i < r; ++i) {
-            if (i & 1) acc1 -= Ab[r * 16 + i] * xs[i];
-            else acc0 -= Ab[r * 16 + i] * xs[i];
+            if (i & 1) acc1 -= Ab[r * kRS + i] * xs[i];
+            else acc0 -= Ab[r * kRS + i] * xs[i];
           }
           xs[r] = acc0 + acc1;
         }
-        float *Tb = TC + blk(bb, bb) * 256;
+        float *Tb = TC + blk(bb, bb) * kBS;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Tb[r * 16 + j] = xs[r];
+        for (int r = 0; r < 16; ++r) Tb[r * kRS + j] = xs[r];
       }
       named_bar_sync(2, kPrep);
       // M_be = D_b A_be for the six blocks below the diagonal, in place
@@ -868,9 +873,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bb = (pw < 1) ? 1 : (pw < 3) ? 2 : 3;
         const int e = (pw < 1) ? 0 : (pw < 3) ? pw - 1 : pw - 3;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        mma16(TC + blk(bb, bb) * 256, AC + blk(bb, e) * 256, acc, lane);
+        mma16(TC + blk(bb, bb) * kBS, AC + blk(bb, e) * kBS, acc, lane);
         __syncwarp();
-        store16(AC + blk(bb, e) * 256, acc, 1.f, lane);
+        store16(AC + blk(bb, e) * kBS, acc, 1.f, lane);
       }
       named_bar_sync(2, kPrep);
       // T_bc = -sum_{c<=e<b} M_be T_ec (T_cc = D_c), level b - c at a time;
@@ -881,8 +886,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int c = pw >> 1, nt = pw & 1, bb = c + lev;
           float acc[4] = {0.f, 0.f, 0.f, 0.f};
           for (int e = c; e < bb; ++e)
-            mma16_nt(AC + blk(bb, e) * 256, TC + blk(e, c) * 256, acc, lane, nt);
-          store16_nt(TC + blk(bb, c) * 256, acc, -1.f, lane, nt);
+            mma16_nt(AC + blk(bb, e) * kBS, TC + blk(e, c) * kBS, acc, lane, nt);
+          store16_nt(TC + blk(bb, c) * kBS, acc, -1.f, lane, nt);
         }
         named_bar_sync(2, kPrep);
       }
@@ -917,7 +922,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float t8[8];
             if (cb <= rb) {
               const float4 *tsrc = reinterpret_cast<const float4 *>(
-                  TC + blk(rb, cb) * 256 + (r & 15) * 16 + ((8 * ch) & 15));
+                  TC + blk(rb, cb) * kBS + (r & 15) * kRS + ((8 * ch) & 15));
               const float4 t0 = tsrc[0], t1 = tsrc[1];
               const float4 f0 = *reinterpret_cast<const float4 *>(fac + 8 * ch);
               const float4 f1 = *reinterpret_cast<const float4 *>(fac + 8 * ch + 4);
