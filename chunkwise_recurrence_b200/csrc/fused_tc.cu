@@ -262,6 +262,14 @@ __device__ __forceinline__ void store16_nt(float *Y, const float acc[4],
 }
 
 // store C fragments (scaled by s) to a row-major 16x16 fp32 block
+__device__ __forceinline__ void load16_nt(const float *Y, float acc[4],
+                                          int lane, int nt) {
+  const int g = lane >> 2, t = lane & 3;
+  acc[0] = Y[g * kRS + 8 * nt + 2 * t];
+  acc[1] = Y[g * kRS + 8 * nt + 2 * t + 1];
+  acc[2] = Y[(g + 8) * kRS + 8 * nt + 2 * t];
+  acc[3] = Y[(g + 8) * kRS + 8 * nt + 2 * t + 1];
+}
 __device__ __forceinline__ void store16(float *Y, const float acc[8], float s,
                                         int lane) {
   const int g = lane >> 2, t = lane & 3;
@@ -878,17 +886,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         store16(AC + blk(bb, e) * kBS, acc, 1.f, lane);
       }
       named_bar_sync(2, kPrep);
-      // T_bc = -sum_{c<=e<b} M_be T_ec (T_cc = D_c), level b - c at a time;
-      // one warp per 8-column half of each block of the level
-#pragma unroll 1
-      for (int lev = 1; lev <= 3; ++lev) {
-        if (pw < 2 * (4 - lev)) {
-          const int c = pw >> 1, nt = pw & 1, bb = c + lev;
+      // T_bc = -sum_{c<=e<b} M_be T_ec (T_cc = D_c), scheduled on the
+      // dependency depth with partial sums kept in the T blocks:
+      //   step 1: T10, T21, T32 = -M D, and P20 = M20 D0, P31 = M31 D1,
+      //           P30 = M30 D0
+      //   step 2: T20 = -(P20 + M21 T10), T31 = -(P31 + M32 T21),
+      //           P30 += M31 T10
+      //   step 3: T30 = -(P30 + M32 T20)
+      // One task = one 8-column half of one block; a task reads only the
+      // half it writes, and inputs that no task of its step writes.
+      {
+        // task (rb, cb, e): block T_{rb,cb} (or its partial sum) from
+        // M_{rb,e} T_{e,cb}, negated or not, added to the stored partial
+        auto run = [&](int rb, int cb, int e, bool neg, bool accum, int nt) {
           float acc[4] = {0.f, 0.f, 0.f, 0.f};
-          for (int e = c; e < bb; ++e)
-            mma16_nt(AC + blk(bb, e) * kBS, TC + blk(e, c) * kBS, acc, lane, nt);
-          store16_nt(TC + blk(bb, c) * kBS, acc, -1.f, lane, nt);
-        }
+          float *dst = TC + blk(rb, cb) * kBS;
+          if (accum) load16_nt(dst, acc, lane, nt);
+          mma16_nt(AC + blk(rb, e) * kBS, TC + blk(e, cb) * kBS, acc, lane,
+                   nt);
+          store16_nt(dst, acc, neg ? -1.f : 1.f, lane, nt);
+        };
+        const int b2 = pw >> 1, nt = pw & 1;
+        // step 1: 12 half-tasks, T10, T21, T32 first
+        if (b2 < 3) run(b2 + 1, b2, b2, true, false, nt);   // T_{b+1,b}
+        else run(2, 0, 0, false, false, nt);                 // P20
+        if (pw < 2) run(3, 1, 1, false, false, nt);          // P31
+        else if (pw < 4) run(3, 0, 0, false, false, nt);     // P30
+        named_bar_sync(2, kPrep);
+        // step 2
+        if (b2 == 0) run(2, 0, 1, true, true, nt);           // T20
+        else if (b2 == 1) run(3, 1, 2, true, true, nt);      // T31
+        else if (b2 == 2) run(3, 0, 1, false, true, nt);     // P30 += M31 T10
+        named_bar_sync(2, kPrep);
+        // step 3
+        if (b2 == 0) run(3, 0, 2, true, true, nt);           // T30
         named_bar_sync(2, kPrep);
       }
       // channel gate: V -> fp16 in place for U = (T diag b) V
