@@ -25,8 +25,10 @@
 //               = one value channel)
 //   warps 6..13 "prep" warps (two per scheduler): gates, cumsum and per-row
 //               decay factors, A and P from K K^T / Q K^T, T = (I+A)^-1,
-//               T-factor operands (bf16 hi + lo), -W operand, in-place
-//               Q . e^g and K . e^{g_C - g} (fp16)
+//               fp16 T-factor operands, -W operand, in-place Q . e^g and
+//               K . e^{g_C - g} (fp16)
+//   warps 14,15 "convert" warps: K and V tiles bf16 -> fp16 in place once
+//               K K^T has read them, for the fp16 U and W products
 // All state lives in tensor memory as S^T (lane = value channel, column =
 // key channel) in fp32; fp16 / bf16 appear only as tensor-core operands.
 //
@@ -53,8 +55,9 @@ using namespace sm100;
 
 constexpr int kC = 64;         // chunk length
 constexpr int kD = 128;        // dk = dv
-constexpr int kThreads = 448;  // 14 warps
+constexpr int kThreads = 512;  // 16 warps
 constexpr int kPrep = 256;     // prep threads (warps 6..13)
+constexpr int kConv = 64;      // convert threads (warps 14, 15)
 // fp32 16x16 blocks: rows kRS floats apart, blocks kBS floats apart.  The
 // padding spreads eight consecutive rows (16-byte accesses) and the tf32
 // fragment rows over distinct banks, and puts neighbouring blocks on
@@ -75,20 +78,20 @@ constexpr uint32_t OFF_P = OFF_OS + 16384;               // P [2][64][64]
 constexpr uint32_t OFF_TP = OFF_P + 16384;               // T-factor tiles
 template <int GATE>
 struct Layout {
-  // scalar / no gate: T diag(b e^g) and T diag(b), each as a bf16 hi + lo
-  // pair (16 significant bits against raw bf16 K and V); channel gate: one
-  // fp16 T diag(b) tile, plus K e^{g_m - g} in bf16.
-  static constexpr uint32_t TP_BYTES = (GATE == 2) ? 8192 : 32768;
-  static constexpr uint32_t TPG_HI = OFF_TP, TPG_LO = OFF_TP + 8192,
-                            TPB_HI = OFF_TP + 16384, TPB_LO = OFF_TP + 24576;
+  // fp16 T-factor tiles: scalar / no gate T diag(b e^g) (TPG) and
+  // T diag(b) (TPB); channel gate T diag(b) only, plus K e^{g_m - g} (bf16)
+  static constexpr uint32_t TP_BYTES = (GATE == 2) ? 8192 : 16384;
+  static constexpr uint32_t TPB = OFF_TP, TPG = OFF_TP + 8192;
   static constexpr uint32_t KN = OFF_TP + TP_BYTES;
   static constexpr uint32_t KN_BYTES = (GATE == 2) ? 16384 : 0;
   static constexpr uint32_t AC = KN + KN_BYTES;   // A blocks fp32 [10][kBS]
   static constexpr uint32_t TC = AC + 40 * kBS;   // T blocks fp32 [10][kBS]
-  static constexpr uint32_t GS = TC + 40 * kBS;   // g [2][64]
-  static constexpr uint32_t FT = GS + 512;        // row factors [2][6][64]
-  static constexpr uint32_t GC = FT + 3072;       // g_C [2][128]
-  static constexpr uint32_t GM = GC + 1024;       // g at row 31 [128] (KDA)
+  // per-chunk gate arrays, three buffers (chunk m uses buffer m % 3): a
+  // chunk's gates are written while the two before it may still be read
+  static constexpr uint32_t GS = TC + 40 * kBS;   // g [3][64]
+  static constexpr uint32_t FT = GS + 768;        // row factors [3][6][64]
+  static constexpr uint32_t GC = FT + 4608;       // g_C [3][128]
+  static constexpr uint32_t GM = GC + 1536;       // g at row 31 [128] (KDA)
   static constexpr uint32_t MISC = GM + 512;      // barriers, tmem base, flags
   static constexpr uint32_t BYTES = MISC + 256;
   static_assert(BYTES + 1024 <= 232448, "shared memory budget");
@@ -101,21 +104,24 @@ constexpr uint32_t ACC_S = 0, ACC_V = 128, ACC_O = 256, ACC_KK = 384,
                    ACC_W = 448;
 
 // mbarrier indices
+// (pairs indexed by chunk parity complete every other chunk, so a waiter
+// that falls one chunk behind cannot mistake a later phase for its own)
 enum {
-  B_FULL0, B_FULL1, B_EMPTY0, B_EMPTY1, B_VFREE, B_KKREADY, B_KKDONE,
+  B_FULL0, B_FULL1, B_EMPTY0, B_EMPTY1, B_VFREE, B_KKREADY,
+  B_KKDONE0, B_KKDONE1,  // K K^T of the chunk done (MMA commit)
   B_TREADY, B_WDONE, B_WREADY, B_SREADY, B_XDONE, B_VNREADY, B_SDONE,
-  B_ODONE, B_DRAIN, B_FULLV, B_COUNT
+  B_ODONE, B_DRAIN, B_FULLV,
+  B_CONV,                // K (scalar / no gate) and V fp16 (convert warps)
+  B_COUNT
 };
 
 // Instruction descriptors (M = 128 everywhere).  Operands built on chip are
-// fp16 (11-bit significand: 8x finer than bf16 at the same tensor-core rate).
-// Products that read the raw bf16 inputs stay bf16: K K^T (exact inputs), and
-// for the scalar / no gate U and W, whose T factor is split into bf16 hi + lo.
-// The channel-gate K K^T reads e^{+-(g - g_m)}-scaled keys, which need bf16's
-// exponent range.
+// fp16 (11-bit significand: 8x finer than bf16 at the same tensor-core rate);
+// V and K are converted to fp16 in place (exact for inputs within fp16's
+// range) for U and W.  K K^T reads the raw bf16 tiles, or for the channel
+// gate keys scaled by e^{+-(g - g_m)}, which need bf16's exponent range.
 constexpr uint32_t ID_KK_B = idesc_f16kind(128, 64, false, false, true);
 constexpr uint32_t ID_UW_H = idesc_f16kind(128, 64, true, false, false);
-constexpr uint32_t ID_UW_B = idesc_f16kind(128, 64, true, false, true);
 constexpr uint32_t ID_XV = idesc_f16kind(128, 64, false, true, false);
 constexpr uint32_t ID_XO = idesc_f16kind(128, 64, false, false, false);
 constexpr uint32_t ID_SU = idesc_f16kind(128, 128, false, true, false);
@@ -127,7 +133,6 @@ constexpr unsigned kErrNonFinite = 1u << 25;  // non-finite output or state
 constexpr float kF16Max = 65504.f;
 
 constexpr long long kWaitCycles = 1ll << 32;   // ~2 s: a wait never lasts this
-constexpr uint32_t kSleepNs = 20000;           // suspend hint per try (20 us)
 
 __device__ unsigned g_fused_error;
 
@@ -152,7 +157,7 @@ __device__ __forceinline__ bool wait_bar(const Ctx &cx, int b,
   if (mbar_try_wait(&cx.bar[b], parity)) return true;
   const long long t0 = clock64();
   for (;;) {
-    if (mbar_try_wait_sleep(&cx.bar[b], parity, kSleepNs)) return true;
+    if (mbar_try_wait(&cx.bar[b], parity)) return true;
     if (*cx.abort_flag) return false;
     if (clock64() - t0 > kWaitCycles) {
       *cx.abort_flag = 1;
@@ -187,6 +192,31 @@ __device__ __forceinline__ void unpack_bf16(uint32_t w, float &lo, float &hi) {
   float2 f = __bfloat1622float2(v);
   lo = f.x;
   hi = f.y;
+}
+// 8 values in place (16 bytes of shared memory): bf16 -> fp16 times sc
+__device__ __forceinline__ void bf16_to_f16_16B(uint8_t *ptr, float sc) {
+  uint4 x = *reinterpret_cast<uint4 *>(ptr);
+  uint32_t *w = reinterpret_cast<uint32_t *>(&x);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
+    float2 f = __bfloat1622float2(b);
+    __half2 hv = __floats2half2_rn(f.x * sc, f.y * sc);
+    w[e] = *reinterpret_cast<uint32_t *>(&hv);
+  }
+  *reinterpret_cast<uint4 *>(ptr) = x;
+}
+// 8 fp16 values in place times sc
+__device__ __forceinline__ void f16_scale_16B(uint8_t *ptr, float sc) {
+  uint4 x = *reinterpret_cast<uint4 *>(ptr);
+  uint32_t *w = reinterpret_cast<uint32_t *>(&x);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float2 f = __half22float2(*reinterpret_cast<__half2 *>(&w[e]));
+    __half2 hv = __floats2half2_rn(f.x * sc, f.y * sc);
+    w[e] = *reinterpret_cast<uint32_t *>(&hv);
+  }
+  *reinterpret_cast<uint4 *>(ptr) = x;
 }
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
@@ -310,8 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const size_t sbase = ((size_t)n * p.H + h) * kD * kD;
 
   if (threadIdx.x == 0) {
-    const uint32_t counts[B_COUNT] = {1, 1, 1, 1, 1, kPrep, 1, kPrep, 1, kPrep,
-                                      128, 1, 128, 1, 1, 1, 1};
+    const uint32_t counts[B_COUNT] = {
+        1, 1, 1, 1, 1, kPrep, 1, 1, kPrep, 1, kPrep, 128, 1, 128, 1, 1, 1, 1,
+        kConv};
     for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], counts[i]);
     *abort_flag = 0;
     fence_mbar_init();
@@ -374,7 +405,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t nw = smem_u32(sm + OFF_NW), vt = smem_u32(sm + OFF_V),
-                     tp = smem_u32(sm + OFF_TP),
                      kn = smem_u32(sm + Lay::KN);
       auto stage = [&](int m) {
         return smem_u32(sm + OFF_STAGE + (m & 1) * kStageBytes);
@@ -397,40 +427,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                   : sdesc_sw128(base + koff, 16, 1024);
           mma_f16kind(tmem + ACC_KK, a, b, ID_KK_B, ks > 0);
         }
-        mma_commit(&bar[B_KKDONE]);
+        mma_commit(&bar[B_KKDONE0 + (m & 1)]);
       };
-      // U^T = V^T (T diag b)^T and W^T = (K e^g)^T (T diag(b e^g))^T
+      // U^T = V^T (T diag b)^T and W^T = (K e^g)^T (T diag(b e^g))^T, all
+      // fp16: V and K are converted in place by the convert warps (for the
+      // channel gate K already holds K e^g, and the factor is T diag(b))
       auto issue_uw = [&](int m) {
-        if (!wait_bar(cx, B_FULLV, m & 1)) return false;
+        if (!wait_bar(cx, B_CONV, m & 1)) return false;
         tc_fence_after();
         const uint32_t base = stage(m);
         const uint32_t accv = tmem + ACC_V + (m & 1) * 64;
-        if (GATE == 2) {
+        const uint32_t tpb = smem_u32(sm + Lay::TPB);
+        const uint32_t tpw = smem_u32(sm + (GATE == 2 ? Lay::TPB : Lay::TPG));
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_f16kind(accv, sdesc_sw128(vt + ks * 2048, 8192, 1024),
-                        sdesc_sw128(tp + ks * 32, 16, 1024), ID_UW_H, ks > 0);
+        for (int ks = 0; ks < 4; ++ks)
+          mma_f16kind(accv, sdesc_sw128(vt + ks * 2048, 8192, 1024),
+                      sdesc_sw128(tpb + ks * 32, 16, 1024), ID_UW_H, ks > 0);
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_f16kind(tmem + ACC_W,
-                        sdesc_sw128(base + ks * 2048, 16384, 1024),
-                        sdesc_sw128(tp + ks * 32, 16, 1024), ID_UW_H, ks > 0);
-        } else {
-          // hi and lo halves of the T factor accumulate into one result
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            mma_f16kind(accv, sdesc_sw128(vt + (ks & 3) * 2048, 8192, 1024),
-                        sdesc_sw128(tp + 16384 + (ks >> 2) * 8192 + (ks & 3) * 32,
-                                    16, 1024),
-                        ID_UW_B, ks > 0);
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            mma_f16kind(tmem + ACC_W,
-                        sdesc_sw128(base + (ks & 3) * 2048, 16384, 1024),
-                        sdesc_sw128(tp + (ks >> 2) * 8192 + (ks & 3) * 32, 16,
-                                    1024),
-                        ID_UW_B, ks > 0);
-        }
+        for (int ks = 0; ks < 4; ++ks)
+          mma_f16kind(tmem + ACC_W, sdesc_sw128(base + ks * 2048, 16384, 1024),
+                      sdesc_sw128(tpw + ks * 32, 16, 1024), ID_UW_H, ks > 0);
         mma_commit(&bar[B_WDONE]);
         mma_commit(&bar[B_VFREE]);
         return true;
@@ -496,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // S update and intra-chunk output
         if (!wait_bar(cx, B_VNREADY, m & 1)) break;
         tc_fence_after();
-        // A = V_new^T, fp16 pairs in tensor memory
+        // A = V_new^T, fp16 pairs in tensor memory; B = K e^{g_C - g}
         const uint32_t vn_op = tmem + ACC_V + (m & 1) * 64;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
@@ -583,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       if (!(ok = group_all(wait_bar(cx, B_TREADY, m & 1), 1, 128))) break;
       tc_fence_after();
-      const float *gcm = gC + (m & 1) * 128;
+      const float *gcm = gC + (m % 3) * 128;
       const float dscal = GATE == 1 ? __expf(gcm[0]) : 1.f;
       // S^T as fp16 pairs (key channels 2j, 2j+1 in column j) into the
       // V_new^T region of the other chunk parity, free from S done(m-1)
@@ -658,6 +674,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!finite) atomicOr(&g_fused_error, kErrNonFinite);
     }
+  } else if (warp >= 14) {
+    // ------------------------------------------------------ convert warps
+    // bf16 -> fp16 in place for the U and W operands: K of chunk m once
+    // K K^T has read it (scalar / no gate; the channel gate's prep warps
+    // write K e^g in fp16 themselves), and V of chunk m once it has landed.
+    const int ct = threadIdx.x - 14 * 32;
+    for (int m = 0; m < NC; ++m) {
+      if (GATE != 2) {
+        if (!group_all(wait_bar(cx, B_KKDONE0 + (m & 1), (m >> 1) & 1), 3,
+                       kConv))
+          break;
+        uint8_t *stg = sm + OFF_STAGE + (m & 1) * kStageBytes;
+        // the two 8 KB K tiles of the stage, 16 bytes per step
+#pragma unroll 4
+        for (int i = ct; i < 1024; i += kConv)
+          bf16_to_f16_16B(stg + (i >> 9) * 16384 + (i & 511) * 16, 1.f);
+      }
+      if (!group_all(wait_bar(cx, B_FULLV, m & 1), 3, kConv)) break;
+#pragma unroll 4
+      for (int i = ct; i < 1024; i += kConv)
+        bf16_to_f16_16B(sm + OFF_V + i * 16, 1.f);
+      fence_proxy_async_smem();
+      mbar_arrive(&bar[B_CONV]);
+    }
   } else {
     // ------------------------------------------------------ prep warps
     // 8 warps, two per scheduler.  pt = 0..255; TMEM lane l (two threads per
@@ -684,15 +724,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (GATE == 1) na = p.log_alpha[(size_t)(tok0 + pt) * p.H + h];
       }
     };
-    if (pt < 64) load_gates(0);
-    for (int m = 0; m < NC; ++m) {
-      const int s = m & 1, tok0 = start + m * kC, L = min(kC, end - tok0);
-      uint8_t *stg = sm + OFF_STAGE + s * kStageBytes;
-      float *g = gS + s * 64, *gc = gC + s * 128;
-      float *F = FT + s * (F_COUNT * 64);
-      // ---- P1: beta, in-chunk cumulative log-decay, per-row factors
+    // ---- P1 of chunk j: beta, in-chunk cumulative log-decay, per-row
+    // factors, into gate buffer j % 3; prefetches the gates of chunk j+1
+    auto p1 = [&](int j) {
+      float *g = gS + (j % 3) * 64, *gc = gC + (j % 3) * 128;
+      float *F = FT + (j % 3) * (F_COUNT * 64);
       float x = na, bb = nb;
-      if (pt < 64) load_gates(m + 1);
+      if (pt < 64) load_gates(j + 1);
       if (GATE != 2) {
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -721,6 +759,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         F[F_EG * 64 + pt] = __expf(gr);
         F[F_EK * 64 + pt] = __expf(gcv - gr);
       }
+    };
+    if (pt < 64) load_gates(0);
+    if (NC > 0) p1(0);
+    for (int m = 0; m < NC; ++m) {
+      const int s = m & 1, tok0 = start + m * kC, L = min(kC, end - tok0);
+      uint8_t *stg = sm + OFF_STAGE + s * kStageBytes;
+      float *g = gS + (m % 3) * 64, *gc = gC + (m % 3) * 128;
+      float *F = FT + (m % 3) * (F_COUNT * 64);
       // ---- P2 (channel gate only): per key channel c, with g_m = g at row
       // 31: Q e^{g-g_m}, K e^{g-g_m}, K e^{g_m-g} (bf16)
       float amax = 0.f;
@@ -768,7 +814,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bar[B_KKREADY]);
       }
       // ---- P3: A (strictly lower, fp32 blocks) and P (lower, fp16 operand)
-      if (!group_all(wait_bar(cx, B_KKDONE, m & 1), 2, kPrep)) break;
+      if (!group_all(wait_bar(cx, B_KKDONE0 + s, (m >> 1) & 1), 2, kPrep))
+        break;
       tc_fence_after();
       const bool fact = (GATE != 1) || (g[0] - g[63] < 80.f);
       {
@@ -922,72 +969,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (b2 == 0) run(3, 0, 2, true, true, nt);           // T30
         named_bar_sync(2, kPrep);
       }
-      // channel gate: V -> fp16 in place for U = (T diag b) V
-      if (GATE == 2) {
-        if (!group_all(wait_bar(cx, B_FULLV, m & 1), 2, kPrep)) break;
-        for (int i = pt; i < 1024; i += kPrep) {
-          uint8_t *ptr = sm + OFF_V + i * 16;
-          uint4 xv = *reinterpret_cast<uint4 *>(ptr);
-          uint32_t *w = reinterpret_cast<uint32_t *>(&xv);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float a0, a1;
-            unpack_bf16(w[e], a0, a1);
-            amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
-            w[e] = pack_f16(a0, a1);
-          }
-          *reinterpret_cast<uint4 *>(ptr) = xv;
-        }
-      }
-      // ---- T-factor operands.  Scalar / no gate: T diag(b e^g) and
-      // T diag(b) as bf16 hi + lo pairs.  Channel gate: T diag(b) in fp16.
+      // ---- T-factor operands in fp16: T diag(b e^g) (scalar / no gate)
+      // and T diag(b).  Item (tile, row r, 16-byte chunk ch); consecutive
+      // threads take consecutive rows.
       {
-        const int r = pt & 63, rb = r >> 4;
-        const int which = (GATE == 2) ? 1 : ((pt >> 6) & 1);   // 0: b e^g, 1: b
-        const int chs = (GATE == 2) ? 0 : ((pt >> 7) * 4);     // chunk range
-        const int che = (GATE == 2) ? 8 : chs + 4;
-        const float *fac = F + (which == 0 ? F_BG : F_B) * 64;
-        if (GATE != 2 || pt < 64) {
-          for (int ch = chs; ch < che; ++ch) {
-            const int cb = (8 * ch) >> 4;
-            float t8[8];
-            if (cb <= rb) {
-              const float4 *tsrc = reinterpret_cast<const float4 *>(
-                  TC + blk(rb, cb) * kBS + (r & 15) * kRS + ((8 * ch) & 15));
-              const float4 t0 = tsrc[0], t1 = tsrc[1];
-              const float4 f0 = *reinterpret_cast<const float4 *>(fac + 8 * ch);
-              const float4 f1 = *reinterpret_cast<const float4 *>(fac + 8 * ch + 4);
-              t8[0] = t0.x * f0.x; t8[1] = t0.y * f0.y; t8[2] = t0.z * f0.z;
-              t8[3] = t0.w * f0.w; t8[4] = t1.x * f1.x; t8[5] = t1.y * f1.y;
-              t8[6] = t1.z * f1.z; t8[7] = t1.w * f1.w;
-            } else {
+        constexpr int kTiles = (GATE == 2) ? 1 : 2;
 #pragma unroll
-              for (int e = 0; e < 8; ++e) t8[e] = 0.f;
-            }
-            if (GATE == 2) {
-              st_smem_v4(sm + OFF_TP + sw128_chunk(r, ch),
-                         pack_f16(t8[0], t8[1]), pack_f16(t8[2], t8[3]),
-                         pack_f16(t8[4], t8[5]), pack_f16(t8[6], t8[7]));
-            } else {
-              uint32_t hw[4], lw[4];
+        for (int it = pt; it < kTiles * 512; it += kPrep) {
+          const int r = it & 63, rb = r >> 4, ch = (it >> 6) & 7;
+          const bool tb = (GATE == 2) || (it >> 9) == 1;   // T diag(b)
+          const float *fac = F + (tb ? F_B : F_BG) * 64;
+          const int cb = ch >> 1;
+          float t8[8];
+          if (cb <= rb) {
+            const float4 *tsrc = reinterpret_cast<const float4 *>(
+                TC + blk(rb, cb) * kBS + (r & 15) * kRS + ((8 * ch) & 15));
+            const float4 t0 = tsrc[0], t1 = tsrc[1];
+            const float4 f0 = *reinterpret_cast<const float4 *>(fac + 8 * ch);
+            const float4 f1 = *reinterpret_cast<const float4 *>(fac + 8 * ch + 4);
+            t8[0] = t0.x * f0.x; t8[1] = t0.y * f0.y; t8[2] = t0.z * f0.z;
+            t8[3] = t0.w * f0.w; t8[4] = t1.x * f1.x; t8[5] = t1.y * f1.y;
+            t8[6] = t1.z * f1.z; t8[7] = t1.w * f1.w;
+          } else {
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const __nv_bfloat16 h0 = __float2bfloat16_rn(t8[2 * e]);
-                const __nv_bfloat16 h1 = __float2bfloat16_rn(t8[2 * e + 1]);
-                hw[e] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
-                lw[e] = pack_bf16(t8[2 * e] - __bfloat162float(h0),
-                                  t8[2 * e + 1] - __bfloat162float(h1));
-              }
-              const uint32_t hi = which == 0 ? Lay::TPG_HI : Lay::TPB_HI;
-              const uint32_t lo = which == 0 ? Lay::TPG_LO : Lay::TPB_LO;
-              st_smem_v4(sm + hi + sw128_chunk(r, ch), hw[0], hw[1], hw[2], hw[3]);
-              st_smem_v4(sm + lo + sw128_chunk(r, ch), lw[0], lw[1], lw[2], lw[3]);
-            }
+            for (int e = 0; e < 8; ++e) t8[e] = 0.f;
           }
+          st_smem_v4(sm + (tb ? Lay::TPB : Lay::TPG) + sw128_chunk(r, ch),
+                     pack_f16(t8[0], t8[1]), pack_f16(t8[2], t8[3]),
+                     pack_f16(t8[4], t8[5]), pack_f16(t8[6], t8[7]));
         }
       }
       fence_proxy_async_smem();
       mbar_arrive(&bar[B_TREADY]);
+      // P1 of the next chunk while U and W run
+      if (m + 1 < NC) p1(m + 1);
       // ---- P5: -W^T operand; Q e^g and K e^{g_C - g} in place (fp16)
       if (!group_all(wait_bar(cx, B_WDONE, m & 1), 2, kPrep)) break;
       tc_fence_after();
@@ -1005,31 +1020,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int idx = pt; idx < kC * 16; idx += kPrep) {
         const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
-        const uint32_t off = kb * 16384 + sw128_chunk(r, cc & 7);
-        uint4 *kp = reinterpret_cast<uint4 *>(stg + off);
-        uint4 kv;
-        uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
+        uint8_t *kp = stg + kb * 16384 + sw128_chunk(r, cc & 7);
         if (GATE != 2) {
-          // raw bf16 -> fp16, scaled by e^g (Q) and e^{g_C - g} (K)
-          uint4 *qp = reinterpret_cast<uint4 *>(stg + off + 8192);
+          // Q: raw bf16 -> fp16 times e^g; K (fp16 since the convert
+          // warps) times e^{g_C - g}
           const float eq = (GATE == 1) ? F[F_EG * 64 + r] : 1.f;
           const float ek = (GATE == 1) ? F[F_EK * 64 + r] : 1.f;
-          uint4 qv = *qp;
-          kv = *kp;
-          uint32_t *qw = reinterpret_cast<uint32_t *>(&qv);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float a0, a1;
-            unpack_bf16(qw[e], a0, a1);
-            qw[e] = pack_f16(a0 * eq, a1 * eq);
-            unpack_bf16(kw[e], a0, a1);
-            kw[e] = pack_f16(a0 * ek, a1 * ek);
-          }
-          *qp = qv;
+          bf16_to_f16_16B(kp + 8192, eq);
+          if (GATE == 1) f16_scale_16B(kp, ek);
         } else {
           // K~ = (K e^{g_m-g}) e^{g_C-g_m}, per channel
-          kv = *reinterpret_cast<const uint4 *>(sm + Lay::KN + kb * 8192 +
-                                                sw128_chunk(r, cc & 7));
+          uint4 kv = *reinterpret_cast<const uint4 *>(
+              sm + Lay::KN + kb * 8192 + sw128_chunk(r, cc & 7));
+          uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
           const int cbase = kb * 64 + (cc & 7) * 8;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -1038,8 +1041,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             kw[e] = pack_f16(a0 * __expf(gc[cbase + 2 * e] - gM[cbase + 2 * e]),
                              a1 * __expf(gc[cbase + 2 * e + 1] - gM[cbase + 2 * e + 1]));
           }
+          *reinterpret_cast<uint4 *>(kp) = kv;
         }
-        *kp = kv;
       }
       if (!(amax <= kF16Max)) atomicOr(&g_fused_error, kErrRange);
       fence_proxy_async_smem();
