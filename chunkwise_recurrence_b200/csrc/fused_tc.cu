@@ -25,10 +25,11 @@
 //               = one value channel)
 //   warps 6..13 "prep" warps (two per scheduler): gates, cumsum and per-row
 //               decay factors, A and P from K K^T / Q K^T, T = (I+A)^-1,
-//               fp16 T-factor operands, -W operand, in-place Q . e^g and
+//               T-factor operands, -W operand, in-place Q . e^g and
 //               K . e^{g_C - g} (fp16)
-//   warps 14,15 "convert" warps: K and V tiles bf16 -> fp16 in place once
-//               K K^T has read them, for the fp16 U and W products
+//   warps 14,15 "convert" warps: channel gate, V tile bf16 -> fp16 in place
+//               for the fp16 U product (the scalar / no gate U and W read
+//               the raw bf16 V and K)
 // All state lives in tensor memory as S^T (lane = value channel, column =
 // key channel) in fp32; fp16 / bf16 appear only as tensor-core operands.
 //
@@ -80,8 +81,15 @@ template <int GATE>
 struct Layout {
   // fp16 T-factor tiles: scalar / no gate T diag(b e^g) (TPG) and
   // T diag(b) (TPB); channel gate T diag(b) only, plus K e^{g_m - g} (bf16)
-  static constexpr uint32_t TP_BYTES = (GATE == 2) ? 8192 : 16384;
-  static constexpr uint32_t TPB = OFF_TP, TPG = OFF_TP + 8192;
+  // T-factor tiles.  Scalar / no gate, bf16 against the raw bf16 V and K:
+  // T diag(b) for U as a hi + lo pair (TPB, TPB_LO: the lo tile holds the
+  // bf16 rounding residual, so U carries about 16 significant bits of the
+  // factor; a single bf16 factor there quadruples the final-state error),
+  // and T diag(b e^g) for W as one tile (TPG).  Channel gate: T diag(b) in
+  // fp16 (TPB) for both, against fp16 V and K e^g.
+  static constexpr uint32_t TP_BYTES = (GATE == 2) ? 8192 : 24576;
+  static constexpr uint32_t TPB = OFF_TP, TPG = OFF_TP + 8192,
+                            TPB_LO = OFF_TP + 16384;
   static constexpr uint32_t KN = OFF_TP + TP_BYTES;
   static constexpr uint32_t KN_BYTES = (GATE == 2) ? 16384 : 0;
   static constexpr uint32_t AC = KN + KN_BYTES;   // A blocks fp32 [10][kBS]
@@ -116,12 +124,14 @@ enum {
 };
 
 // Instruction descriptors (M = 128 everywhere).  Operands built on chip are
-// fp16 (11-bit significand: 8x finer than bf16 at the same tensor-core rate);
-// V and K are converted to fp16 in place (exact for inputs within fp16's
-// range) for U and W.  K K^T reads the raw bf16 tiles, or for the channel
-// gate keys scaled by e^{+-(g - g_m)}, which need bf16's exponent range.
+// fp16 (11-bit significand: 8x finer than bf16 at the same tensor-core rate).
+// Products that read raw bf16 input tiles stay bf16: K K^T, and for the
+// scalar / no gate U and W (their T factors are bf16; U's as a hi + lo
+// pair).  The channel gate's K K^T reads keys scaled by e^{+-(g - g_m)},
+// which need bf16's exponent range; its U and W are fp16.
 constexpr uint32_t ID_KK_B = idesc_f16kind(128, 64, false, false, true);
 constexpr uint32_t ID_UW_H = idesc_f16kind(128, 64, true, false, false);
+constexpr uint32_t ID_UW_B = idesc_f16kind(128, 64, true, false, true);
 constexpr uint32_t ID_XV = idesc_f16kind(128, 64, false, true, false);
 constexpr uint32_t ID_XO = idesc_f16kind(128, 64, false, false, false);
 constexpr uint32_t ID_SU = idesc_f16kind(128, 128, false, true, false);
@@ -201,18 +211,6 @@ __device__ __forceinline__ void bf16_to_f16_16B(uint8_t *ptr, float sc) {
   for (int e = 0; e < 4; ++e) {
     __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
     float2 f = __bfloat1622float2(b);
-    __half2 hv = __floats2half2_rn(f.x * sc, f.y * sc);
-    w[e] = *reinterpret_cast<uint32_t *>(&hv);
-  }
-  *reinterpret_cast<uint4 *>(ptr) = x;
-}
-// 8 fp16 values in place times sc
-__device__ __forceinline__ void f16_scale_16B(uint8_t *ptr, float sc) {
-  uint4 x = *reinterpret_cast<uint4 *>(ptr);
-  uint32_t *w = reinterpret_cast<uint32_t *>(&x);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    float2 f = __half22float2(*reinterpret_cast<__half2 *>(&w[e]));
     __half2 hv = __floats2half2_rn(f.x * sc, f.y * sc);
     w[e] = *reinterpret_cast<uint32_t *>(&hv);
   }
@@ -432,6 +430,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // U^T = V^T (T diag b)^T and W^T = (K e^g)^T (T diag(b e^g))^T, all
       // fp16: V and K are converted in place by the convert warps (for the
       // channel gate K already holds K e^g, and the factor is T diag(b))
+      // scalar / no gate: raw bf16 V and K against bf16 T factors; channel
+      // gate: fp16 (V converted, K e^g written by the prep warps)
+      constexpr uint32_t kIdUW = (GATE == 2) ? ID_UW_H : ID_UW_B;
       auto issue_uw = [&](int m) {
         if (!wait_bar(cx, B_CONV, m & 1)) return false;
         tc_fence_after();
@@ -439,14 +440,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t accv = tmem + ACC_V + (m & 1) * 64;
         const uint32_t tpb = smem_u32(sm + Lay::TPB);
         const uint32_t tpw = smem_u32(sm + (GATE == 2 ? Lay::TPB : Lay::TPG));
+        const uint32_t tplo = smem_u32(sm + Lay::TPB_LO);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           mma_f16kind(accv, sdesc_sw128(vt + ks * 2048, 8192, 1024),
-                      sdesc_sw128(tpb + ks * 32, 16, 1024), ID_UW_H, ks > 0);
+                      sdesc_sw128(tpb + ks * 32, 16, 1024), kIdUW, ks > 0);
+        if (GATE != 2) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_f16kind(accv, sdesc_sw128(vt + ks * 2048, 8192, 1024),
+                        sdesc_sw128(tplo + ks * 32, 16, 1024), kIdUW, 1);
+        }
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           mma_f16kind(tmem + ACC_W, sdesc_sw128(base + ks * 2048, 16384, 1024),
-                      sdesc_sw128(tpw + ks * 32, 16, 1024), ID_UW_H, ks > 0);
+                      sdesc_sw128(tpw + ks * 32, 16, 1024), kIdUW, ks > 0);
         mma_commit(&bar[B_WDONE]);
         mma_commit(&bar[B_VFREE]);
         return true;
@@ -676,26 +684,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 14) {
     // ------------------------------------------------------ convert warps
-    // bf16 -> fp16 in place for the U and W operands: K of chunk m once
-    // K K^T has read it (scalar / no gate; the channel gate's prep warps
-    // write K e^g in fp16 themselves), and V of chunk m once it has landed.
+    // Channel gate: V -> fp16 in place for U = (T diag b) V, once V has
+    // landed.  Scalar / no gate: U and W read the raw bf16 tiles, and these
+    // warps only pass the V arrival on.
     const int ct = threadIdx.x - 14 * 32;
     for (int m = 0; m < NC; ++m) {
-      if (GATE != 2) {
-        if (!group_all(wait_bar(cx, B_KKDONE0 + (m & 1), (m >> 1) & 1), 3,
-                       kConv))
-          break;
-        uint8_t *stg = sm + OFF_STAGE + (m & 1) * kStageBytes;
-        // the two 8 KB K tiles of the stage, 16 bytes per step
+      if (!group_all(wait_bar(cx, B_FULLV, m & 1), 3, kConv)) break;
+      if (GATE == 2) {
 #pragma unroll 4
         for (int i = ct; i < 1024; i += kConv)
-          bf16_to_f16_16B(stg + (i >> 9) * 16384 + (i & 511) * 16, 1.f);
+          bf16_to_f16_16B(sm + OFF_V + i * 16, 1.f);
+        fence_proxy_async_smem();
       }
-      if (!group_all(wait_bar(cx, B_FULLV, m & 1), 3, kConv)) break;
-#pragma unroll 4
-      for (int i = ct; i < 1024; i += kConv)
-        bf16_to_f16_16B(sm + OFF_V + i * 16, 1.f);
-      fence_proxy_async_smem();
       mbar_arrive(&bar[B_CONV]);
     }
   } else {
@@ -969,9 +969,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (b2 == 0) run(3, 0, 2, true, true, nt);           // T30
         named_bar_sync(2, kPrep);
       }
-      // ---- T-factor operands in fp16: T diag(b e^g) (scalar / no gate)
-      // and T diag(b).  Item (tile, row r, 16-byte chunk ch); consecutive
-      // threads take consecutive rows.
+      // ---- T-factor operands: T diag(b e^g) (scalar / no gate) and
+      // T diag(b), with T diag(b)'s bf16 residual tile (scalar / no gate).
+      // Item (tile, row r, 16-byte chunk ch); consecutive threads take
+      // consecutive rows.
       {
         constexpr int kTiles = (GATE == 2) ? 1 : 2;
 #pragma unroll
@@ -994,9 +995,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) t8[e] = 0.f;
           }
+          auto pk = [](float a, float b) {
+            return GATE == 2 ? pack_f16(a, b) : pack_bf16(a, b);
+          };
+          uint32_t hw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) hw[e] = pk(t8[2 * e], t8[2 * e + 1]);
           st_smem_v4(sm + (tb ? Lay::TPB : Lay::TPG) + sw128_chunk(r, ch),
-                     pack_f16(t8[0], t8[1]), pack_f16(t8[2], t8[3]),
-                     pack_f16(t8[4], t8[5]), pack_f16(t8[6], t8[7]));
+                     hw[0], hw[1], hw[2], hw[3]);
+          if (GATE != 2 && tb) {
+            uint32_t lw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float h0, h1;
+              unpack_bf16(hw[e], h0, h1);
+              lw[e] = pack_bf16(t8[2 * e] - h0, t8[2 * e + 1] - h1);
+            }
+            st_smem_v4(sm + Lay::TPB_LO + sw128_chunk(r, ch), lw[0], lw[1],
+                       lw[2], lw[3]);
+          }
         }
       }
       fence_proxy_async_smem();
@@ -1022,12 +1039,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
         uint8_t *kp = stg + kb * 16384 + sw128_chunk(r, cc & 7);
         if (GATE != 2) {
-          // Q: raw bf16 -> fp16 times e^g; K (fp16 since the convert
-          // warps) times e^{g_C - g}
+          // raw bf16 -> fp16: Q times e^g, K times e^{g_C - g}
           const float eq = (GATE == 1) ? F[F_EG * 64 + r] : 1.f;
           const float ek = (GATE == 1) ? F[F_EK * 64 + r] : 1.f;
           bf16_to_f16_16B(kp + 8192, eq);
-          if (GATE == 1) f16_scale_16B(kp, ek);
+          bf16_to_f16_16B(kp, ek);
         } else {
           // K~ = (K e^{g_m-g}) e^{g_C-g_m}, per channel
           uint4 kv = *reinterpret_cast<const uint4 *>(
