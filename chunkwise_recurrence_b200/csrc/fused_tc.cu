@@ -99,8 +99,10 @@ struct Layout {
   static constexpr uint32_t GS = TC + 40 * kBS;   // g [3][64]
   static constexpr uint32_t FT = GS + 768;        // row factors [3][6][64]
   static constexpr uint32_t GC = FT + 4608;       // g_C [3][128]
-  static constexpr uint32_t GM = GC + 1536;       // g at row 31 [128] (KDA)
-  static constexpr uint32_t MISC = GM + 512;      // barriers, tmem base, flags
+  // channel gate, per key channel, for the chunk in progress: e^{g_m}
+  // (g_m = g at row 31) and e^{g_C - g_m}
+  static constexpr uint32_t GM = GC + 1536;       // [2][128]
+  static constexpr uint32_t MISC = GM + 1024;     // barriers, tmem base, flags
   static constexpr uint32_t BYTES = MISC + 256;
   static_assert(BYTES + 1024 <= 232448, "shared memory budget");
 };
@@ -510,13 +512,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      16, 1024),
                          ID_XO, ks > 0);
         mma_commit(&bar[B_XDONE]);
-        // K K^T of chunk m+1 while the state warps turn V_new into an operand
-        if (m + 1 < NC && kk_next == m + 1) {
-          if (!kk_inputs_ready(m + 1)) break;
-          tc_fence_after();
-          issue_kk(m + 1);
-          ++kk_next;
-        }
+        // K K^T of chunk m+1 while the state warps turn V_new into an
+        // operand, if its inputs are in (the channel gate's rescaling may
+        // still be running: the S update must not wait for it)
+        try_kk_early(m + 1);
         // S update and intra-chunk output
         if (!wait_bar(cx, B_VNREADY, m & 1)) break;
         tc_fence_after();
@@ -536,6 +535,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bar[B_SDONE]);
         mma_commit(&bar[B_ODONE]);
         mma_commit(&bar[B_EMPTY0 + (m & 1)]);
+        // K K^T of chunk m+1 now at the latest: its T factors depend on it
+        if (m + 1 < NC && kk_next == m + 1) {
+          if (!kk_inputs_ready(m + 1)) break;
+          tc_fence_after();
+          issue_kk(m + 1);
+          ++kk_next;
+        }
         // U, W of chunk m+1
         if (m + 1 < NC) {
           if (!wait_bar(cx, B_TREADY, (m + 1) & 1)) break;
@@ -623,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (GATE != 0) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            v[j] *= (GATE == 1) ? dscal : __expf(gcm[c0 + j]);
+            v[j] *= (GATE == 1) ? dscal : gcm[c0 + j];   // KDA: e^{g_C}
           tmem_st32(trow + ACC_S + c0, v);
         }
       }
@@ -808,8 +814,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<__nv_bfloat16 *>(knt + off) =
               __float2bfloat16_rn(kv * en);
         }
-        if (half == 0) gM[c] = gm;
-        else gc[c] = gg;
+        // per-channel factors, one exponential each per chunk: e^{g_m}, and
+        // e^{g_C} (decay of S) and e^{g_C - g_m} in gc / gM + 128
+        if (half == 0) {
+          gM[c] = __expf(gm);
+        } else {
+          gc[c] = __expf(gg);
+          gM[128 + c] = __expf(gg - gm);
+        }
         fence_proxy_async_smem();
         mbar_arrive(&bar[B_KKREADY]);
       }
@@ -893,8 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 4; ++e) {
               float a0, a1;
               unpack_bf16(w[e], a0, a1);
-              w[e] = pack_f16(a0 * __expf(gM[cbase + 2 * e]),
-                              a1 * __expf(gM[cbase + 2 * e + 1]));
+              w[e] = pack_f16(a0 * gM[cbase + 2 * e], a1 * gM[cbase + 2 * e + 1]);
             }
             *ptr = xv;
           }
@@ -974,9 +985,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Item (tile, row r, 16-byte chunk ch); consecutive threads take
       // consecutive rows.
       {
-        constexpr int kTiles = (GATE == 2) ? 1 : 2;
+        if (GATE != 2) {
+          // Thread = row r and two 8-column chunks; each T value feeds both
+          // tiles.  All loads are issued before the first store.
+          const int r = pt & 63, rb = r >> 4;
+          float4 t[2][2], fg[2][2], fb[2][2];
 #pragma unroll
-        for (int it = pt; it < kTiles * 512; it += kPrep) {
+          for (int u = 0; u < 2; ++u) {
+            const int ch = (pt >> 6) + 4 * u;
+            if ((ch >> 1) <= rb) {
+              const float4 *tsrc = reinterpret_cast<const float4 *>(
+                  TC + blk(rb, ch >> 1) * kBS + (r & 15) * kRS + ((8 * ch) & 15));
+              t[u][0] = tsrc[0];
+              t[u][1] = tsrc[1];
+            } else {
+              t[u][0] = t[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            fg[u][0] = *reinterpret_cast<const float4 *>(F + F_BG * 64 + 8 * ch);
+            fg[u][1] = *reinterpret_cast<const float4 *>(F + F_BG * 64 + 8 * ch + 4);
+            fb[u][0] = *reinterpret_cast<const float4 *>(F + F_B * 64 + 8 * ch);
+            fb[u][1] = *reinterpret_cast<const float4 *>(F + F_B * 64 + 8 * ch + 4);
+          }
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int ch = (pt >> 6) + 4 * u;
+            const float tv[8] = {t[u][0].x, t[u][0].y, t[u][0].z, t[u][0].w,
+                                 t[u][1].x, t[u][1].y, t[u][1].z, t[u][1].w};
+            const float gv[8] = {fg[u][0].x, fg[u][0].y, fg[u][0].z, fg[u][0].w,
+                                 fg[u][1].x, fg[u][1].y, fg[u][1].z, fg[u][1].w};
+            const float bv[8] = {fb[u][0].x, fb[u][0].y, fb[u][0].z, fb[u][0].w,
+                                 fb[u][1].x, fb[u][1].y, fb[u][1].z, fb[u][1].w};
+            uint32_t gw[4], hw[4], lw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              gw[e] = pack_bf16(tv[2 * e] * gv[2 * e], tv[2 * e + 1] * gv[2 * e + 1]);
+              const float b0 = tv[2 * e] * bv[2 * e], b1 = tv[2 * e + 1] * bv[2 * e + 1];
+              hw[e] = pack_bf16(b0, b1);
+              float h0, h1;
+              unpack_bf16(hw[e], h0, h1);
+              lw[e] = pack_bf16(b0 - h0, b1 - h1);
+            }
+            const uint32_t o = sw128_chunk(r, ch);
+            st_smem_v4(sm + Lay::TPG + o, gw[0], gw[1], gw[2], gw[3]);
+            st_smem_v4(sm + Lay::TPB + o, hw[0], hw[1], hw[2], hw[3]);
+            st_smem_v4(sm + Lay::TPB_LO + o, lw[0], lw[1], lw[2], lw[3]);
+          }
+        }
+        constexpr int kTiles = 1;
+#pragma unroll
+        for (int it = pt; GATE == 2 && it < kTiles * 512; it += kPrep) {
           const int r = it & 63, rb = r >> 4, ch = (it >> 6) & 7;
           const bool tb = (GATE == 2) || (it >> 9) == 1;   // T diag(b)
           const float *fac = F + (tb ? F_B : F_BG) * 64;
@@ -1035,16 +1092,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                      pack_f16(-v[8 * ch + 4], -v[8 * ch + 5]),
                      pack_f16(-v[8 * ch + 6], -v[8 * ch + 7]));
       }
-      for (int idx = pt; idx < kC * 16; idx += kPrep) {
+      if (GATE != 2) {
+        // raw bf16 -> fp16: Q times e^g, K times e^{g_C - g}.  All eight
+        // 16-byte chunks of a thread are loaded before any is stored, so
+        // their shared-memory latencies overlap.
+        constexpr int kIt = kC * 16 / kPrep;   // 4
+        uint4 xq[kIt], xk[kIt];
+        float eq[kIt], ek[kIt];
+        uint32_t off[kIt];
+#pragma unroll
+        for (int u = 0; u < kIt; ++u) {
+          const int idx = pt + u * kPrep;
+          const int r = idx >> 4, cc = idx & 15;
+          off[u] = (cc >> 3) * 16384 + sw128_chunk(r, cc & 7);
+          eq[u] = (GATE == 1) ? F[F_EG * 64 + r] : 1.f;
+          ek[u] = (GATE == 1) ? F[F_EK * 64 + r] : 1.f;
+          xq[u] = *reinterpret_cast<const uint4 *>(stg + off[u] + 8192);
+          xk[u] = *reinterpret_cast<const uint4 *>(stg + off[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kIt; ++u) {
+          uint32_t *wq = reinterpret_cast<uint32_t *>(&xq[u]);
+          uint32_t *wk = reinterpret_cast<uint32_t *>(&xk[u]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float a0, a1;
+            unpack_bf16(wq[e], a0, a1);
+            wq[e] = pack_f16(a0 * eq[u], a1 * eq[u]);
+            unpack_bf16(wk[e], a0, a1);
+            wk[e] = pack_f16(a0 * ek[u], a1 * ek[u]);
+          }
+          *reinterpret_cast<uint4 *>(stg + off[u] + 8192) = xq[u];
+          *reinterpret_cast<uint4 *>(stg + off[u]) = xk[u];
+        }
+      }
+      for (int idx = pt; GATE == 2 && idx < kC * 16; idx += kPrep) {
         const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
         uint8_t *kp = stg + kb * 16384 + sw128_chunk(r, cc & 7);
-        if (GATE != 2) {
-          // raw bf16 -> fp16: Q times e^g, K times e^{g_C - g}
-          const float eq = (GATE == 1) ? F[F_EG * 64 + r] : 1.f;
-          const float ek = (GATE == 1) ? F[F_EK * 64 + r] : 1.f;
-          bf16_to_f16_16B(kp + 8192, eq);
-          bf16_to_f16_16B(kp, ek);
-        } else {
+        {
           // K~ = (K e^{g_m-g}) e^{g_C-g_m}, per channel
           uint4 kv = *reinterpret_cast<const uint4 *>(
               sm + Lay::KN + kb * 8192 + sw128_chunk(r, cc & 7));
@@ -1054,8 +1139,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 4; ++e) {
             float a0, a1;
             unpack_bf16(kw[e], a0, a1);
-            kw[e] = pack_f16(a0 * __expf(gc[cbase + 2 * e] - gM[cbase + 2 * e]),
-                             a1 * __expf(gc[cbase + 2 * e + 1] - gM[cbase + 2 * e + 1]));
+            kw[e] = pack_f16(a0 * gM[128 + cbase + 2 * e],
+                             a1 * gM[128 + cbase + 2 * e + 1]);
           }
           *reinterpret_cast<uint4 *>(kp) = kv;
         }
