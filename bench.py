@@ -429,6 +429,128 @@ def run_ours(args, w):
     return 0
 
 
+DECODE_METRIC = ("tokens/s, single-token decode step (gdr_decode_step), GDN "
+                 "H16 d128 bf16, state resident in HBM; % HBM roofline")
+
+
+def decode_bytes(N, H, dk, dv, esz, gate):
+    """Bytes a decode step must move: the state read and written once (fp32),
+    q, k, v, out in the I/O dtype, beta and log-alpha in fp32."""
+    per = 2 * dk * dv * 4 + esz * (2 * dk + 2 * dv) + 4
+    per += {"none": 0, "scalar": 4, "channel": 4 * dk}[gate]
+    return N * H * per
+
+
+def run_decode(args):
+    """One decode step per sequence per timed step: N sequences x H heads,
+    the state updated in place in HBM (256 MiB at the default size, larger
+    than L2, so no flush is needed)."""
+    import torch
+
+    import chunkwise_recurrence_b200 as gdr
+    from chunkwise_recurrence_b200.inputs import Workload, generate
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        raise SystemExit("--decode runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    N, H, d = args.decode_seqs, 16, 128
+    w = Workload("gdn_decode_h16_d128_bf16", B=N, T=1, H=H, dk=d, dv=d,
+                 chunk=16, dtype="bf16", gate="scalar", decay_lo=0.01,
+                 decay_hi=0.1, init_state=True)
+    inp = generate(w, seed=args.seed)
+    sq = lambda t: t[:, 0].contiguous()  # noqa: E731
+    hq, hk, hv = sq(inp.q), sq(inp.k), sq(inp.v)
+    hb, hla = sq(inp.beta), sq(inp.log_alpha)
+    q, k, v, b, la = (t.to(dev) for t in (hq, hk, hv, hb, hla))
+    state = inp.s0.to(dev)
+    out = torch.empty_like(v)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gdr.decode_step(q, k, v, b, la, state, out=out, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_gpu_index(local)) as clocks:
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    # end to end: the step's token inputs come from pinned host memory and
+    # its outputs go back; the state stays resident on the device
+    pin = lambda t: t.pin_memory()  # noqa: E731
+    pq, pk, pv, pb, pla = (pin(t) for t in (hq, hk, hv, hb, hla))
+    pout = torch.empty_like(hv).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (pq, pk, pv, pb, pla))
+    d2h = pout.numel() * pout.element_size()
+
+    def e2e_step():
+        for dst, src in ((q, pq), (k, pk), (v, pv), (b, pb), (la, pla)):
+            dst.copy_(src, non_blocking=True)
+        step()
+        pout.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    ea, eb = (torch.cuda.Event(enable_timing=True),
+              torch.cuda.Event(enable_timing=True))
+    ea.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    eb.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ea.elapsed_time(eb)
+    ms = total_ms / args.steps
+    by = decode_bytes(N, H, d, d, 2, "scalar")
+    peaks, peak_src = load_peaks()
+    kernel_ms = statistics.mean(per_step)
+    gbs = by / (kernel_ms / 1e3) / 1e9
+    line = {
+        "metric": DECODE_METRIC, "value": N / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "sequences": N, "H": H, "dk": d,
+                   "dv": d, "gate": "scalar",
+                   "l2": f"state {N * H * d * d * 4 >> 20} MiB > L2 (no flush)"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                     "traffic": None, "peak_source": peak_src,
+                     "kernel": "gdr_decode_kernel",
+                     "algorithmic_bytes_per_launch": by},
+        "clocks": clocks.summary(),
+        "e2e": {"value": N * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "entry": "gdr_decode_step, token inputs from pinned host "
+                         "memory, state resident"},
+        "gpu_launches": args.steps,
+        "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
+    }
+    if not args.no_cpu_baseline:
+        import oracle
+        ns = min(N, 32)
+        f = lambda t: t[:ns].double().numpy()  # noqa: E731
+        t0 = time.perf_counter()
+        oracle.decode_step(f(hq), f(hk), f(hv), f(hb), f(hla), gate="scalar",
+                           state=f(inp.s0))
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {
+            "value": ns / dt, "unit": "tokens/s", "cores": cpu_cores(),
+            "kind": "oracle",
+            "sample": f"sequences 0..{ns - 1} of {N} (x {H} heads), one step"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def gdr_fused_available():
     from chunkwise_recurrence_b200 import fused_tc_available
     return fused_tc_available()
@@ -459,10 +581,16 @@ def main(argv=None):
     ap.add_argument("--ref-seqs", type=int, default=2,
                     help="sequences per step in the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the single-token decode step instead")
+    ap.add_argument("--decode-seqs", type=int, default=256,
+                    help="sequences per decode step")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
+    if args.decode and args.impl == "ours":
+        return run_decode(args)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

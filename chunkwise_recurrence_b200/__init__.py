@@ -14,7 +14,7 @@ import os
 
 import torch
 
-__all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_noalloc",
+__all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_noalloc", "decode_step",
            "device_error", "status_string",
            "algo_applies", "fused_tc_available",
            "GdrError", "load_library", "LIB_PATH", "GATES", "ALGOS",
@@ -31,7 +31,7 @@ STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARGUMENT", 2: "GDR_ERR_UNSUPPORTED",
           6: "GDR_ERR_RANGE"}
 EXPORTED_SYMBOLS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_device_error",
                     "gdr_algo_applies", "gdr_status_string",
-                    "gdr_chunk_fwd_noalloc")
+                    "gdr_chunk_fwd_noalloc", "gdr_decode_step")
 # size of the static scratch array behind gdr_chunk_fwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -67,6 +67,9 @@ def load_library(path: str = LIB_PATH):
         f.restype = ctypes.c_int
         f.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, vp,
                       ctypes.POINTER(_Opts)]
+    lib.gdr_decode_step.restype = ctypes.c_int
+    lib.gdr_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i,
+                                    vp, ctypes.POINTER(_Opts)]
     lib.gdr_device_error.restype = ctypes.c_int
     lib.gdr_device_error.argtypes = [vp, i]
     lib.gdr_algo_applies.restype = ctypes.c_int
@@ -196,6 +199,42 @@ def chunk_fwd_host(q, k, v, beta, log_alpha=None, initial_state=None, *,
     if rc != 0:
         raise GdrError(rc, "gdr_chunk_fwd_host")
     return out, final_state
+
+
+def decode_step(q, k, v, beta, log_alpha=None, state=None, *, out=None,
+                state_out=None, gate: str | None = None, stream=None):
+    """Run ``gdr_decode_step`` on CUDA tensors: one token per (sequence, head).
+
+    q, k [N, H, dk]; v [N, H, dv]; beta [N, H]; log_alpha [N, H] (scalar
+    gate), [N, H, dk] (channel gate) or None; state [N, H, dk, dv] fp32 or
+    None (zero).  ``state_out`` defaults to ``state`` itself (an in-place
+    update) when a state is given, else a new tensor.  Returns
+    (out [N, H, dv], state_out).
+    """
+    lib = load_library()
+    if q.dim() != 3 or v.dim() != 3:
+        raise ValueError("q, k, v must be [N, H, d]")
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty_like(v)
+    if state_out is None:
+        state_out = state if state is not None else torch.empty(
+            N, H, dk, dv, dtype=torch.float32, device=q.device)
+    g = gate if gate is not None else (
+        "none" if log_alpha is None else
+        "scalar" if log_alpha.dim() == 2 else "channel")
+    opts = _Opts(DTYPES[q.dtype], GATES[g], None, 0, ALGOS["auto"])
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    rc = lib.gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                             _ptr(beta), _ptr(state), _ptr(state_out),
+                             _ptr(out), N, H, dk, dv,
+                             ctypes.c_void_p(stream.cuda_stream),
+                             ctypes.byref(opts))
+    if rc != 0:
+        raise GdrError(rc, "gdr_decode_step")
+    return out, state_out
 
 
 def device_error(stream=None, clear: bool = True) -> int:

@@ -1,0 +1,237 @@
+// Single-token decode step of libgdr: the recurrent update of a resident
+// state, one token per (sequence, head).
+//
+// Per (sequence, head), with the state S (dk x dv, fp32) and one token:
+//   S~ = D S                   D = I, alpha I or diag(alpha)
+//   r  = S~^T k,  u = beta (v - r)
+//   S' = S~ + k u^T            (= (I - beta k k^T) D S + beta k v^T)
+//   o  = S'^T q = S~^T q + u (k . q)
+// This is the delta rule's one-token step ("DeltaTTT: Layerwise Optimization
+// for Nonlinear Recurrent Memory", §2 Background and §4.1); decoding runs it
+// once per generated token with the state read and written back each time
+// ("Delta-Rule Linear Attention" topic page, GDN decode-accelerator card: one
+// state read and one state write per token, under 1 FLOP per byte).
+//
+// The step moves 2 dk dv 4 bytes of state per (sequence, head) against about
+// 6 dk dv flops, so it is bound by HBM bandwidth.  One CTA of 256 threads per
+// (sequence, head): warp w owns rows [w dk/8, (w+1) dk/8) of S, lane l owns
+// columns [4l, 4l+4), so every load and store of S is a 16-byte access and a
+// warp covers whole 512-byte rows.  S is read once into registers, the two
+// column reductions (S~^T k, S~^T q) go through shared memory, and S' is
+// written back from the same registers: one read and one write of the state.
+// In place (state_in == state_out) is safe: every element is read and written
+// by the same thread.
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "gdr_internal.h"
+
+namespace gdr {
+namespace {
+
+constexpr int kDecThreads = 256;
+
+struct DecodeParams {
+  const void *q, *k, *v;
+  const float *log_alpha, *beta, *s_in;
+  float *s_out;
+  void *out;
+  int dv;
+};
+
+template <typename T>
+__device__ __forceinline__ float ld1(const T *p);
+template <>
+__device__ __forceinline__ float ld1<float>(const float *p) {
+  return *p;
+}
+template <>
+__device__ __forceinline__ float ld1<__nv_bfloat16>(const __nv_bfloat16 *p) {
+  return __bfloat162float(*p);
+}
+// four consecutive elements (8- or 16-byte aligned)
+__device__ __forceinline__ float4 ld4(const float *p) {
+  return *reinterpret_cast<const float4 *>(p);
+}
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
+  const uint2 w = *reinterpret_cast<const uint2 *>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ void st4(float *p, float4 x) {
+  *reinterpret_cast<float4 *>(p) = x;
+}
+__device__ __forceinline__ void st4(__nv_bfloat16 *p, float4 x) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(x.z, x.w);
+  uint2 w;
+  w.x = *reinterpret_cast<const uint32_t *>(&a);
+  w.y = *reinterpret_cast<const uint32_t *>(&b);
+  *reinterpret_cast<uint2 *>(p) = w;
+}
+__device__ __forceinline__ float4 fma4(float s, float4 a, float4 b) {
+  return make_float4(fmaf(s, a.x, b.x), fmaf(s, a.y, b.y), fmaf(s, a.z, b.z),
+                     fmaf(s, a.w, b.w));
+}
+
+template <int DK, typename T, int GATE>
+__global__ void __launch_bounds__(kDecThreads)
+    gdr_decode_kernel(DecodeParams p) {
+  constexpr int R = DK / 8;   // rows of S per warp
+  __shared__ float sk[DK], sq[DK], sa[DK];
+  __shared__ float4 red[2][8][32];   // per warp: partial S~^T k, S~^T q
+  __shared__ float kq_s;
+  const int nh = blockIdx.x;         // (sequence, head), flattened
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int dv = p.dv, j0 = 4 * lane;
+  const bool act = j0 < dv;
+  const T *q = static_cast<const T *>(p.q) + (size_t)nh * DK;
+  const T *k = static_cast<const T *>(p.k) + (size_t)nh * DK;
+  for (int c = threadIdx.x; c < DK; c += kDecThreads) {
+    sk[c] = ld1(k + c);
+    sq[c] = ld1(q + c);
+    sa[c] = GATE == 0   ? 1.f
+            : GATE == 1 ? __expf(p.log_alpha[nh])
+                        : __expf(p.log_alpha[(size_t)nh * DK + c]);
+  }
+  __syncthreads();
+  // S~ = D S for this thread's rows and columns; partial column reductions
+  const size_t sb = (size_t)nh * DK * dv;
+  float4 S[R];
+  float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int c = warp * R + r;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (act && p.s_in) x = ld4(p.s_in + sb + (size_t)c * dv + j0);
+    const float a = sa[c];
+    x = make_float4(a * x.x, a * x.y, a * x.z, a * x.w);
+    S[r] = x;
+    pk = fma4(sk[c], x, pk);
+    pq = fma4(sq[c], x, pq);
+  }
+  red[0][warp][lane] = pk;
+  red[1][warp][lane] = pq;
+  if (warp == 0) {
+    float t = 0.f;
+    for (int c = lane; c < DK; c += 32) t = fmaf(sk[c], sq[c], t);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+      t += __shfl_xor_sync(0xffffffffu, t, off);
+    if (lane == 0) kq_s = t;
+  }
+  __syncthreads();
+  if (!act) return;
+  float4 rk = red[0][0][lane], rq = red[1][0][lane];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) {
+    const float4 a = red[0][w][lane], b = red[1][w][lane];
+    rk = make_float4(rk.x + a.x, rk.y + a.y, rk.z + a.z, rk.w + a.w);
+    rq = make_float4(rq.x + b.x, rq.y + b.y, rq.z + b.z, rq.w + b.w);
+  }
+  // u = beta (v - S~^T k); o = S~^T q + u (k . q)
+  const float bt = p.beta[nh];
+  const float4 vv = ld4(static_cast<const T *>(p.v) + (size_t)nh * dv + j0);
+  const float4 u = make_float4(bt * (vv.x - rk.x), bt * (vv.y - rk.y),
+                               bt * (vv.z - rk.z), bt * (vv.w - rk.w));
+  if (warp == 0)
+    st4(static_cast<T *>(p.out) + (size_t)nh * dv + j0, fma4(kq_s, u, rq));
+  // S' = S~ + k u^T
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int c = warp * R + r;
+    st4(p.s_out + sb + (size_t)c * dv + j0, fma4(sk[c], u, S[r]));
+  }
+}
+
+template <int DK, typename T>
+cudaError_t launch_dk(const DecodeParams &dp, int gate, int nblocks,
+                      cudaStream_t s) {
+  switch (gate) {
+    case 0: gdr_decode_kernel<DK, T, 0><<<nblocks, kDecThreads, 0, s>>>(dp); break;
+    case 1: gdr_decode_kernel<DK, T, 1><<<nblocks, kDecThreads, 0, s>>>(dp); break;
+    default: gdr_decode_kernel<DK, T, 2><<<nblocks, kDecThreads, 0, s>>>(dp); break;
+  }
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_t(const DecodeParams &dp, int dk, int gate, int nblocks,
+                     cudaStream_t s) {
+  switch (dk) {
+    case 16: return launch_dk<16, T>(dp, gate, nblocks, s);
+    case 32: return launch_dk<32, T>(dp, gate, nblocks, s);
+    case 64: return launch_dk<64, T>(dp, gate, nblocks, s);
+    default: return launch_dk<128, T>(dp, gate, nblocks, s);
+  }
+}
+
+bool aligned16(const void *p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+bool dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+}  // namespace
+}  // namespace gdr
+
+extern "C" gdr_status gdr_decode_step(const void *q, const void *k,
+                                      const void *v, const float *log_alpha,
+                                      const float *beta,
+                                      const float *state_in, float *state_out,
+                                      void *out, int N, int H, int dk, int dv,
+                                      cudaStream_t stream,
+                                      const gdr_opts *opts) {
+  gdr_opts o;
+  o.dtype = GDR_BF16;
+  o.gate = GDR_GATE_SCALAR;
+  o.cu_seqlens = nullptr;
+  o.num_seqs = 0;
+  o.algo = GDR_ALGO_AUTO;
+  if (opts) o = *opts;
+  if (N < 0 || H < 0) return GDR_ERR_INVALID_ARGUMENT;
+  if (o.dtype != GDR_BF16 && o.dtype != GDR_FP32) return GDR_ERR_INVALID_ARGUMENT;
+  if (o.gate != GDR_GATE_NONE && o.gate != GDR_GATE_SCALAR &&
+      o.gate != GDR_GATE_CHANNEL)
+    return GDR_ERR_INVALID_ARGUMENT;
+  if (o.cu_seqlens != nullptr || o.num_seqs != 0)
+    return GDR_ERR_INVALID_ARGUMENT;   // one token per sequence: no packing
+  if (o.algo != GDR_ALGO_AUTO) return GDR_ERR_UNSUPPORTED;
+  if (!gdr::dim_ok(dk) || !gdr::dim_ok(dv)) return GDR_ERR_UNSUPPORTED;
+  if ((o.gate == GDR_GATE_NONE) != (log_alpha == nullptr))
+    return GDR_ERR_INVALID_ARGUMENT;
+  const long long nh = (long long)N * H;
+  if (nh > 0x7fffffffLL) return GDR_ERR_UNSUPPORTED;
+  if (nh == 0) return GDR_OK;
+  if (!q || !k || !v || !beta || !state_out || !out)
+    return GDR_ERR_INVALID_ARGUMENT;
+  const void *ptrs[] = {q, k, v, log_alpha, beta, state_in, state_out, out};
+  for (const void *ptr : ptrs)
+    if (ptr && !gdr::aligned16(ptr)) return GDR_ERR_INVALID_ARGUMENT;
+  // state_in and state_out: the same buffer (in-place update) or disjoint
+  if (state_in && state_in != state_out) {
+    const size_t bytes = (size_t)nh * dk * dv * sizeof(float);
+    const uintptr_t a = reinterpret_cast<uintptr_t>(state_in);
+    const uintptr_t b = reinterpret_cast<uintptr_t>(state_out);
+    if (a < b + bytes && b < a + bytes) return GDR_ERR_INVALID_ARGUMENT;
+  }
+  gdr::DecodeParams dp;
+  dp.q = q;
+  dp.k = k;
+  dp.v = v;
+  dp.log_alpha = log_alpha;
+  dp.beta = beta;
+  dp.s_in = state_in;
+  dp.s_out = state_out;
+  dp.out = out;
+  dp.dv = dv;
+  const int nb = (int)nh;
+  const cudaError_t e =
+      o.dtype == GDR_BF16
+          ? gdr::launch_t<__nv_bfloat16>(dp, dk, o.gate, nb, stream)
+          : gdr::launch_t<float>(dp, dk, o.gate, nb, stream);
+  return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}

@@ -219,6 +219,44 @@ GDR_API gdr_status gdr_chunk_fwd_noalloc(const void *q, const void *k,
                                          const gdr_opts *opts);
 
 /*
+ * gdr_decode_step -- one token per (sequence, head): the recurrent update of
+ * a resident state, as used when generating one token at a time after a
+ * forward pass over the prompt.
+ *
+ * The operation is the recurrence above for a single token t (DeltaTTT page,
+ * §2 Background and §4.1: the delta rule's one-token gradient step; "Delta-
+ * Rule Linear Attention" topic page, GDN decode-accelerator card: decoding
+ * reads and writes the whole recurrent state once per token, at under one
+ * flop per byte):
+ *     S' = (I - beta k k^T) D S + beta k v^T,    o = S'^T q
+ *
+ * Device pointers, row-major and contiguous, 16-byte aligned:
+ *   q, k        [N][H][dk]   dtype
+ *   v           [N][H][dv]   dtype
+ *   log_alpha   NULL (GDR_GATE_NONE), [N][H] (SCALAR) or [N][H][dk]
+ *               (CHANNEL), fp32
+ *   beta        [N][H] fp32
+ *   state_in    [N][H][dk][dv] fp32, or NULL for a zero state
+ *   state_out   [N][H][dk][dv] fp32 (written).  It may be the same buffer as
+ *               state_in (the state is then updated in place); otherwise the
+ *               two must not overlap (GDR_ERR_INVALID_ARGUMENT).
+ *   out         [N][H][dv]   dtype (written)
+ *
+ * Sizes: N, H >= 0 (N * H == 0 is a no-op returning GDR_OK), N * H < 2^31;
+ * dk, dv in {16, 32, 64, 128}.  opts may be NULL (bf16, scalar gate);
+ * opts->cu_seqlens must be NULL and opts->num_seqs 0 (one token per
+ * sequence: nothing to pack), opts->algo must be GDR_ALGO_AUTO.
+ * Arithmetic is fp32.  One kernel launch, no scratch memory, no device-side
+ * waits.  Returns GDR_ERR_INVALID_ARGUMENT / GDR_ERR_UNSUPPORTED as described,
+ * GDR_ERR_CUDA if the launch fails.
+ */
+GDR_API gdr_status gdr_decode_step(const void *q, const void *k, const void *v,
+                                   const float *log_alpha, const float *beta,
+                                   const float *state_in, float *state_out,
+                                   void *out, int N, int H, int dk, int dv,
+                                   cudaStream_t stream, const gdr_opts *opts);
+
+/*
  * gdr_device_error -- synchronise `stream`, then read (and clear if `clear`)
  * the library's sticky device-side error word for the current device.
  * Returns GDR_OK if no kernel has reported an error, GDR_ERR_TIMEOUT if a

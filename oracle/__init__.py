@@ -8,6 +8,8 @@ Contents
 --------
 ``gdr_fwd``          the plain token-by-token recurrence (C, fp64, threaded over
                      independent (sequence, head) chains) -- the oracle proper.
+``decode_step``      one token per (sequence, head): the same recurrence for a
+                     single token, applied to a given state.
 ``chunkwise_ref``    an independent fp64 chunkwise reformulation that solves the
                      intra-chunk triangular system with a dense ``solve``; it is a
                      pin for the token loop, not a second oracle for the GPU.
@@ -129,6 +131,25 @@ def gdr_fwd(q, k, v, beta, log_alpha=None, gate="scalar", initial_state=None,
     if rc < 0:
         raise ValueError(f"oracle_gdr_fwd rejected its arguments (code {rc})")
     return out, sT, rc
+
+
+def decode_step(q, k, v, beta, log_alpha=None, gate="scalar", state=None,
+                lib=None):
+    """One token per (sequence, head): the recurrence for a single token.
+
+    q, k [N, H, dk]; v [N, H, dv]; beta [N, H]; log_alpha [N, H] (scalar
+    gate), [N, H, dk] (channel gate) or None; state [N, H, dk, dv] or None.
+    Returns (out [N, H, dv], new state [N, H, dk, dv]).  Decoding applies the
+    delta rule's one-token step once per generated token ("Delta-Rule Linear
+    Attention" topic page, GDN decode-accelerator card); it is the token loop
+    above with one token per sequence, so it reuses it.
+    """
+    q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
+    la = _f64(log_alpha)
+    ex = lambda a: None if a is None else a[:, None]  # noqa: E731  [N,1,...]
+    out, sT, _ = gdr_fwd(ex(q), ex(k), ex(v), ex(beta), ex(la), gate=gate,
+                         initial_state=state, lib=lib)
+    return out[:, 0], sT
 
 
 from .chunkwise_ref import chunkwise_ref  # noqa: E402  (re-export)

@@ -129,6 +129,41 @@ def test_product_never_imports_the_oracle():
                 assert "gdr_oracle" not in text and "liboracle" not in text, f
 
 
+def dcall(lib, *, q=A, k=A, v=A, la=A, beta=A, sin=None, sout=A, out=A, N=4,
+          H=2, dk=128, dv=128, dtype=0, gate=1, cu=None, nseq=0, algo=0):
+    opts = gdr._Opts(dtype, gate, cu, nseq, algo)
+    return lib.gdr_decode_step(q, k, v, la, beta, sin, sout, out, N, H, dk, dv,
+                               None, ctypes.byref(opts))
+
+
+def test_decode_step_rejects_bad_arguments(lib):
+    c = lambda **kw: dcall(lib, **kw)  # noqa: E731
+    assert c(q=None) == INVALID
+    assert c(sout=None) == INVALID                 # the state is written
+    assert c(out=None) == INVALID
+    assert c(v=A + 8) == INVALID                   # misaligned
+    assert c(sin=A + 4) == INVALID
+    assert c(la=None) == INVALID
+    assert c(gate=0) == INVALID
+    assert c(gate=3) == INVALID
+    assert c(dtype=2) == INVALID
+    assert c(N=-1) == INVALID
+    assert c(cu=A) == INVALID                      # nothing to pack
+    assert c(nseq=2) == INVALID
+    assert c(algo=1) == UNSUPPORTED
+    assert c(dk=48) == UNSUPPORTED
+    assert c(dv=8) == UNSUPPORTED
+    assert c(N=1 << 20, H=1 << 12) == UNSUPPORTED  # N * H >= 2^31
+    # partially overlapping input and output states (4*2*128*128*4 bytes)
+    assert c(sin=A, sout=A + 4096) == INVALID
+    assert c(sin=A + 4096, sout=A) == INVALID
+    # no pointer is touched and no CUDA call is made for an empty batch
+    assert c(q=None, k=None, v=None, la=None, beta=None, sout=None, out=None,
+             gate=0, N=0) == OK
+    assert c(q=None, k=None, v=None, la=None, beta=None, sout=None, out=None,
+             gate=0, H=0) == OK
+
+
 def test_algo_applies(lib):
     assert gdr.algo_applies("staged", "fp32", "none", 16, 16, 16)
     assert gdr.algo_applies("auto", "bf16", "channel", 128, 64, 32)

@@ -308,6 +308,59 @@ def test_varlen_equals_separate(oracle_lib):
     assert np.allclose(o2, o, atol=1e-11) and np.allclose(s2, s, atol=1e-11)
 
 
+def test_decode_step_chains_to_the_sequence(oracle_lib):
+    """One-token steps, each handing its state to the next, reproduce the
+    token loop over the whole sequence: outputs and final state (this is what
+    the decode wrapper's reshaping and state handling must preserve)."""
+    rng = np.random.default_rng(11)
+    for gate in ("none", "scalar", "channel"):
+        case = _rand_case(rng, B=3, T=6, H=2, dk=4, dv=3, gate=gate)
+        out, sT, _ = gdr_fwd(**case, lib=oracle_lib)
+        S = case["initial_state"]
+        for t in range(case["q"].shape[1]):
+            la = None if case["log_alpha"] is None else case["log_alpha"][:, t]
+            o, S = oracle.decode_step(case["q"][:, t], case["k"][:, t],
+                                      case["v"][:, t], case["beta"][:, t], la,
+                                      gate=gate, state=S, lib=oracle_lib)
+            np.testing.assert_allclose(o, out[:, t], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(S, sT, rtol=0, atol=1e-13)
+
+
+def test_decode_step_special_cases(oracle_lib):
+    """beta = 0: the step only decays the state, S' = D S and o = (D S)^T q.
+    alpha = beta = 1 from a zero state: one write of (k, v) with a unit key
+    stores v, so reading with q = k returns v exactly (DeltaTTT page, §2: the
+    delta rule corrects the memory's read of the current key to its value)."""
+    rng = np.random.default_rng(12)
+    N, H, dk, dv = 3, 2, 5, 4
+    for gate in ("none", "scalar", "channel"):
+        q = rng.standard_normal((N, H, dk))
+        k = rng.standard_normal((N, H, dk))
+        v = rng.standard_normal((N, H, dv))
+        S = rng.standard_normal((N, H, dk, dv))
+        la = None if gate == "none" else -rng.uniform(
+            0.1, 1.0, size=(N, H) if gate == "scalar" else (N, H, dk))
+        o, S1 = oracle.decode_step(q, k, v, np.zeros((N, H)), la, gate=gate,
+                                   state=S, lib=oracle_lib)
+        for n in range(N):
+            for h in range(H):
+                if gate == "none":
+                    D = np.eye(dk)
+                elif gate == "scalar":
+                    D = np.exp(la[n, h]) * np.eye(dk)
+                else:
+                    D = np.diag(np.exp(la[n, h]))
+                np.testing.assert_allclose(S1[n, h], D @ S[n, h], atol=1e-13)
+                np.testing.assert_allclose(o[n, h], (D @ S[n, h]).T @ q[n, h],
+                                           atol=1e-12)
+    kk = rng.standard_normal((N, H, dk))
+    kk /= np.linalg.norm(kk, axis=-1, keepdims=True)
+    v = rng.standard_normal((N, H, dv))
+    o, _ = oracle.decode_step(kk, kk, v, np.ones((N, H)), None, gate="none",
+                              state=None, lib=oracle_lib)
+    np.testing.assert_allclose(o, v, atol=1e-13)
+
+
 def test_thread_count_does_not_change_bits(oracle_lib):
     rng = np.random.default_rng(10)
     c = _rand_case(rng, B=3, T=15, H=5, dk=4, dv=4, gate="channel")
