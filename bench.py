@@ -68,7 +68,8 @@ def load_peaks():
 
 def kernel_source_hash(algo):
     files = {"fused_tc": ["fused_tc.cu"],
-             "staged": ["staged.cu"]}.get(algo, [])
+             "staged": ["staged.cu"],
+             "decode": ["decode.cu"]}.get(algo, [])
     h = hashlib.sha256()
     for f in files:
         h.update(open(os.path.join(ROOT, "chunkwise_recurrence_b200", "csrc",
@@ -524,7 +525,9 @@ def run_decode(args):
                    "l2": f"state {N * H * d * d * 4 >> 20} MiB > L2 (no flush)"},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
-                     "traffic": None, "peak_source": peak_src,
+                     "traffic": recorded_traffic(
+                         f"decode_{w.name}.md", kernel_source_hash("decode")),
+                     "peak_source": peak_src,
                      "kernel": "gdr_decode_kernel",
                      "algorithmic_bytes_per_launch": by},
         "clocks": clocks.summary(),
