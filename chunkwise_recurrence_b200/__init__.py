@@ -15,6 +15,7 @@ import os
 import torch
 
 __all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_noalloc", "decode_step",
+           "efla_beta",
            "device_error", "status_string",
            "algo_applies", "fused_tc_available",
            "GdrError", "load_library", "LIB_PATH", "GATES", "ALGOS",
@@ -31,7 +32,8 @@ STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARGUMENT", 2: "GDR_ERR_UNSUPPORTED",
           6: "GDR_ERR_RANGE"}
 EXPORTED_SYMBOLS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_device_error",
                     "gdr_algo_applies", "gdr_status_string",
-                    "gdr_chunk_fwd_noalloc", "gdr_decode_step")
+                    "gdr_chunk_fwd_noalloc", "gdr_decode_step",
+                    "gdr_efla_beta")
 # size of the static scratch array behind gdr_chunk_fwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -70,6 +72,8 @@ def load_library(path: str = LIB_PATH):
     lib.gdr_decode_step.restype = ctypes.c_int
     lib.gdr_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i,
                                     vp, ctypes.POINTER(_Opts)]
+    lib.gdr_efla_beta.restype = ctypes.c_int
+    lib.gdr_efla_beta.argtypes = [vp, fp, fp, i, i, i, i, vp]
     lib.gdr_device_error.restype = ctypes.c_int
     lib.gdr_device_error.argtypes = [vp, i]
     lib.gdr_algo_applies.restype = ctypes.c_int
@@ -235,6 +239,27 @@ def decode_step(q, k, v, beta, log_alpha=None, state=None, *, out=None,
     if rc != 0:
         raise GdrError(rc, "gdr_decode_step")
     return out, state_out
+
+
+def efla_beta(k, beta, *, out=None, stream=None):
+    """Run ``gdr_efla_beta``: the exact-flow step size
+    beta' = (1 - exp(-beta |k|^2)) / |k|^2 for keys k [..., H, dk] and beta
+    [..., H] (CUDA tensors; ``out`` may be ``beta`` for an in-place update).
+    Passing beta' to ``chunk_fwd`` or ``decode_step`` runs the EFLA
+    recurrence."""
+    lib = load_library()
+    dk = k.shape[-1]
+    H = k.shape[-2]
+    ntok = k.numel() // (H * dk)
+    if out is None:
+        out = torch.empty_like(beta)
+    if stream is None:
+        stream = torch.cuda.current_stream(k.device)
+    rc = lib.gdr_efla_beta(_ptr(k), _ptr(beta), _ptr(out), ntok, H, dk,
+                           DTYPES[k.dtype], ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise GdrError(rc, "gdr_efla_beta")
+    return out
 
 
 def device_error(stream=None, clear: bool = True) -> int:

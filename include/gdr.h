@@ -257,6 +257,28 @@ GDR_API gdr_status gdr_decode_step(const void *q, const void *k, const void *v,
                                    cudaStream_t stream, const gdr_opts *opts);
 
 /*
+ * gdr_efla_beta -- exact-flow step size (EFLA) for the delta rule.
+ *
+ * The delta rule's update is one explicit Euler step of length beta of the
+ * flow dS/dtau = -k k^T S + k v^T; EFLA takes the exact flow instead, which
+ * for these rank-1 dynamics has the same form ("Delta-Rule Linear Attention"
+ * topic page, EFLA card).  Reading taken (the card prints no formula): the
+ * exact step is the delta rule with step size
+ *     beta'[t][h] = (1 - exp(-beta[t][h] * |k[t][h]|^2)) / |k[t][h]|^2
+ * (beta' = beta where |k| = 0), applied after the decay as usual.  Running
+ * gdr_chunk_fwd or gdr_decode_step with beta' in place of beta gives the
+ * EFLA recurrence with every gate kind.
+ *
+ * Device pointers, 16-byte aligned: k [ntok][H][dk] in `dtype`, beta and
+ * beta_out [ntok][H] fp32.  beta_out may be beta itself (in place);
+ * otherwise the two must not overlap.  dk in {16, 32, 64, 128};
+ * ntok * H == 0 is a no-op.  One launch on `stream`, no scratch.
+ */
+GDR_API gdr_status gdr_efla_beta(const void *k, const float *beta,
+                                 float *beta_out, int ntok, int H, int dk,
+                                 gdr_dtype dtype, cudaStream_t stream);
+
+/*
  * gdr_device_error -- synchronise `stream`, then read (and clear if `clear`)
  * the library's sticky device-side error word for the current device.
  * Returns GDR_OK if no kernel has reported an error, GDR_ERR_TIMEOUT if a

@@ -10,6 +10,9 @@ Contents
                      independent (sequence, head) chains) -- the oracle proper.
 ``decode_step``      one token per (sequence, head): the same recurrence for a
                      single token, applied to a given state.
+``efla_fwd``         the exact-flow (EFLA) variant: each token's update is the
+                     exact flow of the delta rule's dynamics, integrated with a
+                     matrix exponential (small cases only).
 ``chunkwise_ref``    an independent fp64 chunkwise reformulation that solves the
                      intra-chunk triangular system with a dense ``solve``; it is a
                      pin for the token loop, not a second oracle for the GPU.
@@ -153,3 +156,4 @@ def decode_step(q, k, v, beta, log_alpha=None, gate="scalar", state=None,
 
 
 from .chunkwise_ref import chunkwise_ref  # noqa: E402  (re-export)
+from .efla_ref import efla_fwd  # noqa: E402  (re-export)

@@ -164,6 +164,18 @@ def test_decode_step_rejects_bad_arguments(lib):
              gate=0, H=0) == OK
 
 
+def test_efla_beta_rejects_bad_arguments(lib):
+    f = lambda k=A, b=A, o=A + 4096, ntok=8, H=2, dk=64, dt=0: \
+        lib.gdr_efla_beta(k, b, o, ntok, H, dk, dt, None)  # noqa: E731
+    assert f(k=None) == INVALID
+    assert f(b=A + 4) == INVALID        # misaligned
+    assert f(o=A + 16) == INVALID       # overlaps beta (8 x 2 floats)
+    assert f(dt=3) == INVALID
+    assert f(ntok=-1) == INVALID
+    assert f(dk=48) == UNSUPPORTED
+    assert f(k=None, b=None, o=None, ntok=0) == OK   # empty: no-op
+
+
 def test_algo_applies(lib):
     assert gdr.algo_applies("staged", "fp32", "none", 16, 16, 16)
     assert gdr.algo_applies("auto", "bf16", "channel", 128, 64, 32)

@@ -361,6 +361,52 @@ def test_decode_step_special_cases(oracle_lib):
     np.testing.assert_allclose(o, v, atol=1e-13)
 
 
+def _efla_step_size(k, beta):
+    lam = np.sum(np.asarray(k) ** 2, axis=-1)
+    return np.where(lam > 0, -np.expm1(-beta * lam) / np.where(lam > 0, lam, 1),
+                    beta)
+
+
+def test_efla_flow_is_the_delta_rule_with_a_new_step_size(oracle_lib):
+    """The exact flow, integrated by a matrix exponential (oracle.efla_fwd),
+    equals the delta rule run with beta' = (1 - e^{-beta |k|^2}) / |k|^2 --
+    the closed form the library's gdr_efla_beta computes -- for every gate,
+    with unnormalised keys too."""
+    rng = np.random.default_rng(21)
+    for gate in ("none", "scalar", "channel"):
+        case = _rand_case(rng, B=2, T=7, H=2, dk=4, dv=3, gate=gate)
+        case["k"] = case["k"] * rng.uniform(0.3, 2.0, size=case["k"].shape[:-1]
+                                            + (1,))
+        case["beta"] = case["beta"] * 3.0
+        ro, rs = oracle.efla_fwd(**case)
+        bp = _efla_step_size(case["k"], case["beta"])
+        o, sT, _ = gdr_fwd(**{**case, "beta": bp}, lib=oracle_lib)
+        np.testing.assert_allclose(o, ro, atol=1e-10)
+        np.testing.assert_allclose(sT, rs, atol=1e-10)
+
+
+def test_efla_limits():
+    """Small steps: the exact flow and one Euler step (the delta rule) agree
+    to first order in beta.  Long flow with a unit key: the memory converges
+    to the least-squares solution, so reading the key returns the value."""
+    rng = np.random.default_rng(22)
+    dk, dv = 5, 3
+    k = rng.standard_normal((1, 1, 1, dk))
+    k /= np.linalg.norm(k)
+    v = rng.standard_normal((1, 1, 1, dv))
+    S0 = rng.standard_normal((1, 1, dk, dv))
+    for b in (1e-3, 1e-4):
+        _, se = oracle.efla_fwd(k, k, v, np.full((1, 1, 1), b), gate="none",
+                                initial_state=S0)
+        euler = S0[0, 0] - b * np.outer(k[0, 0, 0], S0[0, 0].T @ k[0, 0, 0]
+                                        - v[0, 0, 0])
+        assert np.max(np.abs(se[0, 0] - euler)) < 5 * b * b * (
+            1 + np.max(np.abs(S0)))
+    _, se = oracle.efla_fwd(k, k, v, np.full((1, 1, 1), 60.0), gate="none",
+                            initial_state=S0)
+    np.testing.assert_allclose(se[0, 0].T @ k[0, 0, 0], v[0, 0, 0], atol=1e-12)
+
+
 def test_thread_count_does_not_change_bits(oracle_lib):
     rng = np.random.default_rng(10)
     c = _rand_case(rng, B=3, T=15, H=5, dk=4, dv=4, gate="channel")
