@@ -554,6 +554,81 @@ def run_decode(args):
     return 0
 
 
+BACKWARD_METRIC = ("tokens/s, backward pass (gdr_backward) of the chunked "
+                   "gated-delta fwd; % HBM roofline")
+
+
+def run_backward(args, w):
+    """Backward pass of the workload: upstream gradients of out and of the
+    final state in, gradients of every input out."""
+    import torch
+
+    import chunkwise_recurrence_b200 as gdr
+    from chunkwise_recurrence_b200.inputs import generate
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        raise SystemExit("--backward runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    inp = generate(w, seed=args.seed)
+    g = torch.Generator().manual_seed(args.seed + 1)
+    dO = torch.randn(inp.v.shape, generator=g).to(inp.v.dtype).to(dev)
+    dS = (torch.randn(inp.nseq, w.H, w.dk, w.dv, generator=g) * 0.1).to(dev)
+    c = lambda t: None if t is None else t.to(dev)  # noqa: E731
+    q, k, v, b, la, s0, cu = (c(t) for t in (inp.q, inp.k, inp.v, inp.beta,
+                                             inp.log_alpha, inp.s0,
+                                             inp.cu_seqlens))
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return gdr.backward(q, k, v, b, la, s0, dO, dS, gate=w.gate,
+                            cu_seqlens=cu, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_gpu_index(local)) as clocks:
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    ms = ev[0].elapsed_time(ev[-1]) / args.steps
+    ntok, H, dk, dv = inp.ntok, w.H, w.dk, w.dv
+    esz = 4 if w.dtype == "fp32" else 2
+    la_b = {"none": 0, "scalar": 4, "channel": 4 * dk}[w.gate]
+    # inputs (q, k, v, d_out in the I/O dtype, beta, log-alpha) read once,
+    # gradients (fp32) written once, states in and out
+    by = ntok * H * (esz * (2 * dk + 2 * dv) + 4 + la_b +
+                     4 * (2 * dk + dv) + 4 + la_b)
+    by += inp.nseq * H * dk * dv * 4 * (2 + (1 if inp.s0 is not None else 0))
+    peaks, peak_src = load_peaks()
+    gbs = by / (statistics.mean(per_step) / 1e3) / 1e9
+    line = {
+        "metric": BACKWARD_METRIC, "value": ntok / (ms / 1e3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {**workload_config(w, inp), "algo": "token-level reverse",
+                   "l2": "inputs larger than L2 (no flush)"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                     "traffic": None, "peak_source": peak_src,
+                     "kernel": "gdr_bwd_kernel",
+                     "algorithmic_bytes_per_launch": by},
+        "clocks": clocks.summary(),
+        "gpu_launches": args.steps,
+        "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def gdr_fused_available():
     from chunkwise_recurrence_b200 import fused_tc_available
     return fused_tc_available()
@@ -588,12 +663,16 @@ def main(argv=None):
                     help="time the single-token decode step instead")
     ap.add_argument("--decode-seqs", type=int, default=256,
                     help="sequences per decode step")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (gdr_backward) instead")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
     if args.decode and args.impl == "ours":
         return run_decode(args)
+    if args.backward and args.impl == "ours":
+        return run_backward(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -15,7 +15,7 @@ import os
 import torch
 
 __all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_noalloc", "decode_step",
-           "efla_beta",
+           "efla_beta", "backward",
            "device_error", "status_string",
            "algo_applies", "fused_tc_available",
            "GdrError", "load_library", "LIB_PATH", "GATES", "ALGOS",
@@ -33,7 +33,7 @@ STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARGUMENT", 2: "GDR_ERR_UNSUPPORTED",
 EXPORTED_SYMBOLS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_device_error",
                     "gdr_algo_applies", "gdr_status_string",
                     "gdr_chunk_fwd_noalloc", "gdr_decode_step",
-                    "gdr_efla_beta")
+                    "gdr_efla_beta", "gdr_backward")
 # size of the static scratch array behind gdr_chunk_fwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -72,6 +72,10 @@ def load_library(path: str = LIB_PATH):
     lib.gdr_decode_step.restype = ctypes.c_int
     lib.gdr_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i,
                                     vp, ctypes.POINTER(_Opts)]
+    lib.gdr_backward.restype = ctypes.c_int
+    lib.gdr_backward.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, fp, fp, fp,
+                                 fp, fp, fp, i, i, i, i, i, vp,
+                                 ctypes.POINTER(_Opts)]
     lib.gdr_efla_beta.restype = ctypes.c_int
     lib.gdr_efla_beta.argtypes = [vp, fp, fp, i, i, i, i, vp]
     lib.gdr_device_error.restype = ctypes.c_int
@@ -239,6 +243,39 @@ def decode_step(q, k, v, beta, log_alpha=None, state=None, *, out=None,
     if rc != 0:
         raise GdrError(rc, "gdr_decode_step")
     return out, state_out
+
+
+def backward(q, k, v, beta, log_alpha, initial_state, d_out, d_final_state=None,
+             *, gate: str | None = None, cu_seqlens=None,
+             need_initial_state_grad: bool = True, stream=None):
+    """Run ``gdr_backward``: gradients of the forward pass (same inputs as
+    ``chunk_fwd``) given dL/d out and, optionally, dL/d final_state.
+    Returns a dict of fp32 CUDA tensors dq, dk, dv, dbeta, dlog_alpha (None
+    without a gate) and dinitial_state (None unless requested)."""
+    lib = load_library()
+    B, T, H, dk, dv, nseq = _shapes(q, v, cu_seqlens)
+    g = _gate_of(log_alpha, gate)
+    f32 = lambda t: torch.empty(t.shape, dtype=torch.float32,  # noqa: E731
+                                device=q.device)
+    gq, gk, gv, gb = f32(q), f32(k), f32(v), f32(beta)
+    gla = None if log_alpha is None else f32(log_alpha)
+    gs0 = (torch.empty(nseq, H, dk, dv, dtype=torch.float32, device=q.device)
+           if need_initial_state_grad else None)
+    opts = _Opts(DTYPES[q.dtype], GATES[g],
+                 None if cu_seqlens is None else cu_seqlens.data_ptr(),
+                 nseq if cu_seqlens is not None else 0, ALGOS["auto"])
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    rc = lib.gdr_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                          _ptr(beta), _ptr(initial_state), _ptr(d_out),
+                          _ptr(d_final_state), _ptr(gq), _ptr(gk), _ptr(gv),
+                          _ptr(gla), _ptr(gb), _ptr(gs0), B, T, H, dk, dv,
+                          ctypes.c_void_p(stream.cuda_stream),
+                          ctypes.byref(opts))
+    if rc != 0:
+        raise GdrError(rc, "gdr_backward")
+    return dict(dq=gq, dk=gk, dv=gv, dbeta=gb, dlog_alpha=gla,
+                dinitial_state=gs0)
 
 
 def efla_beta(k, beta, *, out=None, stream=None):

@@ -468,6 +468,47 @@ extern "C" gdr_status gdr_chunk_fwd_noalloc(
                                                             : GDR_ERR_CUDA;
 }
 
+extern "C" gdr_status gdr_backward(
+    const void *q, const void *k, const void *v, const float *log_alpha,
+    const float *beta, const float *initial_state, const void *d_out,
+    const float *d_final_state, float *dq, float *dk, float *dv,
+    float *d_log_alpha, float *d_beta, float *d_initial_state, int B, int T,
+    int H, int dk_, int dv_, cudaStream_t stream, const gdr_opts *opts) {
+  const gdr_opts o = opts ? *opts : default_opts();
+  if (o.algo != GDR_ALGO_AUTO) return GDR_ERR_UNSUPPORTED;
+  Problem p;
+  // the forward pass's checks, with d_out in the place of out and
+  // d_final_state in the place of final_state (chunk plays no part here)
+  gdr_status st = validate(q, k, v, log_alpha, beta, initial_state, d_out,
+                           d_final_state, B, T, H, dk_, dv_, 64, o, &p);
+  if (st != GDR_OK) return st;
+  if (p.nseq == 0 || p.H == 0) return GDR_OK;
+  if (!dq || !dk || !dv || !d_beta) return GDR_ERR_INVALID_ARGUMENT;
+  if ((o.gate == GDR_GATE_NONE) != (d_log_alpha == nullptr))
+    return GDR_ERR_INVALID_ARGUMENT;
+  const void *grads[] = {dq, dk, dv, d_log_alpha, d_beta, d_initial_state};
+  for (const void *ptr : grads)
+    if (ptr && !aligned16(ptr)) return GDR_ERR_INVALID_ARGUMENT;
+  long long total_win = 0;
+  const size_t bytes = gdr::backward_scratch_bytes(p, &total_win);
+  void *ws = nullptr;
+  st = scratch_alloc(&ws, bytes, stream);
+  if (st != GDR_OK) return st;
+  gdr::BackwardIO io;
+  io.dout = d_out;
+  io.dsT = d_final_state;
+  io.dq = dq;
+  io.dk = dk;
+  io.dv = dv;
+  io.dla = d_log_alpha;
+  io.dbeta = d_beta;
+  io.ds0 = d_initial_state;
+  cudaError_t e = gdr::backward_run(p, io, static_cast<float *>(ws), total_win,
+                                    stream);
+  cudaError_t f = cudaFreeAsync(ws, stream);
+  return (e == cudaSuccess && f == cudaSuccess) ? GDR_OK : GDR_ERR_CUDA;
+}
+
 extern "C" gdr_status gdr_device_error(cudaStream_t stream, int clear) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return GDR_ERR_CUDA;
   unsigned word = 0;

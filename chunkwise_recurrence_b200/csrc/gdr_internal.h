@@ -46,4 +46,19 @@ cudaError_t fused_tc_run(const Problem &p, cudaStream_t s);
 // Reads (and optionally clears) the fused kernel's sticky device error word.
 cudaError_t fused_tc_read_error(unsigned *word, bool clear);
 
+// Backward pass (csrc/backward.cu): upstream gradients in, gradients out.
+struct BackwardIO {
+  const void *dout;      // dL/d out, layout of out, dtype of the problem
+  const float *dsT;      // dL/d final_state [N][H][dk][dv], or nullptr
+  float *dq, *dk, *dv;   // fp32, layouts of q, k, v
+  float *dla;            // fp32, layout of log_alpha (nullptr for no gate)
+  float *dbeta;          // fp32 [ntok][H]
+  float *ds0;            // fp32 [N][H][dk][dv], or nullptr
+};
+// Scratch the backward pass needs (bytes); *total_win = the number of
+// checkpoint windows per head, to pass on to backward_run.
+size_t backward_scratch_bytes(const Problem &p, long long *total_win);
+cudaError_t backward_run(const Problem &p, const BackwardIO &io,
+                         float *scratch, long long total_win, cudaStream_t s);
+
 }  // namespace gdr

@@ -257,6 +257,38 @@ GDR_API gdr_status gdr_decode_step(const void *q, const void *k, const void *v,
                                    cudaStream_t stream, const gdr_opts *opts);
 
 /*
+ * gdr_backward -- gradients of gdr_chunk_fwd's outputs with respect to its
+ * inputs (the backward pass for training).
+ *
+ * Given the forward inputs and the upstream gradients dL/d out and
+ * dL/d final_state, it writes dL/dq, dL/dk, dL/dv, dL/d log_alpha,
+ * dL/d beta and dL/d initial_state of the recurrence above (the same
+ * definition gdr_chunk_fwd evaluates, whichever algorithm ran it).  It
+ * runs the recurrence forward, checkpointing the state every 16 tokens in
+ * scratch, then the reverse token recurrence window by window, all in fp32.
+ *
+ * Inputs: q, k, v, log_alpha, beta, initial_state, B, T, H, dk, dv and opts
+ * exactly as for gdr_chunk_fwd (opts->algo must be GDR_ALGO_AUTO);
+ *   d_out          layout and dtype of out (device), required;
+ *   d_final_state  [N][H][dk][dv] fp32, or NULL for a zero gradient.
+ * Outputs (device, fp32, 16-byte aligned, written):
+ *   dq, dk         [B][T][H][dk];   dv [B][T][H][dv];   d_beta [B][T][H];
+ *   d_log_alpha    the layout of log_alpha; NULL iff gate is NONE;
+ *   d_initial_state [N][H][dk][dv], or NULL to skip.
+ * Scratch: about (ntok/16 + N) * H + 16 * N * H states of dk*dv floats,
+ * allocated stream-ordered on `stream` (GDR_ERR_OUT_OF_MEMORY on failure).
+ * Status codes as for gdr_chunk_fwd.
+ */
+GDR_API gdr_status gdr_backward(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta,
+                                const float *initial_state, const void *d_out,
+                                const float *d_final_state, float *dq,
+                                float *dk, float *dv, float *d_log_alpha,
+                                float *d_beta, float *d_initial_state, int B,
+                                int T, int H, int dk_dim, int dv_dim,
+                                cudaStream_t stream, const gdr_opts *opts);
+
+/*
  * gdr_efla_beta -- exact-flow step size (EFLA) for the delta rule.
  *
  * The delta rule's update is one explicit Euler step of length beta of the

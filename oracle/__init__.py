@@ -13,6 +13,8 @@ Contents
 ``efla_fwd``         the exact-flow (EFLA) variant: each token's update is the
                      exact flow of the delta rule's dynamics, integrated with a
                      matrix exponential (small cases only).
+``gdr_grads``        fp64 gradients of the recurrence (PyTorch autograd on the
+                     plain token loop), the reference for the backward pass.
 ``chunkwise_ref``    an independent fp64 chunkwise reformulation that solves the
                      intra-chunk triangular system with a dense ``solve``; it is a
                      pin for the token loop, not a second oracle for the GPU.
@@ -157,3 +159,4 @@ def decode_step(q, k, v, beta, log_alpha=None, gate="scalar", state=None,
 
 from .chunkwise_ref import chunkwise_ref  # noqa: E402  (re-export)
 from .efla_ref import efla_fwd  # noqa: E402  (re-export)
+from .grad_ref import gdr_grads  # noqa: E402  (re-export)

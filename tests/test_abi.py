@@ -176,6 +176,31 @@ def test_efla_beta_rejects_bad_arguments(lib):
     assert f(k=None, b=None, o=None, ntok=0) == OK   # empty: no-op
 
 
+def bcall(lib, *, q=A, k=A, v=A, la=A, beta=A, s0=None, dout=A, dsT=None,
+          dq=A, dk=A, dv=A, dla=A, db=A, ds0=None, B=1, T=32, H=1, dk_=64,
+          dv_=64, gate=1, dtype=0, algo=0, cu=None, nseq=0):
+    opts = gdr._Opts(dtype, gate, cu, nseq, algo)
+    return lib.gdr_backward(q, k, v, la, beta, s0, dout, dsT, dq, dk, dv, dla,
+                            db, ds0, B, T, H, dk_, dv_, None,
+                            ctypes.byref(opts))
+
+
+def test_backward_rejects_bad_arguments(lib):
+    c = lambda **kw: bcall(lib, **kw)  # noqa: E731
+    assert c(dout=None) == INVALID       # the upstream output gradient
+    assert c(dq=None) == INVALID
+    assert c(db=None) == INVALID
+    assert c(dla=None) == INVALID        # a gate needs its gradient
+    assert c(gate=0, la=None) == INVALID  # ... and no gate forbids it
+    assert c(dk=A + 4) == INVALID        # misaligned
+    assert c(ds0=A + 8) == INVALID
+    assert c(algo=1) == UNSUPPORTED
+    assert c(dk_=48) == UNSUPPORTED
+    assert c(T=-1) == INVALID
+    assert c(q=None, k=None, v=None, la=None, beta=None, dout=None, dq=None,
+             dk=None, dv=None, dla=None, db=None, gate=0, B=0) == OK
+
+
 def test_algo_applies(lib):
     assert gdr.algo_applies("staged", "fp32", "none", 16, 16, 16)
     assert gdr.algo_applies("auto", "bf16", "channel", 128, 64, 32)
