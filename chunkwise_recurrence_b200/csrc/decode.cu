@@ -14,13 +14,17 @@
 //
 // The step moves 2 dk dv 4 bytes of state per (sequence, head) against about
 // 6 dk dv flops, so it is bound by HBM bandwidth.  One CTA of 256 threads per
-// (sequence, head): warp w owns rows [w dk/8, (w+1) dk/8) of S, lane l owns
-// columns [4l, 4l+4), so every load and store of S is a 16-byte access and a
-// warp covers whole 512-byte rows.  S is read once into registers, the two
-// column reductions (S~^T k, S~^T q) go through shared memory, and S' is
-// written back from the same registers: one read and one write of the state.
-// In place (state_in == state_out) is safe: every element is read and written
-// by the same thread.
+// (sequence, head).  The state tile (contiguous, dk dv 4 bytes) comes into
+// shared memory with one bulk asynchronous copy (cp.async.bulk, completion on
+// an mbarrier) and leaves with one bulk store, so three CTAs per SM keep
+// up to 3 x 64 KB of state in flight with a handful of instructions.  In
+// shared memory warp w owns rows [w dk/8, (w+1) dk/8) of S and lane l
+// columns [4l, 4l+4) (16-byte accesses, whole 512-byte rows per warp); the
+// two column reductions (S~^T k, S~^T q) meet in shared memory; S' overwrites
+// the tile in place before the store.  state_in == state_out is safe: the
+// tile is read in full before any of it is written back.  The copy wait is
+// bounded; on expiry the CTA skips its step and raises the library's device
+// error word (gdr_device_error: GDR_ERR_TIMEOUT).
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -28,11 +32,38 @@
 #include <cstdint>
 
 #include "gdr_internal.h"
+#include "sm100.cuh"
 
 namespace gdr {
+
+__device__ unsigned g_decode_error;
+
 namespace {
 
+using namespace sm100;
+
 constexpr int kDecThreads = 256;
+constexpr long long kDecWaitCycles = 1ll << 31;   // ~1 s: never reached
+
+__device__ __forceinline__ void bulk_load(void *dst, const void *src,
+                                          uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void bulk_store(void *dst, const void *src,
+                                           uint32_t bytes) {
+  asm volatile(
+      "cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+          reinterpret_cast<uint64_t>(dst)),
+      "r"(smem_u32(src)), "r"(bytes)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  // the source tile must stay in place until the copy has read it
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 
 struct DecodeParams {
   const void *q, *k, *v;
@@ -82,13 +113,27 @@ template <int DK, typename T, int GATE>
 __global__ void __launch_bounds__(kDecThreads)
     gdr_decode_kernel(DecodeParams p) {
   constexpr int R = DK / 8;   // rows of S per warp
+  extern __shared__ __align__(128) float tile[];   // the state, [DK][dv]
   __shared__ float sk[DK], sq[DK], sa[DK];
   __shared__ float4 red[2][8][32];   // per warp: partial S~^T k, S~^T q
   __shared__ float kq_s;
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int copy_ok;
   const int nh = blockIdx.x;         // (sequence, head), flattened
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int dv = p.dv, j0 = 4 * lane;
   const bool act = j0 < dv;
+  const size_t sb = (size_t)nh * DK * dv;
+  const uint32_t bytes = (uint32_t)(DK * dv * 4);
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    copy_ok = 1;
+    if (p.s_in) {
+      mbar_arrive_expect_tx(&bar, bytes);
+      bulk_load(tile, p.s_in + sb, bytes, &bar);
+    }
+  }
   const T *q = static_cast<const T *>(p.q) + (size_t)nh * DK;
   const T *k = static_cast<const T *>(p.k) + (size_t)nh * DK;
   for (int c = threadIdx.x; c < DK; c += kDecThreads) {
@@ -98,19 +143,28 @@ __global__ void __launch_bounds__(kDecThreads)
             : GATE == 1 ? __expf(p.log_alpha[nh])
                         : __expf(p.log_alpha[(size_t)nh * DK + c]);
   }
+  if (threadIdx.x == 0 && p.s_in) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(&bar, 0)) {
+      if (clock64() - t0 > kDecWaitCycles) {
+        copy_ok = 0;
+        atomicOr(&g_decode_error, 1u);
+        break;
+      }
+    }
+  }
   __syncthreads();
+  if (!copy_ok) return;   // uniform: the tile never arrived
   // S~ = D S for this thread's rows and columns; partial column reductions
-  const size_t sb = (size_t)nh * DK * dv;
-  float4 S[R];
   float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     const int c = warp * R + r;
     float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (act && p.s_in) x = ld4(p.s_in + sb + (size_t)c * dv + j0);
+    if (act && p.s_in) x = ld4(tile + c * dv + j0);
     const float a = sa[c];
     x = make_float4(a * x.x, a * x.y, a * x.z, a * x.w);
-    S[r] = x;
+    if (act) st4(tile + c * dv + j0, x);   // S~, kept for the update
     pk = fma4(sk[c], x, pk);
     pq = fma4(sq[c], x, pq);
   }
@@ -125,7 +179,6 @@ __global__ void __launch_bounds__(kDecThreads)
     if (lane == 0) kq_s = t;
   }
   __syncthreads();
-  if (!act) return;
   float4 rk = red[0][0][lane], rq = red[1][0][lane];
 #pragma unroll
   for (int w = 1; w < 8; ++w) {
@@ -133,30 +186,47 @@ __global__ void __launch_bounds__(kDecThreads)
     rk = make_float4(rk.x + a.x, rk.y + a.y, rk.z + a.z, rk.w + a.w);
     rq = make_float4(rq.x + b.x, rq.y + b.y, rq.z + b.z, rq.w + b.w);
   }
-  // u = beta (v - S~^T k); o = S~^T q + u (k . q)
-  const float bt = p.beta[nh];
-  const float4 vv = ld4(static_cast<const T *>(p.v) + (size_t)nh * dv + j0);
-  const float4 u = make_float4(bt * (vv.x - rk.x), bt * (vv.y - rk.y),
-                               bt * (vv.z - rk.z), bt * (vv.w - rk.w));
-  if (warp == 0)
-    st4(static_cast<T *>(p.out) + (size_t)nh * dv + j0, fma4(kq_s, u, rq));
-  // S' = S~ + k u^T
+  if (act) {
+    // u = beta (v - S~^T k); o = S~^T q + u (k . q)
+    const float bt = p.beta[nh];
+    const float4 vv = ld4(static_cast<const T *>(p.v) + (size_t)nh * dv + j0);
+    const float4 u = make_float4(bt * (vv.x - rk.x), bt * (vv.y - rk.y),
+                                 bt * (vv.z - rk.z), bt * (vv.w - rk.w));
+    if (warp == 0)
+      st4(static_cast<T *>(p.out) + (size_t)nh * dv + j0, fma4(kq_s, u, rq));
+    // S' = S~ + k u^T, in place in the tile
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int c = warp * R + r;
-    st4(p.s_out + sb + (size_t)c * dv + j0, fma4(sk[c], u, S[r]));
+    for (int r = 0; r < R; ++r) {
+      const int c = warp * R + r;
+      float *e = tile + c * dv + j0;
+      st4(e, fma4(sk[c], u, ld4(e)));
+    }
   }
+  // the tile's generic-proxy writes, visible to the bulk store
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (threadIdx.x == 0) bulk_store(p.s_out + sb, tile, bytes);
+}
+
+template <int DK, typename T, int GATE>
+cudaError_t launch_g(const DecodeParams &dp, int nblocks, cudaStream_t s) {
+  const int smem = DK * dp.dv * 4;
+  cudaError_t e = cudaFuncSetAttribute(
+      gdr_decode_kernel<DK, T, GATE>,
+      cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  gdr_decode_kernel<DK, T, GATE><<<nblocks, kDecThreads, smem, s>>>(dp);
+  return cudaGetLastError();
 }
 
 template <int DK, typename T>
 cudaError_t launch_dk(const DecodeParams &dp, int gate, int nblocks,
                       cudaStream_t s) {
   switch (gate) {
-    case 0: gdr_decode_kernel<DK, T, 0><<<nblocks, kDecThreads, 0, s>>>(dp); break;
-    case 1: gdr_decode_kernel<DK, T, 1><<<nblocks, kDecThreads, 0, s>>>(dp); break;
-    default: gdr_decode_kernel<DK, T, 2><<<nblocks, kDecThreads, 0, s>>>(dp); break;
+    case 0: return launch_g<DK, T, 0>(dp, nblocks, s);
+    case 1: return launch_g<DK, T, 1>(dp, nblocks, s);
+    default: return launch_g<DK, T, 2>(dp, nblocks, s);
   }
-  return cudaGetLastError();
 }
 
 template <typename T>
@@ -169,6 +239,20 @@ cudaError_t launch_t(const DecodeParams &dp, int dk, int gate, int nblocks,
     default: return launch_dk<128, T>(dp, gate, nblocks, s);
   }
 }
+
+}  // namespace
+
+cudaError_t decode_read_error(unsigned *word, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(word, g_decode_error, sizeof(unsigned));
+  if (e != cudaSuccess) return e;
+  if (clear && *word) {
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_decode_error, &zero, sizeof(unsigned));
+  }
+  return e;
+}
+
+namespace {
 
 bool aligned16(const void *p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;

@@ -491,9 +491,22 @@ extern "C" gdr_status gdr_backward(
     if (ptr && !aligned16(ptr)) return GDR_ERR_INVALID_ARGUMENT;
   long long total_win = 0;
   const size_t bytes = gdr::backward_scratch_bytes(p, &total_win);
-  void *ws = nullptr;
-  st = scratch_alloc(&ws, bytes, stream);
+  // the scratch comes from the library's per-device pool, which keeps its
+  // memory between calls (hundreds of MB at training sizes: mapping it anew
+  // every call would cost more than the copies it saves)
+  if (alloc_fault_injected()) return GDR_ERR_OUT_OF_MEMORY;
+  HostCtx hc;
+  st = host_ctx(&hc);
   if (st != GDR_OK) return st;
+  void *ws = nullptr;
+  {
+    cudaError_t e = cudaMallocFromPoolAsync(&ws, bytes, hc.pool, stream);
+    if (e == cudaErrorMemoryAllocation) {
+      (void)cudaGetLastError();
+      return GDR_ERR_OUT_OF_MEMORY;
+    }
+    if (e != cudaSuccess) return GDR_ERR_CUDA;
+  }
   gdr::BackwardIO io;
   io.dout = d_out;
   io.dsT = d_final_state;
@@ -514,7 +527,10 @@ extern "C" gdr_status gdr_device_error(cudaStream_t stream, int clear) {
   unsigned word = 0;
   if (gdr::fused_tc_read_error(&word, clear != 0) != cudaSuccess)
     return GDR_ERR_CUDA;
-  if (word & 0xFFFFFFu) return GDR_ERR_TIMEOUT;  // an mbarrier wait expired
+  unsigned dword = 0;   // the decode step's bulk copy never completed
+  if (gdr::decode_read_error(&dword, clear != 0) != cudaSuccess)
+    return GDR_ERR_CUDA;
+  if ((word & 0xFFFFFFu) || dword) return GDR_ERR_TIMEOUT;  // a wait expired
   return word ? GDR_ERR_RANGE : GDR_OK;
 }
 

@@ -46,6 +46,10 @@ cudaError_t fused_tc_run(const Problem &p, cudaStream_t s);
 // Reads (and optionally clears) the fused kernel's sticky device error word.
 cudaError_t fused_tc_read_error(unsigned *word, bool clear);
 
+// Decode step: reads (and optionally clears) its sticky device error word
+// (a bulk copy that never completed).
+cudaError_t decode_read_error(unsigned *word, bool clear);
+
 // Backward pass (csrc/backward.cu): upstream gradients in, gradients out.
 struct BackwardIO {
   const void *dout;      // dL/d out, layout of out, dtype of the problem

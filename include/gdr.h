@@ -246,9 +246,10 @@ GDR_API gdr_status gdr_chunk_fwd_noalloc(const void *q, const void *k,
  * dk, dv in {16, 32, 64, 128}.  opts may be NULL (bf16, scalar gate);
  * opts->cu_seqlens must be NULL and opts->num_seqs 0 (one token per
  * sequence: nothing to pack), opts->algo must be GDR_ALGO_AUTO.
- * Arithmetic is fp32.  One kernel launch, no scratch memory, no device-side
- * waits.  Returns GDR_ERR_INVALID_ARGUMENT / GDR_ERR_UNSUPPORTED as described,
- * GDR_ERR_CUDA if the launch fails.
+ * Arithmetic is fp32.  One kernel launch, no scratch memory; each CTA's wait
+ * for its state tile is bounded (an expired wait is reported by
+ * gdr_device_error as GDR_ERR_TIMEOUT).  Returns GDR_ERR_INVALID_ARGUMENT /
+ * GDR_ERR_UNSUPPORTED as described, GDR_ERR_CUDA if the launch fails.
  */
 GDR_API gdr_status gdr_decode_step(const void *q, const void *k, const void *v,
                                    const float *log_alpha, const float *beta,
@@ -276,7 +277,9 @@ GDR_API gdr_status gdr_decode_step(const void *q, const void *k, const void *v,
  *   d_log_alpha    the layout of log_alpha; NULL iff gate is NONE;
  *   d_initial_state [N][H][dk][dv], or NULL to skip.
  * Scratch: about (ntok/16 + N) * H + 16 * N * H states of dk*dv floats,
- * allocated stream-ordered on `stream` (GDR_ERR_OUT_OF_MEMORY on failure).
+ * allocated stream-ordered on `stream` from the library's per-device memory
+ * pool, which keeps its memory between calls (the pool gdr_chunk_fwd_host
+ * uses); GDR_ERR_OUT_OF_MEMORY on failure.
  * Status codes as for gdr_chunk_fwd.
  */
 GDR_API gdr_status gdr_backward(const void *q, const void *k, const void *v,
@@ -314,7 +317,8 @@ GDR_API gdr_status gdr_efla_beta(const void *k, const float *beta,
  * gdr_device_error -- synchronise `stream`, then read (and clear if `clear`)
  * the library's sticky device-side error word for the current device.
  * Returns GDR_OK if no kernel has reported an error, GDR_ERR_TIMEOUT if a
- * bounded wait expired, GDR_ERR_RANGE if the fused kernel produced a
+ * bounded wait expired (the fused kernel's, or the decode step's wait for its
+ * state tile), GDR_ERR_RANGE if the fused kernel produced a
  * non-finite output or final state (an input or intermediate beyond the
  * fp16 operand range, |x| > 65504, or a NaN input) or, for the channel gate,
  * met such an input,
