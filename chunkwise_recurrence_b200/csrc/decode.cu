@@ -30,6 +30,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 
 #include "gdr_internal.h"
 #include "sm100.cuh"
@@ -44,6 +45,9 @@ using namespace sm100;
 
 constexpr int kDecThreads = 256;
 constexpr long long kDecWaitCycles = 1ll << 31;   // ~1 s: never reached
+// GDR_FAULT_INJECT_DECODE_TIMEOUT=1: the state copy is never issued and the
+// wait gives up after this many cycles (tests of the timeout path)
+constexpr long long kDecInjectWaitCycles = 1ll << 20;
 
 __device__ __forceinline__ void bulk_load(void *dst, const void *src,
                                           uint32_t bytes, uint64_t *bar) {
@@ -71,6 +75,10 @@ struct DecodeParams {
   float *s_out;
   void *out;
   int dv;
+  // failure injection (host hook): the state copy is not issued, so the
+  // CTA's wait runs out after wait_cycles and reports a timeout
+  int inject_timeout;
+  long long wait_cycles;
 };
 
 template <typename T>
@@ -131,7 +139,7 @@ __global__ void __launch_bounds__(kDecThreads)
     copy_ok = 1;
     if (p.s_in) {
       mbar_arrive_expect_tx(&bar, bytes);
-      bulk_load(tile, p.s_in + sb, bytes, &bar);
+      if (!p.inject_timeout) bulk_load(tile, p.s_in + sb, bytes, &bar);
     }
   }
   const T *q = static_cast<const T *>(p.q) + (size_t)nh * DK;
@@ -146,7 +154,7 @@ __global__ void __launch_bounds__(kDecThreads)
   if (threadIdx.x == 0 && p.s_in) {
     const long long t0 = clock64();
     while (!mbar_try_wait(&bar, 0)) {
-      if (clock64() - t0 > kDecWaitCycles) {
+      if (clock64() - t0 > p.wait_cycles) {
         copy_ok = 0;
         atomicOr(&g_decode_error, 1u);
         break;
@@ -312,6 +320,10 @@ extern "C" gdr_status gdr_decode_step(const void *q, const void *k,
   dp.s_out = state_out;
   dp.out = out;
   dp.dv = dv;
+  const char *inj = std::getenv("GDR_FAULT_INJECT_DECODE_TIMEOUT");
+  dp.inject_timeout = (inj && inj[0] == '1') ? 1 : 0;
+  dp.wait_cycles = dp.inject_timeout ? gdr::kDecInjectWaitCycles
+                                     : gdr::kDecWaitCycles;
   const int nb = (int)nh;
   const cudaError_t e =
       o.dtype == GDR_BF16

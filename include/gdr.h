@@ -248,7 +248,9 @@ GDR_API gdr_status gdr_chunk_fwd_noalloc(const void *q, const void *k,
  * sequence: nothing to pack), opts->algo must be GDR_ALGO_AUTO.
  * Arithmetic is fp32.  One kernel launch, no scratch memory; each CTA's wait
  * for its state tile is bounded (an expired wait is reported by
- * gdr_device_error as GDR_ERR_TIMEOUT).  Returns GDR_ERR_INVALID_ARGUMENT /
+ * gdr_device_error as GDR_ERR_TIMEOUT; the environment variable
+ * GDR_FAULT_INJECT_DECODE_TIMEOUT=1 makes every wait expire, for tests of that
+ * path: the step is then skipped and state_out is not written).  Returns GDR_ERR_INVALID_ARGUMENT /
  * GDR_ERR_UNSUPPORTED as described, GDR_ERR_CUDA if the launch fails.
  */
 GDR_API gdr_status gdr_decode_step(const void *q, const void *k, const void *v,

@@ -122,3 +122,26 @@ def test_decode_full_size_sampled():
     assert out_err(o[:8], ro, "bf16") <= TOL
     assert rel_err(s[:8], rs) <= TOL
     assert np.isfinite(o).all() and np.isfinite(s).all()
+
+
+def test_decode_wait_timeout_is_reported_and_recovers(monkeypatch):
+    """Failure detection on the GPU without a fault: with the injection hook
+    set, the decode kernel never issues its state copy, so each CTA's bounded
+    wait runs out (after about 10^6 cycles); the CTA skips its step and the
+    host reads GDR_ERR_TIMEOUT.  The state is left untouched, the context
+    stays usable, and the next call is correct."""
+    d = decode_inputs(4, 2, 128, 128, "bf16", "scalar")
+    c = lambda t: None if t is None else t.cuda()  # noqa: E731
+    state = c(d["state"])
+    before = state.clone()
+    monkeypatch.setenv("GDR_FAULT_INJECT_DECODE_TIMEOUT", "1")
+    gdr.decode_step(c(d["q"]), c(d["k"]), c(d["v"]), c(d["beta"]),
+                    c(d["log_alpha"]), state)
+    assert gdr.device_error(clear=True) == 5          # GDR_ERR_TIMEOUT
+    assert torch.equal(state, before)
+    assert gdr.device_error() == 0                    # cleared
+    monkeypatch.delenv("GDR_FAULT_INJECT_DECODE_TIMEOUT")
+    o, s = run_gpu(d)
+    assert gdr.device_error() == 0
+    ro, rs = run_oracle(d, "scalar")
+    assert out_err(o, ro, "bf16") <= TOL and rel_err(s, rs) <= TOL
