@@ -269,10 +269,12 @@ def run_reference(args, w):
     return 0
 
 
-def launches_per_step(algo_used, w):
-    if algo_used == "fused_tc":
-        return 1
-    return 4 + (0 if w.gate == "none" else 1)
+def launches_per_step(algo_used, w, segments=0):
+    one = 1 if algo_used == "fused_tc" else 4 + (0 if w.gate == "none" else 1)
+    if segments:
+        # three forward passes, the identity fill and the combine
+        return 3 * one + 2
+    return one
 
 
 def run_ours(args, w):
@@ -301,6 +303,13 @@ def run_ours(args, w):
     stream = torch.cuda.current_stream(dev)
 
     def step():
+        if args.segments:
+            gdr.chunk_fwd_segmented(q, k, v, beta, la, s0,
+                                    segments=args.segments, chunk=w.chunk,
+                                    gate=w.gate, cu_seqlens=cu, out=out,
+                                    final_state=sT, algo=args.algo,
+                                    stream=stream)
+            return
         gdr.chunk_fwd(q, k, v, beta, la, s0, chunk=w.chunk, gate=w.gate,
                       cu_seqlens=cu, out=out, final_state=sT, algo=args.algo,
                       stream=stream)
@@ -404,6 +413,7 @@ def run_ours(args, w):
                    "seq_len": None if w.varlen_nseq else w.T,
                    "parallelism": f"dp{ws} (independent sequences)",
                    "algo": algo_used,
+                   "segments": args.segments or None,
                    "l2": "inputs larger than L2 (no flush)"},
         "tflops": fl * ws / (ms / 1e3) / 1e12,
         "roofline": roofline,
@@ -411,7 +421,8 @@ def run_ours(args, w):
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d * ws, "d2h_bytes_per_step": d2h * ws,
                 "entry": "gdr_chunk_fwd_host (pinned host buffers)"},
-        "gpu_launches": launches_per_step(algo_used, w) * args.steps,
+        "gpu_launches": launches_per_step(algo_used, w, args.segments) *
+        args.steps,
         "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -665,6 +676,9 @@ def main(argv=None):
                     help="sequences per decode step")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (gdr_backward) instead")
+    ap.add_argument("--segments", type=int, default=0,
+                    help="context-parallel forward (gdr_chunk_fwd_segmented) "
+                         "with this many pieces per sequence")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -14,7 +14,8 @@ import os
 
 import torch
 
-__all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_noalloc", "decode_step",
+__all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_noalloc",
+           "chunk_fwd_segmented", "decode_step",
            "efla_beta", "backward",
            "device_error", "status_string",
            "algo_applies", "fused_tc_available",
@@ -33,7 +34,8 @@ STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARGUMENT", 2: "GDR_ERR_UNSUPPORTED",
 EXPORTED_SYMBOLS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_device_error",
                     "gdr_algo_applies", "gdr_status_string",
                     "gdr_chunk_fwd_noalloc", "gdr_decode_step",
-                    "gdr_efla_beta", "gdr_backward")
+                    "gdr_efla_beta", "gdr_backward",
+                    "gdr_chunk_fwd_segmented")
 # size of the static scratch array behind gdr_chunk_fwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -72,6 +74,10 @@ def load_library(path: str = LIB_PATH):
     lib.gdr_decode_step.restype = ctypes.c_int
     lib.gdr_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i,
                                     vp, ctypes.POINTER(_Opts)]
+    lib.gdr_chunk_fwd_segmented.restype = ctypes.c_int
+    lib.gdr_chunk_fwd_segmented.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i,
+                                            i, i, i, i, i, i, vp,
+                                            ctypes.POINTER(_Opts)]
     lib.gdr_backward.restype = ctypes.c_int
     lib.gdr_backward.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, fp, fp, fp,
                                  fp, fp, fp, i, i, i, i, i, vp,
@@ -155,6 +161,38 @@ def chunk_fwd(q, k, v, beta, log_alpha=None, initial_state=None, *,
                            ctypes.byref(opts))
     if rc != 0:
         raise GdrError(rc, "gdr_chunk_fwd")
+    return out, final_state
+
+
+def chunk_fwd_segmented(q, k, v, beta, log_alpha=None, initial_state=None, *,
+                        segments: int, chunk: int = 64,
+                        gate: str | None = None, cu_seqlens=None, out=None,
+                        final_state=None, output_final_state: bool = True,
+                        algo: str = "auto", stream=None):
+    """Run ``gdr_chunk_fwd_segmented``: the forward pass with every sequence
+    cut into up to ``segments`` pieces whose state maps are computed in
+    parallel (context-parallel state passing).  Same inputs and results as
+    ``chunk_fwd``."""
+    lib = load_library()
+    B, T, H, dk, dv, nseq = _shapes(q, v, cu_seqlens)
+    if out is None:
+        out = torch.empty_like(v)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(nseq, H, dk, dv, dtype=torch.float32,
+                                  device=q.device)
+    g = _gate_of(log_alpha, gate)
+    opts = _Opts(DTYPES[q.dtype], GATES[g],
+                 None if cu_seqlens is None else cu_seqlens.data_ptr(),
+                 nseq if cu_seqlens is not None else 0, ALGOS[algo])
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    rc = lib.gdr_chunk_fwd_segmented(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+        _ptr(initial_state), _ptr(out), _ptr(final_state), B, T, H, dk, dv,
+        chunk, int(segments), ctypes.c_void_p(stream.cuda_stream),
+        ctypes.byref(opts))
+    if rc != 0:
+        raise GdrError(rc, "gdr_chunk_fwd_segmented")
     return out, final_state
 
 

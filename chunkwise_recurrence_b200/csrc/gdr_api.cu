@@ -9,6 +9,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "gdr_internal.h"
 
@@ -466,6 +467,157 @@ extern "C" gdr_status gdr_chunk_fwd_noalloc(
   if (st != GDR_OK) return st;
   return gdr::staged_run(p, scratch, stream) == cudaSuccess ? GDR_OK
                                                             : GDR_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Context-parallel forward pass: every sequence is cut into segments of whole
+// chunks; the segments' state maps (M, N) are computed in parallel, combined
+// in order per sequence, and a final pass runs every segment from its true
+// initial state.
+extern "C" gdr_status gdr_chunk_fwd_segmented(
+    const void *q, const void *k, const void *v, const float *log_alpha,
+    const float *beta, const float *initial_state, void *out,
+    float *final_state, int B, int T, int H, int dk, int dv, int chunk,
+    int segments, cudaStream_t stream, const gdr_opts *opts) {
+  const gdr_opts o = opts ? *opts : default_opts();
+  if (segments < 1) return GDR_ERR_INVALID_ARGUMENT;
+  Problem p;
+  gdr_status st = validate(q, k, v, log_alpha, beta, initial_state, out,
+                           final_state, B, T, H, dk, dv, chunk, o, &p);
+  if (st != GDR_OK) return st;
+  if (p.nseq == 0 || p.H == 0) return GDR_OK;
+  const int nseq = p.nseq;
+  // sequence offsets on the host (packed batches: one synchronous read)
+  std::vector<int64_t> cu(nseq + 1);
+  if (p.cu) {
+    std::vector<int32_t> hcu(nseq + 1);
+    if (cudaMemcpyAsync(hcu.data(), p.cu, (nseq + 1) * sizeof(int32_t),
+                        cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+      return GDR_ERR_CUDA;
+    if (hcu[0] != 0 || hcu[nseq] != p.ntok) return GDR_ERR_INVALID_ARGUMENT;
+    for (int i = 0; i <= nseq; ++i) {
+      if (i > 0 && hcu[i] < hcu[i - 1]) return GDR_ERR_INVALID_ARGUMENT;
+      cu[i] = hcu[i];
+    }
+  } else {
+    for (int i = 0; i <= nseq; ++i) cu[i] = (int64_t)i * T;
+  }
+  // the plan: sequence n of L tokens = ceil(L / chunk) chunks, cut into at
+  // most `segments` pieces of equally many whole chunks
+  std::vector<int32_t> seg_cu(1, 0), seg_first(nseq + 1, 0), seg_last(nseq);
+  int nseg = 0;
+  for (int n = 0; n < nseq; ++n) {
+    seg_first[n] = nseg;
+    const int64_t L = cu[n + 1] - cu[n];
+    const int64_t nch = (L + chunk - 1) / chunk;
+    const int64_t pieces = nch < segments ? nch : segments;
+    const int64_t per = pieces > 0 ? (nch + pieces - 1) / pieces : 0;
+    for (int64_t a = 0; a < L; a += per * chunk) {
+      const int64_t e = a + per * chunk < L ? a + per * chunk : L;
+      seg_cu.back() = (int32_t)(cu[n] + a);
+      seg_cu.push_back((int32_t)(cu[n] + e));
+      ++nseg;
+    }
+    seg_last[n] = nseg - 1;
+  }
+  seg_first[nseq] = nseg;
+  // seg_cu holds nseg + 1 offsets; consecutive segments share boundaries
+  // except across empty sequences, where the next start equals the end
+  const size_t ss = (size_t)dk * dv, sk2 = (size_t)dk * dk;
+  const size_t esz = p.dtype == GDR_FP32 ? 4 : 2;
+  auto up256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const size_t b_cu = up256((size_t)(nseg + 1) * 4);
+  const size_t b_first = up256((size_t)(nseq + 1) * 4);
+  const size_t b_zero = up256((size_t)p.ntok * H * dk * esz);
+  const size_t b_otmp = up256((size_t)p.ntok * H * (dk > dv ? dk : dv) * esz);
+  const size_t b_sq = up256((size_t)nseg * H * sk2 * 4);   // eye, Ms
+  const size_t b_st = up256((size_t)nseg * H * ss * 4);    // Ns, Sin, Sfin
+  const size_t total = b_cu + b_first + b_zero + b_otmp + 2 * b_sq + 3 * b_st;
+  if (alloc_fault_injected()) return GDR_ERR_OUT_OF_MEMORY;
+  HostCtx hc;
+  st = host_ctx(&hc);
+  if (st != GDR_OK) return st;
+  void *block = nullptr;
+  {
+    cudaError_t e = cudaMallocFromPoolAsync(&block, total, hc.pool, stream);
+    if (e == cudaErrorMemoryAllocation) {
+      (void)cudaGetLastError();
+      return GDR_ERR_OUT_OF_MEMORY;
+    }
+    if (e != cudaSuccess) return GDR_ERR_CUDA;
+  }
+  char *c = static_cast<char *>(block);
+  int32_t *d_cu = reinterpret_cast<int32_t *>(c); c += b_cu;
+  int32_t *d_first = reinterpret_cast<int32_t *>(c); c += b_first;
+  void *zero_v = c; c += b_zero;
+  void *otmp = c; c += b_otmp;
+  float *eye = reinterpret_cast<float *>(c); c += b_sq;
+  float *Ms = reinterpret_cast<float *>(c); c += b_sq;
+  float *Ns = reinterpret_cast<float *>(c); c += b_st;
+  float *Sin = reinterpret_cast<float *>(c); c += b_st;
+  float *Sfin = reinterpret_cast<float *>(c);
+  auto ok = [&](cudaError_t e) {
+    if (e != cudaSuccess && st == GDR_OK) st = GDR_ERR_CUDA;
+    return st == GDR_OK;
+  };
+  // the host vectors are pageable: these copies complete before returning
+  ok(cudaMemcpyAsync(d_cu, seg_cu.data(), (nseg + 1) * sizeof(int32_t),
+                     cudaMemcpyHostToDevice, stream));
+  ok(cudaMemcpyAsync(d_first, seg_first.data(), (nseq + 1) * sizeof(int32_t),
+                     cudaMemcpyHostToDevice, stream));
+  if (nseg > 0 && st == GDR_OK) {
+    // the segment problem: the same token axis, segments as sequences
+    Problem sp = p;
+    sp.cu = d_cu;
+    sp.nseq = nseg;
+    sp.T = p.ntok;
+    sp.max_chunks = p.ntok / chunk + nseg;
+    // pass M: transitions, from S = I with v = 0 (dv' = dk)
+    Problem pm = sp;
+    pm.v = zero_v;
+    pm.dv = dk;
+    pm.s0 = eye;
+    pm.out = otmp;
+    pm.sT = Ms;
+    ok(cudaMemsetAsync(zero_v, 0, (size_t)p.ntok * H * dk * esz, stream));
+    ok(gdr::fill_identity(eye, (long long)nseg * H, dk, stream));
+    if (st == GDR_OK) st = run(pm, o.algo, stream);
+    // pass N: offsets, from S = 0
+    Problem pn = sp;
+    pn.s0 = nullptr;
+    pn.out = otmp;
+    pn.sT = Ns;
+    if (st == GDR_OK) st = run(pn, o.algo, stream);
+    // in order per sequence: each segment's initial state
+    if (st == GDR_OK)
+      ok(gdr::segment_combine(p.s0, Ms, Ns, Sin, d_first, nseq, H, dk, dv,
+                              stream));
+    // pass C: every segment from its initial state: out, segment finals
+    Problem pc = sp;
+    pc.s0 = Sin;
+    pc.sT = Sfin;
+    if (st == GDR_OK) st = run(pc, o.algo, stream);
+  }
+  // final states: the last segment's, or the initial state of an empty
+  // sequence
+  if (final_state && st == GDR_OK) {
+    const size_t bytes = (size_t)H * ss * sizeof(float);
+    for (int n = 0; n < nseq && st == GDR_OK; ++n) {
+      float *dst = final_state + (size_t)n * H * ss;
+      if (seg_first[n + 1] > seg_first[n])
+        ok(cudaMemcpyAsync(dst, Sfin + (size_t)seg_last[n] * H * ss, bytes,
+                           cudaMemcpyDeviceToDevice, stream));
+      else if (p.s0)
+        ok(cudaMemcpyAsync(dst, p.s0 + (size_t)n * H * ss, bytes,
+                           cudaMemcpyDeviceToDevice, stream));
+      else
+        ok(cudaMemsetAsync(dst, 0, bytes, stream));
+    }
+  }
+  const cudaError_t f = cudaFreeAsync(block, stream);
+  if (st == GDR_OK && f != cudaSuccess) st = GDR_ERR_CUDA;
+  return st;
 }
 
 extern "C" gdr_status gdr_backward(

@@ -46,6 +46,17 @@ cudaError_t fused_tc_run(const Problem &p, cudaStream_t s);
 // Reads (and optionally clears) the fused kernel's sticky device error word.
 cudaError_t fused_tc_read_error(unsigned *word, bool clear);
 
+// Context-parallel state passing (csrc/segmented.cu): for each sequence n,
+// walk its segments seg_first[n] .. seg_first[n+1]-1 in order, writing each
+// segment's initial state into Sin and advancing S <- M_s S + N_s; S starts
+// from s0[n] (or zero).  Ms [nseg][H][dk][dk], Ns and Sin [nseg][H][dk][dv].
+cudaError_t segment_combine(const float *s0, const float *Ms, const float *Ns,
+                            float *Sin, const int32_t *seg_first, int nseq,
+                            int H, int dk, int dv, cudaStream_t s);
+// eye[i] = I (dk x dk) for nstates consecutive states.
+cudaError_t fill_identity(float *eye, long long nstates, int dk,
+                          cudaStream_t s);
+
 // Decode step: reads (and optionally clears) its sticky device error word
 // (a bulk copy that never completed).
 cudaError_t decode_read_error(unsigned *word, bool clear);

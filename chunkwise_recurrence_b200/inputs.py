@@ -67,6 +67,11 @@ WORKLOADS = {
                  dv=128, chunk=64, dtype="bf16", gate="scalar",
                  decay_lo=0.01, decay_hi=0.1, init_state=True,
                  varlen_nseq=8, varlen_lo=2048, varlen_hi=16384),
+        # long context, one sequence: fewer (sequence, head) chains than SMs
+        # (the case for context-parallel state passing)
+        Workload("gdn_longctx_b1_h16_t65536_d128_bf16", B=1, T=65536, H=16,
+                 dk=128, dv=128, chunk=64, dtype="bf16", gate="scalar",
+                 decay_lo=0.01, decay_hi=0.1, init_state=True),
     ]
 }
 

@@ -178,6 +178,37 @@ GDR_API gdr_status gdr_chunk_fwd_host(const void *q, const void *k, const void *
                               const gdr_opts *opts);
 
 /*
+ * gdr_chunk_fwd_segmented -- gdr_chunk_fwd with context-parallel state
+ * passing along each sequence.
+ *
+ * The update is affine in the preceding state ("DeltaTTT" page, §2
+ * Background), so a segment of a sequence maps its incoming state S to
+ * M S + N.  Every sequence is cut into up to `segments` pieces of equally
+ * many whole chunks; the pieces' M (the recurrence run from the identity
+ * with v = 0) and N (run from a zero state) are computed in parallel by the
+ * forward kernels, a combine kernel walks each sequence's pieces in order to
+ * give every piece its true initial state, and a last forward pass computes
+ * the outputs and final states.  The work is about three forward passes, in
+ * exchange for `segments` times more independent chains: it pays when the
+ * batch has fewer (sequence, head) pairs than the GPU has SMs (one long
+ * sequence, few heads).  segments = 1 gives gdr_chunk_fwd's result (with
+ * three passes).
+ *
+ * Arguments and layouts as for gdr_chunk_fwd, plus segments >= 1
+ * (GDR_ERR_INVALID_ARGUMENT otherwise).  With cu_seqlens, the offsets are
+ * read to the host once (the call synchronises `stream` for that) and
+ * checked: first 0, non-decreasing, last T (else GDR_ERR_INVALID_ARGUMENT).
+ * Scratch (about one bf16 / fp32 copy of v and out, and five dk x max(dk, dv)
+ * fp32 states per piece and head) comes from the library's per-device pool,
+ * stream-ordered on `stream`.
+ */
+GDR_API gdr_status gdr_chunk_fwd_segmented(
+    const void *q, const void *k, const void *v, const float *log_alpha,
+    const float *beta, const float *initial_state, void *out,
+    float *final_state, int B, int T, int H, int dk, int dv, int chunk,
+    int segments, cudaStream_t stream, const gdr_opts *opts);
+
+/*
  * gdr_chunk_fwd_noalloc -- gdr_chunk_fwd without any device allocation.
  *
  * The pages have no counterpart to this entry point: it exists for callers

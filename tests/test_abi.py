@@ -201,6 +201,27 @@ def test_backward_rejects_bad_arguments(lib):
              dk=None, dv=None, dla=None, db=None, gate=0, B=0) == OK
 
 
+def test_segmented_rejects_bad_arguments(lib):
+    def c(segments=4, **kw):
+        args = dict(q=A, k=A, v=A, la=A, beta=A, s0=None, out=A, sT=None, B=1,
+                    T=64, H=1, dk=128, dv=128, chunk=64, dtype=0, gate=1,
+                    cu=None, nseq=0, algo=0)
+        args.update(kw)
+        opts = gdr._Opts(args["dtype"], args["gate"], args["cu"], args["nseq"],
+                         args["algo"])
+        return lib.gdr_chunk_fwd_segmented(
+            args["q"], args["k"], args["v"], args["la"], args["beta"],
+            args["s0"], args["out"], args["sT"], args["B"], args["T"],
+            args["H"], args["dk"], args["dv"], args["chunk"], segments, None,
+            ctypes.byref(opts))
+    assert c(segments=0) == INVALID
+    assert c(segments=-3) == INVALID
+    assert c(q=None) == INVALID
+    assert c(dk=48) == UNSUPPORTED
+    assert c(q=None, k=None, v=None, la=None, beta=None, out=None, gate=0,
+             B=0) == OK
+
+
 def test_algo_applies(lib):
     assert gdr.algo_applies("staged", "fp32", "none", 16, 16, 16)
     assert gdr.algo_applies("auto", "bf16", "channel", 128, 64, 32)
