@@ -102,7 +102,11 @@ struct Layout {
   // channel gate, per key channel, for the chunk in progress: e^{g_m}
   // (g_m = g at row 31) and e^{g_C - g_m}
   static constexpr uint32_t GM = GC + 1536;       // [2][128]
-  static constexpr uint32_t MISC = GM + 1024;     // barriers, tmem base, flags
+  // channel gate: the chunk's log-decays, fp32 [2][64 rows][64 channels]
+  // (channels 0..63, then 64..127), loaded by TMA one chunk ahead
+  static constexpr uint32_t LA = (GM + 1024 + 127) & ~127u;
+  static constexpr uint32_t LA_BYTES = (GATE == 2) ? 32768 : 0;
+  static constexpr uint32_t MISC = LA + LA_BYTES; // barriers, tmem base, flags
   static constexpr uint32_t BYTES = MISC + 256;
   static_assert(BYTES + 1024 <= 232448, "shared memory budget");
 };
@@ -122,6 +126,7 @@ enum {
   B_TREADY, B_WDONE, B_WREADY, B_SREADY, B_XDONE, B_VNREADY, B_SDONE,
   B_ODONE, B_DRAIN, B_FULLV,
   B_CONV,                // K (scalar / no gate) and V fp16 (convert warps)
+  B_LAFULL, B_LAFREE,    // channel gate: log-decay tile landed / read
   B_COUNT
 };
 
@@ -316,7 +321,8 @@ template <int GATE>
 __global__ void __launch_bounds__(kThreads, 1)
     gdr_fused_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                         const __grid_constant__ CUtensorMap tmk,
-                        const __grid_constant__ CUtensorMap tmv, Params p) {
+                        const __grid_constant__ CUtensorMap tmv,
+                        const __grid_constant__ CUtensorMap tmla, Params p) {
   using Lay = Layout<GATE>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-aligned base, derived by pointer arithmetic on the shared array so
@@ -342,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     const uint32_t counts[B_COUNT] = {
         1, 1, 1, 1, 1, kPrep, 1, 1, kPrep, 1, kPrep, 128, 1, 128, 1, 1, 1, 1,
-        kConv};
+        kConv, 1, kPrep};
     for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], counts[i]);
     *abort_flag = 0;
     fence_mbar_init();
@@ -362,9 +368,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_map(&tmq);
       tma_prefetch_map(&tmk);
       tma_prefetch_map(&tmv);
-      int issued = 0, issued_v = 0;
+      if (GATE == 2) tma_prefetch_map(&tmla);
+      int issued = 0, issued_v = 0, issued_la = 0;
       for (int m = 0; m < NC; ++m) {
         const int s = m & 1;
+        if (GATE == 2) {
+          // log-decays of chunk m, once the prep warps have read chunk m-1's
+          if (m >= 1 && !wait_bar(cx, B_LAFREE, (m - 1) & 1)) break;
+          mbar_arrive_expect_tx(&bar[B_LAFULL], 2 * 16384);
+          for (int kb = 0; kb < 2; ++kb)
+            tma_load_3d(sm + Lay::LA + kb * 16384, &tmla, &bar[B_LAFULL],
+                        kb * 64, h, start + m * kC);
+          issued_la = m + 1;
+        }
         if (m >= 2 && !wait_bar(cx, B_EMPTY0 + s, ((m - 2) >> 1) & 1)) break;
         const int tok0 = start + m * kC;
         uint8_t *stg = sm + OFF_STAGE + s * kStageBytes;
@@ -396,6 +412,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (issued_v > 0) {
           const long long t0 = clock64();
           while (!mbar_try_wait(&bar[B_FULLV], (issued_v - 1) & 1) &&
+                 clock64() - t0 < (1ll << 28)) {
+          }
+        }
+        if (issued_la > 0) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(&bar[B_LAFULL], (issued_la - 1) & 1) &&
                  clock64() - t0 < (1ll << 28)) {
           }
         }
@@ -777,16 +799,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // 31: Q e^{g-g_m}, K e^{g-g_m}, K e^{g_m-g} (bf16)
       float amax = 0.f;
       if (GATE == 2) {
-        if (!group_all(wait_bar(cx, B_FULL0 + s, (m >> 1) & 1), 2, kPrep))
+        if (!group_all(wait_bar(cx, B_FULL0 + s, (m >> 1) & 1) &&
+                           wait_bar(cx, B_LAFULL, m & 1),
+                       2, kPrep))
           break;
         const int c = pt & 127, half = pt >> 7;
-        const float *la = p.log_alpha + ((size_t)tok0 * p.H + h) * kD + c;
-        const size_t rs = (size_t)p.H * kD;
+        const float *la = reinterpret_cast<const float *>(sm + Lay::LA) +
+                          (c >> 6) * 4096 + (c & 63);
         float lv[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int r = half * 32 + j;
-          lv[j] = (r < L) ? la[r * rs] : 0.f;
+          lv[j] = (r < L) ? la[r * 64] : 0.f;
         }
         float gm = 0.f;
         if (half == 0) {
@@ -794,8 +818,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 32; ++j) gm += lv[j];
         } else {
 #pragma unroll
-          for (int r = 0; r < 32; ++r) gm += (r < L) ? la[r * rs] : 0.f;
+          for (int r = 0; r < 32; ++r) gm += (r < L) ? la[r * 64] : 0.f;
         }
+        // the tile is in registers: the next chunk's may land
+        mbar_arrive(&bar[B_LAFREE]);
         float gg = half ? gm : 0.f;
         uint8_t *kt = stg + (c >> 6) * 16384, *qt = kt + 8192;
         uint8_t *knt = sm + Lay::KN + (c >> 6) * 8192;
@@ -1180,26 +1206,38 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [ntok][H][128] bf16, box of 64 channels x 1 head x 64 tokens, 128-B swizzle
-bool make_map(CUtensorMap *map, const void *base, int ntok, int H) {
+// [ntok][H][128], box of 64 channels x 1 head x 64 tokens: bf16 with the
+// 128-B swizzle (q, k, v), or fp32 unswizzled (per-channel log-decays)
+bool make_map(CUtensorMap *map, const void *base, int ntok, int H,
+              bool f32 = false) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
+  const cuuint64_t es_bytes = f32 ? 4 : 2;
   const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H,
                               (cuuint64_t)(ntok > 0 ? ntok : 1)};
-  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * es_bytes,
+                                 (cuuint64_t)H * kD * es_bytes};
   const cuuint32_t box[3] = {64, 1, (cuuint32_t)kC};
   const cuuint32_t es[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base),
-             dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return enc(map,
+             f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+             3, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE,
+             f32 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int GATE>
 cudaError_t launch(const Problem &pr, cudaStream_t s) {
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mla;
   if (!make_map(&mq, pr.q, pr.ntok, pr.H) || !make_map(&mk, pr.k, pr.ntok, pr.H) ||
       !make_map(&mv, pr.v, pr.ntok, pr.H))
+    return cudaErrorInvalidValue;
+  // the channel gate's log-decays; the other gates never read this map
+  if (GATE == 2 ? !make_map(&mla, pr.log_alpha, pr.ntok, pr.H, true)
+                : !make_map(&mla, pr.q, pr.ntok, pr.H))
     return cudaErrorInvalidValue;
   Params p;
   p.beta = pr.beta;
@@ -1217,7 +1255,8 @@ cudaError_t launch(const Problem &pr, cudaStream_t s) {
       gdr_fused_tc_kernel<GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
       smem);
   if (e != cudaSuccess) return e;
-  gdr_fused_tc_kernel<GATE><<<pr.nseq * pr.H, kThreads, smem, s>>>(mq, mk, mv, p);
+  gdr_fused_tc_kernel<GATE><<<pr.nseq * pr.H, kThreads, smem, s>>>(mq, mk, mv, mla,
+                                                                 p);
   return cudaGetLastError();
 }
 
