@@ -427,10 +427,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t nw = smem_u32(sm + OFF_NW), vt = smem_u32(sm + OFF_V),
-                     kn = smem_u32(sm + Lay::KN);
-      auto stage = [&](int m) {
-        return smem_u32(sm + OFF_STAGE + (m & 1) * kStageBytes);
-      };
+                     kn = smem_u32(sm + Lay::KN), sm_base_u32 = smem_u32(sm);
+      // Shared-memory descriptors are built once; a K step or sub-tile
+      // only adds its byte offset / 16 to the start-address field (shared
+      // addresses stay below 256 KB, so the 14-bit field never carries).
+      auto dadd = [](uint64_t d, uint32_t bytes) { return d + (bytes >> 4); };
+      const uint64_t st16[2] = {sdesc_sw128(sm_base_u32 + OFF_STAGE, 16, 1024),
+                                sdesc_sw128(sm_base_u32 + OFF_STAGE + kStageBytes,
+                                            16, 1024)};
+      const uint64_t stmn[2] = {
+          sdesc_sw128(sm_base_u32 + OFF_STAGE, 16384, 1024),
+          sdesc_sw128(sm_base_u32 + OFF_STAGE + kStageBytes, 16384, 1024)};
+      auto st_k = [&](int m) { return (m & 1) ? st16[1] : st16[0]; };
+      auto st_mn = [&](int m) { return (m & 1) ? stmn[1] : stmn[0]; };
+      const uint64_t d_kn = sdesc_sw128(kn, 16, 1024);
+      const uint64_t d_vt = sdesc_sw128(vt, 8192, 1024);
+      const uint64_t d_nw = sdesc_sw128(nw, 8192, 1024);
+      const uint64_t d_tpb = sdesc_sw128(smem_u32(sm + Lay::TPB), 16, 1024);
+      const uint64_t d_tpw = sdesc_sw128(
+          smem_u32(sm + (GATE == 2 ? Lay::TPB : Lay::TPG)), 16, 1024);
+      const uint64_t d_tplo = sdesc_sw128(smem_u32(sm + Lay::TPB_LO), 16, 1024);
+      const uint64_t d_p[2] = {sdesc_sw128(smem_u32(sm + OFF_P), 16, 1024),
+                               sdesc_sw128(smem_u32(sm + OFF_P + 8192), 16, 1024)};
       // channel gate: the prep warps rescale Q, K in place first (kk_ready);
       // otherwise K K^T runs straight on the landed bf16 tiles
       auto kk_inputs_ready = [&](int m) {
@@ -438,15 +456,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                          : wait_bar(cx, B_FULL0 + (m & 1), (m >> 1) & 1);
       };
       auto issue_kk = [&](int m) {
-        const uint32_t base = stage(m);
+        const uint64_t base = st_k(m);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-          const uint64_t a = sdesc_sw128(base + koff, 16, 1024);
+          const uint64_t a = dadd(base, koff);
           const uint64_t b =
-              GATE == 2
-                  ? sdesc_sw128(kn + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024)
-                  : sdesc_sw128(base + koff, 16, 1024);
+              GATE == 2 ? dadd(d_kn, (ks >> 2) * 8192 + (ks & 3) * 32) : a;
           mma_f16kind(tmem + ACC_KK, a, b, ID_KK_B, ks > 0);
         }
         mma_commit(&bar[B_KKDONE0 + (m & 1)]);
@@ -460,25 +476,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_uw = [&](int m) {
         if (!wait_bar(cx, B_CONV, m & 1)) return false;
         tc_fence_after();
-        const uint32_t base = stage(m);
+        const uint64_t base = st_mn(m);
         const uint32_t accv = tmem + ACC_V + (m & 1) * 64;
-        const uint32_t tpb = smem_u32(sm + Lay::TPB);
-        const uint32_t tpw = smem_u32(sm + (GATE == 2 ? Lay::TPB : Lay::TPG));
-        const uint32_t tplo = smem_u32(sm + Lay::TPB_LO);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_f16kind(accv, sdesc_sw128(vt + ks * 2048, 8192, 1024),
-                      sdesc_sw128(tpb + ks * 32, 16, 1024), kIdUW, ks > 0);
+          mma_f16kind(accv, dadd(d_vt, ks * 2048), dadd(d_tpb, ks * 32), kIdUW,
+                      ks > 0);
         if (GATE != 2) {
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_f16kind(accv, sdesc_sw128(vt + ks * 2048, 8192, 1024),
-                        sdesc_sw128(tplo + ks * 32, 16, 1024), kIdUW, 1);
+            mma_f16kind(accv, dadd(d_vt, ks * 2048), dadd(d_tplo, ks * 32),
+                        kIdUW, 1);
         }
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_f16kind(tmem + ACC_W, sdesc_sw128(base + ks * 2048, 16384, 1024),
-                      sdesc_sw128(tpw + ks * 32, 16, 1024), kIdUW, ks > 0);
+          mma_f16kind(tmem + ACC_W, dadd(base, ks * 2048), dadd(d_tpw, ks * 32),
+                      kIdUW, ks > 0);
         mma_commit(&bar[B_WDONE]);
         mma_commit(&bar[B_VFREE]);
         return true;
@@ -515,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       for (int m = 0; m < NC && ok; ++m) {
-        const uint32_t base = stage(m);
+        const uint64_t qbase = dadd(st_k(m), 8192), kbase = st_mn(m);
         // X(m): V_new^T = U^T + S^T (-W)^T ; O^T = S^T (Q e^g)^T
         if (!wait_bar(cx, B_SREADY, m & 1) || !wait_bar(cx, B_WREADY, m & 1))
           break;
@@ -525,14 +538,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_f16kind_ts(tmem + ACC_V + (m & 1) * 64, st_op + 8 * ks,
-                         sdesc_sw128(nw + ks * 2048, 8192, 1024), ID_XV, 1);
+                         dadd(d_nw, ks * 2048), ID_XV, 1);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_f16kind_ts(tmem + ACC_O + (m & 1) * 64, st_op + 8 * ks,
-                         sdesc_sw128(base + 8192 + (ks >> 2) * 16384 +
-                                         (ks & 3) * 32,
-                                     16, 1024),
-                         ID_XO, ks > 0);
+                         dadd(qbase, (ks >> 2) * 16384 + (ks & 3) * 32), ID_XO,
+                         ks > 0);
         mma_commit(&bar[B_XDONE]);
         // K K^T of chunk m+1 while the state warps turn V_new into an
         // operand, if its inputs are in (the channel gate's rescaling may
@@ -545,13 +556,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t vn_op = tmem + ACC_V + (m & 1) * 64;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_f16kind_ts(tmem + ACC_S, vn_op + 8 * ks,
-                         sdesc_sw128(base + ks * 2048, 16384, 1024), ID_SU, 1);
-        const uint32_t pt = smem_u32(sm + OFF_P + (m & 1) * 8192);
+          mma_f16kind_ts(tmem + ACC_S, vn_op + 8 * ks, dadd(kbase, ks * 2048),
+                         ID_SU, 1);
+        const uint64_t pbase = (m & 1) ? d_p[1] : d_p[0];
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           mma_f16kind_ts(tmem + ACC_O + (m & 1) * 64, vn_op + 8 * ks,
-                         sdesc_sw128(pt + ks * 32, 16, 1024), ID_OI, 1);
+                         dadd(pbase, ks * 32), ID_OI, 1);
         // S done also covers the intra-chunk output: both read V_new(m),
         // whose columns S^T(m+1) reuses
         mma_commit(&bar[B_SDONE]);
