@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--algo auto|staged|fused_tc]
+                    [--batch B] [--segments S] [--decode] [--backward]
 
 One step = one gdr_chunk_fwd call over one batch of the workload (all four
 stages: log-decay cumsum, WY/UT transform, state passing, output), inputs
@@ -676,6 +677,9 @@ def main(argv=None):
                     help="sequences per decode step")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (gdr_backward) instead")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="run a fixed-length workload with this many "
+                         "sequences instead of its own")
     ap.add_argument("--segments", type=int, default=0,
                     help="context-parallel forward (gdr_chunk_fwd_segmented) "
                          "with this many pieces per sequence")
@@ -683,6 +687,10 @@ def main(argv=None):
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
+    if args.batch:
+        if w.varlen_nseq or args.batch < 1:
+            raise SystemExit("--batch needs a fixed-length workload and B >= 1")
+        w = w.with_(B=args.batch, name=f"{w.name}@B{args.batch}")
     if args.decode and args.impl == "ours":
         return run_decode(args)
     if args.backward and args.impl == "ours":
