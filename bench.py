@@ -567,7 +567,10 @@ def run_decode(args):
 
 
 BACKWARD_METRIC = ("tokens/s, backward pass (gdr_backward) of the chunked "
-                   "gated-delta fwd; % HBM roofline")
+                   "gated-delta fwd; % fp32 ALU roofline")
+# fp32 flops per state element, token and head over the backward's three
+# sweeps: forward and replay 5 each (decay, S~^T k, k u^T), reverse 19
+BACKWARD_FLOPS_PER_ELEM = 29
 
 
 def run_backward(args, w):
@@ -618,8 +621,15 @@ def run_backward(args, w):
     by = ntok * H * (esz * (2 * dk + 2 * dv) + 4 + la_b +
                      4 * (2 * dk + dv) + 4 + la_b)
     by += inp.nseq * H * dk * dv * 4 * (2 + (1 if inp.s0 is not None else 0))
-    peaks, peak_src = load_peaks()
     gbs = by / (statistics.mean(per_step) / 1e3) / 1e9
+    cols = dk >= 32 and dv >= 32   # the column-split kernel + its reduction
+    clk = clocks.summary()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    max_mhz = clk.get("sm_max_mhz") or 1965.0
+    # CUDA-core fp32 peak: SMs x 128 lanes x 2 flops (FMA) x max SM clock
+    alu_peak = sms * 128 * 2 * max_mhz * 1e6 / 1e12
+    tflops = (BACKWARD_FLOPS_PER_ELEM * dk * dv * ntok * H /
+              (statistics.mean(per_step) / 1e3) / 1e12)
     line = {
         "metric": BACKWARD_METRIC, "value": ntok / (ms / 1e3),
         "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
@@ -628,13 +638,19 @@ def run_backward(args, w):
         "data": "synthetic",
         "config": {**workload_config(w, inp), "algo": "token-level reverse",
                    "l2": "inputs larger than L2 (no flush)"},
-        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
-                     "traffic": None, "peak_source": peak_src,
-                     "kernel": "gdr_bwd_kernel",
+        "roofline": {"bound": "alu", "achieved": tflops, "peak": alu_peak,
+                     "unit": "TFLOP/s", "frac": tflops / alu_peak,
+                     "traffic": None,
+                     "peak_source": f"derived: {sms} SMs x 128 fp32 lanes x 2 "
+                                    f"x {max_mhz:.0f} MHz",
+                     "kernel": ("gdr_bwd_cols_kernel" if cols
+                                else "gdr_bwd_kernel"),
+                     "flops_per_step": BACKWARD_FLOPS_PER_ELEM * dk * dv *
+                     ntok * H,
+                     "hbm_gbs_on_algorithmic_bytes": gbs,
                      "algorithmic_bytes_per_launch": by},
-        "clocks": clocks.summary(),
-        "gpu_launches": args.steps,
+        "clocks": clk,
+        "gpu_launches": args.steps * (2 if cols else 1),
         "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
     }
     print(json.dumps(line), flush=True)

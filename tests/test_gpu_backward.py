@@ -62,6 +62,11 @@ def _check(w, seed=0, with_final=True, with_s0_grad=True):
     ("kda_b4_h16_t4096_d128_bf16", dict(B=1, T=33, H=2, dk=64, dv=128)),
     ("kda_b4_h16_t4096_d128_bf16", dict(B=2, T=16, H=1, dk=16, dv=32,
                                         dtype="fp32")),
+    # column-split kernel: two column groups, fp32, channel gate, ragged
+    # last window; no gate with four groups
+    ("kda_b4_h16_t4096_d128_bf16", dict(B=2, T=19, H=2, dk=128, dv=64,
+                                        dtype="fp32")),
+    ("deltanet_b1_h1_t256_d16_fp32", dict(T=45, H=3, dk=32, dv=128)),
 ])
 def test_backward_matches_autograd(name, shape):
     _check(WORKLOADS[name].with_(**shape))
