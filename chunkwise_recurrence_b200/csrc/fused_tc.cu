@@ -102,9 +102,13 @@ struct Layout {
   // channel gate, per key channel, for the chunk in progress: e^{g_m}
   // (g_m = g at row 31) and e^{g_C - g_m}
   static constexpr uint32_t GM = GC + 1536;       // [2][128]
+  // channel gate: each half-chunk's log-decay total per key channel [2][128]
+  static constexpr uint32_t TT = GM + 1024;
+  static constexpr uint32_t TT_BYTES = (GATE == 2) ? 1024 : 0;
   // channel gate: the chunk's log-decays, fp32 [2][64 rows][64 channels]
-  // (channels 0..63, then 64..127), loaded by TMA one chunk ahead
-  static constexpr uint32_t LA = (GM + 1024 + 127) & ~127u;
+  // (channels 0..63, then 64..127), loaded by TMA one chunk ahead; turned
+  // into running sums in place
+  static constexpr uint32_t LA = (TT + TT_BYTES + 127) & ~127u;
   static constexpr uint32_t LA_BYTES = (GATE == 2) ? 32768 : 0;
   static constexpr uint32_t MISC = LA + LA_BYTES; // barriers, tmem base, flags
   static constexpr uint32_t BYTES = MISC + 256;
@@ -814,51 +818,85 @@ __global__ void __launch_bounds__(kThreads, 1)
                            wait_bar(cx, B_LAFULL, m & 1),
                        2, kPrep))
           break;
-        const int c = pt & 127, half = pt >> 7;
-        const float *la = reinterpret_cast<const float *>(sm + Lay::LA) +
-                          (c >> 6) * 4096 + (c & 63);
-        float lv[32];
+        // (a) per key channel c and half of the chunk, the running sum of
+        // the log-decays over the half's rows, in place; each half's total
+        // in TT (rows past the sequence end add nothing)
+        {
+          const int c = pt & 127, half = pt >> 7;
+          float *la = reinterpret_cast<float *>(sm + Lay::LA) +
+                      (c >> 6) * 4096 + (c & 63);
+          float lv[32];   // all loads first: one latency, not 32
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int r = half * 32 + j;
-          lv[j] = (r < L) ? la[r * 64] : 0.f;
+          for (int j = 0; j < 32; ++j) {
+            const int r = half * 32 + j;
+            lv[j] = (r < L) ? la[r * 64] : 0.f;
+          }
+          float run = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            run += lv[j];
+            la[(half * 32 + j) * 64] = run;
+          }
+          reinterpret_cast<float *>(sm + Lay::TT)[half * 128 + c] = run;
         }
-        float gm = 0.f;
-        if (half == 0) {
+        named_bar_sync(2, kPrep);
+        // (b) with g_m = g at row 31 (the first half's total): row r's
+        // g_r - g_m is its running sum minus g_m in the first half, and its
+        // running sum in the second.  Item = row r, 8 channels (16 bytes of
+        // Q, K and K e^{g_m-g}); thread pt takes items pt + 256 u.
+        {
+          const float *gl = reinterpret_cast<const float *>(sm + Lay::LA);
+          const float *T0 = reinterpret_cast<const float *>(sm + Lay::TT);
+#pragma unroll 2
+          for (int u = 0; u < 4; ++u) {
+            const int item = pt + 256 * u, r = item >> 4, ch = item & 15;
+            const int kb = ch >> 3, cc = ch & 7;
+            const float4 *gp = reinterpret_cast<const float4 *>(
+                gl + kb * 4096 + r * 64 + cc * 8);
+            const float4 g0 = gp[0], g1 = gp[1];
+            float x[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+            if (r < 32) {
+              const float4 *tp = reinterpret_cast<const float4 *>(T0 + ch * 8);
+              const float4 t0 = tp[0], t1 = tp[1];
+              x[0] -= t0.x; x[1] -= t0.y; x[2] -= t0.z; x[3] -= t0.w;
+              x[4] -= t1.x; x[5] -= t1.y; x[6] -= t1.z; x[7] -= t1.w;
+            }
+            const uint32_t off = kb * 16384 + sw128_chunk(r, cc);
+            uint4 *qp = reinterpret_cast<uint4 *>(stg + off + 8192);
+            uint4 *kp = reinterpret_cast<uint4 *>(stg + off);
+            uint4 qv = *qp, kv = *kp, nv;
+            uint32_t *qw = reinterpret_cast<uint32_t *>(&qv);
+            uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
+            uint32_t *knw = reinterpret_cast<uint32_t *>(&nv);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) gm += lv[j];
-        } else {
-#pragma unroll
-          for (int r = 0; r < 32; ++r) gm += (r < L) ? la[r * 64] : 0.f;
+            for (int e = 0; e < 4; ++e) {
+              const float ep0 = __expf(x[2 * e]), ep1 = __expf(x[2 * e + 1]);
+              const float en0 = __expf(-x[2 * e]), en1 = __expf(-x[2 * e + 1]);
+              float q0, q1, k0, k1;
+              unpack_bf16(qw[e], q0, q1);
+              unpack_bf16(kw[e], k0, k1);
+              amax = fmaxf(amax, fmaxf(fmaxf(fabsf(q0), fabsf(q1)),
+                                       fmaxf(fabsf(k0), fabsf(k1))));
+              qw[e] = pack_bf16(q0 * ep0, q1 * ep1);
+              kw[e] = pack_bf16(k0 * ep0, k1 * ep1);
+              knw[e] = pack_bf16(k0 * en0, k1 * en1);
+            }
+            *qp = qv;
+            *kp = kv;
+            *reinterpret_cast<uint4 *>(sm + Lay::KN + kb * 8192 +
+                                       sw128_chunk(r, cc)) = nv;
+          }
+          // per-channel factors, one exponential each per chunk: e^{g_m};
+          // e^{g_C} (decay of S) in gc; e^{g_C - g_m} in gM + 128
+          if (pt < 128) {
+            const float t0 = T0[pt], t1 = T0[128 + pt];
+            gM[pt] = __expf(t0);
+            gc[pt] = __expf(t0 + t1);
+            gM[128 + pt] = __expf(t1);
+          }
         }
-        // the tile is in registers: the next chunk's may land
+        // the log-decay tile has been read: the next chunk's may land
         mbar_arrive(&bar[B_LAFREE]);
-        float gg = half ? gm : 0.f;
-        uint8_t *kt = stg + (c >> 6) * 16384, *qt = kt + 8192;
-        uint8_t *knt = sm + Lay::KN + (c >> 6) * 8192;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int r = half * 32 + j;
-          gg += lv[j];
-          const float ep = __expf(gg - gm), en = __expf(gm - gg);
-          const uint32_t off = sw128_off(r, c & 63);
-          __nv_bfloat16 *qe = reinterpret_cast<__nv_bfloat16 *>(qt + off);
-          __nv_bfloat16 *ke = reinterpret_cast<__nv_bfloat16 *>(kt + off);
-          const float qv = __bfloat162float(*qe), kv = __bfloat162float(*ke);
-          amax = fmaxf(amax, fmaxf(fabsf(qv), fabsf(kv)));
-          *qe = __float2bfloat16_rn(qv * ep);
-          *ke = __float2bfloat16_rn(kv * ep);
-          *reinterpret_cast<__nv_bfloat16 *>(knt + off) =
-              __float2bfloat16_rn(kv * en);
-        }
-        // per-channel factors, one exponential each per chunk: e^{g_m}, and
-        // e^{g_C} (decay of S) and e^{g_C - g_m} in gc / gM + 128
-        if (half == 0) {
-          gM[c] = __expf(gm);
-        } else {
-          gc[c] = __expf(gg);
-          gM[128 + c] = __expf(gg - gm);
-        }
         fence_proxy_async_smem();
         mbar_arrive(&bar[B_KKREADY]);
       }
@@ -928,24 +966,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (GATE == 2) {
-        // Q e^{g-g_m}, K e^{g-g_m} (bf16) -> Q e^g, K e^g (fp16), in place
+        // Q e^{g-g_m}, K e^{g-g_m} (bf16) -> Q e^g, K e^g (fp16), in place.
+        // Item = row, 8 channels; the 8 factors e^{g_m} are two vector loads
+        // shared by the Q and the K chunk.
+#pragma unroll 2
         for (int idx = pt; idx < kC * 16; idx += kPrep) {
           const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
           const uint32_t off = kb * 16384 + sw128_chunk(r, cc & 7);
-          const int cbase = kb * 64 + (cc & 7) * 8;
+          const float4 *fp = reinterpret_cast<const float4 *>(gM + cc * 8);
+          const float4 f0 = fp[0], f1 = fp[1];
+          const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+          uint4 *kp = reinterpret_cast<uint4 *>(stg + off);
+          uint4 *qp = reinterpret_cast<uint4 *>(stg + off + 8192);
+          uint4 kv = *kp, qv = *qp;
+          uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
+          uint32_t *qw = reinterpret_cast<uint32_t *>(&qv);
 #pragma unroll
-          for (int part = 0; part < 2; ++part) {
-            uint4 *ptr = reinterpret_cast<uint4 *>(stg + off + part * 8192);
-            uint4 xv = *ptr;
-            uint32_t *w = reinterpret_cast<uint32_t *>(&xv);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float a0, a1;
-              unpack_bf16(w[e], a0, a1);
-              w[e] = pack_f16(a0 * gM[cbase + 2 * e], a1 * gM[cbase + 2 * e + 1]);
-            }
-            *ptr = xv;
+          for (int e = 0; e < 4; ++e) {
+            float a0, a1;
+            unpack_bf16(kw[e], a0, a1);
+            kw[e] = pack_f16(a0 * f[2 * e], a1 * f[2 * e + 1]);
+            unpack_bf16(qw[e], a0, a1);
+            qw[e] = pack_f16(a0 * f[2 * e], a1 * f[2 * e + 1]);
           }
+          *kp = kv;
+          *qp = qv;
         }
       }
       named_bar_sync(2, kPrep);
@@ -1163,24 +1208,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4 *>(stg + off[u]) = xk[u];
         }
       }
+#pragma unroll 2
       for (int idx = pt; GATE == 2 && idx < kC * 16; idx += kPrep) {
         const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
         uint8_t *kp = stg + kb * 16384 + sw128_chunk(r, cc & 7);
-        {
-          // K~ = (K e^{g_m-g}) e^{g_C-g_m}, per channel
-          uint4 kv = *reinterpret_cast<const uint4 *>(
-              sm + Lay::KN + kb * 8192 + sw128_chunk(r, cc & 7));
-          uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
-          const int cbase = kb * 64 + (cc & 7) * 8;
+        // K~ = (K e^{g_m-g}) e^{g_C-g_m}, per channel (8 factors, two
+        // vector loads)
+        const float4 *fp = reinterpret_cast<const float4 *>(gM + 128 + cc * 8);
+        const float4 f0 = fp[0], f1 = fp[1];
+        const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+        uint4 kv = *reinterpret_cast<const uint4 *>(
+            sm + Lay::KN + kb * 8192 + sw128_chunk(r, cc & 7));
+        uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float a0, a1;
-            unpack_bf16(kw[e], a0, a1);
-            kw[e] = pack_f16(a0 * gM[128 + cbase + 2 * e],
-                             a1 * gM[128 + cbase + 2 * e + 1]);
-          }
-          *reinterpret_cast<uint4 *>(kp) = kv;
+        for (int e = 0; e < 4; ++e) {
+          float a0, a1;
+          unpack_bf16(kw[e], a0, a1);
+          kw[e] = pack_f16(a0 * f[2 * e], a1 * f[2 * e + 1]);
         }
+        *reinterpret_cast<uint4 *>(kp) = kv;
       }
       if (!(amax <= kF16Max)) atomicOr(&g_fused_error, kErrRange);
       fence_proxy_async_smem();
