@@ -303,23 +303,40 @@ def run_ours(args, w):
                      device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    def step(s=stream):
         if args.segments:
             gdr.chunk_fwd_segmented(q, k, v, beta, la, s0,
                                     segments=args.segments, chunk=w.chunk,
                                     gate=w.gate, cu_seqlens=cu, out=out,
                                     final_state=sT, algo=args.algo,
-                                    stream=stream)
+                                    stream=s)
             return
         gdr.chunk_fwd(q, k, v, beta, la, s0, chunk=w.chunk, gate=w.gate,
                       cu_seqlens=cu, out=out, final_state=sT, algo=args.algo,
-                      stream=stream)
+                      stream=s)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     if gdr.device_error() != 0:
         raise RuntimeError("device-side error during warm-up")
+    # One step as a CUDA graph (the same launches, without the per-call host
+    # work between steps); the context-parallel call reads the sequence
+    # offsets on the host and runs directly.
+    graph = None
+    if not args.segments:
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(torch.cuda.current_stream(dev))
+            g.replay()
+            torch.cuda.synchronize()
+            if gdr.device_error() == 0:
+                graph = g
+        except RuntimeError:
+            torch.cuda.synchronize()
+            graph = None
+    run_step = graph.replay if graph is not None else step
     algo_used = args.algo
     if algo_used == "auto":
         algo_used = ("fused_tc" if (w.dtype == "bf16" and w.dk == 128 and
@@ -335,7 +352,7 @@ def run_ours(args, w):
         torch.cuda.synchronize()
         ev[0].record(stream)
         for i in range(args.steps):
-            step()
+            run_step()
             ev[i + 1].record(stream)
         torch.cuda.synchronize()
         if ws > 1:
@@ -344,6 +361,8 @@ def run_ours(args, w):
     total_ms = ev[0].elapsed_time(ev[-1])
     if gdr.device_error() != 0:
         raise RuntimeError("device-side error during timing")
+    launch_mode = "cuda graph of one step" if graph is not None else "direct"
+    del graph
 
     # ---- end to end through the host-buffer entry point
     pin = lambda t: None if t is None else t.pin_memory()  # noqa: E731
@@ -415,7 +434,8 @@ def run_ours(args, w):
                    "parallelism": f"dp{ws} (independent sequences)",
                    "algo": algo_used,
                    "segments": args.segments or None,
-                   "l2": "inputs larger than L2 (no flush)"},
+                   "l2": "inputs larger than L2 (no flush)",
+                   "launch": launch_mode},
         "tflops": fl * ws / (ms / 1e3) / 1e12,
         "roofline": roofline,
         "clocks": clocks.summary(),

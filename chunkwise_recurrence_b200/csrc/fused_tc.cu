@@ -129,8 +129,9 @@ enum {
   B_KKDONE0, B_KKDONE1,  // K K^T of the chunk done (MMA commit)
   B_TREADY, B_WDONE, B_WREADY, B_SREADY, B_XDONE, B_VNREADY, B_SDONE,
   B_ODONE, B_DRAIN, B_FULLV,
-  B_CONV,                // K (scalar / no gate) and V fp16 (convert warps)
+  B_CONV,                // channel gate: V, Q, K fp16 (convert warps)
   B_LAFULL, B_LAFREE,    // channel gate: log-decay tile landed / read
+  B_QCONV,               // channel gate: Q e^g fp16 (convert warps)
   B_COUNT
 };
 
@@ -352,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     const uint32_t counts[B_COUNT] = {
         1, 1, 1, 1, 1, kPrep, 1, 1, kPrep, 1, kPrep, 128, 1, 128, 1, 1, 1, 1,
-        kConv, 1, kPrep};
+        kConv, 1, kPrep, kConv};
     for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], counts[i]);
     *abort_flag = 0;
     fence_mbar_init();
@@ -534,7 +535,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int m = 0; m < NC && ok; ++m) {
         const uint64_t qbase = dadd(st_k(m), 8192), kbase = st_mn(m);
         // X(m): V_new^T = U^T + S^T (-W)^T ; O^T = S^T (Q e^g)^T
-        if (!wait_bar(cx, B_SREADY, m & 1) || !wait_bar(cx, B_WREADY, m & 1))
+        if (!wait_bar(cx, B_SREADY, m & 1) || !wait_bar(cx, B_WREADY, m & 1) ||
+            (GATE == 2 && !wait_bar(cx, B_QCONV, m & 1)))
           break;
         tc_fence_after();
         // A = S^T, fp16 pairs in tensor memory (8 columns per K step)
@@ -728,18 +730,53 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 14) {
     // ------------------------------------------------------ convert warps
     // Channel gate: V -> fp16 in place for U = (T diag b) V, once V has
-    // landed.  Scalar / no gate: U and W read the raw bf16 tiles, and these
-    // warps only pass the V arrival on.
+    // landed, and Q, K -> fp16 Q e^g, K e^g once K K^T has read them.
+    // Scalar / no gate: U and W read the raw bf16 tiles, and these warps
+    // only pass the V arrival on.
     const int ct = threadIdx.x - 14 * 32;
+    const float *gM = reinterpret_cast<const float *>(sm + Lay::GM);
     for (int m = 0; m < NC; ++m) {
       if (!group_all(wait_bar(cx, B_FULLV, m & 1), 3, kConv)) break;
       if (GATE == 2) {
 #pragma unroll 4
         for (int i = ct; i < 1024; i += kConv)
           bf16_to_f16_16B(sm + OFF_V + i * 16, 1.f);
-        fence_proxy_async_smem();
+        // once K K^T has read them: K e^{g-g_m}, then Q e^{g-g_m} (bf16)
+        // -> K e^g for W (conv), then Q e^g for X (qconv), fp16 in place.
+        // Item = row, 8 channels; the 8 factors e^{g_m} are two vector loads.
+        if (!group_all(wait_bar(cx, B_KKDONE0 + (m & 1), (m >> 1) & 1), 3,
+                       kConv))
+          break;
+        uint8_t *stg = sm + OFF_STAGE + (m & 1) * kStageBytes;
+        auto to_f16_ge = [&](uint32_t part) {
+#pragma unroll 4
+          for (int idx = ct; idx < kC * 16; idx += kConv) {
+            const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
+            const float4 *fp = reinterpret_cast<const float4 *>(gM + cc * 8);
+            const float4 f0 = fp[0], f1 = fp[1];
+            const float f[8] = {f0.x, f0.y, f0.z, f0.w,
+                                f1.x, f1.y, f1.z, f1.w};
+            uint4 *xp = reinterpret_cast<uint4 *>(
+                stg + kb * 16384 + part + sw128_chunk(r, cc & 7));
+            uint4 xv = *xp;
+            uint32_t *xw = reinterpret_cast<uint32_t *>(&xv);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float a0, a1;
+              unpack_bf16(xw[e], a0, a1);
+              xw[e] = pack_f16(a0 * f[2 * e], a1 * f[2 * e + 1]);
+            }
+            *xp = xv;
+          }
+          fence_proxy_async_smem();
+        };
+        to_f16_ge(0);
+        mbar_arrive(&bar[B_CONV]);
+        to_f16_ge(8192);
+        mbar_arrive(&bar[B_QCONV]);
+      } else {
+        mbar_arrive(&bar[B_CONV]);
       }
-      mbar_arrive(&bar[B_CONV]);
     }
   } else {
     // ------------------------------------------------------ prep warps
@@ -963,34 +1000,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                        pack_f16(v[8 * ch + 2], v[8 * ch + 3]),
                        pack_f16(v[8 * ch + 4], v[8 * ch + 5]),
                        pack_f16(v[8 * ch + 6], v[8 * ch + 7]));
-        }
-      }
-      if (GATE == 2) {
-        // Q e^{g-g_m}, K e^{g-g_m} (bf16) -> Q e^g, K e^g (fp16), in place.
-        // Item = row, 8 channels; the 8 factors e^{g_m} are two vector loads
-        // shared by the Q and the K chunk.
-#pragma unroll 2
-        for (int idx = pt; idx < kC * 16; idx += kPrep) {
-          const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
-          const uint32_t off = kb * 16384 + sw128_chunk(r, cc & 7);
-          const float4 *fp = reinterpret_cast<const float4 *>(gM + cc * 8);
-          const float4 f0 = fp[0], f1 = fp[1];
-          const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-          uint4 *kp = reinterpret_cast<uint4 *>(stg + off);
-          uint4 *qp = reinterpret_cast<uint4 *>(stg + off + 8192);
-          uint4 kv = *kp, qv = *qp;
-          uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
-          uint32_t *qw = reinterpret_cast<uint32_t *>(&qv);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float a0, a1;
-            unpack_bf16(kw[e], a0, a1);
-            kw[e] = pack_f16(a0 * f[2 * e], a1 * f[2 * e + 1]);
-            unpack_bf16(qw[e], a0, a1);
-            qw[e] = pack_f16(a0 * f[2 * e], a1 * f[2 * e + 1]);
-          }
-          *kp = kv;
-          *qp = qv;
         }
       }
       named_bar_sync(2, kPrep);
