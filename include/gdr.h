@@ -298,8 +298,12 @@ GDR_API gdr_status gdr_decode_step(const void *q, const void *k, const void *v,
  * dL/d final_state, it writes dL/dq, dL/dk, dL/dv, dL/d log_alpha,
  * dL/d beta and dL/d initial_state of the recurrence above (the same
  * definition gdr_chunk_fwd evaluates, whichever algorithm ran it).  It
- * runs the recurrence forward, checkpointing the state every 16 tokens in
- * scratch, then the reverse token recurrence window by window, all in fp32.
+ * runs the recurrence forward, checkpointing the state every 8 tokens in
+ * scratch (16 when dk or dv is 16), then the reverse token recurrence window
+ * by window, all in fp32.  For dk, dv >= 32 each (sequence, head) runs on
+ * dv/32 blocks of 32 value columns; their per-token shares of the row sums
+ * (dq, dk, d_log_alpha, d_beta) are added in a fixed order, so the result
+ * does not depend on scheduling.
  *
  * Inputs: q, k, v, log_alpha, beta, initial_state, B, T, H, dk, dv and opts
  * exactly as for gdr_chunk_fwd (opts->algo must be GDR_ALGO_AUTO);
@@ -309,8 +313,10 @@ GDR_API gdr_status gdr_decode_step(const void *q, const void *k, const void *v,
  *   dq, dk         [B][T][H][dk];   dv [B][T][H][dv];   d_beta [B][T][H];
  *   d_log_alpha    the layout of log_alpha; NULL iff gate is NONE;
  *   d_initial_state [N][H][dk][dv], or NULL to skip.
- * Scratch: about (ntok/16 + N) * H + 16 * N * H states of dk*dv floats,
- * allocated stream-ordered on `stream` from the library's per-device memory
+ * Scratch (dk, dv >= 32): (ntok/8 + N) * H + 8 * N * H states of dk*dv
+ * floats, plus the row-sum shares, 2 * (dv/32) * ntok * H * dk floats (3 *
+ * for the channel gate); for dk or dv = 16: (ntok/16 + N) * H + 16 * N * H
+ * states.  Allocated stream-ordered on `stream` from the library's per-device memory
  * pool, which keeps its memory between calls (the pool gdr_chunk_fwd_host
  * uses); GDR_ERR_OUT_OF_MEMORY on failure.
  * Status codes as for gdr_chunk_fwd.
