@@ -153,12 +153,18 @@ extern "C" gdr_status gdr_chunk_fwd(const void *q, const void *k,
 }
 
 // ---------------------------------------------------------------------------
-// Host-buffer entry.  The batch is cut into up to kHostPieces pieces of whole
-// sequences; each piece is an independent sub-problem with its own device
-// buffers.  Three streams overlap the pieces: the host-to-device copies of
-// piece i+1 (upload stream) run while piece i computes (the caller's stream)
-// and the results of piece i-1 come back (download stream), so the host link
-// carries both directions at once and the kernels hide behind the copies.
+// Host-buffer entry.  The work is cut into up to kHostPieces pieces, each
+// with its own device buffers.  Three streams overlap the pieces: the
+// host-to-device copies of piece i+1 (upload stream) run while piece i
+// computes (the caller's stream) and the results of piece i-1 come back
+// (download stream), so the host link carries both directions at once and
+// the kernels hide behind the copies.  Fixed-length batches are cut by time,
+// at chunk boundaries: a piece holds the same token range of every sequence
+// and starts from the state the previous piece ended with (kept on the
+// device), so the last piece -- the part that cannot hide behind an upload --
+// is a few chunks long.  The results are those of one call: the state passes
+// from piece to piece in fp32, exactly as from chunk to chunk.  Packed
+// batches are cut into pieces of whole sequences.
 namespace {
 
 constexpr int kHostPieces = 8;
@@ -234,6 +240,142 @@ struct EventSet {
 
 }  // namespace
 
+namespace {
+
+// Fixed-length host entry, cut by time (see above).
+gdr_status host_by_time(const Problem &p, const gdr_opts &o, const void *q,
+                        const void *k, const void *v, const float *log_alpha,
+                        const float *beta, const float *initial_state,
+                        void *out, float *final_state, cudaStream_t stream) {
+  const int B = p.nseq, T = p.T, C = p.chunk;
+  const int nck = (T + C - 1) / C;
+  const int P = nck < kHostPieces ? nck : kHostPieces;
+  int tb[kHostPieces + 1];   // token boundaries, multiples of C
+  for (int i = 0; i < P; ++i) tb[i] = (int)((long long)nck * i / P) * C;
+  tb[P] = T;
+  const size_t esz = o.dtype == GDR_FP32 ? 4 : 2;
+  const size_t gdim = o.gate == GDR_GATE_NONE     ? 0
+                      : o.gate == GDR_GATE_SCALAR ? 1
+                                                  : (size_t)p.dk;
+  const size_t state1 = (size_t)p.H * p.dk * p.dv * sizeof(float);
+  // per-token bytes, in the order q k v log_alpha beta out
+  const size_t tok_bytes[6] = {
+      (size_t)p.H * p.dk * esz, (size_t)p.H * p.dk * esz,
+      (size_t)p.H * p.dv * esz,
+      log_alpha ? (size_t)p.H * gdim * sizeof(float) : 0,
+      (size_t)p.H * sizeof(float), (size_t)p.H * p.dv * esz};
+  const void *host_in[5] = {q, k, v, log_alpha, beta};
+  auto up256 = [](size_t x) { return (x + 255) & ~size_t(255); };
+  enum { BQ, BK, BV, BLA, BB, BOUT, NBUF };
+  size_t off[kHostPieces][NBUF];
+  // the initial state, then two states that the pieces pass on in turn
+  size_t total = 0;
+  const size_t off_s0 = total;
+  total += initial_state ? up256((size_t)B * state1) : 0;
+  const size_t off_st[2] = {total, total + up256((size_t)B * state1)};
+  total += 2 * up256((size_t)B * state1);
+  for (int i = 0; i < P; ++i) {
+    const size_t nt = (size_t)B * (tb[i + 1] - tb[i]);
+    for (int b = 0; b < NBUF; ++b) {
+      off[i][b] = total;
+      total += up256(nt * tok_bytes[b]);
+    }
+  }
+
+  if (alloc_fault_injected()) return GDR_ERR_OUT_OF_MEMORY;
+  HostCtx hc;
+  gdr_status st = host_ctx(&hc);
+  if (st != GDR_OK) return st;
+  EventSet evs;
+  cudaEvent_t ev_start = evs.make(), ev_up_end = evs.make(),
+              ev_down_end = evs.make();
+  cudaEvent_t ev_in[kHostPieces], ev_run[kHostPieces];
+  for (int i = 0; i < P; ++i) {
+    ev_in[i] = evs.make();
+    ev_run[i] = evs.make();
+  }
+  if (evs.n != 3 + 2 * P) return GDR_ERR_CUDA;
+  void *block = nullptr;
+  {
+    cudaError_t e = cudaMallocFromPoolAsync(&block, total, hc.pool, stream);
+    if (e == cudaErrorMemoryAllocation) {
+      (void)cudaGetLastError();
+      return GDR_ERR_OUT_OF_MEMORY;
+    }
+    if (e != cudaSuccess) return GDR_ERR_CUDA;
+  }
+  char *base = static_cast<char *>(block);
+  auto ok = [&](cudaError_t e) {
+    if (e != cudaSuccess && st == GDR_OK) st = GDR_ERR_CUDA;
+    return st == GDR_OK;
+  };
+  ok(cudaEventRecord(ev_start, stream));
+  ok(cudaStreamWaitEvent(hc.up, ev_start, 0));
+  if (initial_state)
+    ok(cudaMemcpyAsync(base + off_s0, initial_state, (size_t)B * state1,
+                       cudaMemcpyHostToDevice, hc.up));
+  for (int i = 0; i < P && st == GDR_OK; ++i) {
+    const size_t t0 = tb[i], tp = tb[i + 1] - tb[i];
+    char *pb[NBUF];
+    for (int b = 0; b < NBUF; ++b) pb[b] = base + off[i][b];
+    // inputs of piece i: tokens [t0, t0 + tp) of every sequence
+    for (int b = BQ; b <= BB; ++b)
+      if (host_in[b] && tok_bytes[b])
+        ok(cudaMemcpy2DAsync(pb[b], tp * tok_bytes[b],
+                             static_cast<const char *>(host_in[b]) +
+                                 t0 * tok_bytes[b],
+                             (size_t)T * tok_bytes[b], tp * tok_bytes[b], B,
+                             cudaMemcpyHostToDevice, hc.up));
+    ok(cudaEventRecord(ev_in[i], hc.up));
+    if (st != GDR_OK) break;
+    ok(cudaStreamWaitEvent(stream, ev_in[i], 0));
+    Problem pp = p;
+    pp.q = pb[BQ];
+    pp.k = pb[BK];
+    pp.v = pb[BV];
+    pp.log_alpha = log_alpha ? reinterpret_cast<const float *>(pb[BLA])
+                             : nullptr;
+    pp.beta = reinterpret_cast<const float *>(pb[BB]);
+    pp.s0 = i == 0 ? (initial_state
+                          ? reinterpret_cast<const float *>(base + off_s0)
+                          : nullptr)
+                   : reinterpret_cast<const float *>(base + off_st[(i - 1) & 1]);
+    pp.sT = reinterpret_cast<float *>(base + off_st[i & 1]);
+    pp.out = pb[BOUT];
+    pp.T = (int)tp;
+    pp.ntok = (int)(B * tp);
+    pp.cu = nullptr;
+    pp.max_chunks = B * (int)((tp + C - 1) / C);
+    const gdr_status rs = run(pp, o.algo, stream);
+    if (rs != GDR_OK) {
+      st = rs;
+      break;
+    }
+    ok(cudaEventRecord(ev_run[i], stream));
+    // results of piece i
+    ok(cudaStreamWaitEvent(hc.down, ev_run[i], 0));
+    ok(cudaMemcpy2DAsync(static_cast<char *>(out) + t0 * tok_bytes[BOUT],
+                         (size_t)T * tok_bytes[BOUT], pb[BOUT],
+                         tp * tok_bytes[BOUT], tp * tok_bytes[BOUT], B,
+                         cudaMemcpyDeviceToHost, hc.down));
+    if (final_state && i == P - 1)
+      ok(cudaMemcpyAsync(final_state, base + off_st[i & 1], (size_t)B * state1,
+                         cudaMemcpyDeviceToHost, hc.down));
+  }
+  gdr_status fin = GDR_OK;
+  auto fin_ok = [&](cudaError_t e) {
+    if (e != cudaSuccess) fin = GDR_ERR_CUDA;
+  };
+  fin_ok(cudaEventRecord(ev_up_end, hc.up));
+  fin_ok(cudaEventRecord(ev_down_end, hc.down));
+  fin_ok(cudaStreamWaitEvent(stream, ev_up_end, 0));
+  fin_ok(cudaStreamWaitEvent(stream, ev_down_end, 0));
+  fin_ok(cudaFreeAsync(block, stream));
+  return st != GDR_OK ? st : fin;
+}
+
+}  // namespace
+
 extern "C" gdr_status gdr_chunk_fwd_host(const void *q, const void *k,
                                          const void *v, const float *log_alpha,
                                          const float *beta,
@@ -248,6 +390,9 @@ extern "C" gdr_status gdr_chunk_fwd_host(const void *q, const void *k,
                            final_state, B, T, H, dk, dv, chunk, o, &p);
   if (st != GDR_OK) return st;
   if (p.nseq == 0 || p.H == 0) return GDR_OK;
+  if (o.cu_seqlens == nullptr && p.T > chunk)
+    return host_by_time(p, o, q, k, v, log_alpha, beta, initial_state, out,
+                        final_state, stream);
 
   // host offsets are read here, so that every piece is exact
   const bool varlen = o.cu_seqlens != nullptr;

@@ -237,8 +237,9 @@ def test_host_entry_pieces_varlen():
 
 
 def test_host_entry_pieces_fixed_length():
-    # 10 sequences -> 8 pieces (two of two sequences); no initial state, and
-    # no final state requested
+    # fixed length is cut by time at chunk boundaries: T = 100 -> pieces of
+    # 64 and 36 tokens, the second starting from the first's state on the
+    # device; no initial state, and no final state requested
     w = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(B=10, T=100, H=3)
     inp = generate(w, seed=23)
     for algo in algos_for(w):
@@ -247,6 +248,25 @@ def test_host_entry_pieces_fixed_length():
         assert hs is None and np.array_equal(ho, o)
         ro, _ = run_oracle(inp)
         assert out_err(ho, ro, "bf16") <= 2e-2
+
+
+@pytest.mark.parametrize("name,shape", [
+    # 9 chunks -> 8 time pieces of 1 or 2 chunks and a ragged last chunk
+    ("gdn_b8_h16_t4096_d128_bf16", dict(B=3, T=8 * 64 + 37, H=2)),
+    # fp32 staged path, chunk 16: 16 chunks -> 8 pieces of 2
+    ("deltanet_b1_h1_t256_d16_fp32", dict(B=2, H=2)),
+])
+def test_host_entry_time_pieces_match_device_entry(name, shape):
+    # the state passes from piece to piece in fp32, as from chunk to chunk:
+    # the host entry's results are the device entry's, bit for bit, for every
+    # path, with and without an initial state
+    for init in (True, False):
+        w = WORKLOADS[name].with_(**shape, init_state=init)
+        inp = generate(w, seed=24)
+        for algo in algos_for(w):
+            o, s = run_gpu(inp, algo)
+            ho, hs = run_host(inp, algo)
+            assert np.array_equal(ho, o) and np.array_equal(hs, s)
 
 
 def test_deterministic():
