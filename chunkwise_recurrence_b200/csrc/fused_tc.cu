@@ -174,12 +174,16 @@ struct Ctx {
 };
 
 // Bounded wait: true when the phase completed, false on abort or timeout.
+// While the phase is incomplete the thread asks to be suspended (it resumes
+// when the phase completes), so that waiting warps leave their scheduler's
+// issue slots to the warps that work -- the MMA-issuing thread above all.
+constexpr uint32_t kSuspendNs = 20000;
 __device__ __forceinline__ bool wait_bar(const Ctx &cx, int b,
                                          uint32_t parity) {
   if (mbar_try_wait(&cx.bar[b], parity)) return true;
   const long long t0 = clock64();
   for (;;) {
-    if (mbar_try_wait(&cx.bar[b], parity)) return true;
+    if (mbar_try_wait_sleep(&cx.bar[b], parity, kSuspendNs)) return true;
     if (*cx.abort_flag) return false;
     if (clock64() - t0 > kWaitCycles) {
       *cx.abort_flag = 1;
