@@ -648,20 +648,21 @@ __global__ void __launch_bounds__(kBcThreads, 4)
       }
       // per row c: dq = S_t dO, dk = G u - beta S~ du, dla = G~ . S~ over
       // this group's columns; then G = D G~
+      // S_t dO = S~ dO + k (u . dO); G~ . S~ = G . S~ - beta k (S~ du)
       float qk[2 * R], dl[R];
       float dl_tot = 0.f;
+      const float udo = dot4(u, dO);
 #pragma unroll
       for (int i = 0; i < R; ++i) {
         const int c = row_c(i);
-        const float kc = b.k[c];
-        const float4 St = fma4(kc, u, Sm[i]);
-        qk[i] = dot4(St, dO);
-        qk[R + i] = dot4(G[i], u) - bb * dot4(Sm[i], du);
-        const float4 Gt = fma4(-bb * kc, du, G[i]);
-        dl[i] = dot4(Gt, Sm[i]);
+        const float kc = b.k[c], a = decay(b, c), sk = -bb * kc;
+        const float sdu = dot4(Sm[i], du);
+        qk[i] = fmaf(kc, udo, dot4(Sm[i], dO));
+        qk[R + i] = fmaf(-bb, sdu, dot4(G[i], u));
+        dl[i] = fmaf(sk, sdu, dot4(G[i], Sm[i]));
         dl_tot += dl[i];
-        const float a = decay(b, c);
-        G[i] = make_float4(a * Gt.x, a * Gt.y, a * Gt.z, a * Gt.w);
+        G[i] = make_float4(a * fmaf(sk, du.x, G[i].x), a * fmaf(sk, du.y, G[i].y),
+                           a * fmaf(sk, du.z, G[i].z), a * fmaf(sk, du.w, G[i].w));
       }
       {
         const int base = xreduce8<2 * R>(qk, cq);
