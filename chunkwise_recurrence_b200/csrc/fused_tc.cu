@@ -45,6 +45,7 @@
 #include <cuda_fp16.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "gdr_internal.h"
 #include "sm100.cuh"
@@ -103,8 +104,11 @@ struct Layout {
   // (g_m = g at row 31) and e^{g_C - g_m}
   static constexpr uint32_t GM = GC + 1536;       // [2][128]
   // channel gate: each half-chunk's log-decay total per key channel [2][128]
+  // followed by the prep warps' decay-range maxima [8] and, per chunk
+  // parity, whether the chunk's rescaled Q, K use fp16 (else bf16) [2]
   static constexpr uint32_t TT = GM + 1024;
-  static constexpr uint32_t TT_BYTES = (GATE == 2) ? 1024 : 0;
+  static constexpr uint32_t TT_BYTES = (GATE == 2) ? 1024 + 64 : 0;
+  static constexpr uint32_t TT_WMAX = TT + 1024, TT_F16 = TT + 1024 + 32;
   // channel gate: the chunk's log-decays, fp32 [2][64 rows][64 channels]
   // (channels 0..63, then 64..127), loaded by TMA one chunk ahead; turned
   // into running sums in place
@@ -139,9 +143,14 @@ enum {
 // fp16 (11-bit significand: 8x finer than bf16 at the same tensor-core rate).
 // Products that read raw bf16 input tiles stay bf16: K K^T, and for the
 // scalar / no gate U and W (their T factors are bf16; U's as a hi + lo
-// pair).  The channel gate's K K^T reads keys scaled by e^{+-(g - g_m)},
-// which need bf16's exponent range; its U and W are fp16.
+// pair).  The channel gate's K K^T reads keys scaled by e^{+-(g - g_m)}:
+// fp16 when the chunk's decay keeps those factors within e^{+-9}, else bf16
+// for its exponent range; its U and W are fp16.
 constexpr uint32_t ID_KK_B = idesc_f16kind(128, 64, false, false, true);
+constexpr uint32_t ID_KK_H = idesc_f16kind(128, 64, false, false, false);
+// largest |g - g_m| for which the channel gate's rescaled operands use fp16
+// (e^9 = 8103: normalised keys stay far below fp16's 65504)
+constexpr float kF16Range = 9.f;
 constexpr uint32_t ID_UW_H = idesc_f16kind(128, 64, true, false, false);
 constexpr uint32_t ID_UW_B = idesc_f16kind(128, 64, true, false, true);
 constexpr uint32_t ID_XV = idesc_f16kind(128, 64, false, true, false);
@@ -216,6 +225,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ void unpack_bf16(uint32_t w, float &lo, float &hi) {
   __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162 *>(&w);
   float2 f = __bfloat1622float2(v);
+  lo = f.x;
+  hi = f.y;
+}
+__device__ __forceinline__ void unpack_f16(uint32_t w, float &lo, float &hi) {
+  __half2 v = *reinterpret_cast<__half2 *>(&w);
+  float2 f = __half22float2(v);
   lo = f.x;
   hi = f.y;
 }
@@ -466,13 +481,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_kk = [&](int m) {
         const uint64_t base = st_k(m);
+        // channel gate: the prep warps chose fp16 or bf16 for this chunk
+        const uint32_t kk_id =
+            (GATE == 2 &&
+             reinterpret_cast<const volatile int *>(sm + Lay::TT_F16)[m & 1])
+                ? ID_KK_H
+                : ID_KK_B;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
           const uint64_t a = dadd(base, koff);
           const uint64_t b =
               GATE == 2 ? dadd(d_kn, (ks >> 2) * 8192 + (ks & 3) * 32) : a;
-          mma_f16kind(tmem + ACC_KK, a, b, ID_KK_B, ks > 0);
+          mma_f16kind(tmem + ACC_KK, a, b, kk_id, ks > 0);
         }
         mma_commit(&bar[B_KKDONE0 + (m & 1)]);
       };
@@ -752,7 +773,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                        kConv))
           break;
         uint8_t *stg = sm + OFF_STAGE + (m & 1) * kStageBytes;
-        auto to_f16_ge = [&](uint32_t part) {
+        const bool src16 =
+            reinterpret_cast<const volatile int *>(sm + Lay::TT_F16)[m & 1] != 0;
+        auto to_f16_ge = [&](uint32_t part, auto h16) {
+          constexpr bool kH = decltype(h16)::value;
 #pragma unroll 4
           for (int idx = ct; idx < kC * 16; idx += kConv) {
             const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
@@ -767,16 +791,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               float a0, a1;
-              unpack_bf16(xw[e], a0, a1);
+              if (kH) unpack_f16(xw[e], a0, a1);
+              else unpack_bf16(xw[e], a0, a1);
               xw[e] = pack_f16(a0 * f[2 * e], a1 * f[2 * e + 1]);
             }
             *xp = xv;
           }
           fence_proxy_async_smem();
         };
-        to_f16_ge(0);
+        if (src16) to_f16_ge(0, std::true_type{});
+        else to_f16_ge(0, std::false_type{});
         mbar_arrive(&bar[B_CONV]);
-        to_f16_ge(8192);
+        if (src16) to_f16_ge(8192, std::true_type{});
+        else to_f16_ge(8192, std::false_type{});
         mbar_arrive(&bar[B_QCONV]);
       } else {
         mbar_arrive(&bar[B_CONV]);
@@ -872,20 +899,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r = half * 32 + j;
             lv[j] = (r < L) ? la[r * 64] : 0.f;
           }
-          float run = 0.f;
+          float run = 0.f, lo = 0.f, hi = 0.f;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             run += lv[j];
             la[(half * 32 + j) * 64] = run;
+            lo = fminf(lo, run);
+            hi = fmaxf(hi, run);
           }
           reinterpret_cast<float *>(sm + Lay::TT)[half * 128 + c] = run;
+          // largest |g - g_m| of this half: g - g_m = running sum - g_m in
+          // the first half (g_m = its total), the running sum in the second
+          const float ref = half ? 0.f : run;
+          float bnd = fmaxf(fabsf(lo - ref), fabsf(hi - ref));
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1)
+            bnd = fmaxf(bnd, __shfl_xor_sync(0xffffffffu, bnd, off));
+          if (lane == 0)
+            reinterpret_cast<float *>(sm + Lay::TT_WMAX)[warp - 6] = bnd;
         }
         named_bar_sync(2, kPrep);
+        bool use16;
+        {
+          const float *wm = reinterpret_cast<const float *>(sm + Lay::TT_WMAX);
+          float b = wm[0];
+#pragma unroll
+          for (int w8 = 1; w8 < 8; ++w8) b = fmaxf(b, wm[w8]);
+          use16 = b <= kF16Range;   // same decision in every prep thread
+          if (pt == 0)
+            reinterpret_cast<int *>(sm + Lay::TT_F16)[m & 1] = use16 ? 1 : 0;
+        }
         // (b) with g_m = g at row 31 (the first half's total): row r's
         // g_r - g_m is its running sum minus g_m in the first half, and its
         // running sum in the second.  Item = row r, 8 channels (16 bytes of
         // Q, K and K e^{g_m-g}); thread pt takes items pt + 256 u.
-        {
+        // one loop per operand format (the choice is uniform per chunk)
+        auto rescale = [&](auto h16) {
+          constexpr bool kH = decltype(h16)::value;
           const float *gl = reinterpret_cast<const float *>(sm + Lay::LA);
           const float *T0 = reinterpret_cast<const float *>(sm + Lay::TT);
 #pragma unroll 2
@@ -918,15 +968,23 @@ __global__ void __launch_bounds__(kThreads, 1)
               unpack_bf16(kw[e], k0, k1);
               amax = fmaxf(amax, fmaxf(fmaxf(fabsf(q0), fabsf(q1)),
                                        fmaxf(fabsf(k0), fabsf(k1))));
-              qw[e] = pack_bf16(q0 * ep0, q1 * ep1);
-              kw[e] = pack_bf16(k0 * ep0, k1 * ep1);
-              knw[e] = pack_bf16(k0 * en0, k1 * en1);
+              qw[e] = kH ? pack_f16(q0 * ep0, q1 * ep1)
+                         : pack_bf16(q0 * ep0, q1 * ep1);
+              kw[e] = kH ? pack_f16(k0 * ep0, k1 * ep1)
+                         : pack_bf16(k0 * ep0, k1 * ep1);
+              knw[e] = kH ? pack_f16(k0 * en0, k1 * en1)
+                          : pack_bf16(k0 * en0, k1 * en1);
             }
             *qp = qv;
             *kp = kv;
             *reinterpret_cast<uint4 *>(sm + Lay::KN + kb * 8192 +
                                        sw128_chunk(r, cc)) = nv;
           }
+        };
+        if (use16) rescale(std::true_type{});
+        else rescale(std::false_type{});
+        {
+          const float *T0 = reinterpret_cast<const float *>(sm + Lay::TT);
           // per-channel factors, one exponential each per chunk: e^{g_m};
           // e^{g_C} (decay of S) in gc; e^{g_C - g_m} in gM + 128
           if (pt < 128) {
@@ -1221,26 +1279,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4 *>(stg + off[u]) = xk[u];
         }
       }
+      const bool kn16 =
+          GATE == 2 && reinterpret_cast<const int *>(sm + Lay::TT_F16)[m & 1];
+      auto ktilde = [&](auto h16) {
+        constexpr bool kH = decltype(h16)::value;
 #pragma unroll 2
-      for (int idx = pt; GATE == 2 && idx < kC * 16; idx += kPrep) {
-        const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
-        uint8_t *kp = stg + kb * 16384 + sw128_chunk(r, cc & 7);
-        // K~ = (K e^{g_m-g}) e^{g_C-g_m}, per channel (8 factors, two
-        // vector loads)
-        const float4 *fp = reinterpret_cast<const float4 *>(gM + 128 + cc * 8);
-        const float4 f0 = fp[0], f1 = fp[1];
-        const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-        uint4 kv = *reinterpret_cast<const uint4 *>(
-            sm + Lay::KN + kb * 8192 + sw128_chunk(r, cc & 7));
-        uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
+        for (int idx = pt; GATE == 2 && idx < kC * 16; idx += kPrep) {
+          const int r = idx >> 4, cc = idx & 15, kb = cc >> 3;
+          uint8_t *kp = stg + kb * 16384 + sw128_chunk(r, cc & 7);
+          // K~ = (K e^{g_m-g}) e^{g_C-g_m}, per channel (8 factors, two
+          // vector loads)
+          const float4 *fp = reinterpret_cast<const float4 *>(gM + 128 + cc * 8);
+          const float4 f0 = fp[0], f1 = fp[1];
+          const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+          uint4 kv = *reinterpret_cast<const uint4 *>(
+              sm + Lay::KN + kb * 8192 + sw128_chunk(r, cc & 7));
+          uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float a0, a1;
-          unpack_bf16(kw[e], a0, a1);
-          kw[e] = pack_f16(a0 * f[2 * e], a1 * f[2 * e + 1]);
+          for (int e = 0; e < 4; ++e) {
+            float a0, a1;
+            if (kH) unpack_f16(kw[e], a0, a1);
+            else unpack_bf16(kw[e], a0, a1);
+            kw[e] = pack_f16(a0 * f[2 * e], a1 * f[2 * e + 1]);
+          }
+          *reinterpret_cast<uint4 *>(kp) = kv;
         }
-        *reinterpret_cast<uint4 *>(kp) = kv;
-      }
+      };
+      if (kn16) ktilde(std::true_type{});
+      else ktilde(std::false_type{});
       if (!(amax <= kF16Max)) atomicOr(&g_fused_error, kErrRange);
       fence_proxy_async_smem();
       tc_fence_before();

@@ -102,9 +102,10 @@ typedef enum {
    * and is reported by gdr_device_error as GDR_ERR_RANGE.  Accuracy: the
    * scalar and no gate stay within about 5e-3 of the output RMS at any
    * decay; for the channel gate the decay sits inside the contraction, on
-   * operands rounded to bf16 / fp16, and the error grows with it: about
-   * 1.2e-2 at mean log-decays near -0.03 per token and channel, about 3e-2
-   * at -1 to -2.  Where that matters, GDR_ALGO_STAGED is fp32 throughout. */
+   * rescaled operands that are fp16 where a chunk's decay allows (about 3e-3
+   * at mean log-decays down to -0.1 per token and channel) and bf16 beyond
+   * (up to about 3e-2 at -1 to -2).  Where that matters, GDR_ALGO_STAGED is
+   * fp32 throughout. */
   GDR_ALGO_FUSED_TC = 2
 } gdr_algo;
 

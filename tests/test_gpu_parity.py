@@ -336,12 +336,12 @@ def test_strong_decays_scalar_gate(decay):
 
 
 # Channel gate, fused path: the per-channel decay sits inside the contraction,
-# so K K^T, Q K^T and U, W read operands rescaled by e^{+-(g - g_m)} and
-# rounded to bf16 / fp16 (whose subnormals lose bits once e^g < 2^-14).  The
-# error therefore grows with the decay: about 1.2e-2 of the RMS at the KDA
-# workload's decays (mean log-decay about -0.03 per token and channel), up to
-# about 3e-2 at -1 to -2.  This is the documented envelope of the fused
-# channel-gate path; the fp32 staged path meets the bar at any decay.
+# so K K^T, Q K^T and U, W read operands rescaled by e^{+-(g - g_m)}: fp16
+# where the chunk's decay range allows (about 3e-3 of the RMS at the KDA
+# workload's decays), bf16 beyond (whose 8-bit significand gives up to about
+# 3e-2 at mean log-decays of -1 to -2 per token and channel).  This is the
+# documented envelope of the fused channel-gate path; the fp32 staged path
+# meets the bar at any decay.
 KDA_FUSED_STRONG_DECAY_BOUND = 5e-2
 
 
