@@ -18,18 +18,24 @@
 //
 // Everything that does not depend on S (A, T, W, U, the output mask P) for
 // chunk n+1 is computed while the S-dependent chain of chunk n runs:
-//   warp 0      TMA producer: Q, K (two stages) and V tiles, 128-B swizzle
+//   warp 0      TMA producer: Q, K (two stages) and V tiles, 128-B swizzle;
+//               channel gate, the fp32 log-decay tile one chunk ahead
 //   warp 1      tensor-memory allocation and the single MMA-issuing thread
 //   warps 2..5  "state" warps: S -> fp16 operand and decay, V_new -> fp16
 //               operand, output tile -> global (thread = tensor-memory lane
 //               = one value channel)
 //   warps 6..13 "prep" warps (two per scheduler): gates, cumsum and per-row
-//               decay factors, A and P from K K^T / Q K^T, T = (I+A)^-1,
-//               T-factor operands, -W operand, in-place Q . e^g and
-//               K . e^{g_C - g} (fp16)
+//               decay factors (channel gate: per-channel running sums and
+//               Q, K rescaled by e^{+-(g - g_m)}, fp16 or bf16 per chunk),
+//               A and P from K K^T / Q K^T, T = (I+A)^-1, T-factor
+//               operands, -W operand, in-place Q . e^g and K . e^{g_C - g}
+//               (fp16; channel gate: K~ only)
 //   warps 14,15 "convert" warps: channel gate, V tile bf16 -> fp16 in place
-//               for the fp16 U product (the scalar / no gate U and W read
-//               the raw bf16 V and K)
+//               for the fp16 U product, then K . e^g (for W) and Q . e^g
+//               (for X) in place; the scalar / no gate U and W read the raw
+//               bf16 V and K
+// Waiting threads ask to be suspended until their phase completes, so that
+// they leave issue slots to the working warps (the MMA thread above all).
 // All state lives in tensor memory as S^T (lane = value channel, column =
 // key channel) in fp32; fp16 / bf16 appear only as tensor-core operands.
 //
