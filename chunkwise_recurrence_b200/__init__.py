@@ -15,7 +15,7 @@ import os
 import torch
 
 __all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_noalloc",
-           "chunk_fwd_segmented", "decode_step",
+           "chunk_fwd_segmented", "chunk_fwd_gdn2", "decode_step",
            "efla_beta", "backward",
            "device_error", "status_string",
            "algo_applies", "fused_tc_available",
@@ -35,7 +35,7 @@ EXPORTED_SYMBOLS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_device_error",
                     "gdr_algo_applies", "gdr_status_string",
                     "gdr_chunk_fwd_noalloc", "gdr_decode_step",
                     "gdr_efla_beta", "gdr_backward",
-                    "gdr_chunk_fwd_segmented")
+                    "gdr_chunk_fwd_segmented", "gdr_chunk_fwd_gdn2")
 # size of the static scratch array behind gdr_chunk_fwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -74,6 +74,10 @@ def load_library(path: str = LIB_PATH):
     lib.gdr_decode_step.restype = ctypes.c_int
     lib.gdr_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i,
                                     vp, ctypes.POINTER(_Opts)]
+    lib.gdr_chunk_fwd_gdn2.restype = ctypes.c_int
+    lib.gdr_chunk_fwd_gdn2.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, i,
+                                       i, i, i, i, i, vp,
+                                       ctypes.POINTER(_Opts)]
     lib.gdr_chunk_fwd_segmented.restype = ctypes.c_int
     lib.gdr_chunk_fwd_segmented.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i,
                                             i, i, i, i, i, i, vp,
@@ -161,6 +165,39 @@ def chunk_fwd(q, k, v, beta, log_alpha=None, initial_state=None, *,
                            ctypes.byref(opts))
     if rc != 0:
         raise GdrError(rc, "gdr_chunk_fwd")
+    return out, final_state
+
+
+def chunk_fwd_gdn2(q, k, v, erase_gate, write_gate, log_alpha=None,
+                   initial_state=None, *, chunk: int = 64,
+                   gate: str | None = None, cu_seqlens=None, out=None,
+                   final_state=None, output_final_state: bool = True,
+                   algo: str = "auto", stream=None):
+    """Run ``gdr_chunk_fwd_gdn2``: the forward pass with Gated DeltaNet-2's
+    per-key-channel erase gate (``erase_gate``, the layout of k, fp32) and
+    per-value-channel write gate (``write_gate``, the layout of v, fp32) in
+    place of beta (see include/gdr.h for the update).  Returns (out,
+    final_state)."""
+    lib = load_library()
+    B, T, H, dk, dv, nseq = _shapes(q, v, cu_seqlens)
+    if out is None:
+        out = torch.empty_like(v)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(nseq, H, dk, dv, dtype=torch.float32,
+                                  device=q.device)
+    g = _gate_of(log_alpha, gate)
+    opts = _Opts(DTYPES[q.dtype], GATES[g],
+                 None if cu_seqlens is None else cu_seqlens.data_ptr(),
+                 nseq if cu_seqlens is not None else 0, ALGOS[algo])
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    rc = lib.gdr_chunk_fwd_gdn2(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(erase_gate),
+        _ptr(write_gate), _ptr(initial_state), _ptr(out), _ptr(final_state),
+        B, T, H, dk, dv, chunk, ctypes.c_void_p(stream.cuda_stream),
+        ctypes.byref(opts))
+    if rc != 0:
+        raise GdrError(rc, "gdr_chunk_fwd_gdn2")
     return out, final_state
 
 

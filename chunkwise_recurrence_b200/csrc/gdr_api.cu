@@ -119,7 +119,8 @@ gdr_status scratch_alloc(void **ptr, size_t bytes, cudaStream_t s) {
 
 gdr_status run(const Problem &p, gdr_algo algo, cudaStream_t stream) {
   if (p.nseq == 0 || p.H == 0) return GDR_OK;
-  const bool tc = gdr::fused_tc_applies(p);
+  // the Gated DeltaNet-2 gates run on the staged path only
+  const bool tc = p.erase == nullptr && gdr::fused_tc_applies(p);
   if (algo == GDR_ALGO_FUSED_TC && !tc) return GDR_ERR_UNSUPPORTED;
   if (tc && algo != GDR_ALGO_STAGED) {
     cudaError_t e = gdr::fused_tc_run(p, stream);
@@ -150,6 +151,33 @@ extern "C" gdr_status gdr_chunk_fwd(const void *q, const void *k,
                            final_state, B, T, H, dk, dv, chunk, o, &p);
   if (st != GDR_OK) return st;
   return run(p, o.algo, stream);
+}
+
+// Gated DeltaNet-2 gates (erase on the read key, write on the target), on
+// the staged path: see gdr.h.
+extern "C" gdr_status gdr_chunk_fwd_gdn2(const void *q, const void *k,
+                                         const void *v, const float *log_alpha,
+                                         const float *erase_gate,
+                                         const float *write_gate,
+                                         const float *initial_state, void *out,
+                                         float *final_state, int B, int T,
+                                         int H, int dk, int dv, int chunk,
+                                         cudaStream_t stream,
+                                         const gdr_opts *opts) {
+  const gdr_opts o = opts ? *opts : default_opts();
+  if (o.algo == GDR_ALGO_FUSED_TC) return GDR_ERR_UNSUPPORTED;
+  Problem p;
+  // the erase gate stands in for beta in the common checks (presence,
+  // alignment); the write gate is checked here
+  gdr_status st = validate(q, k, v, log_alpha, erase_gate, initial_state, out,
+                           final_state, B, T, H, dk, dv, chunk, o, &p);
+  if (st != GDR_OK) return st;
+  if (p.nseq == 0 || p.H == 0) return GDR_OK;
+  if (!write_gate || !aligned16(write_gate)) return GDR_ERR_INVALID_ARGUMENT;
+  p.beta = nullptr;
+  p.erase = erase_gate;
+  p.write = write_gate;
+  return run(p, GDR_ALGO_STAGED, stream);
 }
 
 // ---------------------------------------------------------------------------

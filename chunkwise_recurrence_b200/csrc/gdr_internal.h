@@ -34,6 +34,10 @@ struct Problem {
   gdr_dtype dtype;
   gdr_gate gate;
   int max_chunks;     // upper bound on the number of chunks over all sequences
+  // Gated DeltaNet-2 gates (staged path only; nullptr otherwise): the
+  // per-key-channel erase gate [ntok][H][dk] and per-value-channel write
+  // gate [ntok][H][dv] that replace beta
+  const float *erase = nullptr, *write = nullptr;
 };
 
 // Staged path: four kernels + a chunk-table kernel, fp32 CUDA-core math.

@@ -97,9 +97,16 @@ __device__ __forceinline__ float gval(const float *Gs, int gdim, int r,
 }
 
 // (b) intra-chunk WY/UT transform of one (chunk, head).
+// With the Gated DeltaNet-2 gates (erase != nullptr), the read key of token
+// r is b_r . k_r (erase gate b_r, per key channel) and its target w_r . v_r
+// (write gate w_r, per value channel), and beta is not used:
+//   A[r][i] = (b_r . k_r)^T Gamma_r Gamma_i^-1 k_i,  W = T ((B . K) . e^g),
+//   U = T (Wg . V).
 template <typename Tin>
 __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
                           const float *__restrict__ beta,
+                          const float *__restrict__ erase,
+                          const float *__restrict__ write,
                           const float *__restrict__ g, float *__restrict__ W,
                           float *__restrict__ U,
                           const ChunkInfo *__restrict__ table,
@@ -116,7 +123,9 @@ __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
   float *As = Gs + C * gd;         // [C][C+1]
   float *Ts = As + C * (C + 1);    // [C][C+1]
   float *bs = Ts + C * (C + 1);    // [C]
+  float *Es = bs + C;              // [C][dk], erase gates (Gated DeltaNet-2)
   const int tid = threadIdx.x, nt = blockDim.x;
+  const bool g2 = erase != nullptr;
 
   for (int idx = tid; idx < L * dk; idx += nt) {
     const int r = idx / dk, c = idx % dk;
@@ -127,8 +136,22 @@ __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
       const int r = idx / gdim, c = idx % gdim;
       Gs[r * gdim + c] = g[((size_t)(ci.tok0 + r) * H + h) * gdim + c];
     }
-  for (int r = tid; r < L; r += nt) bs[r] = beta[(size_t)(ci.tok0 + r) * H + h];
+  if (g2) {
+    for (int idx = tid; idx < L * dk; idx += nt) {
+      const int r = idx / dk, c = idx % dk;
+      Es[r * dk + c] = erase[((size_t)(ci.tok0 + r) * H + h) * dk + c];
+    }
+    for (int r = tid; r < L; r += nt) bs[r] = 1.f;
+  } else {
+    for (int r = tid; r < L; r += nt)
+      bs[r] = beta[(size_t)(ci.tok0 + r) * H + h];
+  }
   __syncthreads();
+  // the read key of row r, channel c: b_r[c] k_r[c] (Gated DeltaNet-2) or
+  // k_r[c]; the row factor bs[r] is then 1 or beta_r
+  auto rk = [&](int r, int c) {
+    return g2 ? Es[r * dk + c] * Ks[r * dk + c] : Ks[r * dk + c];
+  };
 
   // A[r][i] = beta_r sum_c k_r[c] k_i[c] exp(g_r[c] - g_i[c]),  i < r
   for (int idx = tid; idx < L * L; idx += nt) {
@@ -136,11 +159,11 @@ __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
     float a = 0.f;
     if (i < r) {
       if (gdim <= 1) {
-        for (int c = 0; c < dk; ++c) a += Ks[r * dk + c] * Ks[i * dk + c];
+        for (int c = 0; c < dk; ++c) a += rk(r, c) * Ks[i * dk + c];
         if (gdim == 1) a *= __expf(Gs[r] - Gs[i]);
       } else {
         for (int c = 0; c < dk; ++c)
-          a += Ks[r * dk + c] * Ks[i * dk + c] *
+          a += rk(r, c) * Ks[i * dk + c] *
                __expf(Gs[r * gdim + c] - Gs[i * gdim + c]);
       }
       a *= bs[r];
@@ -165,16 +188,17 @@ __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
     const int r = idx / dk, c = idx % dk;
     float acc = 0.f;
     for (int i = 0; i <= r; ++i)
-      acc += Ts[r * (C + 1) + i] * bs[i] * Ks[i * dk + c] *
+      acc += Ts[r * (C + 1) + i] * bs[i] * rk(i, c) *
              __expf(gval(Gs, gdim, i, c));
     W[((size_t)(ci.tok0 + r) * H + h) * dk + c] = acc;
   }
   for (int idx = tid; idx < L * dv; idx += nt) {
     const int r = idx / dv, c = idx % dv;
     float acc = 0.f;
-    for (int i = 0; i <= r; ++i)
-      acc += Ts[r * (C + 1) + i] * bs[i] *
-             to_f(v[((size_t)(ci.tok0 + i) * H + h) * dv + c]);
+    for (int i = 0; i <= r; ++i) {
+      const size_t e = ((size_t)(ci.tok0 + i) * H + h) * dv + c;
+      acc += Ts[r * (C + 1) + i] * bs[i] * to_f(v[e]) * (g2 ? write[e] : 1.f);
+    }
     U[((size_t)(ci.tok0 + r) * H + h) * dv + c] = acc;
   }
 }
@@ -369,14 +393,15 @@ cudaError_t run_typed(const Problem &p, char *ws, cudaStream_t s) {
                                          gdim);
     const size_t wy_smem =
         sizeof(float) * ((size_t)C * p.dk + (size_t)C * gd +
-                         2 * (size_t)C * (C + 1) + C);
+                         2 * (size_t)C * (C + 1) + C +
+                         (p.erase ? (size_t)C * p.dk : 0));
     cudaError_t e = cudaFuncSetAttribute(
         wy_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
         (int)wy_smem);
     if (e != cudaSuccess) return e;
-    wy_kernel<Tin><<<grid, 256, wy_smem, s>>>(k, v, p.beta, g, W, U, table,
-                                             nchunks, p.H, p.dk, p.dv, C,
-                                             gdim);
+    wy_kernel<Tin><<<grid, 256, wy_smem, s>>>(k, v, p.beta, p.erase, p.write,
+                                             g, W, U, table, nchunks, p.H,
+                                             p.dk, p.dv, C, gdim);
   }
   const int DVT = p.dv < 32 ? p.dv : 32;
   const size_t st_smem =

@@ -150,6 +150,16 @@ def generate(w: Workload, seed: int = 0) -> Inputs:
                   log_alpha=log_alpha, s0=s0, cu_seqlens=cu, lengths=lengths)
 
 
+def gdn2_gates(inp: Inputs, seed: int = 0):
+    """Gated DeltaNet-2 gates for a generated batch: an erase gate per key
+    channel (the layout of k) and a write gate per value channel (the layout
+    of v), both sigmoid(N(0, 1)) like beta, fp32, seeded."""
+    g = torch.Generator().manual_seed(1_000_003 + seed)
+    erase = torch.sigmoid(torch.randn(inp.k.shape, generator=g))
+    write = torch.sigmoid(torch.randn(inp.v.shape, generator=g))
+    return erase.float().contiguous(), write.float().contiguous()
+
+
 def head_slice(inp: Inputs, heads) -> Inputs:
     """The same inputs restricted to a subset of heads (chains are independent
     per head, so this is how large workloads are sampled for the oracle)."""

@@ -161,8 +161,12 @@ GDR_API gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v,
  * layouts above; with cu_seqlens the offsets are checked on the host (first
  * 0, non-decreasing, last T), else GDR_ERR_INVALID_ARGUMENT.
  *
- * The batch is cut into up to 8 pieces of whole sequences, each computed as
- * an independent sub-problem.  The call enqueues, and returns without
+ * The work is cut into up to 8 pieces: fixed-length batches by time, at
+ * chunk boundaries (each piece holds the same token range of every sequence
+ * and starts from the state the previous piece ended with, kept on the
+ * device in fp32, so the results are those of gdr_chunk_fwd bit for bit);
+ * packed batches into pieces of whole sequences, each an independent
+ * sub-problem.  The call enqueues, and returns without
  * waiting: per piece, the host-to-device copies of its inputs on an upload
  * stream, its computation on `stream`, and the device-to-host copies of its
  * results on a download stream, so that the copies of neighbouring pieces
@@ -182,6 +186,41 @@ GDR_API gdr_status gdr_chunk_fwd_host(const void *q, const void *k, const void *
                               float *final_state, int B, int T, int H, int dk,
                               int dv, int chunk, cudaStream_t stream,
                               const gdr_opts *opts);
+
+/*
+ * gdr_chunk_fwd_gdn2 -- the forward pass with Gated DeltaNet-2's separate
+ * erase and write gates.
+ *
+ * Gated DeltaNet-2 (abstract on the comparative-study page 2607.07953)
+ * replaces the delta rule's one scalar gate beta, which controls both how
+ * much old content is erased on the key side and how much new content is
+ * written on the value side, by a channel-wise erase gate b_t (per key
+ * channel) and a channel-wise write gate w_t (per value channel), and
+ * reduces to KDA when both collapse to the same scalar.  The pages print no
+ * formula; the update taken here keeps the delta rule's form with the erase
+ * gate on the read key and the write gate on the target:
+ *   S~_t = D_t S_{t-1},   u_t = w_t . v_t - S~_t^T (b_t . k_t),
+ *   S_t  = S~_t + k_t u_t^T,   o_t = S_t^T q_t,
+ * which is gdr_chunk_fwd's recurrence when b_t = beta_t 1 and w_t = beta_t 1.
+ *
+ * Arguments as for gdr_chunk_fwd, with beta replaced by
+ *   erase_gate  [B][T][H][dk] fp32 (device, 16-byte aligned), required;
+ *   write_gate  [B][T][H][dv] fp32 (device, 16-byte aligned), required;
+ * (packed layouts with cu_seqlens as for gdr_chunk_fwd).  The decay form is
+ * opts->gate (NONE, SCALAR or CHANNEL) as before.  Runs the staged path
+ * (fp32 CUDA-core arithmetic, any supported shape): opts->algo AUTO or
+ * STAGED; FUSED_TC returns GDR_ERR_UNSUPPORTED.  Status codes as for
+ * gdr_chunk_fwd.
+ */
+GDR_API gdr_status gdr_chunk_fwd_gdn2(const void *q, const void *k,
+                                      const void *v, const float *log_alpha,
+                                      const float *erase_gate,
+                                      const float *write_gate,
+                                      const float *initial_state, void *out,
+                                      float *final_state, int B, int T, int H,
+                                      int dk, int dv, int chunk,
+                                      cudaStream_t stream,
+                                      const gdr_opts *opts);
 
 /*
  * gdr_chunk_fwd_segmented -- gdr_chunk_fwd with context-parallel state

@@ -222,6 +222,29 @@ def test_segmented_rejects_bad_arguments(lib):
              B=0) == OK
 
 
+def test_gdn2_rejects_bad_arguments(lib):
+    def c(**kw):
+        args = dict(q=A, k=A, v=A, la=A, er=A, wr=A, s0=None, out=A, sT=None,
+                    B=1, T=64, H=1, dk=128, dv=128, chunk=64, dtype=0, gate=2,
+                    cu=None, nseq=0, algo=0)
+        args.update(kw)
+        opts = gdr._Opts(args["dtype"], args["gate"], args["cu"], args["nseq"],
+                         args["algo"])
+        return lib.gdr_chunk_fwd_gdn2(
+            args["q"], args["k"], args["v"], args["la"], args["er"],
+            args["wr"], args["s0"], args["out"], args["sT"], args["B"],
+            args["T"], args["H"], args["dk"], args["dv"], args["chunk"], None,
+            ctypes.byref(opts))
+    assert c(er=None) == INVALID          # both gates are required
+    assert c(wr=None) == INVALID
+    assert c(wr=A + 4) == INVALID         # 16-byte alignment
+    assert c(la=None) == INVALID          # a decay gate needs log_alpha
+    assert c(algo=2) == UNSUPPORTED       # staged path only
+    assert c(dk=48) == UNSUPPORTED
+    assert c(q=None, k=None, v=None, la=None, er=None, wr=None, out=None,
+             gate=0, B=0) == OK
+
+
 def test_algo_applies(lib):
     assert gdr.algo_applies("staged", "fp32", "none", 16, 16, 16)
     assert gdr.algo_applies("auto", "bf16", "channel", 128, 64, 32)

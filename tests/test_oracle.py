@@ -407,6 +407,63 @@ def test_efla_limits():
     np.testing.assert_allclose(se[0, 0].T @ k[0, 0, 0], v[0, 0, 0], atol=1e-12)
 
 
+@pytest.mark.parametrize("gate", ["none", "scalar", "channel"])
+def test_gdn2_reduces_to_the_delta_rule(oracle_lib, gate):
+    """Erase and write gates equal to beta_t on every channel give the delta
+    rule: the Gated DeltaNet-2 loop matches the C oracle."""
+    rng = np.random.default_rng(31)
+    c = _rand_case(rng, B=2, T=13, H=2, dk=4, dv=3, gate=gate)
+    o, s, _ = gdr_fwd(**c)
+    b = c["beta"]
+    go, gs = oracle.gdn2_fwd(c["q"], c["k"], c["v"],
+                             np.repeat(b[..., None], 4, axis=-1),
+                             np.repeat(b[..., None], 3, axis=-1),
+                             c["log_alpha"], gate, c["initial_state"])
+    assert np.allclose(go, o, atol=1e-13) and np.allclose(gs, s, atol=1e-13)
+
+
+def test_gdn2_without_erase_is_decayed_linear_attention(oracle_lib):
+    """b = 0: nothing is erased, so S_t = sum_{s<=t} (prod_{s<tau<=t} D_tau)
+    k_s (w_s . v_s)^T (+ the decayed initial state), summed directly."""
+    rng = np.random.default_rng(32)
+    c = _rand_case(rng, B=1, T=9, H=1, dk=3, dv=2, gate="channel")
+    w = rng.uniform(0.1, 1.0, size=(1, 9, 1, 2))
+    go, gs = oracle.gdn2_fwd(c["q"], c["k"], c["v"], np.zeros((1, 9, 1, 3)),
+                             w, c["log_alpha"], "channel", c["initial_state"])
+    la = c["log_alpha"][0, :, 0]
+    for t in range(9):
+        S = np.exp(la[:t + 1].sum(axis=0))[:, None] * c["initial_state"][0, 0]
+        for s_ in range(t + 1):
+            dec = np.exp(la[s_ + 1:t + 1].sum(axis=0))
+            S = S + np.outer(dec * c["k"][0, s_, 0], w[0, s_, 0] * c["v"][0, s_, 0])
+        assert np.allclose(go[0, t, 0], S.T @ c["q"][0, t, 0], atol=1e-13)
+    assert np.allclose(gs[0, 0], S, atol=1e-13)
+
+
+def test_gdn2_one_hot_keys_update_rows_independently(oracle_lib):
+    """With k_t = e_c, only row c of S changes, and it follows
+    S_c <- (1 - b_t[c]) a_t[c] S_c + w_t . v_t (a = the decay of row c)."""
+    rng = np.random.default_rng(33)
+    T, dk, dv = 10, 3, 4
+    cs = rng.integers(0, dk, size=T)
+    k = np.zeros((1, T, 1, dk))
+    k[0, np.arange(T), 0, cs] = 1.0
+    q = rng.standard_normal((1, T, 1, dk))
+    v = rng.standard_normal((1, T, 1, dv))
+    b = rng.uniform(0, 1, size=(1, T, 1, dk))
+    w = rng.uniform(0, 1, size=(1, T, 1, dv))
+    la = -rng.uniform(0.05, 0.5, size=(1, T, 1, dk))
+    S0 = rng.standard_normal((1, 1, dk, dv))
+    go, gs = oracle.gdn2_fwd(q, k, v, b, w, la, "channel", S0)
+    S = S0[0, 0].copy()
+    for t in range(T):
+        S = np.exp(la[0, t, 0])[:, None] * S
+        c = cs[t]
+        S[c] = (1 - b[0, t, 0, c]) * S[c] + w[0, t, 0] * v[0, t, 0]
+        assert np.allclose(go[0, t, 0], S.T @ q[0, t, 0], atol=1e-13)
+    assert np.allclose(gs[0, 0], S, atol=1e-13)
+
+
 def test_gradients_match_finite_differences(oracle_lib):
     """The autograd gradients (oracle.gdr_grads, on a PyTorch token loop) agree
     with central differences of the C token loop's loss, element by element,
