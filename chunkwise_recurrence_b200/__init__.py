@@ -35,7 +35,8 @@ EXPORTED_SYMBOLS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_device_error",
                     "gdr_algo_applies", "gdr_status_string",
                     "gdr_chunk_fwd_noalloc", "gdr_decode_step",
                     "gdr_efla_beta", "gdr_backward",
-                    "gdr_chunk_fwd_segmented", "gdr_chunk_fwd_gdn2")
+                    "gdr_chunk_fwd_segmented", "gdr_chunk_fwd_gdn2",
+                    "gdr_decode_step_gdn2")
 # size of the static scratch array behind gdr_chunk_fwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -74,6 +75,10 @@ def load_library(path: str = LIB_PATH):
     lib.gdr_decode_step.restype = ctypes.c_int
     lib.gdr_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i,
                                     vp, ctypes.POINTER(_Opts)]
+    lib.gdr_decode_step_gdn2.restype = ctypes.c_int
+    lib.gdr_decode_step_gdn2.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp,
+                                         i, i, i, i, vp,
+                                         ctypes.POINTER(_Opts)]
     lib.gdr_chunk_fwd_gdn2.restype = ctypes.c_int
     lib.gdr_chunk_fwd_gdn2.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, i,
                                        i, i, i, i, i, vp,
@@ -317,6 +322,40 @@ def decode_step(q, k, v, beta, log_alpha=None, state=None, *, out=None,
                              ctypes.byref(opts))
     if rc != 0:
         raise GdrError(rc, "gdr_decode_step")
+    return out, state_out
+
+
+def decode_step_gdn2(q, k, v, erase_gate, write_gate, log_alpha=None,
+                     state=None, *, out=None, state_out=None,
+                     gate: str | None = None, stream=None):
+    """Run ``gdr_decode_step_gdn2`` on CUDA tensors: one token per (sequence,
+    head) with Gated DeltaNet-2's gates in place of beta.  ``erase_gate``
+    [N, H, dk] and ``write_gate`` [N, H, dv] are fp32; everything else is as
+    in ``decode_step``.  Returns (out [N, H, dv], state_out)."""
+    lib = load_library()
+    if q.dim() != 3 or v.dim() != 3:
+        raise ValueError("q, k, v must be [N, H, d]")
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty_like(v)
+    if state_out is None:
+        state_out = state if state is not None else torch.empty(
+            N, H, dk, dv, dtype=torch.float32, device=q.device)
+    g = gate if gate is not None else (
+        "none" if log_alpha is None else
+        "scalar" if log_alpha.dim() == 2 else "channel")
+    opts = _Opts(DTYPES[q.dtype], GATES[g], None, 0, ALGOS["auto"])
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    rc = lib.gdr_decode_step_gdn2(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                  _ptr(erase_gate), _ptr(write_gate),
+                                  _ptr(state), _ptr(state_out), _ptr(out),
+                                  N, H, dk, dv,
+                                  ctypes.c_void_p(stream.cuda_stream),
+                                  ctypes.byref(opts))
+    if rc != 0:
+        raise GdrError(rc, "gdr_decode_step_gdn2")
     return out, state_out
 
 

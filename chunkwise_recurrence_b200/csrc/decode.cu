@@ -25,6 +25,11 @@
 // tile is read in full before any of it is written back.  The copy wait is
 // bounded; on expiry the CTA skips its step and raises the library's device
 // error word (gdr_device_error: GDR_ERR_TIMEOUT).
+//
+// With Gated DeltaNet-2's gates (erase != nullptr) the read key is b . k
+// (erase gate b, per key channel) and the target w . v (write gate w, per
+// value channel), without beta:  u = w . v - S~^T (b . k),  S' = S~ + k u^T,
+// o = S~^T q + u (k . q)  (gdr_decode_step_gdn2).
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -75,6 +80,8 @@ struct DecodeParams {
   float *s_out;
   void *out;
   int dv;
+  // Gated DeltaNet-2 gates [N*H][dk] and [N*H][dv], or nullptr
+  const float *erase, *write;
   // failure injection (host hook): the state copy is not issued, so the
   // CTA's wait runs out after wait_cycles and reports a timeout
   int inject_timeout;
@@ -122,7 +129,7 @@ __global__ void __launch_bounds__(kDecThreads)
     gdr_decode_kernel(DecodeParams p) {
   constexpr int R = DK / 8;   // rows of S per warp
   extern __shared__ __align__(128) float tile[];   // the state, [DK][dv]
-  __shared__ float sk[DK], sq[DK], sa[DK];
+  __shared__ float sk[DK], sq[DK], sa[DK], sr[DK];   // sr: read key
   __shared__ float4 red[2][8][32];   // per warp: partial S~^T k, S~^T q
   __shared__ float kq_s;
   __shared__ __align__(8) uint64_t bar;
@@ -150,6 +157,7 @@ __global__ void __launch_bounds__(kDecThreads)
     sa[c] = GATE == 0   ? 1.f
             : GATE == 1 ? __expf(p.log_alpha[nh])
                         : __expf(p.log_alpha[(size_t)nh * DK + c]);
+    sr[c] = p.erase ? p.erase[(size_t)nh * DK + c] * sk[c] : sk[c];
   }
   if (threadIdx.x == 0 && p.s_in) {
     const long long t0 = clock64();
@@ -173,7 +181,7 @@ __global__ void __launch_bounds__(kDecThreads)
     const float a = sa[c];
     x = make_float4(a * x.x, a * x.y, a * x.z, a * x.w);
     if (act) st4(tile + c * dv + j0, x);   // S~, kept for the update
-    pk = fma4(sk[c], x, pk);
+    pk = fma4(sr[c], x, pk);
     pq = fma4(sq[c], x, pq);
   }
   red[0][warp][lane] = pk;
@@ -195,11 +203,19 @@ __global__ void __launch_bounds__(kDecThreads)
     rq = make_float4(rq.x + b.x, rq.y + b.y, rq.z + b.z, rq.w + b.w);
   }
   if (act) {
-    // u = beta (v - S~^T k); o = S~^T q + u (k . q)
-    const float bt = p.beta[nh];
+    // u = beta (v - S~^T k) (Gated DeltaNet-2: w . v - S~^T (b . k));
+    // o = S~^T q + u (k . q)
     const float4 vv = ld4(static_cast<const T *>(p.v) + (size_t)nh * dv + j0);
-    const float4 u = make_float4(bt * (vv.x - rk.x), bt * (vv.y - rk.y),
-                                 bt * (vv.z - rk.z), bt * (vv.w - rk.w));
+    float4 u;
+    if (p.erase) {
+      const float4 wg = ld4(p.write + (size_t)nh * dv + j0);
+      u = make_float4(wg.x * vv.x - rk.x, wg.y * vv.y - rk.y,
+                      wg.z * vv.z - rk.z, wg.w * vv.w - rk.w);
+    } else {
+      const float bt = p.beta[nh];
+      u = make_float4(bt * (vv.x - rk.x), bt * (vv.y - rk.y),
+                      bt * (vv.z - rk.z), bt * (vv.w - rk.w));
+    }
     if (warp == 0)
       st4(static_cast<T *>(p.out) + (size_t)nh * dv + j0, fma4(kq_s, u, rq));
     // S' = S~ + k u^T, in place in the tile
@@ -270,13 +286,15 @@ bool dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 }  // namespace
 }  // namespace gdr
 
-extern "C" gdr_status gdr_decode_step(const void *q, const void *k,
-                                      const void *v, const float *log_alpha,
-                                      const float *beta,
-                                      const float *state_in, float *state_out,
-                                      void *out, int N, int H, int dk, int dv,
-                                      cudaStream_t stream,
-                                      const gdr_opts *opts) {
+namespace gdr {
+namespace {
+
+gdr_status decode_entry(const void *q, const void *k, const void *v,
+                        const float *log_alpha, const float *beta,
+                        const float *erase, const float *write,
+                        const float *state_in, float *state_out, void *out,
+                        int N, int H, int dk, int dv, cudaStream_t stream,
+                        const gdr_opts *opts) {
   gdr_opts o;
   o.dtype = GDR_BF16;
   o.gate = GDR_GATE_SCALAR;
@@ -292,17 +310,19 @@ extern "C" gdr_status gdr_decode_step(const void *q, const void *k,
   if (o.cu_seqlens != nullptr || o.num_seqs != 0)
     return GDR_ERR_INVALID_ARGUMENT;   // one token per sequence: no packing
   if (o.algo != GDR_ALGO_AUTO) return GDR_ERR_UNSUPPORTED;
-  if (!gdr::dim_ok(dk) || !gdr::dim_ok(dv)) return GDR_ERR_UNSUPPORTED;
+  if (!dim_ok(dk) || !dim_ok(dv)) return GDR_ERR_UNSUPPORTED;
   if ((o.gate == GDR_GATE_NONE) != (log_alpha == nullptr))
     return GDR_ERR_INVALID_ARGUMENT;
   const long long nh = (long long)N * H;
   if (nh > 0x7fffffffLL) return GDR_ERR_UNSUPPORTED;
   if (nh == 0) return GDR_OK;
-  if (!q || !k || !v || !beta || !state_out || !out)
-    return GDR_ERR_INVALID_ARGUMENT;
-  const void *ptrs[] = {q, k, v, log_alpha, beta, state_in, state_out, out};
+  const bool g2 = erase != nullptr || write != nullptr;
+  if (!q || !k || !v || !state_out || !out) return GDR_ERR_INVALID_ARGUMENT;
+  if (g2 ? (!erase || !write) : !beta) return GDR_ERR_INVALID_ARGUMENT;
+  const void *ptrs[] = {q, k, v, log_alpha, beta, erase, write, state_in,
+                        state_out, out};
   for (const void *ptr : ptrs)
-    if (ptr && !gdr::aligned16(ptr)) return GDR_ERR_INVALID_ARGUMENT;
+    if (ptr && !aligned16(ptr)) return GDR_ERR_INVALID_ARGUMENT;
   // state_in and state_out: the same buffer (in-place update) or disjoint
   if (state_in && state_in != state_out) {
     const size_t bytes = (size_t)nh * dk * dv * sizeof(float);
@@ -310,7 +330,7 @@ extern "C" gdr_status gdr_decode_step(const void *q, const void *k,
     const uintptr_t b = reinterpret_cast<uintptr_t>(state_out);
     if (a < b + bytes && b < a + bytes) return GDR_ERR_INVALID_ARGUMENT;
   }
-  gdr::DecodeParams dp;
+  DecodeParams dp;
   dp.q = q;
   dp.k = k;
   dp.v = v;
@@ -320,14 +340,41 @@ extern "C" gdr_status gdr_decode_step(const void *q, const void *k,
   dp.s_out = state_out;
   dp.out = out;
   dp.dv = dv;
+  dp.erase = g2 ? erase : nullptr;
+  dp.write = g2 ? write : nullptr;
   const char *inj = std::getenv("GDR_FAULT_INJECT_DECODE_TIMEOUT");
   dp.inject_timeout = (inj && inj[0] == '1') ? 1 : 0;
-  dp.wait_cycles = dp.inject_timeout ? gdr::kDecInjectWaitCycles
-                                     : gdr::kDecWaitCycles;
+  dp.wait_cycles = dp.inject_timeout ? kDecInjectWaitCycles : kDecWaitCycles;
   const int nb = (int)nh;
   const cudaError_t e =
       o.dtype == GDR_BF16
-          ? gdr::launch_t<__nv_bfloat16>(dp, dk, o.gate, nb, stream)
-          : gdr::launch_t<float>(dp, dk, o.gate, nb, stream);
+          ? launch_t<__nv_bfloat16>(dp, dk, o.gate, nb, stream)
+          : launch_t<float>(dp, dk, o.gate, nb, stream);
   return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace gdr
+
+extern "C" gdr_status gdr_decode_step(const void *q, const void *k,
+                                      const void *v, const float *log_alpha,
+                                      const float *beta,
+                                      const float *state_in, float *state_out,
+                                      void *out, int N, int H, int dk, int dv,
+                                      cudaStream_t stream,
+                                      const gdr_opts *opts) {
+  return gdr::decode_entry(q, k, v, log_alpha, beta, nullptr, nullptr,
+                           state_in, state_out, out, N, H, dk, dv, stream,
+                           opts);
+}
+
+extern "C" gdr_status gdr_decode_step_gdn2(
+    const void *q, const void *k, const void *v, const float *log_alpha,
+    const float *erase_gate, const float *write_gate, const float *state_in,
+    float *state_out, void *out, int N, int H, int dk, int dv,
+    cudaStream_t stream, const gdr_opts *opts) {
+  if (!erase_gate || !write_gate) return GDR_ERR_INVALID_ARGUMENT;
+  return gdr::decode_entry(q, k, v, log_alpha, nullptr, erase_gate,
+                           write_gate, state_in, state_out, out, N, H, dk, dv,
+                           stream, opts);
 }

@@ -336,6 +336,30 @@ GDR_API gdr_status gdr_decode_step(const void *q, const void *k, const void *v,
                                    cudaStream_t stream, const gdr_opts *opts);
 
 /*
+ * gdr_decode_step_gdn2 -- gdr_decode_step with Gated DeltaNet-2's separate
+ * erase and write gates (the update gdr_chunk_fwd_gdn2 documents) for one
+ * token per (sequence, head):
+ *     S~ = D S,   u = w . v - S~^T (b . k),   S' = S~ + k u^T,   o = S'^T q
+ * so that a prompt run through gdr_chunk_fwd_gdn2 can be continued one token
+ * at a time.
+ *
+ * Arguments as for gdr_decode_step, with beta replaced by
+ *   erase_gate  [N][H][dk] fp32 (device, 16-byte aligned), required;
+ *   write_gate  [N][H][dv] fp32 (device, 16-byte aligned), required.
+ * Same kernel, limits, bounded wait and status codes as gdr_decode_step;
+ * a NULL gate returns GDR_ERR_INVALID_ARGUMENT.
+ */
+GDR_API gdr_status gdr_decode_step_gdn2(const void *q, const void *k,
+                                        const void *v, const float *log_alpha,
+                                        const float *erase_gate,
+                                        const float *write_gate,
+                                        const float *state_in,
+                                        float *state_out, void *out, int N,
+                                        int H, int dk, int dv,
+                                        cudaStream_t stream,
+                                        const gdr_opts *opts);
+
+/*
  * gdr_backward -- gradients of gdr_chunk_fwd's outputs with respect to its
  * inputs (the backward pass for training).
  *
