@@ -3,6 +3,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--algo auto|staged|fused_tc]
                     [--batch B] [--segments S] [--decode] [--backward]
+                    [--gdn2]
 
 One step = one gdr_chunk_fwd call over one batch of the workload (all four
 stages: log-decay cumsum, WY/UT transform, state passing, output), inputs
@@ -464,12 +465,17 @@ def run_ours(args, w):
 
 DECODE_METRIC = ("tokens/s, single-token decode step (gdr_decode_step), GDN "
                  "H16 d128 bf16, state resident in HBM; % HBM roofline")
+DECODE_GDN2_METRIC = ("tokens/s, single-token decode step with Gated "
+                      "DeltaNet-2 gates (gdr_decode_step_gdn2), H16 d128 bf16, "
+                      "state resident in HBM; % HBM roofline")
 
 
-def decode_bytes(N, H, dk, dv, esz, gate):
+def decode_bytes(N, H, dk, dv, esz, gate, gdn2=False):
     """Bytes a decode step must move: the state read and written once (fp32),
-    q, k, v, out in the I/O dtype, beta and log-alpha in fp32."""
-    per = 2 * dk * dv * 4 + esz * (2 * dk + 2 * dv) + 4
+    q, k, v, out in the I/O dtype, beta (or the erase and write gates) and
+    log-alpha in fp32."""
+    per = 2 * dk * dv * 4 + esz * (2 * dk + 2 * dv)
+    per += 4 * (dk + dv) if gdn2 else 4
     per += {"none": 0, "scalar": 4, "channel": 4 * dk}[gate]
     return N * H * per
 
@@ -489,7 +495,9 @@ def run_decode(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     N, H, d = args.decode_seqs, 16, 128
-    w = Workload("gdn_decode_h16_d128_bf16", B=N, T=1, H=H, dk=d, dv=d,
+    g2 = args.gdn2
+    w = Workload("gdn2_decode_h16_d128_bf16" if g2 else
+                 "gdn_decode_h16_d128_bf16", B=N, T=1, H=H, dk=d, dv=d,
                  chunk=16, dtype="bf16", gate="scalar", decay_lo=0.01,
                  decay_hi=0.1, init_state=True)
     inp = generate(w, seed=args.seed)
@@ -497,12 +505,20 @@ def run_decode(args):
     hq, hk, hv = sq(inp.q), sq(inp.k), sq(inp.v)
     hb, hla = sq(inp.beta), sq(inp.log_alpha)
     q, k, v, b, la = (t.to(dev) for t in (hq, hk, hv, hb, hla))
+    if g2:
+        from chunkwise_recurrence_b200.inputs import gdn2_gates
+        her, hwr = (sq(t) for t in gdn2_gates(inp, seed=args.seed))
+        er, wr = her.to(dev), hwr.to(dev)
     state = inp.s0.to(dev)
     out = torch.empty_like(v)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        gdr.decode_step(q, k, v, b, la, state, out=out, stream=stream)
+        if g2:
+            gdr.decode_step_gdn2(q, k, v, er, wr, la, state, out=out,
+                                 stream=stream)
+        else:
+            gdr.decode_step(q, k, v, b, la, state, out=out, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -520,13 +536,14 @@ def run_decode(args):
     # end to end: the step's token inputs come from pinned host memory and
     # its outputs go back; the state stays resident on the device
     pin = lambda t: t.pin_memory()  # noqa: E731
-    pq, pk, pv, pb, pla = (pin(t) for t in (hq, hk, hv, hb, hla))
+    pairs = [(q, pin(hq)), (k, pin(hk)), (v, pin(hv)), (la, pin(hla))]
+    pairs += ([(er, pin(her)), (wr, pin(hwr))] if g2 else [(b, pin(hb))])
     pout = torch.empty_like(hv).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (pq, pk, pv, pb, pla))
+    h2d = sum(t.numel() * t.element_size() for _, t in pairs)
     d2h = pout.numel() * pout.element_size()
 
     def e2e_step():
-        for dst, src in ((q, pq), (k, pk), (v, pv), (b, pb), (la, pla)):
+        for dst, src in pairs:
             dst.copy_(src, non_blocking=True)
         step()
         pout.copy_(out, non_blocking=True)
@@ -543,12 +560,13 @@ def run_decode(args):
     torch.cuda.synchronize()
     e2e_ms = ea.elapsed_time(eb)
     ms = total_ms / args.steps
-    by = decode_bytes(N, H, d, d, 2, "scalar")
+    by = decode_bytes(N, H, d, d, 2, "scalar", gdn2=g2)
     peaks, peak_src = load_peaks()
     kernel_ms = statistics.mean(per_step)
     gbs = by / (kernel_ms / 1e3) / 1e9
     line = {
-        "metric": DECODE_METRIC, "value": N / (ms / 1e3), "unit": "tokens/s",
+        "metric": DECODE_GDN2_METRIC if g2 else DECODE_METRIC,
+        "value": N / (ms / 1e3), "unit": "tokens/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -565,8 +583,8 @@ def run_decode(args):
         "clocks": clocks.summary(),
         "e2e": {"value": N * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "entry": "gdr_decode_step, token inputs from pinned host "
-                         "memory, state resident"},
+                "entry": ("gdr_decode_step_gdn2" if g2 else "gdr_decode_step")
+                + ", token inputs from pinned host memory, state resident"},
         "gpu_launches": args.steps,
         "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
     }
@@ -575,11 +593,18 @@ def run_decode(args):
         ns = min(N, 32)
         f = lambda t: t[:ns].double().numpy()  # noqa: E731
         t0 = time.perf_counter()
-        oracle.decode_step(f(hq), f(hk), f(hv), f(hb), f(hla), gate="scalar",
-                           state=f(inp.s0))
+        if g2:
+            u = lambda t: t[:ns, None].double().numpy()  # noqa: E731
+            oracle.gdn2_fwd(u(hq), u(hk), u(hv), u(her), u(hwr), u(hla),
+                            "scalar", f(inp.s0))
+            cores = 1   # a numpy token loop on one thread
+        else:
+            oracle.decode_step(f(hq), f(hk), f(hv), f(hb), f(hla),
+                               gate="scalar", state=f(inp.s0))
+            cores = cpu_cores()
         dt = time.perf_counter() - t0
         line["cpu_baseline"] = {
-            "value": ns / dt, "unit": "tokens/s", "cores": cpu_cores(),
+            "value": ns / dt, "unit": "tokens/s", "cores": cores,
             "kind": "oracle",
             "sample": f"sequences 0..{ns - 1} of {N} (x {H} heads), one step"}
     print(json.dumps(line), flush=True)
@@ -677,6 +702,134 @@ def run_backward(args, w):
     return 0
 
 
+GDN2_METRIC = ("tokens/s, chunked forward with Gated DeltaNet-2 erase and "
+               "write gates (gdr_chunk_fwd_gdn2, staged path); % HBM roofline")
+
+
+def run_gdn2(args, w):
+    """The workload's forward pass with Gated DeltaNet-2's per-channel erase
+    and write gates in place of beta (the staged path)."""
+    import torch
+
+    import chunkwise_recurrence_b200 as gdr
+    from chunkwise_recurrence_b200.inputs import gdn2_gates, generate
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        raise SystemExit("--gdn2 runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    inp = generate(w, seed=args.seed)
+    her, hwr = gdn2_gates(inp, seed=args.seed)
+    host = dict(q=inp.q, k=inp.k, v=inp.v, er=her, wr=hwr,
+                la=inp.log_alpha, s0=inp.s0, cu=inp.cu_seqlens)
+    d = {n: None if t is None else t.to(dev) for n, t in host.items()}
+    out = torch.empty_like(d["v"])
+    sT = torch.empty(inp.nseq, w.H, w.dk, w.dv, dtype=torch.float32,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gdr.chunk_fwd_gdn2(d["q"], d["k"], d["v"], d["er"], d["wr"], d["la"],
+                           d["s0"], chunk=w.chunk, gate=w.gate,
+                           cu_seqlens=d["cu"], out=out, final_state=sT,
+                           stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_gpu_index(local)) as clocks:
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+    if gdr.device_error() != 0:
+        raise RuntimeError("device-side error during timing")
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    ms = ev[0].elapsed_time(ev[-1]) / args.steps
+    # end to end: every input from pinned host memory, out and the final
+    # state back, through the same device entry point
+    pinned = {n: None if t is None else t.pin_memory()
+              for n, t in host.items()}
+    hout = torch.empty_like(inp.v).pin_memory()
+    hsT = torch.empty(inp.nseq, w.H, w.dk, w.dv).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values()
+              if t is not None)
+    d2h = hout.numel() * hout.element_size() + hsT.numel() * 4
+
+    def e2e_step():
+        for n, t in pinned.items():
+            if t is not None:
+                d[n].copy_(t, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+        hsT.copy_(sT, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(1, min(args.steps, 10))
+    ea, eb = (torch.cuda.Event(enable_timing=True),
+              torch.cuda.Event(enable_timing=True))
+    ea.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    eb.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ea.elapsed_time(eb)
+    ntok, H, dk, dv = inp.ntok, w.H, w.dk, w.dv
+    esz = 4 if w.dtype == "fp32" else 2
+    la_b = {"none": 0, "scalar": 4, "channel": 4 * dk}[w.gate]
+    # q, k, v, out in the I/O dtype, the two gates and log-alpha in fp32,
+    # each read or written once; the states in and out
+    by = ntok * H * (esz * (2 * dk + 2 * dv) + 4 * (dk + dv) + la_b)
+    by += inp.nseq * H * dk * dv * 4 * (1 + (1 if inp.s0 is not None else 0))
+    peaks, peak_src = load_peaks()
+    gbs = by / (statistics.mean(per_step) / 1e3) / 1e9
+    line = {
+        "metric": GDN2_METRIC, "value": ntok / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {**workload_config(w, inp), "algo": "staged",
+                   "gates": "erase [.., dk], write [.., dv], sigmoid(N(0,1))",
+                   "l2": "inputs larger than L2 (no flush)",
+                   "launch": "direct"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                     "traffic": None, "peak_source": peak_src,
+                     "kernel": "staged path (whole call)",
+                     "algorithmic_bytes_per_launch": by},
+        "clocks": clocks.summary(),
+        "e2e": {"value": ntok * e2e_steps / (e2e_ms / 1e3),
+                "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "entry": "gdr_chunk_fwd_gdn2, inputs copied from pinned host "
+                         "memory and results back each step"},
+        "gpu_launches": launches_per_step("staged", w) * args.steps,
+        "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
+    }
+    if not args.no_cpu_baseline:
+        import oracle
+        f = lambda t, n: None if t is None else t[:n].double().numpy()  # noqa
+        n = 1
+        t0 = time.perf_counter()
+        oracle.gdn2_fwd(f(inp.q, n), f(inp.k, n), f(inp.v, n), f(her, n),
+                        f(hwr, n), f(inp.log_alpha, n), w.gate,
+                        f(inp.s0, n))
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {
+            "value": n * w.T / dt, "unit": "tokens/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"sequence 0 of {inp.nseq} ({w.T} tokens x {H} heads), "
+                      "numpy token loop on one thread"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def gdr_fused_available():
     from chunkwise_recurrence_b200 import fused_tc_available
     return fused_tc_available()
@@ -719,6 +872,10 @@ def main(argv=None):
     ap.add_argument("--segments", type=int, default=0,
                     help="context-parallel forward (gdr_chunk_fwd_segmented) "
                          "with this many pieces per sequence")
+    ap.add_argument("--gdn2", action="store_true",
+                    help="with Gated DeltaNet-2 erase and write gates "
+                         "(gdr_chunk_fwd_gdn2; with --decode, "
+                         "gdr_decode_step_gdn2)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -731,6 +888,10 @@ def main(argv=None):
         return run_decode(args)
     if args.backward and args.impl == "ours":
         return run_backward(args, w)
+    if args.gdn2 and args.impl == "ours":
+        if w.varlen_nseq:
+            raise SystemExit("--gdn2 takes a fixed-length workload")
+        return run_gdn2(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

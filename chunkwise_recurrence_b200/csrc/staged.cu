@@ -102,6 +102,10 @@ __device__ __forceinline__ float gval(const float *Gs, int gdim, int r,
 // (write gate w_r, per value channel), and beta is not used:
 //   A[r][i] = (b_r . k_r)^T Gamma_r Gamma_i^-1 k_i,  W = T ((B . K) . e^g),
 //   U = T (Wg . V).
+// Shared memory: the key rows are padded to dk + 1 floats so that the A
+// products, whose lanes walk rows, read distinct banks; the factors of W and
+// U (beta_i (read key) e^{g_i} and beta_i (target)) are formed once per
+// chunk, not once per (row, column) of the product.
 template <typename Tin>
 __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
                           const float *__restrict__ beta,
@@ -117,54 +121,55 @@ __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
   const ChunkInfo ci = table[j];
   const int L = ci.len;
   const int gd = gdim == 0 ? 1 : gdim;
-  extern __shared__ float sm[];
-  float *Ks = sm;                  // [C][dk]
-  float *Gs = Ks + C * dk;         // [C][gd]
+  const int dkp = dk + 1;
+  const bool g2 = erase != nullptr;
+  extern __shared__ __align__(16) float sm[];
+  float *Ks = sm;                  // [C][dkp]
+  float *Gs = Ks + C * dkp;        // [C][gd]
   float *As = Gs + C * gd;         // [C][C+1]
   float *Ts = As + C * (C + 1);    // [C][C+1]
   float *bs = Ts + C * (C + 1);    // [C]
-  float *Es = bs + C;              // [C][dk], erase gates (Gated DeltaNet-2)
+  float *Vs = bs + C;              // [C][dv], beta_i v_i (or w_i . v_i)
+  float *Es = Vs + C * dv;         // [C][dkp], b_r . k_r (Gated DeltaNet-2)
+  // the read keys: b_r . k_r (Gated DeltaNet-2) or k_r; the row factor
+  // bs[r] is then 1 or beta_r
+  float *Rs = g2 ? Es : Ks;
   const int tid = threadIdx.x, nt = blockDim.x;
-  const bool g2 = erase != nullptr;
 
   for (int idx = tid; idx < L * dk; idx += nt) {
     const int r = idx / dk, c = idx % dk;
-    Ks[r * dk + c] = to_f(k[((size_t)(ci.tok0 + r) * H + h) * dk + c]);
+    const size_t off = ((size_t)(ci.tok0 + r) * H + h) * dk + c;
+    const float kv = to_f(k[off]);
+    Ks[r * dkp + c] = kv;
+    if (g2) Es[r * dkp + c] = erase[off] * kv;
   }
   if (gdim)
     for (int idx = tid; idx < L * gdim; idx += nt) {
       const int r = idx / gdim, c = idx % gdim;
       Gs[r * gdim + c] = g[((size_t)(ci.tok0 + r) * H + h) * gdim + c];
     }
-  if (g2) {
-    for (int idx = tid; idx < L * dk; idx += nt) {
-      const int r = idx / dk, c = idx % dk;
-      Es[r * dk + c] = erase[((size_t)(ci.tok0 + r) * H + h) * dk + c];
-    }
-    for (int r = tid; r < L; r += nt) bs[r] = 1.f;
-  } else {
-    for (int r = tid; r < L; r += nt)
-      bs[r] = beta[(size_t)(ci.tok0 + r) * H + h];
-  }
+  for (int r = tid; r < L; r += nt)
+    bs[r] = g2 ? 1.f : beta[(size_t)(ci.tok0 + r) * H + h];
   __syncthreads();
-  // the read key of row r, channel c: b_r[c] k_r[c] (Gated DeltaNet-2) or
-  // k_r[c]; the row factor bs[r] is then 1 or beta_r
-  auto rk = [&](int r, int c) {
-    return g2 ? Es[r * dk + c] * Ks[r * dk + c] : Ks[r * dk + c];
-  };
+  for (int idx = tid; idx < L * dv; idx += nt) {
+    const int r = idx / dv, c = idx % dv;
+    const size_t e = ((size_t)(ci.tok0 + r) * H + h) * dv + c;
+    Vs[r * dv + c] = bs[r] * (g2 ? write[e] * to_f(v[e]) : to_f(v[e]));
+  }
 
-  // A[r][i] = beta_r sum_c k_r[c] k_i[c] exp(g_r[c] - g_i[c]),  i < r
+  // A[r][i] = beta_r sum_c rk_r[c] k_i[c] exp(g_r[c] - g_i[c]),  i < r
   for (int idx = tid; idx < L * L; idx += nt) {
     const int r = idx / L, i = idx % L;
     float a = 0.f;
     if (i < r) {
+      const float *rr = Rs + r * dkp, *ki = Ks + i * dkp;
       if (gdim <= 1) {
-        for (int c = 0; c < dk; ++c) a += rk(r, c) * Ks[i * dk + c];
+        for (int c = 0; c < dk; ++c) a += rr[c] * ki[c];
         if (gdim == 1) a *= __expf(Gs[r] - Gs[i]);
       } else {
+        const float *gr = Gs + r * gdim, *gi = Gs + i * gdim;
         for (int c = 0; c < dk; ++c)
-          a += rk(r, c) * Ks[i * dk + c] *
-               __expf(Gs[r * gdim + c] - Gs[i * gdim + c]);
+          a += rr[c] * ki[c] * __expf(gr[c] - gi[c]);
       }
       a *= bs[r];
     }
@@ -172,6 +177,13 @@ __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
     Ts[r * (C + 1) + i] = (r == i) ? 1.f : 0.f;
   }
   __syncthreads();
+
+  // the factor of W, in place of the read keys (A no longer needs them):
+  // X[i][c] = beta_i rk_i[c] e^{g_i[c]}
+  for (int idx = tid; idx < L * dk; idx += nt) {
+    const int i = idx / dk, c = idx % dk;
+    Rs[i * dkp + c] = bs[i] * Rs[i * dkp + c] * __expf(gval(Gs, gdim, i, c));
+  }
 
   // T = (I + A)^-1, row by row: T[r][j] = -sum_{j<=i<r} A[r][i] T[i][j]
   for (int r = 1; r < L; ++r) {
@@ -182,28 +194,28 @@ __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
     }
     __syncthreads();
   }
+  if (L <= 1) __syncthreads();   // the X and Vs writes before their reads
 
-  // W = T diag(beta) (K . e^g),  U = T diag(beta) V
+  // W = T X,  U = T Vs
   for (int idx = tid; idx < L * dk; idx += nt) {
     const int r = idx / dk, c = idx % dk;
+    const float *tr = Ts + r * (C + 1);
     float acc = 0.f;
-    for (int i = 0; i <= r; ++i)
-      acc += Ts[r * (C + 1) + i] * bs[i] * rk(i, c) *
-             __expf(gval(Gs, gdim, i, c));
+    for (int i = 0; i <= r; ++i) acc += tr[i] * Rs[i * dkp + c];
     W[((size_t)(ci.tok0 + r) * H + h) * dk + c] = acc;
   }
   for (int idx = tid; idx < L * dv; idx += nt) {
     const int r = idx / dv, c = idx % dv;
+    const float *tr = Ts + r * (C + 1);
     float acc = 0.f;
-    for (int i = 0; i <= r; ++i) {
-      const size_t e = ((size_t)(ci.tok0 + i) * H + h) * dv + c;
-      acc += Ts[r * (C + 1) + i] * bs[i] * to_f(v[e]) * (g2 ? write[e] : 1.f);
-    }
+    for (int i = 0; i <= r; ++i) acc += tr[i] * Vs[i * dv + c];
     U[((size_t)(ci.tok0 + r) * H + h) * dv + c] = acc;
   }
 }
 
 // (c) sequential state passing for one (sequence, head, dv tile).
+// Per chunk the rows k_r . e^{g_C - g_r} are formed once in shared memory
+// (one exponential per row and channel) before the state update reads them.
 template <typename Tin>
 __global__ void state_kernel(const Tin *__restrict__ k,
                              const float *__restrict__ g,
@@ -216,10 +228,11 @@ __global__ void state_kernel(const Tin *__restrict__ k,
                              const int *__restrict__ seq_first, int H, int dk,
                              int dv, int C, int gdim, int DVT) {
   const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * DVT;
-  extern __shared__ float sm[];
+  extern __shared__ __align__(16) float sm[];
   float *S = sm;              // [dk][DVT]
   float *V = S + dk * DVT;    // [C][DVT]
   float *gl = V + C * DVT;    // [dk]
+  float *Kt = gl + dk;        // [C][dk], k_r . e^{g_C - g_r}
   const int tid = threadIdx.x, nt = blockDim.x;
   const size_t sbase = ((size_t)n * H + h) * dk * dv;
 
@@ -252,16 +265,18 @@ __global__ void state_kernel(const Tin *__restrict__ k,
                         : g[((size_t)(ci.tok0 + L - 1) * H + h) * gdim +
                             (gdim == 1 ? 0 : c)];
     __syncthreads();
+    for (int idx = tid; idx < L * dk; idx += nt) {
+      const int r = idx / dk, c = idx % dk;
+      const size_t row = (size_t)(ci.tok0 + r) * H + h;
+      const float gr = gdim == 0 ? 0.f : g[row * gdim + (gdim == 1 ? 0 : c)];
+      Kt[idx] = to_f(k[row * dk + c]) * __expf(gl[c] - gr);
+    }
+    __syncthreads();
     // S <- Gamma_C S + (K . e^{g_C - g})^T V_new
     for (int idx = tid; idx < dk * DVT; idx += nt) {
       const int c = idx / DVT, jj = idx % DVT;
       float acc = __expf(gl[c]) * S[idx];
-      for (int r = 0; r < L; ++r) {
-        const size_t row = (size_t)(ci.tok0 + r) * H + h;
-        const float gr =
-            gdim == 0 ? 0.f : g[row * gdim + (gdim == 1 ? 0 : c)];
-        acc += to_f(k[row * dk + c]) * __expf(gl[c] - gr) * V[r * DVT + jj];
-      }
+      for (int r = 0; r < L; ++r) acc += Kt[r * dk + c] * V[r * DVT + jj];
       S[idx] = acc;
     }
     __syncthreads();
@@ -273,7 +288,12 @@ __global__ void state_kernel(const Tin *__restrict__ k,
     }
 }
 
-// (d) chunk output for one (chunk, head).
+// (d) chunk output for one (chunk, head).  After the masked products P, the
+// rows of Q are scaled in place to Q . e^g; each thread then owns one value
+// column and blocks of kOutRows rows, so that a state element read from
+// memory serves kOutRows outputs.
+constexpr int kOutRows = 8;
+
 template <typename Tin>
 __global__ void output_kernel(const Tin *__restrict__ q,
                               const Tin *__restrict__ k,
@@ -289,17 +309,18 @@ __global__ void output_kernel(const Tin *__restrict__ q,
   const ChunkInfo ci = table[j];
   const int L = ci.len;
   const int gd = gdim == 0 ? 1 : gdim;
-  extern __shared__ float sm[];
+  const int dkp = dk + 1;
+  extern __shared__ __align__(16) float sm[];
   float *Qs = sm;               // [C][dk]
-  float *Ks = Qs + C * dk;      // [C][dk]
-  float *Gs = Ks + C * dk;      // [C][gd]
+  float *Ks = Qs + C * dk;      // [C][dkp]
+  float *Gs = Ks + C * dkp;     // [C][gd]
   float *Ps = Gs + C * gd;      // [C][C+1]
   const int tid = threadIdx.x, nt = blockDim.x;
   for (int idx = tid; idx < L * dk; idx += nt) {
     const int r = idx / dk, c = idx % dk;
     const size_t off = ((size_t)(ci.tok0 + r) * H + h) * dk + c;
     Qs[r * dk + c] = to_f(q[off]);
-    Ks[r * dk + c] = to_f(k[off]);
+    Ks[r * dkp + c] = to_f(k[off]);
   }
   if (gdim)
     for (int idx = tid; idx < L * gdim; idx += nt) {
@@ -312,29 +333,60 @@ __global__ void output_kernel(const Tin *__restrict__ q,
     const int r = idx / L, i = idx % L;
     float a = 0.f;
     if (i <= r) {
+      const float *qr = Qs + r * dk, *ki = Ks + i * dkp;
       if (gdim <= 1) {
-        for (int c = 0; c < dk; ++c) a += Qs[r * dk + c] * Ks[i * dk + c];
+        for (int c = 0; c < dk; ++c) a += qr[c] * ki[c];
         if (gdim == 1) a *= __expf(Gs[r] - Gs[i]);
       } else {
+        const float *gr = Gs + r * gdim, *gi = Gs + i * gdim;
         for (int c = 0; c < dk; ++c)
-          a += Qs[r * dk + c] * Ks[i * dk + c] *
-               __expf(Gs[r * gdim + c] - Gs[i * gdim + c]);
+          a += qr[c] * ki[c] * __expf(gr[c] - gi[c]);
       }
     }
     Ps[r * (C + 1) + i] = a;
   }
   __syncthreads();
+  for (int idx = tid; idx < L * dk; idx += nt) {
+    const int r = idx / dk, c = idx % dk;
+    Qs[idx] = Qs[idx] * __expf(gval(Gs, gdim, r, c));
+  }
+  __syncthreads();
   const float *Sn = Sbuf + ((size_t)j * H + h) * dk * dv;
-  for (int idx = tid; idx < L * dv; idx += nt) {
-    const int r = idx / dv, c = idx % dv;
-    float acc = 0.f;
-    for (int e = 0; e < dk; ++e)
-      acc += Qs[r * dk + e] * __expf(gval(Gs, gdim, r, e)) *
-             Sn[(size_t)e * dv + c];
-    for (int i = 0; i <= r; ++i)
-      acc += Ps[r * (C + 1) + i] *
-             Vn[((size_t)(ci.tok0 + i) * H + h) * dv + c];
-    out[((size_t)(ci.tok0 + r) * H + h) * dv + c] = from_f<Tin>(acc);
+  const int groups = nt / dv;   // dv divides the block size
+  const int c = tid % dv;
+  for (int r0 = (tid / dv) * kOutRows; r0 < L; r0 += groups * kOutRows) {
+    // rows r0 .. r0 + kOutRows - 1 lie inside the C-row tiles (C is a
+    // multiple of kOutRows); rows >= L hold stale values and are not stored
+    float acc[kOutRows];
+#pragma unroll
+    for (int i = 0; i < kOutRows; ++i) acc[i] = 0.f;
+    for (int e = 0; e < dk; e += 4) {
+      const float s0 = Sn[(size_t)e * dv + c];
+      const float s1 = Sn[(size_t)(e + 1) * dv + c];
+      const float s2 = Sn[(size_t)(e + 2) * dv + c];
+      const float s3 = Sn[(size_t)(e + 3) * dv + c];
+#pragma unroll
+      for (int i = 0; i < kOutRows; ++i) {
+        const float4 qv =
+            *reinterpret_cast<const float4 *>(Qs + (r0 + i) * dk + e);
+        acc[i] += qv.x * s0;
+        acc[i] += qv.y * s1;
+        acc[i] += qv.z * s2;
+        acc[i] += qv.w * s3;
+      }
+    }
+    const int iend = min(L, r0 + kOutRows);
+    for (int i2 = 0; i2 < iend; ++i2) {
+      const float vn = Vn[((size_t)(ci.tok0 + i2) * H + h) * dv + c];
+#pragma unroll
+      for (int i = 0; i < kOutRows; ++i)
+        if (i2 <= r0 + i) acc[i] += Ps[(r0 + i) * (C + 1) + i2] * vn;
+    }
+#pragma unroll
+    for (int i = 0; i < kOutRows; ++i)
+      if (r0 + i < L)
+        out[((size_t)(ci.tok0 + r0 + i) * H + h) * dv + c] =
+            from_f<Tin>(acc[i]);
   }
 }
 
@@ -391,10 +443,11 @@ cudaError_t run_typed(const Problem &p, char *ws, cudaStream_t s) {
     if (gdim)
       cumsum_kernel<<<grid, 128, 0, s>>>(p.log_alpha, g, table, nchunks, p.H,
                                          gdim);
+    const size_t dkp = (size_t)p.dk + 1;
     const size_t wy_smem =
-        sizeof(float) * ((size_t)C * p.dk + (size_t)C * gd +
-                         2 * (size_t)C * (C + 1) + C +
-                         (p.erase ? (size_t)C * p.dk : 0));
+        sizeof(float) * ((size_t)C * dkp + (size_t)C * gd +
+                         2 * (size_t)C * (C + 1) + C + (size_t)C * p.dv +
+                         (p.erase ? (size_t)C * dkp : 0));
     cudaError_t e = cudaFuncSetAttribute(
         wy_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
         (int)wy_smem);
@@ -403,16 +456,23 @@ cudaError_t run_typed(const Problem &p, char *ws, cudaStream_t s) {
                                              g, W, U, table, nchunks, p.H,
                                              p.dk, p.dv, C, gdim);
   }
-  const int DVT = p.dv < 32 ? p.dv : 32;
+  const int DVT = p.dv < 64 ? p.dv : 64;
   const size_t st_smem =
-      sizeof(float) * ((size_t)p.dk * DVT + (size_t)C * DVT + p.dk);
+      sizeof(float) * ((size_t)p.dk * DVT + (size_t)C * DVT + p.dk +
+                       (size_t)C * p.dk);
+  {
+    cudaError_t e = cudaFuncSetAttribute(
+        state_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)st_smem);
+    if (e != cudaSuccess) return e;
+  }
   state_kernel<Tin><<<dim3(p.nseq, p.H, p.dv / DVT), 256, st_smem, s>>>(
       k, g, W, U, p.s0, p.sT, Sbuf, Vn, table, seq_first, p.H, p.dk, p.dv, C,
       gdim, DVT);
   if (p.max_chunks > 0) {
     const size_t o_smem =
-        sizeof(float) * (2 * (size_t)C * p.dk + (size_t)C * gd +
-                         (size_t)C * (C + 1));
+        sizeof(float) * ((size_t)C * p.dk + (size_t)C * (p.dk + 1) +
+                         (size_t)C * gd + (size_t)C * (C + 1));
     cudaError_t e = cudaFuncSetAttribute(
         output_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
         (int)o_smem);
