@@ -16,7 +16,8 @@ with D_t = I, alpha_t I or diag(alpha_t) as for the other gates.  Plain numpy
 loops over tokens; small cases only.  Pinned in tests/test_oracle.py by its
 reduction to the C oracle (b_t = w_t = beta_t 1), the no-erase closed form
 (b = 0: a decayed sum of write outer products) and one-hot keys (each row of
-S then follows its own scalar recurrence).
+S then follows its own scalar recurrence); the same file checks that
+plausible mistakes planted in a copy of this loop fail those pins.
 """
 from __future__ import annotations
 

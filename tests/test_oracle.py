@@ -407,40 +407,40 @@ def test_efla_limits():
     np.testing.assert_allclose(se[0, 0].T @ k[0, 0, 0], v[0, 0, 0], atol=1e-12)
 
 
-@pytest.mark.parametrize("gate", ["none", "scalar", "channel"])
-def test_gdn2_reduces_to_the_delta_rule(oracle_lib, gate):
+def _gdn2_reduction(fn, gate):
     """Erase and write gates equal to beta_t on every channel give the delta
     rule: the Gated DeltaNet-2 loop matches the C oracle."""
     rng = np.random.default_rng(31)
     c = _rand_case(rng, B=2, T=13, H=2, dk=4, dv=3, gate=gate)
     o, s, _ = gdr_fwd(**c)
     b = c["beta"]
-    go, gs = oracle.gdn2_fwd(c["q"], c["k"], c["v"],
-                             np.repeat(b[..., None], 4, axis=-1),
-                             np.repeat(b[..., None], 3, axis=-1),
-                             c["log_alpha"], gate, c["initial_state"])
-    assert np.allclose(go, o, atol=1e-13) and np.allclose(gs, s, atol=1e-13)
+    go, gs = fn(c["q"], c["k"], c["v"], np.repeat(b[..., None], 4, axis=-1),
+                np.repeat(b[..., None], 3, axis=-1), c["log_alpha"], gate,
+                c["initial_state"])
+    return np.allclose(go, o, atol=1e-13) and np.allclose(gs, s, atol=1e-13)
 
 
-def test_gdn2_without_erase_is_decayed_linear_attention(oracle_lib):
+def _gdn2_no_erase(fn):
     """b = 0: nothing is erased, so S_t = sum_{s<=t} (prod_{s<tau<=t} D_tau)
     k_s (w_s . v_s)^T (+ the decayed initial state), summed directly."""
     rng = np.random.default_rng(32)
     c = _rand_case(rng, B=1, T=9, H=1, dk=3, dv=2, gate="channel")
     w = rng.uniform(0.1, 1.0, size=(1, 9, 1, 2))
-    go, gs = oracle.gdn2_fwd(c["q"], c["k"], c["v"], np.zeros((1, 9, 1, 3)),
-                             w, c["log_alpha"], "channel", c["initial_state"])
+    go, gs = fn(c["q"], c["k"], c["v"], np.zeros((1, 9, 1, 3)), w,
+                c["log_alpha"], "channel", c["initial_state"])
     la = c["log_alpha"][0, :, 0]
+    ok = True
     for t in range(9):
         S = np.exp(la[:t + 1].sum(axis=0))[:, None] * c["initial_state"][0, 0]
         for s_ in range(t + 1):
             dec = np.exp(la[s_ + 1:t + 1].sum(axis=0))
-            S = S + np.outer(dec * c["k"][0, s_, 0], w[0, s_, 0] * c["v"][0, s_, 0])
-        assert np.allclose(go[0, t, 0], S.T @ c["q"][0, t, 0], atol=1e-13)
-    assert np.allclose(gs[0, 0], S, atol=1e-13)
+            S = S + np.outer(dec * c["k"][0, s_, 0],
+                             w[0, s_, 0] * c["v"][0, s_, 0])
+        ok &= np.allclose(go[0, t, 0], S.T @ c["q"][0, t, 0], atol=1e-13)
+    return ok and np.allclose(gs[0, 0], S, atol=1e-13)
 
 
-def test_gdn2_one_hot_keys_update_rows_independently(oracle_lib):
+def _gdn2_one_hot(fn):
     """With k_t = e_c, only row c of S changes, and it follows
     S_c <- (1 - b_t[c]) a_t[c] S_c + w_t . v_t (a = the decay of row c)."""
     rng = np.random.default_rng(33)
@@ -454,14 +454,88 @@ def test_gdn2_one_hot_keys_update_rows_independently(oracle_lib):
     w = rng.uniform(0, 1, size=(1, T, 1, dv))
     la = -rng.uniform(0.05, 0.5, size=(1, T, 1, dk))
     S0 = rng.standard_normal((1, 1, dk, dv))
-    go, gs = oracle.gdn2_fwd(q, k, v, b, w, la, "channel", S0)
+    go, gs = fn(q, k, v, b, w, la, "channel", S0)
     S = S0[0, 0].copy()
+    ok = True
     for t in range(T):
         S = np.exp(la[0, t, 0])[:, None] * S
         c = cs[t]
         S[c] = (1 - b[0, t, 0, c]) * S[c] + w[0, t, 0] * v[0, t, 0]
-        assert np.allclose(go[0, t, 0], S.T @ q[0, t, 0], atol=1e-13)
-    assert np.allclose(gs[0, 0], S, atol=1e-13)
+        ok &= np.allclose(go[0, t, 0], S.T @ q[0, t, 0], atol=1e-13)
+    return ok and np.allclose(gs[0, 0], S, atol=1e-13)
+
+
+def _gdn2_battery(fn):
+    """Names of the Gated DeltaNet-2 pins that `fn` fails (an exception
+    counts as a failure)."""
+    pins = {f"reduction_{g}": (lambda g=g: _gdn2_reduction(fn, g))
+            for g in ("none", "scalar", "channel")}
+    pins["no_erase"] = lambda: _gdn2_no_erase(fn)
+    pins["one_hot"] = lambda: _gdn2_one_hot(fn)
+    fails = []
+    for name, pin in pins.items():
+        try:
+            ok = pin()
+        except Exception:  # noqa: BLE001  (a crash is a failed pin)
+            ok = False
+        if not ok:
+            fails.append(name)
+    return fails
+
+
+@pytest.mark.parametrize("gate", ["none", "scalar", "channel"])
+def test_gdn2_reduces_to_the_delta_rule(oracle_lib, gate):
+    assert _gdn2_reduction(oracle.gdn2_fwd, gate)
+
+
+def test_gdn2_without_erase_is_decayed_linear_attention(oracle_lib):
+    assert _gdn2_no_erase(oracle.gdn2_fwd)
+
+
+def test_gdn2_one_hot_keys_update_rows_independently(oracle_lib):
+    assert _gdn2_one_hot(oracle.gdn2_fwd)
+
+
+# plausible mistakes in the Gated DeltaNet-2 token loop, as (text, mutant)
+GDN2_MUTANTS = {
+    "erase_gate_dropped": (
+        "r = S.T @ (erase[b, t, h] * k[b, t, h])", "r = S.T @ k[b, t, h]"),
+    "write_gate_dropped": (
+        "u = write[b, t, h] * v[b, t, h] - r", "u = v[b, t, h] - r"),
+    "write_gate_on_the_residual": (
+        "u = write[b, t, h] * v[b, t, h] - r",
+        "u = write[b, t, h] * (v[b, t, h] - r)"),
+    "written_along_the_read_key": (
+        "S = S + np.outer(k[b, t, h], u)",
+        "S = S + np.outer(erase[b, t, h] * k[b, t, h], u)"),
+    "residual_sign": (
+        "u = write[b, t, h] * v[b, t, h] - r",
+        "u = write[b, t, h] * v[b, t, h] + r"),
+    "scalar_decay_sign": (
+        "S = np.exp(la[b, t, h]) * S", "S = np.exp(-la[b, t, h]) * S"),
+    "channel_decay_dropped": (
+        "S = np.exp(la[b, t, h])[:, None] * S", "S = S"),
+    "read_before_write": (
+        "out[b, t, h] = S.T @ q[b, t, h]",
+        "out[b, t, h] = (S - np.outer(k[b, t, h], u)).T @ q[b, t, h]"),
+    "initial_state_ignored": (
+        "else np.array(initial_state[n, h], np.float64))",
+        "else np.zeros((dk, dv)))"),
+}
+
+
+def test_gdn2_pins_catch_planted_mistakes(oracle_lib):
+    """Each plausible mistake, planted in a copy of the Gated DeltaNet-2 loop,
+    fails at least one of its pins; the loop as written fails none."""
+    assert _gdn2_battery(oracle.gdn2_fwd) == []
+    src = open(os.path.join(os.path.dirname(oracle.__file__),
+                            "gdn2_ref.py")).read()
+    for name, (text, mutant) in GDN2_MUTANTS.items():
+        assert src.count(text) == 1, name
+        ns = {"__name__": f"gdn2_mutant_{name}"}
+        exec(compile(src.replace(text, mutant), name, "exec"), ns)
+        assert _gdn2_battery(ns["gdn2_fwd"]), (
+            f"planted mistake '{name}' passed every pin")
 
 
 def test_gradients_match_finite_differences(oracle_lib):
