@@ -367,25 +367,27 @@ def _efla_step_size(k, beta):
                     beta)
 
 
-def test_efla_flow_is_the_delta_rule_with_a_new_step_size(oracle_lib):
-    """The exact flow, integrated by a matrix exponential (oracle.efla_fwd),
-    equals the delta rule run with beta' = (1 - e^{-beta |k|^2}) / |k|^2 --
-    the closed form the library's gdr_efla_beta computes -- for every gate,
-    with unnormalised keys too."""
+def _efla_flow(fn, lib=None):
+    """The exact flow, integrated by a matrix exponential, equals the delta
+    rule run with beta' = (1 - e^{-beta |k|^2}) / |k|^2 -- the closed form the
+    library's gdr_efla_beta computes -- for every gate, with unnormalised keys
+    too."""
     rng = np.random.default_rng(21)
+    ok = True
     for gate in ("none", "scalar", "channel"):
         case = _rand_case(rng, B=2, T=7, H=2, dk=4, dv=3, gate=gate)
         case["k"] = case["k"] * rng.uniform(0.3, 2.0, size=case["k"].shape[:-1]
                                             + (1,))
         case["beta"] = case["beta"] * 3.0
-        ro, rs = oracle.efla_fwd(**case)
+        ro, rs = fn(**case)
         bp = _efla_step_size(case["k"], case["beta"])
-        o, sT, _ = gdr_fwd(**{**case, "beta": bp}, lib=oracle_lib)
-        np.testing.assert_allclose(o, ro, atol=1e-10)
-        np.testing.assert_allclose(sT, rs, atol=1e-10)
+        o, sT, _ = gdr_fwd(**{**case, "beta": bp}, lib=lib)
+        ok &= np.allclose(o, ro, rtol=0, atol=1e-10)
+        ok &= np.allclose(sT, rs, rtol=0, atol=1e-10)
+    return ok
 
 
-def test_efla_limits():
+def _efla_limits(fn):
     """Small steps: the exact flow and one Euler step (the delta rule) agree
     to first order in beta.  Long flow with a unit key: the memory converges
     to the least-squares solution, so reading the key returns the value."""
@@ -395,16 +397,69 @@ def test_efla_limits():
     k /= np.linalg.norm(k)
     v = rng.standard_normal((1, 1, 1, dv))
     S0 = rng.standard_normal((1, 1, dk, dv))
+    ok = True
     for b in (1e-3, 1e-4):
-        _, se = oracle.efla_fwd(k, k, v, np.full((1, 1, 1), b), gate="none",
-                                initial_state=S0)
+        _, se = fn(k, k, v, np.full((1, 1, 1), b), gate="none",
+                   initial_state=S0)
         euler = S0[0, 0] - b * np.outer(k[0, 0, 0], S0[0, 0].T @ k[0, 0, 0]
                                         - v[0, 0, 0])
-        assert np.max(np.abs(se[0, 0] - euler)) < 5 * b * b * (
-            1 + np.max(np.abs(S0)))
-    _, se = oracle.efla_fwd(k, k, v, np.full((1, 1, 1), 60.0), gate="none",
-                            initial_state=S0)
-    np.testing.assert_allclose(se[0, 0].T @ k[0, 0, 0], v[0, 0, 0], atol=1e-12)
+        ok &= bool(np.max(np.abs(se[0, 0] - euler)) < 5 * b * b * (
+            1 + np.max(np.abs(S0))))
+    _, se = fn(k, k, v, np.full((1, 1, 1), 60.0), gate="none",
+               initial_state=S0)
+    return ok and np.allclose(se[0, 0].T @ k[0, 0, 0], v[0, 0, 0], rtol=0,
+                              atol=1e-12)
+
+
+def test_efla_flow_is_the_delta_rule_with_a_new_step_size(oracle_lib):
+    assert _efla_flow(oracle.efla_fwd, oracle_lib)
+
+
+def test_efla_limits():
+    assert _efla_limits(oracle.efla_fwd)
+
+
+# plausible mistakes in the EFLA flow integration, as (text, mutant)
+EFLA_MUTANTS = {
+    "flow_sign": ("M[:dk, :dk] = -np.outer(kt, kt)",
+                  "M[:dk, :dk] = np.outer(kt, kt)"),
+    "forcing_sign": ("M[:dk, dk:] = np.outer(kt, vt)",
+                     "M[:dk, dk:] = -np.outer(kt, vt)"),
+    "forcing_dropped": ("S = E[:dk, :dk] @ S + E[:dk, dk:]",
+                        "S = E[:dk, :dk] @ S"),
+    "step_length_ignored": ("E = expm(beta[b, t, h] * M)", "E = expm(M)"),
+    "read_before_update": (
+        "S = E[:dk, :dk] @ S + E[:dk, dk:]\n"
+        "                out[b, t, h] = S.T @ q[b, t, h]",
+        "out[b, t, h] = S.T @ q[b, t, h]\n"
+        "                S = E[:dk, :dk] @ S + E[:dk, dk:]"),
+    "scalar_decay_sign": ("S = np.exp(log_alpha[b, t, h]) * S",
+                          "S = np.exp(-log_alpha[b, t, h]) * S"),
+    "channel_decay_dropped": (
+        "S = np.exp(np.asarray(log_alpha[b, t, h]))[:, None] * S", "S = S"),
+}
+
+
+def test_efla_pins_catch_planted_mistakes(oracle_lib):
+    """Each plausible mistake, planted in a copy of the EFLA loop, fails at
+    least one of its pins."""
+    src = open(os.path.join(os.path.dirname(oracle.__file__),
+                            "efla_ref.py")).read()
+    for name, (text, mutant) in EFLA_MUTANTS.items():
+        assert src.count(text) == 1, name
+        ns = {"__name__": f"efla_mutant_{name}"}
+        exec(compile(src.replace(text, mutant), name, "exec"), ns)
+        fn = ns["efla_fwd"]
+        fails = []
+        for pin, call in (("flow", lambda: _efla_flow(fn, oracle_lib)),
+                          ("limits", lambda: _efla_limits(fn))):
+            try:
+                ok = call()
+            except Exception:  # noqa: BLE001  (a crash is a failed pin)
+                ok = False
+            if not ok:
+                fails.append(pin)
+        assert fails, f"planted mistake '{name}' passed every pin"
 
 
 def _gdn2_reduction(fn, gate):
