@@ -18,6 +18,8 @@ Contents
 ``gdn2_fwd``         the Gated DeltaNet-2 reading: separate per-key-channel erase
                      and per-value-channel write gates in place of beta (numpy
                      token loop, small cases).
+``gdn2_grads``       fp64 gradients of the Gated DeltaNet-2 loop (autograd), the
+                     reference for a gate-aware backward pass.
 ``chunkwise_ref``    an independent fp64 chunkwise reformulation that solves the
                      intra-chunk triangular system with a dense ``solve``; it is a
                      pin for the token loop, not a second oracle for the GPU.
@@ -163,4 +165,4 @@ def decode_step(q, k, v, beta, log_alpha=None, gate="scalar", state=None,
 from .chunkwise_ref import chunkwise_ref  # noqa: E402  (re-export)
 from .efla_ref import efla_fwd  # noqa: E402  (re-export)
 from .gdn2_ref import gdn2_fwd  # noqa: E402  (re-export)
-from .grad_ref import gdr_grads  # noqa: E402  (re-export)
+from .grad_ref import gdn2_grads, gdr_grads  # noqa: E402  (re-export)

@@ -8,6 +8,11 @@ Attention" topic page, FG^2-GDN card).  The loss is sum(out * d_out) +
 sum(final_state * d_final_state), so the returned gradients are the
 vector-Jacobian products the library's backward pass computes.  Small cases
 only (one autograd node per token operation).
+
+``gdn2_grads`` does the same for Gated DeltaNet-2's separate gates (the
+update of oracle/gdn2_ref.py: read key b_t . k_t, target w_t . v_t, no beta;
+Gated DeltaNet-2 abstract on the comparative-study page 2607.07953, which
+credits the model with a gate-aware backward pass).
 """
 from __future__ import annotations
 
@@ -15,7 +20,7 @@ import numpy as np
 import torch
 
 
-def _loop(q, k, v, beta, log_alpha, gate, s0, cu):
+def _loop(q, k, v, beta, log_alpha, gate, s0, cu, erase=None, write=None):
     H, dk = q.shape[-2], q.shape[-1]
     dv = v.shape[-1]
     outs = []
@@ -31,8 +36,12 @@ def _loop(q, k, v, beta, log_alpha, gate, s0, cu):
                 elif gate == "channel":
                     S = torch.exp(log_alpha[t, h])[:, None] * S
                 kt = k[t, h]
-                r = S.T @ kt
-                u = beta[t, h] * (v[t, h] - r)
+                if erase is None:
+                    r = S.T @ kt
+                    u = beta[t, h] * (v[t, h] - r)
+                else:
+                    r = S.T @ (erase[t, h] * kt)
+                    u = write[t, h] * v[t, h] - r
                 S = S + torch.outer(kt, u)
                 outs.append(((t, h), S.T @ q[t, h]))
             for_heads.append(S)
@@ -43,6 +52,23 @@ def _loop(q, k, v, beta, log_alpha, gate, s0, cu):
 def gdr_grads(q, k, v, beta, log_alpha=None, gate="scalar",
               initial_state=None, d_out=None, d_final_state=None,
               cu_seqlens=None):
+    return _grads(q, k, v, beta, None, None, log_alpha, gate, initial_state,
+                  d_out, d_final_state, cu_seqlens)
+
+
+def gdn2_grads(q, k, v, erase, write, log_alpha=None, gate="channel",
+               initial_state=None, d_out=None, d_final_state=None,
+               cu_seqlens=None):
+    """Gradients of sum(out * d_out) + sum(final * d_final_state) through the
+    Gated DeltaNet-2 loop.  erase has the layout of k, write that of v.
+    Returns dq, dk, dv, derase, dwrite, dlog_alpha, dinitial_state, out and
+    final_state (dbeta is None)."""
+    return _grads(q, k, v, None, erase, write, log_alpha, gate,
+                  initial_state, d_out, d_final_state, cu_seqlens)
+
+
+def _grads(q, k, v, beta, erase, write, log_alpha, gate, initial_state,
+           d_out, d_final_state, cu_seqlens):
     """Gradients of sum(out * d_out) + sum(final * d_final_state).
 
     Layouts as for ``oracle.gdr_fwd`` (fixed length [B, T, H, d] or varlen
@@ -59,10 +85,11 @@ def gdr_grads(q, k, v, beta, log_alpha=None, gate="scalar",
     flat = lambda a: None if a is None else a.reshape(  # noqa: E731
         (-1,) + tuple(a.shape[2:]))
     tq, tk, tv, tb = t64(q), t64(k), t64(v), t64(beta)
+    te, tw = t64(erase), t64(write)
     tla = t64(log_alpha) if gate != "none" else None
     ts0 = t64(initial_state)
     outs, final = _loop(flat(tq), flat(tk), flat(tv), flat(tb), flat(tla),
-                        gate, ts0, cu)
+                        gate, ts0, cu, flat(te), flat(tw))
     H, dv = np.shape(v)[2], np.shape(v)[3]
     out = torch.zeros(Bq * T, H, dv, dtype=torch.float64)
     loss = torch.zeros((), dtype=torch.float64)
@@ -75,12 +102,13 @@ def gdr_grads(q, k, v, beta, log_alpha=None, gate="scalar",
     if d_final_state is not None:
         loss = loss + (final * torch.tensor(
             np.asarray(d_final_state, np.float64))).sum()
-    leaves = [x for x in (tq, tk, tv, tb, tla, ts0) if x is not None]
+    leaves = [x for x in (tq, tk, tv, tb, te, tw, tla, ts0) if x is not None]
     grads = torch.autograd.grad(loss, leaves, allow_unused=True)
     gm = dict(zip([id(x) for x in leaves], grads))
     g = lambda x: None if x is None else (  # noqa: E731
         np.zeros(x.shape) if gm[id(x)] is None else gm[id(x)].numpy())
     return dict(dq=g(tq), dk=g(tk), dv=g(tv), dbeta=g(tb),
+                derase=g(te), dwrite=g(tw),
                 dlog_alpha=g(tla), dinitial_state=g(ts0),
                 out=out.reshape(np.shape(v)).numpy(),
                 final_state=final.detach().numpy())

@@ -629,6 +629,80 @@ def test_gradients_match_finite_differences(oracle_lib):
         np.testing.assert_allclose(g["final_state"], sT, atol=1e-13)
 
 
+def test_gdn2_gradients_match_finite_differences():
+    """The Gated DeltaNet-2 autograd gradients (oracle.gdn2_grads, a PyTorch
+    token loop) agree with central differences of the numpy loop's loss
+    (oracle.gdn2_fwd), element by element, for every input -- the erase and
+    write gates included -- and every gate kind."""
+    rng = np.random.default_rng(41)
+    for gate in ("none", "scalar", "channel"):
+        c = _rand_case(rng, B=1, T=5, H=1, dk=3, dv=2, gate=gate)
+        case = dict(q=c["q"], k=c["k"], v=c["v"],
+                    erase=rng.uniform(0.1, 0.9, size=(1, 5, 1, 3)),
+                    write=rng.uniform(0.1, 0.9, size=(1, 5, 1, 2)),
+                    log_alpha=c["log_alpha"], initial_state=c["initial_state"])
+        dO = rng.standard_normal(c["v"].shape)
+        dS = rng.standard_normal((1, 1, 3, 2))
+        g = oracle.gdn2_grads(**case, gate=gate, d_out=dO, d_final_state=dS)
+
+        def loss(x):
+            o, sT = oracle.gdn2_fwd(x["q"], x["k"], x["v"], x["erase"],
+                                    x["write"], x["log_alpha"], gate,
+                                    x["initial_state"])
+            return float((o * dO).sum() + (sT * dS).sum())
+
+        names = ["q", "k", "v", "erase", "write", "initial_state"]
+        if gate != "none":
+            names.append("log_alpha")
+        eps = 1e-6
+        for key in names:
+            x = case[key]
+            fd = np.zeros_like(x)
+            for i in np.ndindex(x.shape):
+                xp, xm = x.copy(), x.copy()
+                xp[i] += eps
+                xm[i] -= eps
+                fd[i] = (loss({**case, key: xp}) - loss({**case, key: xm})) / (
+                    2 * eps)
+            np.testing.assert_allclose(g["d" + key], fd, atol=2e-7, rtol=1e-6,
+                                       err_msg=f"{gate} {key}")
+        assert g["dbeta"] is None
+        o, sT = oracle.gdn2_fwd(case["q"], case["k"], case["v"],
+                                case["erase"], case["write"],
+                                case["log_alpha"], gate,
+                                case["initial_state"])
+        np.testing.assert_allclose(g["out"], o, atol=1e-13)
+        np.testing.assert_allclose(g["final_state"], sT, atol=1e-13)
+
+
+def test_gdn2_gradients_reduce_to_the_delta_rule():
+    """Both gates equal to beta_t on every channel: the Gated DeltaNet-2
+    gradients of q, k, v, log-alpha and the initial state are the delta
+    rule's, and the delta rule's d beta_t is the sum of the two gates'
+    gradients over their channels (chain rule through b = w = beta 1)."""
+    rng = np.random.default_rng(42)
+    for gate in ("none", "scalar", "channel"):
+        c = _rand_case(rng, B=2, T=6, H=2, dk=4, dv=3, gate=gate)
+        dO = rng.standard_normal(c["v"].shape)
+        dS = rng.standard_normal((2, 2, 4, 3))
+        g1 = oracle.gdr_grads(**c, d_out=dO, d_final_state=dS)
+        b = c["beta"]
+        g2 = oracle.gdn2_grads(c["q"], c["k"], c["v"],
+                               np.repeat(b[..., None], 4, axis=-1),
+                               np.repeat(b[..., None], 3, axis=-1),
+                               c["log_alpha"], gate, c["initial_state"],
+                               d_out=dO, d_final_state=dS)
+        for key in ("dq", "dk", "dv", "dlog_alpha", "dinitial_state"):
+            if g1[key] is None:
+                assert g2[key] is None
+            else:
+                np.testing.assert_allclose(g2[key], g1[key], atol=1e-12,
+                                           err_msg=f"{gate} {key}")
+        np.testing.assert_allclose(
+            g2["derase"].sum(-1) + g2["dwrite"].sum(-1), g1["dbeta"],
+            atol=1e-12, err_msg=gate)
+
+
 def test_thread_count_does_not_change_bits(oracle_lib):
     rng = np.random.default_rng(10)
     c = _rand_case(rng, B=3, T=15, H=5, dk=4, dv=4, gate="channel")
