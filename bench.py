@@ -188,6 +188,55 @@ def dist_env():
     return ws, rank, local
 
 
+def free_port():
+    """A free TCP port on 127.0.0.1 for the ranks' rendezvous."""
+    import socket
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        return sock.getsockname()[1]
+
+
+def relaunch_command(argv, n, port):
+    """This script as n ranks on one node (one process per GPU) under
+    torch.distributed.run, rendezvous on 127.0.0.1."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr", "127.0.0.1",
+            "--master-port", str(port), os.path.abspath(__file__), *argv]
+
+
+def launch_ranks(argv, n):
+    """Runs the benchmark as n ranks and returns the launcher's exit code.
+    A hard limit well above the ranks' own collective timeouts ends a run
+    whose ranks wait on one another for good."""
+    import subprocess
+    env = dict(os.environ)
+    env.setdefault("OMP_NUM_THREADS", "1")
+    cmd = ["timeout", "-k", "60", "1800",
+           *relaunch_command(argv, n, free_port())]
+    return subprocess.run(cmd, env=env).returncode
+
+
+def run_launch_check(args):
+    """The multi-rank plumbing without a GPU: every rank joins a gloo group,
+    the ranks' numbers go through the max-over-ranks reduction, and rank 0
+    prints one JSON line with the world size it saw."""
+    import torch.distributed as dist
+    from datetime import timedelta
+    ws, rank, _ = dist_env()
+    if ws > 1:
+        dist.init_process_group("gloo", timeout=timedelta(seconds=60))
+    ranks = max_over_ranks([float(r == rank) * (r + 1) for r in range(ws)],
+                           ws)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps({"launch_check": True, "n_gpus": ws,
+                          "ranks_seen": [int(x) - 1 for x in ranks]}),
+              flush=True)
+    return 0
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -872,6 +921,9 @@ def main(argv=None):
     ap.add_argument("--segments", type=int, default=0,
                     help="context-parallel forward (gdr_chunk_fwd_segmented) "
                          "with this many pieces per sequence")
+    ap.add_argument("--launch-check", action="store_true",
+                    help="check the multi-rank launcher on CPU (gloo ranks, "
+                         "no GPU work)")
     ap.add_argument("--gdn2", action="store_true",
                     help="with Gated DeltaNet-2 erase and write gates "
                          "(gdr_chunk_fwd_gdn2; with --decode, "
@@ -879,6 +931,19 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be >= 1")
+    # --gpus N runs N ranks, one per GPU: launched here unless a launcher
+    # (torch.distributed.run) already did, in which case the two must agree
+    if "WORLD_SIZE" not in os.environ:
+        if args.gpus > 1:
+            return launch_ranks(sys.argv[1:] if argv is None else list(argv),
+                                args.gpus)
+    elif int(os.environ["WORLD_SIZE"]) != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE="
+                         f"{os.environ['WORLD_SIZE']}")
+    if args.launch_check:
+        return run_launch_check(args)
     w = WORKLOADS[args.workload]
     if args.batch:
         if w.varlen_nseq or args.batch < 1:

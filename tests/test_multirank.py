@@ -89,3 +89,40 @@ def test_reference_arm_prints_one_json_line():
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _bench(*args, env_extra=None):
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"),
+                           *args], capture_output=True, text=True, env=env,
+                          timeout=300)
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    # run directly, --gpus 2 re-executes bench.py as two ranks (one per
+    # GPU) under torch.distributed.run; the launch check does the rank
+    # plumbing over gloo without a GPU and rank 0 alone prints
+    r = _bench("--gpus", "2", "--launch-check")
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    import json
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["ranks_seen"] == [0, 1]
+
+
+def test_gpus_flag_must_match_the_launchers_world_size():
+    r = _bench("--gpus", "2", "--launch-check",
+               env_extra={"WORLD_SIZE": "3", "RANK": "0", "LOCAL_RANK": "0"})
+    assert r.returncode != 0
+    assert "WORLD_SIZE=3" in (r.stderr + r.stdout)
+
+
+def test_relaunch_command_is_one_node_on_loopback():
+    cmd = bench.relaunch_command(["--gpus", "4", "--steps", "3"], 4, 29500)
+    assert cmd[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"]
+    assert "--nproc-per-node=4" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-3:] == ["--gpus", "4", "--steps", "3"][-3:]
