@@ -79,18 +79,67 @@ def kernel_source_hash(algo):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel_file, src_hash):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", kernel_file)
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
+# the kernel whose DRAM traffic the roofline line reports, per path
+TRAFFIC_KERNEL = {"fused_tc": "gdr_fused_tc_kernel",
+                  "decode": "decode"}
+
+
+def recorded_traffic(key, src_hash, path=TRAFFIC_JSON):
+    """DRAM bytes per launch recorded for `key` ("<algo>:<workload>") from
+    an ncu capture, if it was taken on the current kernel source (else
+    None)."""
     if not os.path.exists(path):
         return None
-    text = open(path).read()
-    m_h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
-    m_t = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_h or not m_t or m_h.group(1) != src_hash:
+    rec = json.load(open(path)).get(key)
+    if not rec or rec.get("source_sha256_16") != src_hash:
         return None
-    return float(m_t.group(1))
+    return float(rec["dram_bytes_per_launch"])
+
+
+_BYTE_UNITS = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9,
+               "Tbyte": 1e12, "KB": 1e3, "MB": 1e6, "GB": 1e9}
+
+
+def traffic_from_ncu_csv(csv_path, kernel_regex):
+    """Mean DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per
+    captured launch of the kernels matching `kernel_regex`, from the output
+    of `ncu --csv --metrics dram__bytes_read.sum,dram__bytes_write.sum`;
+    and the number of launches."""
+    import csv
+    rows = list(csv.reader(l for l in open(csv_path) if l.startswith('"')))
+    hdr = rows[0]
+    per_launch = {}
+    for r in rows[1:]:
+        d = dict(zip(hdr, r))
+        if not re.search(kernel_regex, d.get("Kernel Name", "")):
+            continue
+        if d.get("Metric Name") not in ("dram__bytes_read.sum",
+                                        "dram__bytes_write.sum"):
+            continue
+        val = float(d["Metric Value"].replace(",", ""))
+        val *= _BYTE_UNITS.get(d.get("Metric Unit", "byte"), 1.0)
+        per_launch[d["ID"]] = per_launch.get(d["ID"], 0.0) + val
+    if not per_launch:
+        raise SystemExit(f"no dram__bytes rows for /{kernel_regex}/ in "
+                         f"{csv_path}")
+    return sum(per_launch.values()) / len(per_launch), len(per_launch)
+
+
+def record_traffic(csv_path, algo, workload, command, path=TRAFFIC_JSON):
+    """Writes the traffic of `algo` on `workload` from an ncu capture into
+    the committed record, with the hash of the kernel source it was taken
+    on (bench.py reports it only while that source is unchanged)."""
+    by, n = traffic_from_ncu_csv(csv_path, TRAFFIC_KERNEL[algo])
+    recs = json.load(open(path)) if os.path.exists(path) else {}
+    recs[f"{algo}:{workload}"] = {
+        "kernel": TRAFFIC_KERNEL[algo],
+        "source_sha256_16": kernel_source_hash(algo),
+        "dram_bytes_per_launch": by, "launches": n, "command": command}
+    with open(path, "w") as f:
+        json.dump(recs, f, indent=1, sort_keys=True)
+        f.write("\n")
+    return by
 
 
 class ClockSampler:
@@ -264,11 +313,14 @@ def oracle_sample(inp, nseq_sample):
     return f, tokens
 
 
-def time_oracle(inp, nseq_sample):
+def time_oracle(inp, nseq_sample, nthreads=0):
+    """The oracle on the first `nseq_sample` sequences (all heads), on
+    `nthreads` host threads (0: all cores): tokens/s, threads, seconds,
+    tokens."""
     import oracle
     f, tokens = oracle_sample(inp, nseq_sample)
     t0 = time.perf_counter()
-    _, _, threads = oracle.gdr_fwd(**f)
+    _, _, threads = oracle.gdr_fwd(**f, nthreads=nthreads)
     dt = time.perf_counter() - t0
     return tokens / dt, threads, dt, tokens
 
@@ -318,6 +370,25 @@ def run_reference(args, w):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def sampled_parity(inp, out, final_state, head=3):
+    """The timed result against the fp64 oracle on one head of every
+    sequence (the chains are independent, so a head is an exact
+    sub-problem): max|gpu - oracle| / RMS(oracle) for out (less half an ulp
+    of its storage dtype) and for the final state, beside the bar."""
+    import oracle
+    from chunkwise_recurrence_b200.inputs import head_slice, out_err, rel_err
+    w = inp.w
+    h = min(head, w.H - 1)
+    ro, rs, _ = oracle.gdr_fwd(**head_slice(inp, [h]).f64())
+    o = out.float().cpu().numpy()[:, :, [h]]
+    st = final_state.cpu().numpy()[:, [h]]
+    return {"head": h, "out_err": out_err(o, ro, w.dtype),
+            "state_err": rel_err(st, rs),
+            "bar": 1e-4 if w.dtype == "fp32" else 2e-2,
+            "metric": "max |gpu - fp64 oracle| / RMS(oracle), all sequences "
+                      "of one head; out less half an ulp of its dtype"}
 
 
 def launches_per_step(algo_used, w, segments=0):
@@ -459,7 +530,7 @@ def run_ours(args, w):
     kernel_ms = statistics.mean(per_step)
     achieved_gbs = by / (kernel_ms / 1e3) / 1e9
     src_hash = kernel_source_hash(algo_used)
-    traffic = recorded_traffic(f"{algo_used}_{w.name}.md", src_hash)
+    traffic = recorded_traffic(f"{algo_used}:{w.name}", src_hash)
     roofline = {
         "bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
         "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
@@ -496,14 +567,21 @@ def run_ours(args, w):
         args.steps,
         "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
     }
+    if rank == 0:
+        line["parity"] = sampled_parity(inp, out, sT)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         nsample = max(1, min(args.cpu_seqs, len(inp.lengths)))
         val, threads, dt, tok = time_oracle(inp, nsample)
+        v1, _, dt1, tok1 = time_oracle(inp, 1, nthreads=1)
         line["cpu_baseline"] = {
             "value": val, "unit": "tokens/s", "cores": threads,
             "kind": "oracle",
             "sample": (f"sequences 0..{nsample - 1} of {len(inp.lengths)} "
-                       f"({tok} tokens x {w.H} heads), {dt:.1f} s wall")}
+                       f"({tok} tokens x {w.H} heads), {dt:.1f} s wall"),
+            "single_core": {
+                "value": v1, "unit": "tokens/s", "cores": 1,
+                "sample": (f"sequence 0 of {len(inp.lengths)} ({tok1} tokens "
+                           f"x {w.H} heads), {dt1:.1f} s wall")}}
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -625,7 +703,7 @@ def run_decode(args):
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                      "traffic": recorded_traffic(
-                         f"decode_{w.name}.md", kernel_source_hash("decode")),
+                         f"decode:{w.name}", kernel_source_hash("decode")),
                      "peak_source": peak_src,
                      "kernel": "gdr_decode_kernel",
                      "algorithmic_bytes_per_launch": by},
@@ -921,6 +999,12 @@ def main(argv=None):
     ap.add_argument("--segments", type=int, default=0,
                     help="context-parallel forward (gdr_chunk_fwd_segmented) "
                          "with this many pieces per sequence")
+    ap.add_argument("--record-traffic", metavar="NCU_CSV",
+                    help="record the DRAM traffic of --algo (fused_tc or "
+                         "decode) on --workload from an ncu --csv capture "
+                         "into profiles/traffic.json, and exit")
+    ap.add_argument("--capture-command", default="",
+                    help="with --record-traffic: the command that made it")
     ap.add_argument("--launch-check", action="store_true",
                     help="check the multi-rank launcher on CPU (gloo ranks, "
                          "no GPU work)")
@@ -933,6 +1017,17 @@ def main(argv=None):
         raise SystemExit("--warmup must be >= 3")
     if args.gpus < 1:
         raise SystemExit("--gpus must be >= 1")
+    if args.record_traffic:
+        algo = "decode" if args.decode else args.algo
+        if algo not in TRAFFIC_KERNEL:
+            raise SystemExit("--record-traffic takes --algo fused_tc or "
+                             "--decode")
+        wname = "gdn_decode_h16_d128_bf16" if args.decode else args.workload
+        by = record_traffic(args.record_traffic, algo, wname,
+                            args.capture_command)
+        print(json.dumps({"recorded": f"{algo}:{wname}",
+                          "dram_bytes_per_launch": by}))
+        return 0
     # --gpus N runs N ranks, one per GPU: launched here unless a launcher
     # (torch.distributed.run) already did, in which case the two must agree
     if "WORLD_SIZE" not in os.environ:

@@ -9,7 +9,6 @@ written once, plus the fp32 states; and the six dense tile products per
 token-head (K K^T, T K and Q K^T at 2 C dk flops each, T V and the masked
 (Q K^T) V_new at 2 C dv, and W S, K^T V_new and Q S at 2 dk dv)."""
 import os
-import re
 import sys
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -66,15 +65,50 @@ def test_launches_per_step():
     assert bench.launches_per_step("fused_tc", w, segments=4) == 5
 
 
-def test_recorded_traffic_follows_the_source_hash():
-    for name, algo in (("fused_tc_gdn_b8_h16_t4096_d128_bf16.md", "fused_tc"),
-                       ("decode_gdn_decode_h16_d128_bf16.md", "decode"),
-                       ("staged_gdn_b8_h16_t4096_d128_bf16.md", "staged")):
-        text = open(os.path.join(ROOT, "profiles", name)).read()
-        h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text).group(1)
-        t = float(re.search(r"dram_bytes_per_launch:\s*([0-9.]+)",
-                            text).group(1))
-        assert bench.recorded_traffic(name, h) == t
-        assert bench.recorded_traffic(name, "0" * 16) is None
-        assert len(bench.kernel_source_hash(algo)) == 16
-    assert bench.recorded_traffic("no_such_profile.md", "0" * 16) is None
+def _ncu_csv(path, rows):
+    hdr = ['"ID"', '"Kernel Name"', '"Metric Name"', '"Metric Unit"',
+           '"Metric Value"']
+    with open(path, "w") as f:
+        f.write("==PROF== a line ncu prints that is not data\n")
+        f.write(",".join(hdr) + "\n")
+        for r in rows:
+            f.write(",".join(f'"{x}"' for x in r) + "\n")
+
+
+def test_traffic_from_an_ncu_capture(tmp_path):
+    # two captured launches of the kernel (units as ncu prints them) and a
+    # launch of another kernel that must not count
+    p = tmp_path / "cap.csv"
+    _ncu_csv(p, [
+        ("0", "void gdr::gdr_fused_tc_kernel<1>(...)", "dram__bytes_read.sum",
+         "Mbyte", "400.5"),
+        ("0", "void gdr::gdr_fused_tc_kernel<1>(...)", "dram__bytes_write.sum",
+         "byte", "1,000"),
+        ("1", "void gdr::gdr_fused_tc_kernel<1>(...)", "dram__bytes_read.sum",
+         "Mbyte", "399.5"),
+        ("1", "void gdr::gdr_fused_tc_kernel<1>(...)", "dram__bytes_write.sum",
+         "Kbyte", "3"),
+        ("2", "fill_kernel", "dram__bytes_read.sum", "Gbyte", "9"),
+    ])
+    by, n = bench.traffic_from_ncu_csv(str(p), "gdr_fused_tc_kernel")
+    assert n == 2
+    assert by == (400.5e6 + 1000 + 399.5e6 + 3e3) / 2
+
+
+def test_recorded_traffic_follows_the_source_hash(tmp_path):
+    p = tmp_path / "cap.csv"
+    _ncu_csv(p, [("0", "gdr_fused_tc_kernel", "dram__bytes_read.sum", "byte",
+                  "100"),
+                 ("0", "gdr_fused_tc_kernel", "dram__bytes_write.sum", "byte",
+                  "20")])
+    rec = tmp_path / "traffic.json"
+    assert bench.record_traffic(str(p), "fused_tc", "w", "ncu ...",
+                                path=str(rec)) == 120.0
+    h = bench.kernel_source_hash("fused_tc")
+    assert len(h) == 16
+    assert bench.recorded_traffic("fused_tc:w", h, path=str(rec)) == 120.0
+    # a record taken on other source is not reported
+    assert bench.recorded_traffic("fused_tc:w", "0" * 16, path=str(rec)) is None
+    assert bench.recorded_traffic("fused_tc:other", h, path=str(rec)) is None
+    assert bench.recorded_traffic("fused_tc:w", h,
+                                  path=str(tmp_path / "none.json")) is None
