@@ -254,12 +254,16 @@ def chunk_fwd_noalloc(q, k, v, beta, log_alpha=None, initial_state=None, *,
                  nseq if cu_seqlens is not None else 0, ALGOS[algo])
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    rc = lib.gdr_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v),
-                                   _ptr(log_alpha), _ptr(beta),
-                                   _ptr(initial_state), _ptr(out),
-                                   _ptr(final_state), B, T, H, dk, dv, chunk,
-                                   ctypes.c_void_p(stream.cuda_stream),
-                                   ctypes.byref(opts))
+    # the library finds its scratch array through the current device, which
+    # must be the device of the stream and the tensors
+    with torch.cuda.device(q.device):
+        rc = lib.gdr_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(log_alpha), _ptr(beta),
+                                       _ptr(initial_state), _ptr(out),
+                                       _ptr(final_state), B, T, H, dk, dv,
+                                       chunk,
+                                       ctypes.c_void_p(stream.cuda_stream),
+                                       ctypes.byref(opts))
     if rc != 0:
         raise GdrError(rc, "gdr_chunk_fwd_noalloc")
     return out, final_state

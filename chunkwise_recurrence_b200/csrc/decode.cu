@@ -168,6 +168,16 @@ __global__ void __launch_bounds__(kDecThreads)
         break;
       }
     }
+    // After an expired wait the tile is not used, but the CTA stays until
+    // the copy it issued has landed (a second bounded wait), so that a late
+    // copy never writes into shared memory another CTA has since been
+    // given.  (An injected expiry issued no copy.)  A copy still in flight
+    // after that leaves the context suspect: see GDR_ERR_TIMEOUT.
+    if (!copy_ok && !p.inject_timeout) {
+      const long long t1 = clock64();
+      while (!mbar_try_wait(&bar, 0) && clock64() - t1 < 4 * p.wait_cycles) {
+      }
+    }
   }
   __syncthreads();
   if (!copy_ok) return;   // uniform: the tile never arrived

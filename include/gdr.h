@@ -275,7 +275,9 @@ GDR_API gdr_status gdr_chunk_fwd_segmented(
  *  - the current device must be the device of `stream`.  The first call on
  *    each device looks up that device's address of the array
  *    (cudaGetSymbolAddress, once per device, cached); make that first call
- *    before any stream capture;
+ *    before any stream capture.  The cached address is not looked up again:
+ *    after a cudaDeviceReset in the calling process this entry point must
+ *    not be used on that device again;
  *  - every call on a device shares the one array, which keeps the last call's
  *    contents (nothing in it needs to start at zero: every scratch word is
  *    written before it is read).  Calls whose execution overlaps on the GPU
@@ -326,7 +328,13 @@ GDR_API gdr_status gdr_chunk_fwd_noalloc(const void *q, const void *k,
  * for its state tile is bounded (an expired wait is reported by
  * gdr_device_error as GDR_ERR_TIMEOUT; the environment variable
  * GDR_FAULT_INJECT_DECODE_TIMEOUT=1 makes every wait expire, for tests of that
- * path: the step is then skipped and state_out is not written).  Returns GDR_ERR_INVALID_ARGUMENT /
+ * path: the step is then skipped and state_out is not written).  After a
+ * wait that expires on its own (not injected) the CTA skips its work but
+ * stays, under a second bounded wait, until the copy it issued has landed,
+ * so that no late copy writes into shared memory another CTA has since been
+ * given; such a GDR_ERR_TIMEOUT means the device is not answering as it
+ * should, and the caller should treat the CUDA context as suspect (finish
+ * and restart rather than continue).  Returns GDR_ERR_INVALID_ARGUMENT /
  * GDR_ERR_UNSUPPORTED as described, GDR_ERR_CUDA if the launch fails.
  */
 GDR_API gdr_status gdr_decode_step(const void *q, const void *k, const void *v,
