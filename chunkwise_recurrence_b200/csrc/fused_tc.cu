@@ -932,8 +932,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int w8 = 1; w8 < 8; ++w8) b = fmaxf(b, wm[w8]);
           use16 = b <= kF16Range;   // same decision in every prep thread
-          if (pt == 0)
+          if (pt == 0) {
             reinterpret_cast<int *>(sm + Lay::TT_F16)[m & 1] = use16 ? 1 : 0;
+            // beyond the fp16 window the rescaled operands fall back to
+            // bf16, whose 8-bit significand does not keep the result within
+            // the accuracy of the fp16 path: the call says so
+            if (!use16) atomicOr(&g_fused_error, kErrRange);
+          }
         }
         // (b) with g_m = g at row 31 (the first half's total): row r's
         // g_r - g_m is its running sum minus g_m in the first half, and its

@@ -96,16 +96,18 @@ typedef enum {
    * tcgen05 tensor cores: fp16 operands (inputs converted on chip), fp32
    * accumulation in tensor memory, fp32 state.  bf16 I/O, dk = dv = 128,
    * chunk = 64.  Inputs and on-chip intermediates must lie within fp16
-   * range (|x| <= 65504); for the channel gate, each key channel's
-   * log-decay must move by at most ~88 between a chunk's row 31 and its
-   * first or last row.  A violation shows as a non-finite output or state
-   * and is reported by gdr_device_error as GDR_ERR_RANGE.  Accuracy: the
-   * scalar and no gate stay within about 5e-3 of the output RMS at any
-   * decay; for the channel gate the decay sits inside the contraction, on
-   * rescaled operands that are fp16 where a chunk's decay allows (about 3e-3
-   * at mean log-decays down to -0.1 per token and channel) and bf16 beyond
-   * (up to about 3e-2 at -1 to -2).  Where that matters, GDR_ALGO_STAGED is
-   * fp32 throughout. */
+   * range (|x| <= 65504); a violation shows as a non-finite output or
+   * state and is reported by gdr_device_error as GDR_ERR_RANGE.  Accuracy:
+   * the scalar and no gate stay within about 5e-3 of the output RMS at any
+   * decay.  For the channel gate the decay sits inside the contraction, on
+   * operands rescaled by e^{+-(g - g_m)} (g_m: the log-decay at a chunk's
+   * row 31), which are fp16 while every key channel's log-decay moves by at
+   * most 9 between row 31 and the chunk's first or last row (about 3e-3 of
+   * the output RMS; the KDA workload's decays stay well inside).  A chunk
+   * beyond that window is computed on bf16 operands instead, which are less
+   * accurate (up to about 3e-2 at mean log-decays of -1 to -2 per token and
+   * channel), and the call reports GDR_ERR_RANGE through gdr_device_error:
+   * run such inputs with GDR_ALGO_STAGED, fp32 throughout. */
   GDR_ALGO_FUSED_TC = 2
 } gdr_algo;
 

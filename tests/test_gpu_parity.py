@@ -337,12 +337,24 @@ def test_strong_decays_scalar_gate(decay):
 
 # Channel gate, fused path: the per-channel decay sits inside the contraction,
 # so K K^T, Q K^T and U, W read operands rescaled by e^{+-(g - g_m)}: fp16
-# where the chunk's decay range allows (about 3e-3 of the RMS at the KDA
-# workload's decays), bf16 beyond (whose 8-bit significand gives up to about
-# 3e-2 at mean log-decays of -1 to -2 per token and channel).  This is the
-# documented envelope of the fused channel-gate path; the fp32 staged path
-# meets the bar at any decay.
-KDA_FUSED_STRONG_DECAY_BOUND = 5e-2
+# while a chunk's decay stays within the fp16 window (about 3e-3 of the RMS at
+# the KDA workload's decays); a chunk beyond it is computed on bf16 operands
+# and the call reports GDR_ERR_RANGE.  So every fused result either meets the
+# bar or is reported; the fp32 staged path meets the bar at any decay.
+def fused_meets_bar_or_reports(inp):
+    w = inp.w
+    o, s = gdr.chunk_fwd(_dev(inp.q), _dev(inp.k), _dev(inp.v),
+                         _dev(inp.beta), _dev(inp.log_alpha), _dev(inp.s0),
+                         chunk=w.chunk, gate=w.gate, algo="fused_tc")
+    err = gdr.device_error(clear=True)
+    assert err in (0, 6)                       # OK or GDR_ERR_RANGE
+    if err == 0:
+        ro, rs = run_oracle(inp)
+        o, s = o.float().cpu().numpy(), s.cpu().numpy()
+        assert np.isfinite(o).all() and np.isfinite(s).all()
+        assert out_err(o, ro, w.dtype) <= TOL[w.dtype]
+        assert rel_err(s, rs) <= TOL[w.dtype]
+    return err
 
 
 @pytest.mark.parametrize("decay", [1.0, 2.0])
@@ -352,32 +364,19 @@ def test_strong_decays_channel_gate(decay):
     inp = generate(w, seed=31)
     check(inp, "staged")
     if "fused_tc" in algos_for(w):
-        o, s = run_gpu(inp, "fused_tc")
-        ro, rs = run_oracle(inp)
-        assert np.isfinite(o).all() and np.isfinite(s).all()
-        assert out_err(o, ro, "bf16") <= KDA_FUSED_STRONG_DECAY_BOUND
-        assert rel_err(s, rs) <= KDA_FUSED_STRONG_DECAY_BOUND
+        fused_meets_bar_or_reports(inp)
 
 
-def test_channel_gate_extreme_decays_are_bounded_or_reported():
-    """Log-decays of about -4 per token and channel overflow the fused
-    kernel's bf16 factors e^{g - g_m} (g - g_m beyond 88 inside a chunk).
-    The call must then report GDR_ERR_RANGE; a result it does not report
-    must be within the channel gate's fused envelope."""
+def test_channel_gate_reports_decays_beyond_its_window():
+    """Log-decays of about -4 per token and channel: every chunk leaves the
+    fused channel gate's fp16 window, so the call must report GDR_ERR_RANGE;
+    at the KDA workload's own decays it reports nothing and meets the bar."""
     w = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(
         B=1, T=2 * 64 + 9, H=2, decay_lo=5.0, decay_hi=5.0)
     if "fused_tc" not in algos_for(w):
         pytest.skip("fused path not built")
     inp = generate(w, seed=32)
-    o, s = gdr.chunk_fwd(_dev(inp.q), _dev(inp.k), _dev(inp.v),
-                         _dev(inp.beta), _dev(inp.log_alpha), _dev(inp.s0),
-                         chunk=w.chunk, gate=w.gate, algo="fused_tc")
-    err = gdr.device_error(clear=True)
-    assert err in (0, 6)                       # OK or GDR_ERR_RANGE
-    if err == 0:
-        ro, rs = run_oracle(inp)
-        o, s = o.float().cpu().numpy(), s.cpu().numpy()
-        assert out_err(o, ro, w.dtype) <= KDA_FUSED_STRONG_DECAY_BOUND
-        assert rel_err(s, rs) <= KDA_FUSED_STRONG_DECAY_BOUND
-    # the staged path handles any decay in fp32
-    check(inp, "staged")
+    assert fused_meets_bar_or_reports(inp) == 6
+    check(inp, "staged")                       # any decay in fp32
+    w = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(B=1, T=2 * 64 + 9, H=2)
+    assert fused_meets_bar_or_reports(generate(w, seed=32)) == 0
