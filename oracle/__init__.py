@@ -166,3 +166,4 @@ from .chunkwise_ref import chunkwise_ref  # noqa: E402  (re-export)
 from .efla_ref import efla_fwd  # noqa: E402  (re-export)
 from .gdn2_ref import gdn2_fwd  # noqa: E402  (re-export)
 from .grad_ref import gdn2_grads, gdr_grads  # noqa: E402  (re-export)
+from .fg2_ref import fg2_fwd  # noqa: E402  (re-export)

@@ -593,6 +593,198 @@ def test_gdn2_pins_catch_planted_mistakes(oracle_lib):
             f"planted mistake '{name}' passed every pin")
 
 
+def _fg2_case(rng, B=1, T=7, H=1, dk=3, dv=4, gate="channel"):
+    c = _rand_case(rng, B=B, T=T, H=H, dk=dk, dv=dv, gate=gate)
+    c["beta_k"] = rng.uniform(0.05, 1.0, size=(B, T, H, dk))
+    c["beta_v"] = rng.uniform(0.1, 1.5, size=(B, T, H, dv))
+    return c
+
+
+def _fg2_reduction(fn, gate):
+    """A key-side rate equal to beta_t on every channel (no value scaling,
+    or a value scaling of ones) gives the delta rule: the loop matches the
+    C oracle."""
+    rng = np.random.default_rng(41)
+    c = _rand_case(rng, B=2, T=13, H=2, dk=4, dv=3, gate=gate)
+    o, s, _ = gdr_fwd(**c)
+    bk = np.repeat(c["beta"][..., None], 4, axis=-1)
+    ok = True
+    for bv in (None, np.ones_like(c["v"])):
+        fo, fs = fn(c["q"], c["k"], c["v"], bk, bv, c["log_alpha"], gate,
+                    c["initial_state"])
+        ok &= np.allclose(fo, o, atol=1e-13) and np.allclose(fs, s, atol=1e-13)
+    return ok
+
+
+def _fd_grad(loss, S, h=1e-3):
+    """Central differences of loss at S, entry by entry (exact up to rounding
+    for a quadratic loss)."""
+    G = np.zeros_like(S)
+    for idx in np.ndindex(*S.shape):
+        E = np.zeros_like(S)
+        E[idx] = h
+        G[idx] = (loss(S + E) - loss(S - E)) / (2 * h)
+    return G
+
+
+def _fg2_gradient_step(fn, value_scale=True):
+    """Token by token, the state is the decayed state minus diag(beta_k)
+    times the gradient of L(S) = 1/2 ||S^T k - c . v||^2, the gradient taken
+    by central differences of L around the decayed state; the output reads
+    the state after the token's write."""
+    rng = np.random.default_rng(42)
+    T, dk, dv = 6, 3, 4
+    c = _fg2_case(rng, T=T, dk=dk, dv=dv, gate="channel")
+    bv = c["beta_v"] if value_scale else None
+    fo, fs = fn(c["q"], c["k"], c["v"], c["beta_k"], bv, c["log_alpha"],
+                "channel", c["initial_state"])
+    S = c["initial_state"][0, 0].copy()
+    ok = True
+    for t in range(T):
+        S = np.exp(c["log_alpha"][0, t, 0])[:, None] * S
+        k = c["k"][0, t, 0]
+        tgt = (bv[0, t, 0] if value_scale else 1.0) * c["v"][0, t, 0]
+        G = _fd_grad(lambda X: 0.5 * np.sum((X.T @ k - tgt) ** 2), S)
+        S = S - c["beta_k"][0, t, 0][:, None] * G
+        ok &= np.allclose(fo[0, t, 0], S.T @ c["q"][0, t, 0], atol=1e-8)
+    return ok and np.allclose(fs[0, 0], S, atol=1e-8)
+
+
+def _fg2_one_hot(fn):
+    """With k_t = e_c only row c of the state changes, and it moves a
+    fraction beta_k[c] of the way to the scaled target:
+    S_c <- (1 - beta_k[c]) a_t[c] S_c + beta_k[c] (c_t . v_t)."""
+    rng = np.random.default_rng(43)
+    T, dk, dv = 10, 3, 4
+    cs = rng.integers(0, dk, size=T)
+    k = np.zeros((1, T, 1, dk))
+    k[0, np.arange(T), 0, cs] = 1.0
+    q = rng.standard_normal((1, T, 1, dk))
+    v = rng.standard_normal((1, T, 1, dv))
+    bk = rng.uniform(0, 1, size=(1, T, 1, dk))
+    bv = rng.uniform(0, 2, size=(1, T, 1, dv))
+    la = -rng.uniform(0.05, 0.5, size=(1, T, 1, dk))
+    S0 = rng.standard_normal((1, 1, dk, dv))
+    fo, fs = fn(q, k, v, bk, bv, la, "channel", S0)
+    S = S0[0, 0].copy()
+    ok = True
+    for t in range(T):
+        S = np.exp(la[0, t, 0])[:, None] * S
+        r = cs[t]
+        S[r] = (1 - bk[0, t, 0, r]) * S[r] + bk[0, t, 0, r] * bv[0, t, 0] * v[0, t, 0]
+        ok &= np.allclose(fo[0, t, 0], S.T @ q[0, t, 0], atol=1e-13)
+    return ok and np.allclose(fs[0, 0], S, atol=1e-13)
+
+
+def _fg2_scalar_gate(fn):
+    """The scalar decay alpha_t scales the whole state: it equals the channel
+    gate with the same log-decay on every channel."""
+    rng = np.random.default_rng(44)
+    c = _fg2_case(rng, B=2, T=9, H=2, dk=3, dv=2, gate="scalar")
+    la_c = np.repeat(c["log_alpha"][..., None], 3, axis=-1)
+    a = fn(c["q"], c["k"], c["v"], c["beta_k"], c["beta_v"], c["log_alpha"],
+           "scalar", c["initial_state"])
+    b = fn(c["q"], c["k"], c["v"], c["beta_k"], c["beta_v"], la_c,
+           "channel", c["initial_state"])
+    return all(np.allclose(x, y, atol=1e-13) for x, y in zip(a, b))
+
+
+def _fg2_battery(fn):
+    """Names of the FG^2-GDN pins that `fn` fails (an exception counts as a
+    failure)."""
+    pins = {f"reduction_{g}": (lambda g=g: _fg2_reduction(fn, g))
+            for g in ("none", "scalar", "channel")}
+    pins["gradient_step"] = lambda: _fg2_gradient_step(fn)
+    pins["gradient_step_no_value_scale"] = (
+        lambda: _fg2_gradient_step(fn, value_scale=False))
+    pins["one_hot"] = lambda: _fg2_one_hot(fn)
+    pins["scalar_gate"] = lambda: _fg2_scalar_gate(fn)
+    fails = []
+    for name, pin in pins.items():
+        try:
+            ok = pin()
+        except Exception:  # noqa: BLE001  (a crash is a failed pin)
+            ok = False
+        if not ok:
+            fails.append(name)
+    return fails
+
+
+@pytest.mark.parametrize("gate", ["none", "scalar", "channel"])
+def test_fg2_reduces_to_the_delta_rule(oracle_lib, gate):
+    assert _fg2_reduction(oracle.fg2_fwd, gate)
+
+
+@pytest.mark.parametrize("value_scale", [False, True])
+def test_fg2_is_a_per_key_channel_gradient_step(value_scale):
+    assert _fg2_gradient_step(oracle.fg2_fwd, value_scale)
+
+
+def test_fg2_one_hot_keys_move_one_row_toward_the_target():
+    assert _fg2_one_hot(oracle.fg2_fwd)
+
+
+def test_fg2_packed_sequences_equal_separate_calls():
+    rng = np.random.default_rng(45)
+    lens = [5, 1, 8]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    c = _fg2_case(rng, B=1, T=int(cu[-1]), H=2, dk=3, dv=2)
+    S0 = rng.standard_normal((3, 2, 3, 2))
+    po, ps = oracle.fg2_fwd(c["q"], c["k"], c["v"], c["beta_k"], c["beta_v"],
+                            c["log_alpha"], "channel", S0, cu_seqlens=cu)
+    for n in range(3):
+        sl = slice(int(cu[n]), int(cu[n + 1]))
+        o, s = oracle.fg2_fwd(c["q"][:, sl], c["k"][:, sl], c["v"][:, sl],
+                              c["beta_k"][:, sl], c["beta_v"][:, sl],
+                              c["log_alpha"][:, sl], "channel", S0[n:n + 1])
+        assert np.array_equal(po[:, sl], o) and np.array_equal(ps[n], s[0])
+
+
+# plausible mistakes in the FG^2-GDN token loop, as (text, mutant)
+_FG2_U = "u = bv[b, t, h] * v[b, t, h] - S.T @ k[b, t, h]"
+_FG2_W = "S = S + np.outer(bk[b, t, h] * k[b, t, h], u)"
+FG2_MUTANTS = {
+    "key_rate_dropped": (_FG2_W, "S = S + np.outer(k[b, t, h], u)"),
+    "key_rate_on_the_read_key_too": (
+        _FG2_U, "u = bv[b, t, h] * v[b, t, h] - S.T @ (bk[b, t, h] * k[b, t, h])"),
+    "key_rate_on_the_read_key_only": (
+        _FG2_U + "\n                " + _FG2_W,
+        "u = bv[b, t, h] * v[b, t, h] - S.T @ (bk[b, t, h] * k[b, t, h])"
+        "\n                S = S + np.outer(k[b, t, h], u)"),
+    "value_scale_dropped": (_FG2_U, "u = v[b, t, h] - S.T @ k[b, t, h]"),
+    "value_scale_on_the_residual": (
+        _FG2_U, "u = bv[b, t, h] * (v[b, t, h] - S.T @ k[b, t, h])"),
+    "residual_sign": (_FG2_U, "u = bv[b, t, h] * v[b, t, h] + S.T @ k[b, t, h]"),
+    "scalar_decay_sign": (
+        "S = np.exp(la[b, t, h]) * S", "S = np.exp(-la[b, t, h]) * S"),
+    "channel_decay_dropped": (
+        "S = np.exp(la[b, t, h])[:, None] * S", "S = S"),
+    "channel_decay_on_value_channels": (
+        "S = np.exp(la[b, t, h])[:, None] * S",
+        "S = S * np.exp(la[b, t, h])[:S.shape[1]][None, :]"),
+    "read_before_write": (
+        "out[b, t, h] = S.T @ q[b, t, h]",
+        "out[b, t, h] = (S - np.outer(bk[b, t, h] * k[b, t, h], u)).T @ q[b, t, h]"),
+    "initial_state_ignored": (
+        "else np.array(initial_state[n, h], np.float64))",
+        "else np.zeros((dk, dv)))"),
+}
+
+
+def test_fg2_pins_catch_planted_mistakes(oracle_lib):
+    """Each plausible mistake, planted in a copy of the FG^2-GDN loop, fails
+    at least one of its pins; the loop as written fails none."""
+    assert _fg2_battery(oracle.fg2_fwd) == []
+    src = open(os.path.join(os.path.dirname(oracle.__file__),
+                            "fg2_ref.py")).read()
+    for name, (text, mutant) in FG2_MUTANTS.items():
+        assert src.count(text) == 1, name
+        ns = {"__name__": f"fg2_mutant_{name}"}
+        exec(compile(src.replace(text, mutant), name, "exec"), ns)
+        assert _fg2_battery(ns["fg2_fwd"]), (
+            f"planted mistake '{name}' passed every pin")
+
+
 def test_gradients_match_finite_differences(oracle_lib):
     """The autograd gradients (oracle.gdr_grads, on a PyTorch token loop) agree
     with central differences of the C token loop's loss, element by element,
