@@ -3,7 +3,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--algo auto|staged|fused_tc]
                     [--batch B] [--segments S] [--decode] [--backward]
-                    [--gdn2]
+                    [--gdn2 | --fg2]
 
 One step = one gdr_chunk_fwd call over one batch of the workload (all four
 stages: log-decay cumsum, WY/UT transform, state passing, output), inputs
@@ -831,23 +831,43 @@ def run_backward(args, w):
 
 GDN2_METRIC = ("tokens/s, chunked forward with Gated DeltaNet-2 erase and "
                "write gates (gdr_chunk_fwd_gdn2, staged path); % HBM roofline")
+FG2_METRIC = ("tokens/s, chunked forward with FG^2-GDN+ per-key-channel rate "
+              "and per-value-channel target scaling (gdr_chunk_fwd_fg2, "
+              "staged path); % HBM roofline")
+
+# per gate variant: metric, the gate generator's name in inputs, the binding,
+# the C entry, the oracle's token loop, and what the two gate tensors are
+TWO_GATES = {
+    "gdn2": (GDN2_METRIC, "gdn2_gates", "chunk_fwd_gdn2",
+             "gdr_chunk_fwd_gdn2", "gdn2_fwd",
+             "erase [.., dk], write [.., dv], sigmoid(N(0,1))"),
+    "fg2": (FG2_METRIC, "fg2_gates", "chunk_fwd_fg2", "gdr_chunk_fwd_fg2",
+            "fg2_fwd",
+            "key-side rate [.., dk], value-side scaling [.., dv], "
+            "sigmoid(N(0,1))"),
+}
 
 
-def run_gdn2(args, w):
-    """The workload's forward pass with Gated DeltaNet-2's per-channel erase
-    and write gates in place of beta (the staged path)."""
+def run_gdn2(args, w, kind="gdn2"):
+    """The workload's forward pass with two per-channel gate tensors in place
+    of beta, on the staged path: Gated DeltaNet-2's erase and write gates
+    (kind "gdn2") or FG^2-GDN+'s key-side rate and value-side scaling
+    (kind "fg2")."""
     import torch
 
     import chunkwise_recurrence_b200 as gdr
-    from chunkwise_recurrence_b200.inputs import gdn2_gates, generate
+    from chunkwise_recurrence_b200 import inputs as inputs_mod
+    from chunkwise_recurrence_b200.inputs import generate
 
+    metric, gen_name, fn_name, entry, oracle_name, gate_desc = TWO_GATES[kind]
     ws, rank, local = dist_env()
     if ws > 1:
-        raise SystemExit("--gdn2 runs on one GPU")
+        raise SystemExit(f"--{kind} runs on one GPU")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     inp = generate(w, seed=args.seed)
-    her, hwr = gdn2_gates(inp, seed=args.seed)
+    her, hwr = getattr(inputs_mod, gen_name)(inp, seed=args.seed)
+    fwd = getattr(gdr, fn_name)
     host = dict(q=inp.q, k=inp.k, v=inp.v, er=her, wr=hwr,
                 la=inp.log_alpha, s0=inp.s0, cu=inp.cu_seqlens)
     d = {n: None if t is None else t.to(dev) for n, t in host.items()}
@@ -857,10 +877,9 @@ def run_gdn2(args, w):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        gdr.chunk_fwd_gdn2(d["q"], d["k"], d["v"], d["er"], d["wr"], d["la"],
-                           d["s0"], chunk=w.chunk, gate=w.gate,
-                           cu_seqlens=d["cu"], out=out, final_state=sT,
-                           stream=stream)
+        fwd(d["q"], d["k"], d["v"], d["er"], d["wr"], d["la"], d["s0"],
+            chunk=w.chunk, gate=w.gate, cu_seqlens=d["cu"], out=out,
+            final_state=sT, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -917,12 +936,12 @@ def run_gdn2(args, w):
     peaks, peak_src = load_peaks()
     gbs = by / (statistics.mean(per_step) / 1e3) / 1e9
     line = {
-        "metric": GDN2_METRIC, "value": ntok / (ms / 1e3), "unit": "tokens/s",
+        "metric": metric, "value": ntok / (ms / 1e3), "unit": "tokens/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {**workload_config(w, inp), "algo": "staged",
-                   "gates": "erase [.., dk], write [.., dv], sigmoid(N(0,1))",
+                   "gates": gate_desc,
                    "l2": "inputs larger than L2 (no flush)",
                    "launch": "direct"},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
@@ -934,7 +953,7 @@ def run_gdn2(args, w):
         "e2e": {"value": ntok * e2e_steps / (e2e_ms / 1e3),
                 "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "entry": "gdr_chunk_fwd_gdn2, inputs copied from pinned host "
+                "entry": f"{entry}, inputs copied from pinned host "
                          "memory and results back each step"},
         "gpu_launches": launches_per_step("staged", w) * args.steps,
         "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
@@ -944,9 +963,9 @@ def run_gdn2(args, w):
         f = lambda t, n: None if t is None else t[:n].double().numpy()  # noqa
         n = 1
         t0 = time.perf_counter()
-        oracle.gdn2_fwd(f(inp.q, n), f(inp.k, n), f(inp.v, n), f(her, n),
-                        f(hwr, n), f(inp.log_alpha, n), w.gate,
-                        f(inp.s0, n))
+        getattr(oracle, oracle_name)(
+            f(inp.q, n), f(inp.k, n), f(inp.v, n), f(her, n), f(hwr, n),
+            f(inp.log_alpha, n), w.gate, f(inp.s0, n))
         dt = time.perf_counter() - t0
         line["cpu_baseline"] = {
             "value": n * w.T / dt, "unit": "tokens/s", "cores": 1,
@@ -1012,6 +1031,10 @@ def main(argv=None):
                     help="with Gated DeltaNet-2 erase and write gates "
                          "(gdr_chunk_fwd_gdn2; with --decode, "
                          "gdr_decode_step_gdn2)")
+    ap.add_argument("--fg2", action="store_true",
+                    help="with FG^2-GDN+'s per-key-channel rate and "
+                         "per-value-channel target scaling "
+                         "(gdr_chunk_fwd_fg2)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -1044,14 +1067,19 @@ def main(argv=None):
         if w.varlen_nseq or args.batch < 1:
             raise SystemExit("--batch needs a fixed-length workload and B >= 1")
         w = w.with_(B=args.batch, name=f"{w.name}@B{args.batch}")
+    if args.fg2 and (args.decode or args.backward):
+        raise SystemExit("--fg2 times the chunked forward pass only")
     if args.decode and args.impl == "ours":
         return run_decode(args)
     if args.backward and args.impl == "ours":
         return run_backward(args, w)
-    if args.gdn2 and args.impl == "ours":
+    if (args.gdn2 or args.fg2) and args.impl == "ours":
+        kind = "gdn2" if args.gdn2 else "fg2"
+        if args.gdn2 and args.fg2:
+            raise SystemExit("--gdn2 and --fg2 are exclusive")
         if w.varlen_nseq:
-            raise SystemExit("--gdn2 takes a fixed-length workload")
-        return run_gdn2(args, w)
+            raise SystemExit(f"--{kind} takes a fixed-length workload")
+        return run_gdn2(args, w, kind)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

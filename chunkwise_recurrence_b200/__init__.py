@@ -15,7 +15,8 @@ import os
 import torch
 
 __all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_noalloc",
-           "chunk_fwd_segmented", "chunk_fwd_gdn2", "decode_step",
+           "chunk_fwd_segmented", "chunk_fwd_gdn2", "chunk_fwd_fg2",
+           "decode_step", "decode_step_gdn2", "decode_step_fg2",
            "efla_beta", "backward",
            "device_error", "status_string",
            "algo_applies", "fused_tc_available",
@@ -36,7 +37,8 @@ EXPORTED_SYMBOLS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_device_error",
                     "gdr_chunk_fwd_noalloc", "gdr_decode_step",
                     "gdr_efla_beta", "gdr_backward",
                     "gdr_chunk_fwd_segmented", "gdr_chunk_fwd_gdn2",
-                    "gdr_decode_step_gdn2")
+                    "gdr_decode_step_gdn2", "gdr_chunk_fwd_fg2",
+                    "gdr_decode_step_fg2")
 # size of the static scratch array behind gdr_chunk_fwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -75,14 +77,16 @@ def load_library(path: str = LIB_PATH):
     lib.gdr_decode_step.restype = ctypes.c_int
     lib.gdr_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i,
                                     vp, ctypes.POINTER(_Opts)]
-    lib.gdr_decode_step_gdn2.restype = ctypes.c_int
-    lib.gdr_decode_step_gdn2.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp,
-                                         i, i, i, i, vp,
-                                         ctypes.POINTER(_Opts)]
-    lib.gdr_chunk_fwd_gdn2.restype = ctypes.c_int
-    lib.gdr_chunk_fwd_gdn2.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, i,
-                                       i, i, i, i, i, vp,
-                                       ctypes.POINTER(_Opts)]
+    for name in ("gdr_decode_step_gdn2", "gdr_decode_step_fg2"):
+        f = getattr(lib, name)
+        f.restype = ctypes.c_int
+        f.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp, i, i, i, i, vp,
+                      ctypes.POINTER(_Opts)]
+    for name in ("gdr_chunk_fwd_gdn2", "gdr_chunk_fwd_fg2"):
+        f = getattr(lib, name)
+        f.restype = ctypes.c_int
+        f.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, i, i, i, i, i, i, vp,
+                      ctypes.POINTER(_Opts)]
     lib.gdr_chunk_fwd_segmented.restype = ctypes.c_int
     lib.gdr_chunk_fwd_segmented.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i,
                                             i, i, i, i, i, i, vp,
@@ -183,6 +187,31 @@ def chunk_fwd_gdn2(q, k, v, erase_gate, write_gate, log_alpha=None,
     per-value-channel write gate (``write_gate``, the layout of v, fp32) in
     place of beta (see include/gdr.h for the update).  Returns (out,
     final_state)."""
+    return _chunk_fwd_two_gates(
+        "gdr_chunk_fwd_gdn2", q, k, v, erase_gate, write_gate, log_alpha,
+        initial_state, chunk, gate, cu_seqlens, out, final_state,
+        output_final_state, algo, stream)
+
+
+def chunk_fwd_fg2(q, k, v, beta_k, beta_v=None, log_alpha=None,
+                  initial_state=None, *, chunk: int = 64,
+                  gate: str | None = None, cu_seqlens=None, out=None,
+                  final_state=None, output_final_state: bool = True,
+                  algo: str = "auto", stream=None):
+    """Run ``gdr_chunk_fwd_fg2``: the forward pass with FG^2-GDN's
+    per-key-channel learning rate ``beta_k`` (the layout of k, fp32) and,
+    for FG^2-GDN+, the per-value-channel target scaling ``beta_v`` (the
+    layout of v, fp32; None for FG^2-GDN) in place of beta (see
+    include/gdr.h for the update).  Returns (out, final_state)."""
+    return _chunk_fwd_two_gates(
+        "gdr_chunk_fwd_fg2", q, k, v, beta_k, beta_v, log_alpha,
+        initial_state, chunk, gate, cu_seqlens, out, final_state,
+        output_final_state, algo, stream)
+
+
+def _chunk_fwd_two_gates(name, q, k, v, gate_k, gate_v, log_alpha,
+                         initial_state, chunk, gate, cu_seqlens, out,
+                         final_state, output_final_state, algo, stream):
     lib = load_library()
     B, T, H, dk, dv, nseq = _shapes(q, v, cu_seqlens)
     if out is None:
@@ -196,13 +225,13 @@ def chunk_fwd_gdn2(q, k, v, erase_gate, write_gate, log_alpha=None,
                  nseq if cu_seqlens is not None else 0, ALGOS[algo])
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    rc = lib.gdr_chunk_fwd_gdn2(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(erase_gate),
-        _ptr(write_gate), _ptr(initial_state), _ptr(out), _ptr(final_state),
+    rc = getattr(lib, name)(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(gate_k),
+        _ptr(gate_v), _ptr(initial_state), _ptr(out), _ptr(final_state),
         B, T, H, dk, dv, chunk, ctypes.c_void_p(stream.cuda_stream),
         ctypes.byref(opts))
     if rc != 0:
-        raise GdrError(rc, "gdr_chunk_fwd_gdn2")
+        raise GdrError(rc, name)
     return out, final_state
 
 
@@ -336,6 +365,25 @@ def decode_step_gdn2(q, k, v, erase_gate, write_gate, log_alpha=None,
     head) with Gated DeltaNet-2's gates in place of beta.  ``erase_gate``
     [N, H, dk] and ``write_gate`` [N, H, dv] are fp32; everything else is as
     in ``decode_step``.  Returns (out [N, H, dv], state_out)."""
+    return _decode_two_gates("gdr_decode_step_gdn2", q, k, v, erase_gate,
+                             write_gate, log_alpha, state, out, state_out,
+                             gate, stream)
+
+
+def decode_step_fg2(q, k, v, beta_k, beta_v=None, log_alpha=None,
+                    state=None, *, out=None, state_out=None,
+                    gate: str | None = None, stream=None):
+    """Run ``gdr_decode_step_fg2`` on CUDA tensors: one token per (sequence,
+    head) with FG^2-GDN's per-key-channel rate ``beta_k`` [N, H, dk] and
+    optional value-side scaling ``beta_v`` [N, H, dv] (fp32) in place of
+    beta; everything else is as in ``decode_step``.  Returns (out [N, H,
+    dv], state_out)."""
+    return _decode_two_gates("gdr_decode_step_fg2", q, k, v, beta_k, beta_v,
+                             log_alpha, state, out, state_out, gate, stream)
+
+
+def _decode_two_gates(name, q, k, v, gate_k, gate_v, log_alpha, state, out,
+                      state_out, gate, stream):
     lib = load_library()
     if q.dim() != 3 or v.dim() != 3:
         raise ValueError("q, k, v must be [N, H, d]")
@@ -352,14 +400,13 @@ def decode_step_gdn2(q, k, v, erase_gate, write_gate, log_alpha=None,
     opts = _Opts(DTYPES[q.dtype], GATES[g], None, 0, ALGOS["auto"])
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    rc = lib.gdr_decode_step_gdn2(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
-                                  _ptr(erase_gate), _ptr(write_gate),
-                                  _ptr(state), _ptr(state_out), _ptr(out),
-                                  N, H, dk, dv,
-                                  ctypes.c_void_p(stream.cuda_stream),
-                                  ctypes.byref(opts))
+    rc = getattr(lib, name)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                            _ptr(gate_k), _ptr(gate_v), _ptr(state),
+                            _ptr(state_out), _ptr(out), N, H, dk, dv,
+                            ctypes.c_void_p(stream.cuda_stream),
+                            ctypes.byref(opts))
     if rc != 0:
-        raise GdrError(rc, "gdr_decode_step_gdn2")
+        raise GdrError(rc, name)
     return out, state_out
 
 

@@ -29,7 +29,10 @@
 // With Gated DeltaNet-2's gates (erase != nullptr) the read key is b . k
 // (erase gate b, per key channel) and the target w . v (write gate w, per
 // value channel), without beta:  u = w . v - S~^T (b . k),  S' = S~ + k u^T,
-// o = S~^T q + u (k . q)  (gdr_decode_step_gdn2).
+// o = S~^T q + u (k . q)  (gdr_decode_step_gdn2).  With FG^2-GDN's rate
+// (wkey != nullptr) the write key is a . k (rate a, per key channel) and the
+// target (c .) v:  u = (c .) v - S~^T k,  S' = S~ + (a . k) u^T,
+// o = S~^T q + u ((a . k) . q)  (gdr_decode_step_fg2).
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -82,6 +85,9 @@ struct DecodeParams {
   int dv;
   // Gated DeltaNet-2 gates [N*H][dk] and [N*H][dv], or nullptr
   const float *erase, *write;
+  // FG^2-GDN's key-side rate [N*H][dk], or nullptr (`write` is then the
+  // optional value-side scaling)
+  const float *wkey;
   // failure injection (host hook): the state copy is not issued, so the
   // CTA's wait runs out after wait_cycles and reports a timeout
   int inject_timeout;
@@ -129,7 +135,8 @@ __global__ void __launch_bounds__(kDecThreads)
     gdr_decode_kernel(DecodeParams p) {
   constexpr int R = DK / 8;   // rows of S per warp
   extern __shared__ __align__(128) float tile[];   // the state, [DK][dv]
-  __shared__ float sk[DK], sq[DK], sa[DK], sr[DK];   // sr: read key
+  // sr: read key; sw: write key
+  __shared__ float sk[DK], sq[DK], sa[DK], sr[DK], sw[DK];
   __shared__ float4 red[2][8][32];   // per warp: partial S~^T k, S~^T q
   __shared__ float kq_s;
   __shared__ __align__(8) uint64_t bar;
@@ -158,6 +165,7 @@ __global__ void __launch_bounds__(kDecThreads)
             : GATE == 1 ? __expf(p.log_alpha[nh])
                         : __expf(p.log_alpha[(size_t)nh * DK + c]);
     sr[c] = p.erase ? p.erase[(size_t)nh * DK + c] * sk[c] : sk[c];
+    sw[c] = p.wkey ? p.wkey[(size_t)nh * DK + c] * sk[c] : sk[c];
   }
   if (threadIdx.x == 0 && p.s_in) {
     const long long t0 = clock64();
@@ -198,7 +206,7 @@ __global__ void __launch_bounds__(kDecThreads)
   red[1][warp][lane] = pq;
   if (warp == 0) {
     float t = 0.f;
-    for (int c = lane; c < DK; c += 32) t = fmaf(sk[c], sq[c], t);
+    for (int c = lane; c < DK; c += 32) t = fmaf(sw[c], sq[c], t);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1)
       t += __shfl_xor_sync(0xffffffffu, t, off);
@@ -213,12 +221,13 @@ __global__ void __launch_bounds__(kDecThreads)
     rq = make_float4(rq.x + b.x, rq.y + b.y, rq.z + b.z, rq.w + b.w);
   }
   if (act) {
-    // u = beta (v - S~^T k) (Gated DeltaNet-2: w . v - S~^T (b . k));
-    // o = S~^T q + u (k . q)
+    // u = beta (v - S~^T k) (Gated DeltaNet-2: w . v - S~^T (b . k);
+    // FG^2-GDN: (c .) v - S~^T k);  o = S~^T q + u (write key . q)
     const float4 vv = ld4(static_cast<const T *>(p.v) + (size_t)nh * dv + j0);
     float4 u;
-    if (p.erase) {
-      const float4 wg = ld4(p.write + (size_t)nh * dv + j0);
+    if (p.erase || p.wkey) {
+      const float4 wg = p.write ? ld4(p.write + (size_t)nh * dv + j0)
+                                : make_float4(1.f, 1.f, 1.f, 1.f);
       u = make_float4(wg.x * vv.x - rk.x, wg.y * vv.y - rk.y,
                       wg.z * vv.z - rk.z, wg.w * vv.w - rk.w);
     } else {
@@ -228,12 +237,12 @@ __global__ void __launch_bounds__(kDecThreads)
     }
     if (warp == 0)
       st4(static_cast<T *>(p.out) + (size_t)nh * dv + j0, fma4(kq_s, u, rq));
-    // S' = S~ + k u^T, in place in the tile
+    // S' = S~ + (write key) u^T, in place in the tile
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int c = warp * R + r;
       float *e = tile + c * dv + j0;
-      st4(e, fma4(sk[c], u, ld4(e)));
+      st4(e, fma4(sw[c], u, ld4(e)));
     }
   }
   // the tile's generic-proxy writes, visible to the bulk store
@@ -299,9 +308,12 @@ bool dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 namespace gdr {
 namespace {
 
+// The gate form follows from which of beta, erase, wkey is given: exactly
+// one of them (erase with write, wkey with an optional write).
 gdr_status decode_entry(const void *q, const void *k, const void *v,
                         const float *log_alpha, const float *beta,
                         const float *erase, const float *write,
+                        const float *wkey,
                         const float *state_in, float *state_out, void *out,
                         int N, int H, int dk, int dv, cudaStream_t stream,
                         const gdr_opts *opts) {
@@ -326,11 +338,13 @@ gdr_status decode_entry(const void *q, const void *k, const void *v,
   const long long nh = (long long)N * H;
   if (nh > 0x7fffffffLL) return GDR_ERR_UNSUPPORTED;
   if (nh == 0) return GDR_OK;
-  const bool g2 = erase != nullptr || write != nullptr;
   if (!q || !k || !v || !state_out || !out) return GDR_ERR_INVALID_ARGUMENT;
-  if (g2 ? (!erase || !write) : !beta) return GDR_ERR_INVALID_ARGUMENT;
-  const void *ptrs[] = {q, k, v, log_alpha, beta, erase, write, state_in,
-                        state_out, out};
+  if ((beta != nullptr) + (erase != nullptr) + (wkey != nullptr) != 1)
+    return GDR_ERR_INVALID_ARGUMENT;
+  if (beta && write) return GDR_ERR_INVALID_ARGUMENT;
+  if (erase && !write) return GDR_ERR_INVALID_ARGUMENT;
+  const void *ptrs[] = {q, k, v, log_alpha, beta, erase, write, wkey,
+                        state_in, state_out, out};
   for (const void *ptr : ptrs)
     if (ptr && !aligned16(ptr)) return GDR_ERR_INVALID_ARGUMENT;
   // state_in and state_out: the same buffer (in-place update) or disjoint
@@ -350,8 +364,9 @@ gdr_status decode_entry(const void *q, const void *k, const void *v,
   dp.s_out = state_out;
   dp.out = out;
   dp.dv = dv;
-  dp.erase = g2 ? erase : nullptr;
-  dp.write = g2 ? write : nullptr;
+  dp.erase = erase;
+  dp.write = write;
+  dp.wkey = wkey;
   const char *inj = std::getenv("GDR_FAULT_INJECT_DECODE_TIMEOUT");
   dp.inject_timeout = (inj && inj[0] == '1') ? 1 : 0;
   dp.wait_cycles = dp.inject_timeout ? kDecInjectWaitCycles : kDecWaitCycles;
@@ -374,8 +389,8 @@ extern "C" gdr_status gdr_decode_step(const void *q, const void *k,
                                       cudaStream_t stream,
                                       const gdr_opts *opts) {
   return gdr::decode_entry(q, k, v, log_alpha, beta, nullptr, nullptr,
-                           state_in, state_out, out, N, H, dk, dv, stream,
-                           opts);
+                           nullptr, state_in, state_out, out, N, H, dk, dv,
+                           stream, opts);
 }
 
 extern "C" gdr_status gdr_decode_step_gdn2(
@@ -385,6 +400,17 @@ extern "C" gdr_status gdr_decode_step_gdn2(
     cudaStream_t stream, const gdr_opts *opts) {
   if (!erase_gate || !write_gate) return GDR_ERR_INVALID_ARGUMENT;
   return gdr::decode_entry(q, k, v, log_alpha, nullptr, erase_gate,
-                           write_gate, state_in, state_out, out, N, H, dk, dv,
+                           write_gate, nullptr, state_in, state_out, out, N, H,
+                           dk, dv, stream, opts);
+}
+
+extern "C" gdr_status gdr_decode_step_fg2(
+    const void *q, const void *k, const void *v, const float *log_alpha,
+    const float *beta_k, const float *beta_v, const float *state_in,
+    float *state_out, void *out, int N, int H, int dk, int dv,
+    cudaStream_t stream, const gdr_opts *opts) {
+  if (!beta_k) return GDR_ERR_INVALID_ARGUMENT;
+  return gdr::decode_entry(q, k, v, log_alpha, nullptr, nullptr, beta_v,
+                           beta_k, state_in, state_out, out, N, H, dk, dv,
                            stream, opts);
 }

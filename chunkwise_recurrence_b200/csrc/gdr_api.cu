@@ -119,8 +119,10 @@ gdr_status scratch_alloc(void **ptr, size_t bytes, cudaStream_t s) {
 
 gdr_status run(const Problem &p, gdr_algo algo, cudaStream_t stream) {
   if (p.nseq == 0 || p.H == 0) return GDR_OK;
-  // the Gated DeltaNet-2 gates run on the staged path only
-  const bool tc = p.erase == nullptr && gdr::fused_tc_applies(p);
+  // the Gated DeltaNet-2 gates and FG^2-GDN's rate run on the staged path
+  // only
+  const bool tc = p.erase == nullptr && p.write == nullptr &&
+                  p.wkey == nullptr && gdr::fused_tc_applies(p);
   if (algo == GDR_ALGO_FUSED_TC && !tc) return GDR_ERR_UNSUPPORTED;
   if (tc && algo != GDR_ALGO_STAGED) {
     cudaError_t e = gdr::fused_tc_run(p, stream);
@@ -177,6 +179,33 @@ extern "C" gdr_status gdr_chunk_fwd_gdn2(const void *q, const void *k,
   p.beta = nullptr;
   p.erase = erase_gate;
   p.write = write_gate;
+  return run(p, GDR_ALGO_STAGED, stream);
+}
+
+// FG^2-GDN's per-key-channel rate on the write key (and FG^2-GDN+'s
+// per-value-channel target scaling), on the staged path: see gdr.h.
+extern "C" gdr_status gdr_chunk_fwd_fg2(const void *q, const void *k,
+                                        const void *v, const float *log_alpha,
+                                        const float *beta_k,
+                                        const float *beta_v,
+                                        const float *initial_state, void *out,
+                                        float *final_state, int B, int T,
+                                        int H, int dk, int dv, int chunk,
+                                        cudaStream_t stream,
+                                        const gdr_opts *opts) {
+  const gdr_opts o = opts ? *opts : default_opts();
+  if (o.algo == GDR_ALGO_FUSED_TC) return GDR_ERR_UNSUPPORTED;
+  Problem p;
+  // the key-side rate stands in for beta in the common checks (presence,
+  // alignment); the optional value-side scaling is checked here
+  gdr_status st = validate(q, k, v, log_alpha, beta_k, initial_state, out,
+                           final_state, B, T, H, dk, dv, chunk, o, &p);
+  if (st != GDR_OK) return st;
+  if (p.nseq == 0 || p.H == 0) return GDR_OK;
+  if (beta_v && !aligned16(beta_v)) return GDR_ERR_INVALID_ARGUMENT;
+  p.beta = nullptr;
+  p.wkey = beta_k;
+  p.write = beta_v;
   return run(p, GDR_ALGO_STAGED, stream);
 }
 

@@ -38,6 +38,10 @@ struct Problem {
   // per-key-channel erase gate [ntok][H][dk] and per-value-channel write
   // gate [ntok][H][dv] that replace beta
   const float *erase = nullptr, *write = nullptr;
+  // FG^2-GDN's per-key-channel rate [ntok][H][dk] (staged path and decode
+  // only; nullptr otherwise): the write key of token t is wkey_t . k_t and
+  // the read key k_t; `write` (or nullptr for ones) then scales the target
+  const float *wkey = nullptr;
 };
 
 // Staged path: four kernels + a chunk-table kernel, fp32 CUDA-core math.

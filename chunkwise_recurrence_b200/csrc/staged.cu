@@ -10,6 +10,16 @@
 //                        S_{n+1} = Gamma_C S_n + (K . e^{g_C - g})^T V_new
 //   (d) output_kernel  : O = (Q . e^g) S_n + mask_{i<=r}[(Q . e^g)(K . e^-g)^T] V_new
 //
+// The gate variants change only which vectors enter these products.  Each
+// token has a read key (the key the state is read with before the write), a
+// write key (the key its correction is written along) and a target:
+//   delta rule         : read k,      write k,      target v,     rows x beta
+//   Gated DeltaNet-2   : read b . k,  write k,      target w . v
+//   FG^2-GDN (+)       : read k,      write a . k,  target (c .) v
+// A[r][i] pairs the read key of r with the write key of i, W is built from
+// the read keys, U from the targets, and the state update and the
+// intra-chunk output use the write keys.
+//
 // The chunkwise form rests on the update being affine in the preceding memory
 // ("DeltaTTT: Layerwise Optimization for Nonlinear Recurrent Memory",
 // §2 Background) and on the WY form with the decay folded into the erase
@@ -102,6 +112,10 @@ __device__ __forceinline__ float gval(const float *Gs, int gdim, int r,
 // (write gate w_r, per value channel), and beta is not used:
 //   A[r][i] = (b_r . k_r)^T Gamma_r Gamma_i^-1 k_i,  W = T ((B . K) . e^g),
 //   U = T (Wg . V).
+// With FG^2-GDN's rate (wkey != nullptr) the write key of token i is
+// a_i . k_i and the target (c_r .) v_r, with write = c or nullptr:
+//   A[r][i] = k_r^T Gamma_r Gamma_i^-1 (a_i . k_i),  W = T (K . e^g),
+//   U = T ((C .) V).
 // Shared memory: the key rows are padded to dk + 1 floats so that the A
 // products, whose lanes walk rows, read distinct banks; the factors of W and
 // U (beta_i (read key) e^{g_i} and beta_i (target)) are formed once per
@@ -111,6 +125,7 @@ __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
                           const float *__restrict__ beta,
                           const float *__restrict__ erase,
                           const float *__restrict__ write,
+                          const float *__restrict__ wkey,
                           const float *__restrict__ g, float *__restrict__ W,
                           float *__restrict__ U,
                           const ChunkInfo *__restrict__ table,
@@ -123,25 +138,28 @@ __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
   const int gd = gdim == 0 ? 1 : gdim;
   const int dkp = dk + 1;
   const bool g2 = erase != nullptr;
+  // a read key that differs from the write key needs a tile of its own
+  const bool split = g2 || wkey != nullptr;
   extern __shared__ __align__(16) float sm[];
-  float *Ks = sm;                  // [C][dkp]
+  float *Ks = sm;                  // [C][dkp], the write keys
   float *Gs = Ks + C * dkp;        // [C][gd]
   float *As = Gs + C * gd;         // [C][C+1]
   float *Ts = As + C * (C + 1);    // [C][C+1]
   float *bs = Ts + C * (C + 1);    // [C]
-  float *Vs = bs + C;              // [C][dv], beta_i v_i (or w_i . v_i)
-  float *Es = Vs + C * dv;         // [C][dkp], b_r . k_r (Gated DeltaNet-2)
-  // the read keys: b_r . k_r (Gated DeltaNet-2) or k_r; the row factor
-  // bs[r] is then 1 or beta_r
-  float *Rs = g2 ? Es : Ks;
+  float *Vs = bs + C;              // [C][dv], the targets (times beta_i)
+  float *Es = Vs + C * dv;         // [C][dkp], the read keys when split
+  // the read keys: b_r . k_r (Gated DeltaNet-2), k_r (FG^2-GDN; the write
+  // keys are then a_r . k_r) or the write keys themselves; the row factor
+  // bs[r] is beta_r for the delta rule and 1 otherwise
+  float *Rs = split ? Es : Ks;
   const int tid = threadIdx.x, nt = blockDim.x;
 
   for (int idx = tid; idx < L * dk; idx += nt) {
     const int r = idx / dk, c = idx % dk;
     const size_t off = ((size_t)(ci.tok0 + r) * H + h) * dk + c;
     const float kv = to_f(k[off]);
-    Ks[r * dkp + c] = kv;
-    if (g2) Es[r * dkp + c] = erase[off] * kv;
+    Ks[r * dkp + c] = wkey ? wkey[off] * kv : kv;
+    if (split) Es[r * dkp + c] = g2 ? erase[off] * kv : kv;
   }
   if (gdim)
     for (int idx = tid; idx < L * gdim; idx += nt) {
@@ -149,15 +167,15 @@ __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
       Gs[r * gdim + c] = g[((size_t)(ci.tok0 + r) * H + h) * gdim + c];
     }
   for (int r = tid; r < L; r += nt)
-    bs[r] = g2 ? 1.f : beta[(size_t)(ci.tok0 + r) * H + h];
+    bs[r] = split ? 1.f : beta[(size_t)(ci.tok0 + r) * H + h];
   __syncthreads();
   for (int idx = tid; idx < L * dv; idx += nt) {
     const int r = idx / dv, c = idx % dv;
     const size_t e = ((size_t)(ci.tok0 + r) * H + h) * dv + c;
-    Vs[r * dv + c] = bs[r] * (g2 ? write[e] * to_f(v[e]) : to_f(v[e]));
+    Vs[r * dv + c] = bs[r] * (write ? write[e] * to_f(v[e]) : to_f(v[e]));
   }
 
-  // A[r][i] = beta_r sum_c rk_r[c] k_i[c] exp(g_r[c] - g_i[c]),  i < r
+  // A[r][i] = beta_r sum_c rk_r[c] wk_i[c] exp(g_r[c] - g_i[c]),  i < r
   for (int idx = tid; idx < L * L; idx += nt) {
     const int r = idx / L, i = idx % L;
     float a = 0.f;
@@ -218,6 +236,7 @@ __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
 // (one exponential per row and channel) before the state update reads them.
 template <typename Tin>
 __global__ void state_kernel(const Tin *__restrict__ k,
+                             const float *__restrict__ wkey,
                              const float *__restrict__ g,
                              const float *__restrict__ W,
                              const float *__restrict__ U,
@@ -232,7 +251,7 @@ __global__ void state_kernel(const Tin *__restrict__ k,
   float *S = sm;              // [dk][DVT]
   float *V = S + dk * DVT;    // [C][DVT]
   float *gl = V + C * DVT;    // [dk]
-  float *Kt = gl + dk;        // [C][dk], k_r . e^{g_C - g_r}
+  float *Kt = gl + dk;        // [C][dk], (write key)_r . e^{g_C - g_r}
   const int tid = threadIdx.x, nt = blockDim.x;
   const size_t sbase = ((size_t)n * H + h) * dk * dv;
 
@@ -269,7 +288,8 @@ __global__ void state_kernel(const Tin *__restrict__ k,
       const int r = idx / dk, c = idx % dk;
       const size_t row = (size_t)(ci.tok0 + r) * H + h;
       const float gr = gdim == 0 ? 0.f : g[row * gdim + (gdim == 1 ? 0 : c)];
-      Kt[idx] = to_f(k[row * dk + c]) * __expf(gl[c] - gr);
+      const float kw = to_f(k[row * dk + c]) * (wkey ? wkey[row * dk + c] : 1.f);
+      Kt[idx] = kw * __expf(gl[c] - gr);
     }
     __syncthreads();
     // S <- Gamma_C S + (K . e^{g_C - g})^T V_new
@@ -297,6 +317,7 @@ constexpr int kOutRows = 8;
 template <typename Tin>
 __global__ void output_kernel(const Tin *__restrict__ q,
                               const Tin *__restrict__ k,
+                              const float *__restrict__ wkey,
                               const float *__restrict__ g,
                               const float *__restrict__ Sbuf,
                               const float *__restrict__ Vn,
@@ -312,7 +333,7 @@ __global__ void output_kernel(const Tin *__restrict__ q,
   const int dkp = dk + 1;
   extern __shared__ __align__(16) float sm[];
   float *Qs = sm;               // [C][dk]
-  float *Ks = Qs + C * dk;      // [C][dkp]
+  float *Ks = Qs + C * dk;      // [C][dkp], the write keys
   float *Gs = Ks + C * dkp;     // [C][gd]
   float *Ps = Gs + C * gd;      // [C][C+1]
   const int tid = threadIdx.x, nt = blockDim.x;
@@ -320,7 +341,7 @@ __global__ void output_kernel(const Tin *__restrict__ q,
     const int r = idx / dk, c = idx % dk;
     const size_t off = ((size_t)(ci.tok0 + r) * H + h) * dk + c;
     Qs[r * dk + c] = to_f(q[off]);
-    Ks[r * dkp + c] = to_f(k[off]);
+    Ks[r * dkp + c] = to_f(k[off]) * (wkey ? wkey[off] : 1.f);
   }
   if (gdim)
     for (int idx = tid; idx < L * gdim; idx += nt) {
@@ -447,14 +468,14 @@ cudaError_t run_typed(const Problem &p, char *ws, cudaStream_t s) {
     const size_t wy_smem =
         sizeof(float) * ((size_t)C * dkp + (size_t)C * gd +
                          2 * (size_t)C * (C + 1) + C + (size_t)C * p.dv +
-                         (p.erase ? (size_t)C * dkp : 0));
+                         ((p.erase || p.wkey) ? (size_t)C * dkp : 0));
     cudaError_t e = cudaFuncSetAttribute(
         wy_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
         (int)wy_smem);
     if (e != cudaSuccess) return e;
     wy_kernel<Tin><<<grid, 256, wy_smem, s>>>(k, v, p.beta, p.erase, p.write,
-                                             g, W, U, table, nchunks, p.H,
-                                             p.dk, p.dv, C, gdim);
+                                             p.wkey, g, W, U, table, nchunks,
+                                             p.H, p.dk, p.dv, C, gdim);
   }
   const int DVT = p.dv < 64 ? p.dv : 64;
   const size_t st_smem =
@@ -467,8 +488,8 @@ cudaError_t run_typed(const Problem &p, char *ws, cudaStream_t s) {
     if (e != cudaSuccess) return e;
   }
   state_kernel<Tin><<<dim3(p.nseq, p.H, p.dv / DVT), 256, st_smem, s>>>(
-      k, g, W, U, p.s0, p.sT, Sbuf, Vn, table, seq_first, p.H, p.dk, p.dv, C,
-      gdim, DVT);
+      k, p.wkey, g, W, U, p.s0, p.sT, Sbuf, Vn, table, seq_first, p.H, p.dk,
+      p.dv, C, gdim, DVT);
   if (p.max_chunks > 0) {
     const size_t o_smem =
         sizeof(float) * ((size_t)C * p.dk + (size_t)C * (p.dk + 1) +
@@ -478,7 +499,8 @@ cudaError_t run_typed(const Problem &p, char *ws, cudaStream_t s) {
         (int)o_smem);
     if (e != cudaSuccess) return e;
     output_kernel<Tin><<<dim3(p.max_chunks, p.H), 256, o_smem, s>>>(
-        q, k, g, Sbuf, Vn, out, table, nchunks, p.H, p.dk, p.dv, C, gdim);
+        q, k, p.wkey, g, Sbuf, Vn, out, table, nchunks, p.H, p.dk, p.dv, C,
+        gdim);
   }
   return cudaGetLastError();
 }

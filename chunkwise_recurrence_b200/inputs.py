@@ -160,6 +160,16 @@ def gdn2_gates(inp: Inputs, seed: int = 0):
     return erase.float().contiguous(), write.float().contiguous()
 
 
+def fg2_gates(inp: Inputs, seed: int = 0):
+    """FG^2-GDN rates for a generated batch: a learning rate per key channel
+    (the layout of k) and, for FG^2-GDN+, a target scaling per value channel
+    (the layout of v), both sigmoid(N(0, 1)) like beta, fp32, seeded."""
+    g = torch.Generator().manual_seed(2_000_003 + seed)
+    beta_k = torch.sigmoid(torch.randn(inp.k.shape, generator=g))
+    beta_v = torch.sigmoid(torch.randn(inp.v.shape, generator=g))
+    return beta_k.float().contiguous(), beta_v.float().contiguous()
+
+
 def head_slice(inp: Inputs, heads) -> Inputs:
     """The same inputs restricted to a subset of heads (chains are independent
     per head, so this is how large workloads are sampled for the oracle)."""

@@ -18,7 +18,8 @@
  *    §4.1: a gradient step on a linear-regression objective in the memory
  *    matrix is a delta-rule update.  App. B: keys are normalised.
  *  - "Delta-Rule Linear Attention" topic page, FG^2-GDN card: KDA refines the
- *    head-wise decay of Gated DeltaNet into a channel-wise decay.
+ *    head-wise decay of Gated DeltaNet into a channel-wise decay; FG^2-GDN
+ *    makes the learning rate channel-wise too (gdr_chunk_fwd_fg2).
  *  - Gated DeltaNet-2 abstract, comparative-study page (2607.07953): a
  *    chunkwise WY algorithm with channel-wise decay absorbed into the erase
  *    factors; GDN-2 reduces to KDA and then to Gated DeltaNet.
@@ -225,6 +226,41 @@ GDR_API gdr_status gdr_chunk_fwd_gdn2(const void *q, const void *k,
                                       const gdr_opts *opts);
 
 /*
+ * gdr_chunk_fwd_fg2 -- the forward pass with FG^2-GDN's channel-wise
+ * learning rate (and FG^2-GDN+'s value-side scaling).
+ *
+ * FG^2-GDN ("Delta-Rule Linear Attention" topic page, FG^2-GDN card) turns
+ * the delta rule's scalar learning rate beta_t into a vector over channels,
+ * as per-coordinate optimisers refine SGD; FG^2-GDN+ scales keys and values
+ * separately.  The pages print no formula; the update taken here reads the
+ * delta rule as one gradient step on 1/2 ||S^T k_t - v_t||^2 ("DeltaTTT"
+ * page, sec. 4.1) with a rate per key channel (row of S), and FG^2-GDN+ as
+ * a per-value-channel scaling c_t of the target:
+ *   S~_t = D_t S_{t-1},   u_t = c_t . v_t - S~_t^T k_t,
+ *   S_t  = S~_t + (beta_t . k_t) u_t^T,   o_t = S_t^T q_t,
+ * i.e. write key beta_t . k_t, read key k_t.  beta_t = beta_t 1 with c = 1
+ * is gdr_chunk_fwd's recurrence.
+ *
+ * Arguments as for gdr_chunk_fwd, with beta replaced by
+ *   beta_k  [B][T][H][dk] fp32 (device, 16-byte aligned), required: the
+ *           per-key-channel rate;
+ *   beta_v  [B][T][H][dv] fp32 (device, 16-byte aligned), or NULL for
+ *           FG^2-GDN (c = 1): FG^2-GDN+'s per-value-channel scaling;
+ * (packed layouts with cu_seqlens as for gdr_chunk_fwd).  The decay form is
+ * opts->gate (NONE, SCALAR or CHANNEL).  Runs the staged path (fp32
+ * CUDA-core arithmetic, any supported shape): opts->algo AUTO or STAGED;
+ * FUSED_TC returns GDR_ERR_UNSUPPORTED.  Status codes as for gdr_chunk_fwd.
+ */
+GDR_API gdr_status gdr_chunk_fwd_fg2(const void *q, const void *k,
+                                     const void *v, const float *log_alpha,
+                                     const float *beta_k, const float *beta_v,
+                                     const float *initial_state, void *out,
+                                     float *final_state, int B, int T, int H,
+                                     int dk, int dv, int chunk,
+                                     cudaStream_t stream,
+                                     const gdr_opts *opts);
+
+/*
  * gdr_chunk_fwd_segmented -- gdr_chunk_fwd with context-parallel state
  * passing along each sequence.
  *
@@ -368,6 +404,31 @@ GDR_API gdr_status gdr_decode_step_gdn2(const void *q, const void *k,
                                         int H, int dk, int dv,
                                         cudaStream_t stream,
                                         const gdr_opts *opts);
+
+/*
+ * gdr_decode_step_fg2 -- gdr_decode_step with FG^2-GDN's per-key-channel
+ * rate (and FG^2-GDN+'s value-side scaling; the update gdr_chunk_fwd_fg2
+ * documents) for one token per (sequence, head):
+ *     S~ = D S,   u = c . v - S~^T k,   S' = S~ + (beta_k . k) u^T,
+ *     o = S'^T q
+ * so that a prompt run through gdr_chunk_fwd_fg2 can be continued one token
+ * at a time.
+ *
+ * Arguments as for gdr_decode_step, with beta replaced by
+ *   beta_k  [N][H][dk] fp32 (device, 16-byte aligned), required;
+ *   beta_v  [N][H][dv] fp32 (device, 16-byte aligned), or NULL (c = 1).
+ * Same kernel, limits, bounded wait and status codes as gdr_decode_step;
+ * a NULL beta_k returns GDR_ERR_INVALID_ARGUMENT.
+ */
+GDR_API gdr_status gdr_decode_step_fg2(const void *q, const void *k,
+                                       const void *v, const float *log_alpha,
+                                       const float *beta_k,
+                                       const float *beta_v,
+                                       const float *state_in,
+                                       float *state_out, void *out, int N,
+                                       int H, int dk, int dv,
+                                       cudaStream_t stream,
+                                       const gdr_opts *opts);
 
 /*
  * gdr_backward -- gradients of gdr_chunk_fwd's outputs with respect to its

@@ -245,6 +245,54 @@ def test_gdn2_rejects_bad_arguments(lib):
              gate=0, B=0) == OK
 
 
+def test_fg2_rejects_bad_arguments(lib):
+    def c(**kw):
+        args = dict(q=A, k=A, v=A, la=A, bk=A, bv=None, s0=None, out=A,
+                    sT=None, B=1, T=64, H=1, dk=128, dv=128, chunk=64,
+                    dtype=0, gate=2, cu=None, nseq=0, algo=0)
+        args.update(kw)
+        opts = gdr._Opts(args["dtype"], args["gate"], args["cu"], args["nseq"],
+                         args["algo"])
+        return lib.gdr_chunk_fwd_fg2(
+            args["q"], args["k"], args["v"], args["la"], args["bk"],
+            args["bv"], args["s0"], args["out"], args["sT"], args["B"],
+            args["T"], args["H"], args["dk"], args["dv"], args["chunk"], None,
+            ctypes.byref(opts))
+    assert c(bk=None) == INVALID          # the key-side rate is required
+    assert c(bk=A + 4) == INVALID         # 16-byte alignment
+    assert c(bv=A + 8) == INVALID
+    assert c(la=None) == INVALID          # a decay gate needs log_alpha
+    assert c(algo=2) == UNSUPPORTED       # staged path only
+    assert c(algo=2, bv=A) == UNSUPPORTED
+    assert c(dk=48) == UNSUPPORTED
+    assert c(q=None, k=None, v=None, la=None, bk=None, out=None, gate=0,
+             B=0) == OK
+
+
+def test_decode_fg2_rejects_bad_arguments(lib):
+    def c(**kw):
+        args = dict(q=A, k=A, v=A, la=A, bk=A, bv=None, s0=None, s1=A, out=A,
+                    N=1, H=1, dk=128, dv=128, dtype=0, gate=1, cu=None,
+                    nseq=0, algo=0)
+        args.update(kw)
+        opts = gdr._Opts(args["dtype"], args["gate"], args["cu"], args["nseq"],
+                         args["algo"])
+        return lib.gdr_decode_step_fg2(
+            args["q"], args["k"], args["v"], args["la"], args["bk"],
+            args["bv"], args["s0"], args["s1"], args["out"], args["N"],
+            args["H"], args["dk"], args["dv"], None, ctypes.byref(opts))
+    assert c(bk=None) == INVALID          # the key-side rate is required
+    assert c(bk=A + 4) == INVALID         # 16-byte alignment
+    assert c(bv=A + 8) == INVALID
+    assert c(la=None) == INVALID
+    assert c(cu=A, nseq=1) == INVALID     # one token per sequence
+    assert c(algo=2) == UNSUPPORTED
+    assert c(dv=48) == UNSUPPORTED
+    assert c(s0=A, s1=A + 64) == INVALID  # overlapping, not identical states
+    assert c(q=None, k=None, v=None, la=None, s1=None, out=None, gate=0,
+             N=0) == OK
+
+
 def test_decode_gdn2_rejects_bad_arguments(lib):
     def c(**kw):
         args = dict(q=A, k=A, v=A, la=A, er=A, wr=A, s0=None, s1=A, out=A,
