@@ -830,10 +830,10 @@ def run_backward(args, w):
 
 
 GDN2_METRIC = ("tokens/s, chunked forward with Gated DeltaNet-2 erase and "
-               "write gates (gdr_chunk_fwd_gdn2, staged path); % HBM roofline")
+               "write gates (gdr_chunk_fwd_gdn2); % HBM roofline")
 FG2_METRIC = ("tokens/s, chunked forward with FG^2-GDN+ per-key-channel rate "
-              "and per-value-channel target scaling (gdr_chunk_fwd_fg2, "
-              "staged path); % HBM roofline")
+              "and per-value-channel target scaling (gdr_chunk_fwd_fg2); "
+              "% HBM roofline")
 
 # per gate variant: metric, the gate generator's name in inputs, the binding,
 # the C entry, the oracle's token loop, and what the two gate tensors are
@@ -850,9 +850,9 @@ TWO_GATES = {
 
 def run_gdn2(args, w, kind="gdn2"):
     """The workload's forward pass with two per-channel gate tensors in place
-    of beta, on the staged path: Gated DeltaNet-2's erase and write gates
-    (kind "gdn2") or FG^2-GDN+'s key-side rate and value-side scaling
-    (kind "fg2")."""
+    of beta: Gated DeltaNet-2's erase and write gates (kind "gdn2") or
+    FG^2-GDN+'s key-side rate and value-side scaling (kind "fg2"); the fused
+    kernel with the channel-wise decay, else the staged path."""
     import torch
 
     import chunkwise_recurrence_b200 as gdr
@@ -875,11 +875,20 @@ def run_gdn2(args, w, kind="gdn2"):
     sT = torch.empty(inp.nseq, w.H, w.dk, w.dv, dtype=torch.float32,
                      device=dev)
     stream = torch.cuda.current_stream(dev)
+    # the fused kernel takes these gates with the channel-wise decay (bf16,
+    # d = 128, C = 64); every other shape runs the staged path
+    algo_used = args.algo
+    if algo_used == "auto":
+        algo_used = ("fused_tc" if (w.gate == "channel" and
+                                    w.dtype == "bf16" and w.dk == 128 and
+                                    w.dv == 128 and w.chunk == 64 and
+                                    gdr_fused_available())
+                     else "staged")
 
     def step():
         fwd(d["q"], d["k"], d["v"], d["er"], d["wr"], d["la"], d["s0"],
             chunk=w.chunk, gate=w.gate, cu_seqlens=d["cu"], out=out,
-            final_state=sT, stream=stream)
+            final_state=sT, stream=stream, algo=algo_used)
 
     for _ in range(args.warmup):
         step()
@@ -940,14 +949,15 @@ def run_gdn2(args, w, kind="gdn2"):
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {**workload_config(w, inp), "algo": "staged",
+        "config": {**workload_config(w, inp), "algo": algo_used,
                    "gates": gate_desc,
                    "l2": "inputs larger than L2 (no flush)",
                    "launch": "direct"},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                      "traffic": None, "peak_source": peak_src,
-                     "kernel": "staged path (whole call)",
+                     "kernel": ("gdr_fused_tc_kernel" if algo_used == "fused_tc"
+                                else "staged path (whole call)"),
                      "algorithmic_bytes_per_launch": by},
         "clocks": clocks.summary(),
         "e2e": {"value": ntok * e2e_steps / (e2e_ms / 1e3),
@@ -955,7 +965,7 @@ def run_gdn2(args, w, kind="gdn2"):
                 "d2h_bytes_per_step": d2h,
                 "entry": f"{entry}, inputs copied from pinned host "
                          "memory and results back each step"},
-        "gpu_launches": launches_per_step("staged", w) * args.steps,
+        "gpu_launches": launches_per_step(algo_used, w) * args.steps,
         "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
     }
     if not args.no_cpu_baseline:

@@ -34,6 +34,16 @@
 //               for the fp16 U product, then K . e^g (for W) and Q . e^g
 //               (for X) in place; the scalar / no gate U and W read the raw
 //               bf16 V and K
+// The channel gate also runs the per-channel gate variants (template GV):
+//   GV = 1  Gated DeltaNet-2: the read key is b . k (erase gate b, per key
+//           channel) and the target w . v (write gate w, per value channel);
+//   GV = 2  FG^2-GDN: the write key is a . k (rate a, per key channel) and
+//           the target (c .) v (FG^2-GDN+'s value scaling c, optional).
+// beta is then 1 (0 past the sequence end, which masks those rows as
+// before).  The prep warps fold b into the M-side key block or a into the
+// write-key tile when they rescale them (one fp32 product, one rounding);
+// the convert warps fold w or c into V when they convert it to fp16.  The
+// TMA producer prefetches each chunk's gate rows into L2 one chunk ahead.
 // Waiting threads ask to be suspended until their phase completes, so that
 // they leave issue slots to the working warps (the MMA thread above all).
 // All state lives in tensor memory as S^T (lane = value channel, column =
@@ -175,6 +185,10 @@ __device__ unsigned g_fused_error;
 
 struct Params {
   const float *beta;
+  // per-channel gate variants (GV != 0): the key-side gate [ntok][H][128]
+  // (erase gate b or rate a) and the value-side gate (write gate w or
+  // scaling c; nullptr for none)
+  const float *gk, *gv;
   const float *log_alpha;
   const float *s0;
   __nv_bfloat16 *out;
@@ -241,6 +255,35 @@ __device__ __forceinline__ void unpack_f16(uint32_t w, float &lo, float &hi) {
   hi = f.y;
 }
 // 8 values in place (16 bytes of shared memory): bf16 -> fp16 times sc
+// 8 values in place (16 bytes of shared memory): bf16 -> fp16 times sc[e]
+__device__ __forceinline__ void bf16_to_f16_16B_each(uint8_t *ptr,
+                                                     const float *sc) {
+  uint4 x = *reinterpret_cast<uint4 *>(ptr);
+  uint32_t *w = reinterpret_cast<uint32_t *>(&x);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
+    float2 f = __bfloat1622float2(b);
+    __half2 hv = __floats2half2_rn(f.x * sc[2 * e], f.y * sc[2 * e + 1]);
+    w[e] = *reinterpret_cast<uint32_t *>(&hv);
+  }
+  *reinterpret_cast<uint4 *>(ptr) = x;
+}
+// 8 consecutive fp32 gate values of row `row` (two 16-byte loads); zeros for
+// a row past the chunk's last token, whose token may lie beyond the tensor
+__device__ __forceinline__ void load_gate8(float *g8, const float *base,
+                                           size_t row, int ch, bool live) {
+  if (live) {
+    const float4 *gp =
+        reinterpret_cast<const float4 *>(base + row * kD + ch);
+    const float4 a = __ldg(gp), b = __ldg(gp + 1);
+    g8[0] = a.x; g8[1] = a.y; g8[2] = a.z; g8[3] = a.w;
+    g8[4] = b.x; g8[5] = b.y; g8[6] = b.z; g8[7] = b.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) g8[e] = 0.f;
+  }
+}
 __device__ __forceinline__ void bf16_to_f16_16B(uint8_t *ptr, float sc) {
   uint4 x = *reinterpret_cast<uint4 *>(ptr);
   uint32_t *w = reinterpret_cast<uint32_t *>(&x);
@@ -347,12 +390,15 @@ __device__ __forceinline__ void store16(float *Y, const float acc[8], float s,
   }
 }
 
-template <int GATE>
+template <int GATE, int GV>
 __global__ void __launch_bounds__(kThreads, 1)
     gdr_fused_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                         const __grid_constant__ CUtensorMap tmk,
                         const __grid_constant__ CUtensorMap tmv,
-                        const __grid_constant__ CUtensorMap tmla, Params p) {
+                        const __grid_constant__ CUtensorMap tmla,
+                        const __grid_constant__ CUtensorMap tmgk,
+                        const __grid_constant__ CUtensorMap tmgv, Params p) {
+  static_assert(GV == 0 || GATE == 2, "gate variants need the channel gate");
   using Lay = Layout<GATE>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-aligned base, derived by pointer arithmetic on the shared array so
@@ -399,6 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_map(&tmk);
       tma_prefetch_map(&tmv);
       if (GATE == 2) tma_prefetch_map(&tmla);
+      if (GV != 0) {
+        tma_prefetch_map(&tmgk);
+        if (p.gv) tma_prefetch_map(&tmgv);
+      }
       int issued = 0, issued_v = 0, issued_la = 0;
       for (int m = 0; m < NC; ++m) {
         const int s = m & 1;
@@ -410,6 +460,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(sm + Lay::LA + kb * 16384, &tmla, &bar[B_LAFULL],
                         kb * 64, h, start + m * kC);
           issued_la = m + 1;
+          // the gate rows of chunk m into L2, a chunk before they are read
+          if (GV != 0) {
+            for (int kb = 0; kb < 2; ++kb) {
+              tma_prefetch_l2_3d(&tmgk, kb * 64, h, start + m * kC);
+              if (p.gv) tma_prefetch_l2_3d(&tmgv, kb * 64, h, start + m * kC);
+            }
+          }
         }
         if (m >= 2 && !wait_bar(cx, B_EMPTY0 + s, ((m - 2) >> 1) & 1)) break;
         const int tok0 = start + m * kC;
@@ -769,9 +826,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int m = 0; m < NC; ++m) {
       if (!group_all(wait_bar(cx, B_FULLV, m & 1), 3, kConv)) break;
       if (GATE == 2) {
+        if (GV != 0 && p.gv) {
+          // V . (write gate or value scaling): item i is row r and the
+          // physical 16-byte chunk i & 7 of block i >> 9, i.e. channels
+          // 64 (i >> 9) + 8 ((i & 7) ^ (r & 7)) .. + 7 (128-B swizzle)
+          const int tok0 = start + m * kC, L = min(kC, end - tok0);
 #pragma unroll 4
-        for (int i = ct; i < 1024; i += kConv)
-          bf16_to_f16_16B(sm + OFF_V + i * 16, 1.f);
+          for (int i = ct; i < 1024; i += kConv) {
+            const int r = (i >> 3) & 63;
+            const int c = (i >> 9) * 64 + (((i & 7) ^ (r & 7)) << 3);
+            float gw[8];
+            load_gate8(gw, p.gv, (size_t)(tok0 + r) * p.H + h, c, r < L);
+            bf16_to_f16_16B_each(sm + OFF_V + i * 16, gw);
+          }
+        } else {
+#pragma unroll 4
+          for (int i = ct; i < 1024; i += kConv)
+            bf16_to_f16_16B(sm + OFF_V + i * 16, 1.f);
+        }
         // once K K^T has read them: K e^{g-g_m}, then Q e^{g-g_m} (bf16)
         // -> K e^g for W (conv), then Q e^g for X (qconv), fp16 in place.
         // Item = row, 8 channels; the 8 factors e^{g_m} are two vector loads.
@@ -837,7 +909,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       na = 0.f;
       const int tok0 = start + m * kC, L = min(kC, end - tok0);
       if (m < NC && pt < L) {
-        nb = p.beta[(size_t)(tok0 + pt) * p.H + h];
+        nb = GV != 0 ? 1.f : p.beta[(size_t)(tok0 + pt) * p.H + h];
         if (GATE == 1) na = p.log_alpha[(size_t)(tok0 + pt) * p.H + h];
       }
     };
@@ -970,6 +1042,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t *qw = reinterpret_cast<uint32_t *>(&qv);
             uint32_t *kw = reinterpret_cast<uint32_t *>(&kv);
             uint32_t *knw = reinterpret_cast<uint32_t *>(&nv);
+            // the key-side gate: erase gate on the read key (GV 1, the
+            // M-side block) or rate on the write key (GV 2, K e^{g_m-g})
+            float gk[8];
+            if (GV != 0)
+              load_gate8(gk, p.gk, (size_t)(tok0 + r) * p.H + h,
+                         kb * 64 + cc * 8, r < L);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float ep0 = __expf(x[2 * e]), ep1 = __expf(x[2 * e + 1]);
@@ -977,14 +1055,25 @@ __global__ void __launch_bounds__(kThreads, 1)
               float q0, q1, k0, k1;
               unpack_bf16(qw[e], q0, q1);
               unpack_bf16(kw[e], k0, k1);
+              float kr0 = k0, kr1 = k1, kn0 = k0, kn1 = k1;
+              if (GV == 1) {
+                kr0 *= gk[2 * e];
+                kr1 *= gk[2 * e + 1];
+              } else if (GV == 2) {
+                kn0 *= gk[2 * e];
+                kn1 *= gk[2 * e + 1];
+              }
               amax = fmaxf(amax, fmaxf(fmaxf(fabsf(q0), fabsf(q1)),
                                        fmaxf(fabsf(k0), fabsf(k1))));
+              if (GV != 0)
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(kr0), fabsf(kr1)),
+                                         fmaxf(fabsf(kn0), fabsf(kn1))));
               qw[e] = kH ? pack_f16(q0 * ep0, q1 * ep1)
                          : pack_bf16(q0 * ep0, q1 * ep1);
-              kw[e] = kH ? pack_f16(k0 * ep0, k1 * ep1)
-                         : pack_bf16(k0 * ep0, k1 * ep1);
-              knw[e] = kH ? pack_f16(k0 * en0, k1 * en1)
-                          : pack_bf16(k0 * en0, k1 * en1);
+              kw[e] = kH ? pack_f16(kr0 * ep0, kr1 * ep1)
+                         : pack_bf16(kr0 * ep0, kr1 * ep1);
+              knw[e] = kH ? pack_f16(kn0 * en0, kn1 * en1)
+                          : pack_bf16(kn0 * en0, kn1 * en1);
             }
             *qp = qv;
             *kp = kv;
@@ -1376,9 +1465,10 @@ bool make_map(CUtensorMap *map, const void *base, int ntok, int H,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int GATE>
-cudaError_t launch(const Problem &pr, cudaStream_t s) {
-  CUtensorMap mq, mk, mv, mla;
+template <int GATE, int GV>
+cudaError_t launch(const Problem &pr, const float *gk, const float *gv,
+                   cudaStream_t s) {
+  CUtensorMap mq, mk, mv, mla, mgk, mgv;
   if (!make_map(&mq, pr.q, pr.ntok, pr.H) || !make_map(&mk, pr.k, pr.ntok, pr.H) ||
       !make_map(&mv, pr.v, pr.ntok, pr.H))
     return cudaErrorInvalidValue;
@@ -1386,8 +1476,17 @@ cudaError_t launch(const Problem &pr, cudaStream_t s) {
   if (GATE == 2 ? !make_map(&mla, pr.log_alpha, pr.ntok, pr.H, true)
                 : !make_map(&mla, pr.q, pr.ntok, pr.H))
     return cudaErrorInvalidValue;
+  // the gate variants' gate tensors (fp32, the layout of the log-decays);
+  // a map the kernel never reads describes q
+  if (!(GV != 0 ? make_map(&mgk, gk, pr.ntok, pr.H, true)
+                : make_map(&mgk, pr.q, pr.ntok, pr.H)) ||
+      !(GV != 0 && gv ? make_map(&mgv, gv, pr.ntok, pr.H, true)
+                      : make_map(&mgv, pr.q, pr.ntok, pr.H)))
+    return cudaErrorInvalidValue;
   Params p;
   p.beta = pr.beta;
+  p.gk = gk;
+  p.gv = gv;
   p.log_alpha = pr.log_alpha;
   p.s0 = pr.s0;
   p.out = static_cast<__nv_bfloat16 *>(pr.out);
@@ -1399,26 +1498,31 @@ cudaError_t launch(const Problem &pr, cudaStream_t s) {
   p.H = pr.H;
   const int smem = Layout<GATE>::BYTES + 1024;
   cudaError_t e = cudaFuncSetAttribute(
-      gdr_fused_tc_kernel<GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-      smem);
+      gdr_fused_tc_kernel<GATE, GV>,
+      cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  gdr_fused_tc_kernel<GATE><<<pr.nseq * pr.H, kThreads, smem, s>>>(mq, mk, mv, mla,
-                                                                 p);
+  gdr_fused_tc_kernel<GATE, GV><<<pr.nseq * pr.H, kThreads, smem, s>>>(
+      mq, mk, mv, mla, mgk, mgv, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool fused_tc_applies(const Problem &p) {
+  // the per-channel gate variants run with the channel-wise decay only
+  const bool variant = p.erase || p.write || p.wkey;
   return p.dtype == GDR_BF16 && p.dk == kD && p.dv == kD && p.chunk == kC &&
-         (long long)p.nseq * p.H < (1ll << 31);
+         (long long)p.nseq * p.H < (1ll << 31) &&
+         (!variant || p.gate == GDR_GATE_CHANNEL);
 }
 
 cudaError_t fused_tc_run(const Problem &p, cudaStream_t s) {
+  if (p.erase) return launch<2, 1>(p, p.erase, p.write, s);
+  if (p.wkey) return launch<2, 2>(p, p.wkey, p.write, s);
   switch (p.gate) {
-    case GDR_GATE_NONE: return launch<0>(p, s);
-    case GDR_GATE_SCALAR: return launch<1>(p, s);
-    default: return launch<2>(p, s);
+    case GDR_GATE_NONE: return launch<0, 0>(p, nullptr, nullptr, s);
+    case GDR_GATE_SCALAR: return launch<1, 0>(p, nullptr, nullptr, s);
+    default: return launch<2, 0>(p, nullptr, nullptr, s);
   }
 }
 

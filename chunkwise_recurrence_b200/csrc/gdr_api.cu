@@ -119,10 +119,9 @@ gdr_status scratch_alloc(void **ptr, size_t bytes, cudaStream_t s) {
 
 gdr_status run(const Problem &p, gdr_algo algo, cudaStream_t stream) {
   if (p.nseq == 0 || p.H == 0) return GDR_OK;
-  // the Gated DeltaNet-2 gates and FG^2-GDN's rate run on the staged path
-  // only
-  const bool tc = p.erase == nullptr && p.write == nullptr &&
-                  p.wkey == nullptr && gdr::fused_tc_applies(p);
+  // (the Gated DeltaNet-2 gates and FG^2-GDN's rate run on the fused path
+  // with the channel-wise decay only: fused_tc_applies)
+  const bool tc = gdr::fused_tc_applies(p);
   if (algo == GDR_ALGO_FUSED_TC && !tc) return GDR_ERR_UNSUPPORTED;
   if (tc && algo != GDR_ALGO_STAGED) {
     cudaError_t e = gdr::fused_tc_run(p, stream);
@@ -167,7 +166,6 @@ extern "C" gdr_status gdr_chunk_fwd_gdn2(const void *q, const void *k,
                                          cudaStream_t stream,
                                          const gdr_opts *opts) {
   const gdr_opts o = opts ? *opts : default_opts();
-  if (o.algo == GDR_ALGO_FUSED_TC) return GDR_ERR_UNSUPPORTED;
   Problem p;
   // the erase gate stands in for beta in the common checks (presence,
   // alignment); the write gate is checked here
@@ -179,7 +177,7 @@ extern "C" gdr_status gdr_chunk_fwd_gdn2(const void *q, const void *k,
   p.beta = nullptr;
   p.erase = erase_gate;
   p.write = write_gate;
-  return run(p, GDR_ALGO_STAGED, stream);
+  return run(p, o.algo, stream);
 }
 
 // FG^2-GDN's per-key-channel rate on the write key (and FG^2-GDN+'s
@@ -194,7 +192,6 @@ extern "C" gdr_status gdr_chunk_fwd_fg2(const void *q, const void *k,
                                         cudaStream_t stream,
                                         const gdr_opts *opts) {
   const gdr_opts o = opts ? *opts : default_opts();
-  if (o.algo == GDR_ALGO_FUSED_TC) return GDR_ERR_UNSUPPORTED;
   Problem p;
   // the key-side rate stands in for beta in the common checks (presence,
   // alignment); the optional value-side scaling is checked here
@@ -206,7 +203,7 @@ extern "C" gdr_status gdr_chunk_fwd_fg2(const void *q, const void *k,
   p.beta = nullptr;
   p.wkey = beta_k;
   p.write = beta_v;
-  return run(p, GDR_ALGO_STAGED, stream);
+  return run(p, o.algo, stream);
 }
 
 // ---------------------------------------------------------------------------

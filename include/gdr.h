@@ -210,10 +210,14 @@ GDR_API gdr_status gdr_chunk_fwd_host(const void *q, const void *k, const void *
  *   erase_gate  [B][T][H][dk] fp32 (device, 16-byte aligned), required;
  *   write_gate  [B][T][H][dv] fp32 (device, 16-byte aligned), required;
  * (packed layouts with cu_seqlens as for gdr_chunk_fwd).  The decay form is
- * opts->gate (NONE, SCALAR or CHANNEL) as before.  Runs the staged path
- * (fp32 CUDA-core arithmetic, any supported shape): opts->algo AUTO or
- * STAGED; FUSED_TC returns GDR_ERR_UNSUPPORTED.  Status codes as for
- * gdr_chunk_fwd.
+ * opts->gate (NONE, SCALAR or CHANNEL) as before.  Paths as for
+ * gdr_chunk_fwd, except that the fused tensor-core kernel takes these gates
+ * with the channel-wise decay (CHANNEL, bf16, dk = dv = 128, chunk = 64)
+ * only: AUTO runs it there and the staged path (fp32 CUDA-core arithmetic)
+ * everywhere else; FUSED_TC on another decay form returns
+ * GDR_ERR_UNSUPPORTED.  On the fused path b . k and w . v are formed in
+ * fp32 and rounded once to the fp16 operands.  Status codes as for
+ * gdr_chunk_fwd (GDR_ERR_RANGE from the fused path as there).
  */
 GDR_API gdr_status gdr_chunk_fwd_gdn2(const void *q, const void *k,
                                       const void *v, const float *log_alpha,
@@ -247,9 +251,11 @@ GDR_API gdr_status gdr_chunk_fwd_gdn2(const void *q, const void *k,
  *   beta_v  [B][T][H][dv] fp32 (device, 16-byte aligned), or NULL for
  *           FG^2-GDN (c = 1): FG^2-GDN+'s per-value-channel scaling;
  * (packed layouts with cu_seqlens as for gdr_chunk_fwd).  The decay form is
- * opts->gate (NONE, SCALAR or CHANNEL).  Runs the staged path (fp32
- * CUDA-core arithmetic, any supported shape): opts->algo AUTO or STAGED;
- * FUSED_TC returns GDR_ERR_UNSUPPORTED.  Status codes as for gdr_chunk_fwd.
+ * opts->gate (NONE, SCALAR or CHANNEL).  Paths as for gdr_chunk_fwd_gdn2:
+ * the fused tensor-core kernel with the channel-wise decay (bf16,
+ * dk = dv = 128, chunk = 64), where it forms beta_k . k and c . v in fp32
+ * and rounds them once to its fp16 operands; the staged path otherwise.
+ * Status codes as for gdr_chunk_fwd.
  */
 GDR_API gdr_status gdr_chunk_fwd_fg2(const void *q, const void *k,
                                      const void *v, const float *log_alpha,

@@ -104,8 +104,8 @@ def test_fg2_with_a_uniform_rate_is_the_delta_rule():
     assert rel_err(o2.cpu().numpy(), o1.cpu().numpy()) <= 1e-5
 
 
-def test_fg2_fused_algo_is_unsupported():
-    w = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(B=1, T=64, H=1)
+def test_fg2_fused_algo_needs_the_channel_decay():
+    w = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=1, T=64, H=1)
     inp = generate(w, seed=55)
     beta_k, _ = fg2_gates(inp, seed=55)
     with pytest.raises(gdr.GdrError):

@@ -86,8 +86,8 @@ def test_gdn2_with_gates_equal_to_beta_is_the_delta_rule():
     assert rel_err(o2.cpu().numpy(), o1.cpu().numpy()) <= 1e-5
 
 
-def test_gdn2_fused_algo_is_unsupported():
-    w = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(B=1, T=64, H=1)
+def test_gdn2_fused_algo_needs_the_channel_decay():
+    w = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=1, T=64, H=1)
     inp = generate(w, seed=44)
     erase, write = gdn2_gates(inp, seed=44)
     with pytest.raises(gdr.GdrError):
