@@ -740,9 +740,21 @@ def run_decode(args):
 
 BACKWARD_METRIC = ("tokens/s, backward pass (gdr_backward) of the chunked "
                    "gated-delta fwd; % fp32 ALU roofline")
-# fp32 flops per state element, token and head over the backward's three
-# sweeps: forward and replay 5 each (decay, S~^T k, k u^T), reverse 19
+# reverse token recurrence: fp32 flops per state element, token and head over
+# its three sweeps: forward and replay 5 each (decay, S~^T k, k u^T), reverse 19
 BACKWARD_FLOPS_PER_ELEM = 29
+
+
+def chunked_backward_flops_per_chunk(dk, dv, C=64):
+    """fp32 flops of one (chunk, head) of the chunked backward, from its
+    products (multiply-adds x 2): 9 C dk dv (W S and the state update in the
+    forward scan; Kc Lambda, Qd^T dO, W^T dV_new in the reverse scan;
+    (K e^g) S and the three slice products dO S^T, Z S^T, V_new Lambda^T in
+    the gradient kernel), C^2 (7 dk + 4.5 dv) (A, W, U in the WY kernel; P;
+    P^T dO; Z, dT, dP; M and the four key/query products of A and P) and
+    2.17 C^3 (the inverse, T^T dT, dA)."""
+    return 2 * (9 * C * dk * dv + C * C * (7 * dk + 4.5 * dv)
+                + 2.17 * C ** 3)
 
 
 def run_backward(args, w):
@@ -768,9 +780,13 @@ def run_backward(args, w):
                                              inp.cu_seqlens))
     stream = torch.cuda.current_stream(dev)
 
+    # --algo staged: the chunked backward; auto / recurrent: the reverse
+    # token recurrence (what gdr_backward's AUTO runs)
+    algo = "staged" if args.algo == "staged" else "recurrent"
+
     def step():
         return gdr.backward(q, k, v, b, la, s0, dO, dS, gate=w.gate,
-                            cu_seqlens=cu, stream=stream)
+                            cu_seqlens=cu, stream=stream, algo=algo)
 
     for _ in range(args.warmup):
         step()
@@ -800,29 +816,39 @@ def run_backward(args, w):
     max_mhz = clk.get("sm_max_mhz") or 1965.0
     # CUDA-core fp32 peak: SMs x 128 lanes x 2 flops (FMA) x max SM clock
     alu_peak = sms * 128 * 2 * max_mhz * 1e6 / 1e12
-    tflops = (BACKWARD_FLOPS_PER_ELEM * dk * dv * ntok * H /
-              (statistics.mean(per_step) / 1e3) / 1e12)
+    if algo == "recurrent":
+        flops = BACKWARD_FLOPS_PER_ELEM * dk * dv * ntok * H
+        kernel = "gdr_bwd_cols_kernel" if cols else "gdr_bwd_kernel"
+        launches = 2 if cols else 1
+        algo_name = "reverse token recurrence"
+    else:
+        nchunks = sum((n + 63) // 64 for n in inp.lengths)
+        flops = chunked_backward_flops_per_chunk(dk, dv) * nchunks * H
+        kernel = ("chunked backward, whole call (WY, P, forward scan, "
+                  "reverse scan, gradient kernels)")
+        # chunk table, cumsum (with a gate), WY, P, two scans, gradients
+        launches = 6 + (0 if w.gate == "none" else 1)
+        algo_name = "chunked (64-token chunks, fp32)"
+    tflops = flops / (statistics.mean(per_step) / 1e3) / 1e12
     line = {
         "metric": BACKWARD_METRIC, "value": ntok / (ms / 1e3),
         "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic",
-        "config": {**workload_config(w, inp), "algo": "token-level reverse",
+        "config": {**workload_config(w, inp), "algo": algo_name,
                    "l2": "inputs larger than L2 (no flush)"},
         "roofline": {"bound": "alu", "achieved": tflops, "peak": alu_peak,
                      "unit": "TFLOP/s", "frac": tflops / alu_peak,
                      "traffic": None,
                      "peak_source": f"derived: {sms} SMs x 128 fp32 lanes x 2 "
                                     f"x {max_mhz:.0f} MHz",
-                     "kernel": ("gdr_bwd_cols_kernel" if cols
-                                else "gdr_bwd_kernel"),
-                     "flops_per_step": BACKWARD_FLOPS_PER_ELEM * dk * dv *
-                     ntok * H,
+                     "kernel": kernel,
+                     "flops_per_step": flops,
                      "hbm_gbs_on_algorithmic_bytes": gbs,
                      "algorithmic_bytes_per_launch": by},
         "clocks": clk,
-        "gpu_launches": args.steps * (2 if cols else 1),
+        "gpu_launches": args.steps * launches,
         "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
     }
     print(json.dumps(line), flush=True)
@@ -1009,7 +1035,9 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS))
     ap.add_argument("--algo", default="auto",
-                    choices=["auto", "staged", "fused_tc"])
+                    choices=["auto", "staged", "fused_tc", "recurrent"],
+                    help="with --backward: staged = the chunked backward, "
+                         "recurrent (or auto) = the reverse token recurrence")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seqs", type=int, default=4,
                     help="sequences in the CPU-baseline sample")
@@ -1077,6 +1105,8 @@ def main(argv=None):
         if w.varlen_nseq or args.batch < 1:
             raise SystemExit("--batch needs a fixed-length workload and B >= 1")
         w = w.with_(B=args.batch, name=f"{w.name}@B{args.batch}")
+    if args.algo == "recurrent" and not args.backward:
+        raise SystemExit("--algo recurrent is a backward algorithm")
     if args.fg2 and (args.decode or args.backward):
         raise SystemExit("--fg2 times the chunked forward pass only")
     if args.decode and args.impl == "ours":

@@ -27,7 +27,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdr.so")
 
 GATES = {"none": 0, "scalar": 1, "channel": 2}
-ALGOS = {"auto": 0, "staged": 1, "fused_tc": 2}
+ALGOS = {"auto": 0, "staged": 1, "fused_tc": 2, "recurrent": 3}
 DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARGUMENT", 2: "GDR_ERR_UNSUPPORTED",
           3: "GDR_ERR_CUDA", 4: "GDR_ERR_OUT_OF_MEMORY", 5: "GDR_ERR_TIMEOUT",
@@ -412,11 +412,14 @@ def _decode_two_gates(name, q, k, v, gate_k, gate_v, log_alpha, state, out,
 
 def backward(q, k, v, beta, log_alpha, initial_state, d_out, d_final_state=None,
              *, gate: str | None = None, cu_seqlens=None,
-             need_initial_state_grad: bool = True, stream=None):
+             need_initial_state_grad: bool = True, algo: str = "auto",
+             stream=None):
     """Run ``gdr_backward``: gradients of the forward pass (same inputs as
     ``chunk_fwd``) given dL/d out and, optionally, dL/d final_state.
-    Returns a dict of fp32 CUDA tensors dq, dk, dv, dbeta, dlog_alpha (None
-    without a gate) and dinitial_state (None unless requested)."""
+    ``algo``: "staged" (the chunked backward) or "recurrent" / "auto" (the
+    reverse token recurrence).  Returns a dict of fp32 CUDA tensors dq, dk,
+    dv, dbeta, dlog_alpha (None without a gate) and dinitial_state (None
+    unless requested)."""
     lib = load_library()
     B, T, H, dk, dv, nseq = _shapes(q, v, cu_seqlens)
     g = _gate_of(log_alpha, gate)
@@ -428,7 +431,7 @@ def backward(q, k, v, beta, log_alpha, initial_state, d_out, d_final_state=None,
            if need_initial_state_grad else None)
     opts = _Opts(DTYPES[q.dtype], GATES[g],
                  None if cu_seqlens is None else cu_seqlens.data_ptr(),
-                 nseq if cu_seqlens is not None else 0, ALGOS["auto"])
+                 nseq if cu_seqlens is not None else 0, ALGOS[algo])
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     rc = lib.gdr_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),

@@ -48,8 +48,10 @@ gdr_status validate(const void *q, const void *k, const void *v,
       o.gate != GDR_GATE_CHANNEL)
     return GDR_ERR_INVALID_ARGUMENT;
   if (o.algo != GDR_ALGO_AUTO && o.algo != GDR_ALGO_STAGED &&
-      o.algo != GDR_ALGO_FUSED_TC)
+      o.algo != GDR_ALGO_FUSED_TC && o.algo != GDR_ALGO_RECURRENT)
     return GDR_ERR_INVALID_ARGUMENT;
+  // the reverse token recurrence is a backward algorithm only
+  if (o.algo == GDR_ALGO_RECURRENT) return GDR_ERR_UNSUPPORTED;
   if (!pow2_in(dk, 16, 128) || !pow2_in(dv, 16, 128) ||
       !pow2_in(chunk, 16, 64))
     return GDR_ERR_UNSUPPORTED;
@@ -826,12 +828,16 @@ extern "C" gdr_status gdr_backward(
     float *d_log_alpha, float *d_beta, float *d_initial_state, int B, int T,
     int H, int dk_, int dv_, cudaStream_t stream, const gdr_opts *opts) {
   const gdr_opts o = opts ? *opts : default_opts();
-  if (o.algo != GDR_ALGO_AUTO) return GDR_ERR_UNSUPPORTED;
+  if (o.algo == GDR_ALGO_FUSED_TC) return GDR_ERR_UNSUPPORTED;
+  const bool recurrent = o.algo == GDR_ALGO_RECURRENT;
+  gdr_opts ov = o;
+  if (recurrent) ov.algo = GDR_ALGO_AUTO;
   Problem p;
   // the forward pass's checks, with d_out in the place of out and
-  // d_final_state in the place of final_state (chunk plays no part here)
+  // d_final_state in the place of final_state (the chunked backward runs
+  // chunks of 64 tokens whatever the forward used)
   gdr_status st = validate(q, k, v, log_alpha, beta, initial_state, d_out,
-                           d_final_state, B, T, H, dk_, dv_, 64, o, &p);
+                           d_final_state, B, T, H, dk_, dv_, 64, ov, &p);
   if (st != GDR_OK) return st;
   if (p.nseq == 0 || p.H == 0) return GDR_OK;
   if (!dq || !dk || !dv || !d_beta) return GDR_ERR_INVALID_ARGUMENT;
@@ -840,8 +846,13 @@ extern "C" gdr_status gdr_backward(
   const void *grads[] = {dq, dk, dv, d_log_alpha, d_beta, d_initial_state};
   for (const void *ptr : grads)
     if (ptr && !aligned16(ptr)) return GDR_ERR_INVALID_ARGUMENT;
+  // AUTO takes the reverse token recurrence, which is the faster of the two
+  // on every measured shape so far; STAGED names the chunked backward
+  const bool chunked = o.algo == GDR_ALGO_STAGED &&
+                       gdr::backward_chunked_applies(p);
   long long total_win = 0;
-  const size_t bytes = gdr::backward_scratch_bytes(p, &total_win);
+  const size_t bytes = chunked ? gdr::backward_chunked_bytes(p)
+                               : gdr::backward_scratch_bytes(p, &total_win);
   // the scratch comes from the library's per-device pool, which keeps its
   // memory between calls (hundreds of MB at training sizes: mapping it anew
   // every call would cost more than the copies it saves)
@@ -867,8 +878,10 @@ extern "C" gdr_status gdr_backward(
   io.dla = d_log_alpha;
   io.dbeta = d_beta;
   io.ds0 = d_initial_state;
-  cudaError_t e = gdr::backward_run(p, io, static_cast<float *>(ws), total_win,
-                                    stream);
+  cudaError_t e =
+      chunked ? gdr::backward_chunked_run(p, io, ws, stream)
+              : gdr::backward_run(p, io, static_cast<float *>(ws), total_win,
+                                  stream);
   cudaError_t f = cudaFreeAsync(ws, stream);
   return (e == cudaSuccess && f == cudaSuccess) ? GDR_OK : GDR_ERR_CUDA;
 }

@@ -47,6 +47,21 @@ struct Problem {
 // Staged path: four kernels + a chunk-table kernel, fp32 CUDA-core math.
 size_t staged_workspace_bytes(const Problem &p);
 cudaError_t staged_run(const Problem &p, void *workspace, cudaStream_t s);
+// The staged path's scratch regions inside a workspace of
+// staged_workspace_bytes(p) bytes: the chunk table, per-sequence first chunk
+// (nseq + 1 entries; the last is the chunk count), in-chunk cumulative
+// log-decays g [ntok][H][gdim], W [ntok][H][dk], U and V_new [ntok][H][dv],
+// chunk-start states [max_chunks][H][dk][dv].
+struct StagedBufs {
+  ChunkInfo *table;
+  int *seq_first, *nchunks;
+  float *g, *W, *U, *Vn, *Sbuf;
+};
+StagedBufs staged_bufs(const Problem &p, void *workspace);
+// The chunk table, g, W and U (and T [max_chunks][H][C][C] into Tout when
+// not nullptr) of every (chunk, head); no state pass, no output.
+cudaError_t staged_wy_run(const Problem &p, void *workspace, float *Tout,
+                          cudaStream_t s);
 
 // Fused tensor-core path.
 bool fused_tc_applies(const Problem &p);
@@ -78,6 +93,13 @@ struct BackwardIO {
   float *dbeta;          // fp32 [ntok][H]
   float *ds0;            // fp32 [N][H][dk][dv], or nullptr
 };
+// Chunked backward pass (csrc/backward_chunked.cu): the gradients of the
+// chunked forward product by product, fp32, chunk-parallel except for one
+// forward and one reverse scan over the chunk boundaries.  p.chunk must be 64.
+bool backward_chunked_applies(const Problem &p);
+size_t backward_chunked_bytes(const Problem &p);
+cudaError_t backward_chunked_run(const Problem &p, const BackwardIO &io,
+                                 void *workspace, cudaStream_t s);
 // Scratch the backward pass needs (bytes); *total_win = the number of
 // checkpoint windows per head, to pass on to backward_run.
 size_t backward_scratch_bytes(const Problem &p, long long *total_win);

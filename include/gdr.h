@@ -109,7 +109,10 @@ typedef enum {
    * accurate (up to about 3e-2 at mean log-decays of -1 to -2 per token and
    * channel), and the call reports GDR_ERR_RANGE through gdr_device_error:
    * run such inputs with GDR_ALGO_STAGED, fp32 throughout. */
-  GDR_ALGO_FUSED_TC = 2
+  GDR_ALGO_FUSED_TC = 2,
+  /* gdr_backward only: the reverse token recurrence (see there); every
+   * forward entry returns GDR_ERR_UNSUPPORTED for it. */
+  GDR_ALGO_RECURRENT = 3
 } gdr_algo;
 
 typedef struct {
@@ -443,26 +446,43 @@ GDR_API gdr_status gdr_decode_step_fg2(const void *q, const void *k,
  * Given the forward inputs and the upstream gradients dL/d out and
  * dL/d final_state, it writes dL/dq, dL/dk, dL/dv, dL/d log_alpha,
  * dL/d beta and dL/d initial_state of the recurrence above (the same
- * definition gdr_chunk_fwd evaluates, whichever algorithm ran it).  It
- * runs the recurrence forward, checkpointing the state every 8 tokens in
- * scratch (16 when dk or dv is 16), then the reverse token recurrence window
- * by window, all in fp32.  For dk, dv >= 32 each (sequence, head) runs on
- * dv/32 blocks of 32 value columns; their per-token shares of the row sums
- * (dq, dk, d_log_alpha, d_beta) are added in a fixed order, so the result
- * does not depend on scheduling.
+ * definition gdr_chunk_fwd evaluates, whichever algorithm ran it), all in
+ * fp32.  Two algorithms (AUTO runs the recurrent one, the faster on every
+ * shape measured so far):
+ *  - STAGED: the chunked backward.  The gradients of the chunkwise
+ *    (WY) forward, taken product by product over chunks of 64 tokens: the
+ *    staged path's per-chunk W, U and T, a forward scan over the chunk
+ *    boundaries for the chunk-start states, a reverse scan for dL/dS at
+ *    every chunk end, then every chunk's input gradients in parallel
+ *    (register-blocked fp32 products on CUDA cores).  The update being
+ *    affine in the preceding memory ("DeltaTTT" page, §2 Background) is
+ *    what makes the two scans exact.  Deterministic except for the order in
+ *    which a chunk's per-channel shares of the decay gradient are added.
+ *  - RECURRENT (and AUTO): the reverse token recurrence.  It runs the
+ *    recurrence
+ *    forward, checkpointing the state every 8 tokens in scratch (16 when dk
+ *    or dv is 16), then the reverse token recurrence window by window.  For
+ *    dk, dv >= 32 each (sequence, head) runs on dv/32 blocks of 32 value
+ *    columns; their per-token shares of the row sums (dq, dk, d_log_alpha,
+ *    d_beta) are added in a fixed order, so the result does not depend on
+ *    scheduling.
+ * FUSED_TC returns GDR_ERR_UNSUPPORTED.
  *
  * Inputs: q, k, v, log_alpha, beta, initial_state, B, T, H, dk, dv and opts
- * exactly as for gdr_chunk_fwd (opts->algo must be GDR_ALGO_AUTO);
+ * exactly as for gdr_chunk_fwd (opts->algo AUTO, STAGED or RECURRENT);
  *   d_out          layout and dtype of out (device), required;
  *   d_final_state  [N][H][dk][dv] fp32, or NULL for a zero gradient.
  * Outputs (device, fp32, 16-byte aligned, written):
  *   dq, dk         [B][T][H][dk];   dv [B][T][H][dv];   d_beta [B][T][H];
  *   d_log_alpha    the layout of log_alpha; NULL iff gate is NONE;
  *   d_initial_state [N][H][dk][dv], or NULL to skip.
- * Scratch (dk, dv >= 32): (ntok/8 + N) * H + 8 * N * H states of dk*dv
- * floats, plus the row-sum shares, 2 * (dv/32) * ntok * H * dk floats (3 *
- * for the channel gate); for dk or dv = 16: (ntok/16 + N) * H + 16 * N * H
- * states.  Allocated stream-ordered on `stream` from the library's per-device memory
+ * Scratch, chunked: the staged path's (about (2 dk + 2 dv) ntok H floats
+ * plus one state per chunk and head), T and P of every chunk (2 * 64 * 64
+ * floats per chunk and head), one more state per chunk and head, and
+ * ntok * H * dv floats.  Recurrent (dk, dv >= 32): (ntok/8 + N) * H + 8 * N
+ * * H states of dk*dv floats, plus the row-sum shares, 2 * (dv/32) * ntok *
+ * H * dk floats (3 * for the channel gate); for dk or dv = 16: (ntok/16 +
+ * N) * H + 16 * N * H states.  Allocated stream-ordered on `stream` from the library's per-device memory
  * pool, which keeps its memory between calls (the pool gdr_chunk_fwd_host
  * uses); GDR_ERR_OUT_OF_MEMORY on failure.
  * Status codes as for gdr_chunk_fwd.

@@ -194,7 +194,9 @@ def test_backward_rejects_bad_arguments(lib):
     assert c(gate=0, la=None) == INVALID  # ... and no gate forbids it
     assert c(dk=A + 4) == INVALID        # misaligned
     assert c(ds0=A + 8) == INVALID
-    assert c(algo=1) == UNSUPPORTED
+    assert c(algo=2) == UNSUPPORTED      # no fused backward
+    assert c(algo=4) == INVALID          # not an algorithm
+    assert c(algo=3, dk_=48) == UNSUPPORTED
     assert c(dk_=48) == UNSUPPORTED
     assert c(T=-1) == INVALID
     assert c(q=None, k=None, v=None, la=None, beta=None, dout=None, dq=None,

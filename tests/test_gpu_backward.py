@@ -1,11 +1,12 @@
 """GPU parity of the backward pass (gdr_backward, through the C ABI) against
 fp64 autograd gradients of the token loop (oracle.gdr_grads, itself pinned by
-finite differences of the C oracle).
+finite differences of the C oracle), for both algorithms: the chunked
+backward (STAGED) and the reverse token recurrence (RECURRENT, which AUTO
+runs).
 
-Tolerance: the kernel computes in fp32 (no operand rounding) over a reverse
-recurrence of T tokens; every gradient tensor must satisfy
-max |gpu - oracle| / RMS(oracle) <= 1e-3 (fp32 accumulation over a few hundred
-dependent steps stays two orders of magnitude below that)."""
+Tolerance: both compute in fp32 (no operand rounding); every gradient tensor
+must satisfy max |gpu - oracle| / RMS(oracle) <= 1e-3 (fp32 accumulation over
+a few hundred dependent steps stays two orders of magnitude below that)."""
 import numpy as np
 import pytest
 import torch
@@ -19,7 +20,7 @@ pytestmark = pytest.mark.gpu
 TOL = 1e-3
 
 
-def _check(w, seed=0, with_final=True, with_s0_grad=True):
+def _check(w, seed=0, with_final=True, with_s0_grad=True, algo="auto"):
     inp = generate(w, seed=seed)
     g = torch.Generator().manual_seed(seed + 100)
     dO = torch.randn(inp.v.shape, generator=g).to(inp.v.dtype)
@@ -30,7 +31,7 @@ def _check(w, seed=0, with_final=True, with_s0_grad=True):
     res = gdr.backward(c(inp.q), c(inp.k), c(inp.v), c(inp.beta),
                        c(inp.log_alpha), c(inp.s0), c(dO), c(dS), gate=w.gate,
                        cu_seqlens=c(inp.cu_seqlens),
-                       need_initial_state_grad=with_s0_grad)
+                       need_initial_state_grad=with_s0_grad, algo=algo)
     torch.cuda.synchronize()
     f = inp.f64()
     ref = oracle.gdr_grads(f["q"], f["k"], f["v"], f["beta"], f["log_alpha"],
@@ -68,16 +69,46 @@ def _check(w, seed=0, with_final=True, with_s0_grad=True):
                                         dtype="fp32")),
     ("deltanet_b1_h1_t256_d16_fp32", dict(T=45, H=3, dk=32, dv=128)),
 ])
-def test_backward_matches_autograd(name, shape):
-    _check(WORKLOADS[name].with_(**shape))
+@pytest.mark.parametrize("algo", ["staged", "recurrent"])
+def test_backward_matches_autograd(name, shape, algo):
+    _check(WORKLOADS[name].with_(**shape), algo=algo)
 
 
-def test_backward_varlen_and_optional_gradients():
+@pytest.mark.parametrize("algo", ["staged", "recurrent"])
+def test_backward_varlen_and_optional_gradients(algo):
     w = WORKLOADS["gdn_varlen8_h16_d128_bf16"].with_(
         varlen_nseq=3, varlen_lo=5, varlen_hi=40, H=2, dk=32, dv=32)
-    _check(w, with_final=False, with_s0_grad=True)
+    _check(w, with_final=False, with_s0_grad=True, algo=algo)
     w2 = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=1, T=20, H=1)
-    _check(w2, with_final=True, with_s0_grad=False)
+    _check(w2, with_final=True, with_s0_grad=False, algo=algo)
+
+
+@pytest.mark.parametrize("gate", ["none", "scalar", "channel"])
+@pytest.mark.parametrize("dtype,dk,dv", [("bf16", 128, 128), ("fp32", 64, 32),
+                                         ("bf16", 16, 64)])
+def test_chunked_backward_several_chunks(gate, dtype, dk, dv):
+    """Several 64-token chunks and a ragged last one: the chunk-boundary
+    scans carry the state forward and its gradient backward."""
+    w = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(
+        B=2, T=3 * 64 + 17, H=2, dk=dk, dv=dv, dtype=dtype, gate=gate,
+        init_state=True)
+    _check(w, seed=3, algo="staged")
+
+
+def test_chunked_backward_varlen_many_sequences():
+    w = WORKLOADS["gdn_varlen8_h16_d128_bf16"].with_(
+        varlen_nseq=5, varlen_lo=1, varlen_hi=300, H=2, gate="channel")
+    _check(w, seed=4, algo="staged")
+
+
+@pytest.mark.parametrize("decay", [0.3, 3.0])
+def test_chunked_backward_strong_channel_decay(decay):
+    """Mean log-decays of -0.3 and -3 per token and channel: the second puts
+    a chunk's spread beyond the factored range, so the gradient kernel takes
+    its one-exponential-per-element path (and P too)."""
+    w = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(
+        B=1, T=2 * 64 + 9, H=2, decay_lo=decay, decay_hi=decay)
+    _check(w, seed=5, algo="staged")
 
 
 def test_backward_headline_shape_sampled():
@@ -85,5 +116,6 @@ def test_backward_headline_shape_sampled():
     (T = 4096, d = 128) on one sequence and two heads: 4096 dependent reverse
     steps, compared with autograd in full."""
     w = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=1, H=2)
-    errs = _check(w)
-    assert max(errs.values()) <= TOL
+    for algo in ("staged", "recurrent"):
+        errs = _check(w, algo=algo)
+        assert max(errs.values()) <= TOL
