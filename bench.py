@@ -780,9 +780,9 @@ def run_backward(args, w):
                                              inp.cu_seqlens))
     stream = torch.cuda.current_stream(dev)
 
-    # --algo staged: the chunked backward; auto / recurrent: the reverse
-    # token recurrence (what gdr_backward's AUTO runs)
-    algo = "staged" if args.algo == "staged" else "recurrent"
+    # --algo auto / staged: the chunked backward (gdr_backward's AUTO);
+    # recurrent: the reverse token recurrence
+    algo = "recurrent" if args.algo == "recurrent" else "auto"
 
     def step():
         return gdr.backward(q, k, v, b, la, s0, dO, dS, gate=w.gate,
@@ -824,10 +824,11 @@ def run_backward(args, w):
     else:
         nchunks = sum((n + 63) // 64 for n in inp.lengths)
         flops = chunked_backward_flops_per_chunk(dk, dv) * nchunks * H
-        kernel = ("chunked backward, whole call (WY, P, forward scan, "
-                  "reverse scan, gradient kernels)")
-        # chunk table, cumsum (with a gate), WY, P, two scans, gradients
-        launches = 6 + (0 if w.gate == "none" else 1)
+        kernel = ("chunked backward, whole call (WY, state maps, two "
+                  "scans, V_new, gradient kernels)")
+        # chunk table, cumsum (with a gate), WY, prep, two scans, V_new,
+        # gradients
+        launches = 7 + (0 if w.gate == "none" else 1)
         algo_name = "chunked (64-token chunks, fp32)"
     tflops = flops / (statistics.mean(per_step) / 1e3) / 1e12
     line = {
@@ -1036,8 +1037,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS))
     ap.add_argument("--algo", default="auto",
                     choices=["auto", "staged", "fused_tc", "recurrent"],
-                    help="with --backward: staged = the chunked backward, "
-                         "recurrent (or auto) = the reverse token recurrence")
+                    help="with --backward: auto / staged = the chunked "
+                         "backward, recurrent = the reverse token recurrence")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seqs", type=int, default=4,
                     help="sequences in the CPU-baseline sample")

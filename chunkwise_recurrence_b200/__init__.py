@@ -416,7 +416,7 @@ def backward(q, k, v, beta, log_alpha, initial_state, d_out, d_final_state=None,
              stream=None):
     """Run ``gdr_backward``: gradients of the forward pass (same inputs as
     ``chunk_fwd``) given dL/d out and, optionally, dL/d final_state.
-    ``algo``: "staged" (the chunked backward) or "recurrent" / "auto" (the
+    ``algo``: "auto" / "staged" (the chunked backward) or "recurrent" (the
     reverse token recurrence).  Returns a dict of fp32 CUDA tensors dq, dk,
     dv, dbeta, dlog_alpha (None without a gate) and dinitial_state (None
     unless requested)."""

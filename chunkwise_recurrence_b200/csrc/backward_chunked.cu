@@ -22,9 +22,9 @@
 // the erase factors is the one the Gated DeltaNet-2 abstract (comparative-
 // study page 2607.07953) names.
 //
-// Kernels (per call): the staged path's chunk table, cumsum and WY kernel
-// (W, U and T of every chunk), then
-//   bw_p_kernel      P of every (chunk, head), in parallel;
+// Kernels (per call): the staged path's chunk table and cumsum, then
+//   bw_wy_kernel     per (chunk, head), in parallel: A, P, T = (I + A)^-1,
+//                    W and U;
 //   bw_prep_kernel   per (chunk, head), in parallel: the chunk's state map
 //                    S' = Cm S + Dm and the adjoint's input Bm;
 //   bw_scan_kernel   per (sequence, head): the chunk-start states (forward),
@@ -47,11 +47,13 @@ namespace gdr {
 namespace {
 
 constexpr int kBC = 64;      // chunk length
-constexpr int kNT = 256;     // threads per CTA
+constexpr int kNT = 512;     // threads per CTA
 constexpr int kSl = 16;      // key rows per slice in bw_grad_kernel
-// shared-memory row strides: d-wide rows (d <= 128) and C-wide rows, one
-// float of padding each so that column walks spread over the banks
-constexpr int kP = 129, kCP = kBC + 1;
+// shared-memory row strides: d-wide rows (d <= 128) and C-wide rows, each
+// 4 (mod 32) floats, so that an MMA fragment's 8 rows x 4 columns fall in 32
+// distinct banks (and its 4 rows x 8 columns, the transposed walk, in at
+// most two per bank)
+constexpr int kP = 132, kCP = kBC + 4;
 // largest in-chunk spread |g - g_ref| of a channel-wise decay for which the
 // gradient kernel factors e^{g_r - g_i} as e^{g_r - g_ref} e^{g_ref - g_i}
 // (both stay far inside fp32 for normalised keys); wider chunks take one
@@ -149,29 +151,35 @@ __device__ __forceinline__ void gemm_tc(int M, int N, int K, FA A, FB B,
   const int nb = N / (8 * NT), total = (M / 16) * nb;
   for (int blk = warp; blk < total; blk += kNT / 32) {
     const int m0 = (blk / nb) * 16, n0 = (blk % nb) * 8 * NT;
-    float c[NT][4];
+    // the main products and the two correction products in accumulators of
+    // their own, so that consecutive MMAs do not wait on one another
+    float c[NT][4], e[NT][4];
 #pragma unroll
-    for (int j = 0; j < NT; ++j) c[j][0] = c[j][1] = c[j][2] = c[j][3] = 0.f;
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int x = 0; x < 4; ++x) c[j][x] = e[j][x] = 0.f;
     for (int k0 = 0; k0 < K; k0 += 8) {
-      uint32_t ah[4], al[4];
+      uint32_t ah[4], al[4], bh[NT][2], bl[NT][2];
       load_a(A, m0, k0, g, t, ah, al);
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
-        uint32_t bh0, bl0, bh1, bl1;
-        tf32_split(B(k0 + t, n0 + 8 * j + g), bh0, bl0);
-        tf32_split(B(k0 + t + 4, n0 + 8 * j + g), bh1, bl1);
-        mma_tf32(c[j], al, bh0, bh1);
-        mma_tf32(c[j], ah, bl0, bl1);
-        mma_tf32(c[j], ah, bh0, bh1);
+        tf32_split(B(k0 + t, n0 + 8 * j + g), bh[j][0], bl[j][0]);
+        tf32_split(B(k0 + t + 4, n0 + 8 * j + g), bh[j][1], bl[j][1]);
       }
+#pragma unroll
+      for (int j = 0; j < NT; ++j) mma_tf32(c[j], ah, bh[j][0], bh[j][1]);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) mma_tf32(e[j], al, bh[j][0], bh[j][1]);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) mma_tf32(e[j], ah, bl[j][0], bl[j][1]);
     }
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
       const int n = n0 + 8 * j + 2 * t;
-      out(m0 + g, n, c[j][0]);
-      out(m0 + g, n + 1, c[j][1]);
-      out(m0 + g + 8, n, c[j][2]);
-      out(m0 + g + 8, n + 1, c[j][3]);
+      out(m0 + g, n, c[j][0] + e[j][0]);
+      out(m0 + g, n + 1, c[j][1] + e[j][1]);
+      out(m0 + g + 8, n, c[j][2] + e[j][2]);
+      out(m0 + g + 8, n + 1, c[j][3] + e[j][3]);
     }
   }
 }
@@ -226,11 +234,15 @@ __device__ __forceinline__ void gemm_tc4(int M, int N, int K, FA1 A1, FB1 B1,
 
 // gemm_tc with the widest column block that divides N (N is a runtime
 // multiple of 8)
+// (but narrower when that leaves warps without a block: the products here
+// are latency-bound, and a block per warp matters more than fragment reuse)
 template <class FA, class FB, class FO>
 __device__ __forceinline__ void gemm_tcn(int M, int N, int K, FA A, FB B,
                                          FO out) {
-  if (N % 32 == 0) gemm_tc<4>(M, N, K, A, B, out);
-  else if (N % 16 == 0) gemm_tc<2>(M, N, K, A, B, out);
+  const int rows = M / 16, warps = kNT / 32;
+  if (N % 32 == 0 && rows * (N / 32) >= warps) gemm_tc<4>(M, N, K, A, B, out);
+  else if (N % 16 == 0 && rows * (N / 16) >= warps)
+    gemm_tc<2>(M, N, K, A, B, out);
   else gemm_tc<1>(M, N, K, A, B, out);
 }
 
@@ -254,78 +266,195 @@ __device__ __forceinline__ float gv(const float *g, int gdim, size_t row,
 }
 
 // ---------------------------------------------------------------------------
-// P[t][i] = sum_c q_t[c] k_i[c] e^{g_t[c] - g_i[c]} for i <= t < L, else 0,
-// per (chunk, head), [max_chunks][H][C][C].
-template <typename Tin>
+// T = (I + A)^-1 for the strictly lower 64 x 64 A (rows kCP floats apart), in
+// fp32, by 16 x 16 blocks: the diagonal blocks D_b = (I + A_bb)^-1 by forward
+// substitution in registers (one thread per block column), then the blocks
+// below them level by level, T_bc = -D_b sum_{c <= e < b} A_be T_ec, each
+// level's sum (into Mt) and its product with D_b as independent dot
+// products.  Six barriers in all.  Ts must not alias As; Mt is [3][16][16].
+__device__ __forceinline__ void invert_unit_lower(const float *As, float *Ts,
+                                                  float *Mt) {
+  const int tid = threadIdx.x;
+  for (int idx = tid; idx < kBC * kBC; idx += kNT)
+    Ts[(idx / kBC) * kCP + idx % kBC] = 0.f;
+  __syncthreads();
+  if (tid < 64) {
+    const int b = tid >> 4, jc = tid & 15, o = 16 * b;
+    float x[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      float a0 = (r == jc) ? 1.f : 0.f, a1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < r; ++i) {
+        const float a = As[(o + r) * kCP + o + i];
+        if (i & 1) a1 -= a * x[i];
+        else a0 -= a * x[i];
+      }
+      x[r] = a0 + a1;
+    }
+#pragma unroll
+    for (int r = 0; r < 16; ++r) Ts[(o + r) * kCP + o + jc] = x[r];
+  }
+  __syncthreads();
+  // level d = b - c: blocks (c + d, c), c = 0 .. 3 - d
+  for (int d = 1; d < 4; ++d) {
+    const int nblk = 4 - d;
+    for (int idx = tid; idx < nblk * 256; idx += kNT) {
+      const int c = idx >> 8, r = (idx >> 4) & 15, col = idx & 15;
+      const int bb = c + d;
+      // M = sum_{c <= e < b} A_{b e} T_{e c}
+      float acc = 0.f;
+      for (int e = c; e < bb; ++e)
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          acc += As[(16 * bb + r) * kCP + 16 * e + i] *
+                 Ts[(16 * e + i) * kCP + 16 * c + col];
+      Mt[idx] = acc;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < nblk * 256; idx += kNT) {
+      const int c = idx >> 8, r = (idx >> 4) & 15, col = idx & 15;
+      const int bb = c + d;
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        acc += Ts[(16 * bb + r) * kCP + 16 * bb + i] * Mt[c * 256 + i * 16 + col];
+      Ts[(16 * bb + r) * kCP + 16 * c + col] = -acc;
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The WY quantities of one (chunk, head), in parallel over all chunks:
+//   A[r][i] = beta_r sum_c k_r[c] k_i[c] e^{g_r[c] - g_i[c]}   (i < r < L)
+//   P[t][i] =        sum_c q_t[c] k_i[c] e^{g_t[c] - g_i[c]}   (i <= t < L)
+//   T = (I + A)^-1,  W = T diag(beta) (K . e^g),  U = T diag(beta) V.
+// A and P share their key operand; for the channel-wise decay the weights
+// are factored around the chunk's middle row (e^{g - g_ref} on the row side,
+// e^{g_ref - g} on the column side) while the chunk's spread allows it, else
+// formed one exponential per element; the scalar decay multiplies the
+// products by the C x C matrix e^{g_r - g_i}.  T, P go to [chunks][H][C][C];
+// W, U to the staged path's [ntok][H][d] buffers.
+template <typename Tin, int GATE>
 __global__ void __launch_bounds__(kNT)
-    bw_p_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
-                const float *__restrict__ g, float *__restrict__ Pout,
-                const ChunkInfo *__restrict__ table,
-                const int *__restrict__ nchunks, int H, int dk, int gdim) {
+    bw_wy_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
+                 const Tin *__restrict__ v, const float *__restrict__ beta,
+                 const float *__restrict__ g, float *__restrict__ Tout,
+                 float *__restrict__ Pout, float *__restrict__ Wout,
+                 float *__restrict__ Uout, const ChunkInfo *__restrict__ table,
+                 const int *__restrict__ nchunks, int H, int dk, int dv) {
   const int j = blockIdx.x, h = blockIdx.y;
   if (j >= *nchunks) return;
   const ChunkInfo ci = table[j];
-  const int L = ci.len, dkp = dk + 1;
+  const int L = ci.len;
+  const int gdim = GATE == 0 ? 0 : GATE == 1 ? 1 : dk;
   extern __shared__ float sm[];
-  float *Qs = sm;                    // [C][dkp]
-  float *Ks = Qs + kBC * dkp;        // [C][dkp]
-  float *Gs = Ks + kBC * dkp;        // [C][dkp] (channel gate) or [C]
-  __shared__ float red[kNT / 32];
+  float *Qu = sm;                    // [C][kP]: q e^{g - g_ref}; then the
+                                     //   W operand beta k e^g
+  float *Ku = Qu + kBC * kP;         // [C][kP]: k e^{g - g_ref}; then beta v
+  float *Kd = Ku + kBC * kP;         // [C][kP]: k e^{g_ref - g}
+  float *As = Kd + kBC * kP;         // [C][kCP]: A
+  float *Ts = As + kBC * kCP;        // [C][kCP]: T
+  float *Gh = Ts + kBC * kCP;        // [C][kCP]: e^{g_r - g_i} (scalar gate)
+  float *bs = Gh + kBC * kCP;        // [C]
+  float *red = bs + kBC;             // [kNT / 32]
   const int tid = threadIdx.x;
-  for (int idx = tid; idx < kBC * dk; idx += kNT) {
-    const int r = idx / dk, c = idx % dk;
-    const size_t row = (size_t)(ci.tok0 + r) * H + h;
-    const bool live = r < L;
-    Qs[r * dkp + c] = live ? ldf(q + row * dk + c) : 0.f;
-    Ks[r * dkp + c] = live ? ldf(k + row * dk + c) : 0.f;
-    if (gdim > 1) Gs[r * dkp + c] = live ? g[row * gdim + c] : 0.f;
-  }
-  if (gdim == 1)
-    for (int r = tid; r < kBC; r += kNT)
-      Gs[r] = r < L ? g[(size_t)(ci.tok0 + r) * H + h] : 0.f;
-  __syncthreads();
-  float *Pg = Pout + ((size_t)j * H + h) * kBC * kBC;
-  bool fact = true;
+  const size_t base = (size_t)ci.tok0 * H + h;
+  auto row = [&](int t) { return base + (size_t)t * H; };
+  auto gt = [&](int t, int c) { return gv(g, gdim, row(t), c); };
   const int ref = (L - 1) / 2;
-  if (gdim > 1) {
-    // factor e^{g_t - g_i} = e^{g_t - g_ref} e^{g_ref - g_i} when the
-    // chunk's spread allows it
+  bool fact = true;
+  if (GATE == 2) {
     float spread = 0.f;
     for (int idx = tid; idx < L * dk; idx += kNT) {
-      const int r = idx / dk, c = idx % dk;
-      spread = fmaxf(spread, fabsf(Gs[r * dkp + c] - Gs[ref * dkp + c]));
+      const int t = idx / dk, c = idx % dk;
+      spread = fmaxf(spread, fabsf(gt(t, c) - gt(ref, c)));
     }
     fact = block_max(spread, red) <= kFactRange;
-    if (fact) {
-      for (int idx = tid; idx < L * dk; idx += kNT) {
-        const int r = idx / dk, c = idx % dk;
-        const float d = Gs[r * dkp + c] - Gs[ref * dkp + c];
-        Qs[r * dkp + c] *= __expf(d);
-        Ks[r * dkp + c] *= __expf(-d);
-      }
-      __syncthreads();
-    }
   }
-  if (fact) {
+  for (int idx = tid; idx < kBC * dk; idx += kNT) {
+    const int t = idx / dk, c = idx % dk;
+    float kv = 0.f, qv = 0.f, d = 0.f;
+    if (t < L) {
+      kv = ldf(k + row(t) * dk + c);
+      qv = ldf(q + row(t) * dk + c);
+      if (GATE == 2 && fact) d = gt(t, c) - gt(ref, c);
+    }
+    const float up = __expf(d), dn = __expf(-d);
+    Qu[t * kP + c] = qv * up;
+    Ku[t * kP + c] = kv * up;
+    Kd[t * kP + c] = kv * dn;
+  }
+  for (int t = tid; t < kBC; t += kNT) bs[t] = t < L ? beta[row(t)] : 0.f;
+  if (GATE == 1)
+    for (int idx = tid; idx < kBC * kBC; idx += kNT) {
+      const int r = idx / kBC, i = idx % kBC;
+      Gh[r * kCP + i] =
+          (i <= r && r < L) ? __expf(gt(r, 0) - gt(i, 0)) : 0.f;
+    }
+  __syncthreads();
+  float *Pg = Pout + ((size_t)j * H + h) * kBC * kBC;
+  if (GATE != 2 || fact) {
     gemm_tcn(
-        kBC, kBC, dk, [&](int m, int c) { return Qs[m * dkp + c]; },
-        [&](int c, int n) { return Ks[n * dkp + c]; },
-        [&](int m, int n, float v) {
-          float w = (n <= m && m < L) ? v : 0.f;
-          if (gdim == 1 && n <= m && m < L) w *= __expf(Gs[m] - Gs[n]);
-          Pg[m * kBC + n] = w;
+        kBC, kBC, dk, [&](int r, int c) { return Ku[r * kP + c]; },
+        [&](int c, int i) { return Kd[i * kP + c]; },
+        [&](int r, int i, float x) {
+          float a = (i < r && r < L) ? bs[r] * x : 0.f;
+          if (GATE == 1) a *= Gh[r * kCP + i];
+          As[r * kCP + i] = a;
+        });
+    gemm_tcn(
+        kBC, kBC, dk, [&](int t, int c) { return Qu[t * kP + c]; },
+        [&](int c, int i) { return Kd[i * kP + c]; },
+        [&](int t, int i, float x) {
+          float w = (i <= t && t < L) ? x : 0.f;
+          if (GATE == 1) w *= Gh[t * kCP + i];
+          Pg[t * kBC + i] = w;
         });
   } else {
+    // the chunk's channel-wise decay is too wide to factor
     for (int idx = tid; idx < kBC * kBC; idx += kNT) {
-      const int t = idx / kBC, i = idx % kBC;
-      float a = 0.f;
-      if (i <= t && t < L)
-        for (int c = 0; c < dk; ++c)
-          a += Qs[t * dkp + c] * Ks[i * dkp + c] *
-               __expf(Gs[t * dkp + c] - Gs[i * dkp + c]);
-      Pg[idx] = a;
+      const int r = idx / kBC, i = idx % kBC;
+      float a = 0.f, pp = 0.f;
+      if (i <= r && r < L)
+        for (int c = 0; c < dk; ++c) {
+          const float e = Kd[i * kP + c] * __expf(gt(r, c) - gt(i, c));
+          a += Ku[r * kP + c] * e;
+          pp += Qu[r * kP + c] * e;
+        }
+      As[r * kCP + i] = i < r ? bs[r] * a : 0.f;
+      Pg[idx] = pp;
     }
   }
+  __syncthreads();
+  invert_unit_lower(As, Ts, Gh);   // Gh (no longer needed) as the scratch
+  float *Tg = Tout + ((size_t)j * H + h) * kBC * kBC;
+  for (int idx = tid; idx < kBC * kBC; idx += kNT)
+    Tg[idx] = Ts[(idx / kBC) * kCP + idx % kBC];
+  // the W and U operands: beta k e^g over Qu, beta v over Ku
+  for (int idx = tid; idx < kBC * dk; idx += kNT) {
+    const int t = idx / dk, c = idx % dk;
+    Qu[t * kP + c] =
+        t < L ? bs[t] * ldf(k + row(t) * dk + c) * __expf(gt(t, c)) : 0.f;
+  }
+  for (int idx = tid; idx < kBC * dv; idx += kNT) {
+    const int t = idx / dv, c = idx % dv;
+    Ku[t * kP + c] = t < L ? bs[t] * ldf(v + row(t) * dv + c) : 0.f;
+  }
+  __syncthreads();
+  gemm_tcn(
+      kBC, dk, kBC, [&](int r, int s2) { return Ts[r * kCP + s2]; },
+      [&](int s2, int c) { return Qu[s2 * kP + c]; },
+      [&](int r, int c, float x) {
+        if (r < L) Wout[row(r) * dk + c] = x;
+      });
+  gemm_tcn(
+      kBC, dv, kBC, [&](int r, int s2) { return Ts[r * kCP + s2]; },
+      [&](int s2, int c) { return Ku[s2 * kP + c]; },
+      [&](int r, int c, float x) {
+        if (r < L) Uout[row(r) * dv + c] = x;
+      });
 }
 
 // ---------------------------------------------------------------------------
@@ -477,7 +606,7 @@ __global__ void __launch_bounds__(kNT)
   const int j = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kVH;
   if (j >= *nchunks) return;
   const ChunkInfo ci = table[j];
-  const int L = ci.len, DV = min(kVH, dv), vp = kVH + 1;
+  const int L = ci.len, DV = min(kVH, dv), vp = kVH + 4;
   extern __shared__ float sm[];
   float *Ws = sm;                    // [C][kP]: W
   float *Ks = Ws + kBC * kP;         // [C][kP]: Kc
@@ -545,7 +674,7 @@ __global__ void __launch_bounds__(kNT)
 //   SL  the slice tiles S, Lambda [16][129] and (K . e^g) [C][17]; then dP
 //   XT  the slice products X1, X2, X3 [3][C][16]
 //   small per-row and per-channel sums
-constexpr int kRS = kSl + 1;
+constexpr int kRS = kSl + 4;
 constexpr int kTS = 0;
 constexpr int kBIG = kTS + kBC * kCP;
 constexpr int kSLo = kBIG + 5 * kBC * kP;
@@ -553,7 +682,8 @@ constexpr int kXT = kSLo + 2 * kSl * kP + kBC * kRS;
 constexpr int kSM = kXT + 3 * kBC * kSl;
 constexpr int kSmall = 64 * 3 + 128 * 2 + 16;
 constexpr int kGradSmemFloats = kSM + kSmall;
-static_assert(kBIG + 24768 + 3 * kBC * kCP <= kSLo, "phase-2 tiles");
+static_assert(kBIG + 3 * kBC * kP + 3 * kBC * kCP <= kSLo, "phase-2 tiles");
+static_assert(kGradSmemFloats * 4 <= 232448, "shared memory");
 static_assert(kBC * kCP <= 2 * kSl * kP + kBC * kRS, "dP tile");
 
 template <typename Tin, int GATE>
@@ -693,7 +823,7 @@ __global__ void __launch_bounds__(kNT)
     dvg[row(t) * dv + c] = bs[t] * Zs[t * kP + c];
   }
   __syncthreads();
-  float *dTs = sm + kBIG + 24768;          // over Z (phase 2: then dA)
+  float *dTs = sm + kBIG + 3 * kBC * kP;   // over Z (phase 2: then dA)
   float *Xi = dTs + kBC * kCP;
   float *Ms = Xi + kBC * kCP;
   float *dPs = sm + kSLo;                  // over the slice tiles
@@ -815,10 +945,10 @@ __global__ void __launch_bounds__(kNT)
     auto bk = [&](int i, int c) { return Kd[i * kP + c]; };
     auto bu = [&](int i, int c) { return Ku[i * kP + c]; };
     auto bq = [&](int i, int c) { return Qu[i * kP + c]; };
-    if (dk % 32 == 0)
-      gemm_tc4<4>(kBC, dk, kBC, a1, bk, a2, bu, a3, bk, a4, bq, pair_out);
-    else
+    if (dk % 16 == 0 && (kBC / 16) * (dk / 16) >= kNT / 32)
       gemm_tc4<2>(kBC, dk, kBC, a1, bk, a2, bu, a3, bk, a4, bq, pair_out);
+    else
+      gemm_tc4<1>(kBC, dk, kBC, a1, bk, a2, bu, a3, bk, a4, bq, pair_out);
   } else {
     // channel-wise decay too wide to factor: one exponential per element
     for (int idx = tid; idx < L * dk; idx += kNT) {
@@ -911,6 +1041,22 @@ cudaError_t run_grad(const Problem &p, const BackwardIO &io,
   return cudaGetLastError();
 }
 
+template <typename Tin, int GATE>
+cudaError_t run_wy(const Problem &p, const StagedBufs &b, float *Tb, float *Pb,
+                   cudaStream_t s) {
+  const int smem =
+      (int)sizeof(float) * (3 * kBC * kP + 3 * kBC * kCP + kBC + kNT / 32);
+  cudaError_t e = cudaFuncSetAttribute(
+      bw_wy_kernel<Tin, GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      smem);
+  if (e != cudaSuccess) return e;
+  bw_wy_kernel<Tin, GATE><<<dim3(p.max_chunks, p.H), kNT, smem, s>>>(
+      static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k),
+      static_cast<const Tin *>(p.v), p.beta, b.g, Tb, Pb, b.W, b.U, b.table,
+      b.nchunks, p.H, p.dk, p.dv);
+  return cudaGetLastError();
+}
+
 template <typename Tin>
 cudaError_t run_typed(const Problem &p, const BackwardIO &io, char *ws,
                       cudaStream_t s) {
@@ -919,22 +1065,20 @@ cudaError_t run_typed(const Problem &p, const BackwardIO &io, char *ws,
   float *Pb = reinterpret_cast<float *>(ws + l.P);
   float *Lam = reinterpret_cast<float *>(ws + l.Lam);
   float *dVn = reinterpret_cast<float *>(ws + l.dVn);
-  cudaError_t e = staged_wy_run(p, ws + l.staged, Tb, s);
+  cudaError_t e = staged_chunks_run(p, ws + l.staged, s);
   if (e != cudaSuccess) return e;
   const StagedBufs b = staged_bufs(p, ws + l.staged);
   const int gdim = p.gate == GDR_GATE_NONE ? 0
                    : p.gate == GDR_GATE_SCALAR ? 1
                                                : p.dk;
-  const int dkp = p.dk + 1;
   const Tin *q = static_cast<const Tin *>(p.q);
   const Tin *k = static_cast<const Tin *>(p.k);
   if (p.max_chunks > 0) {
-    const int smem = (int)sizeof(float) * 3 * kBC * dkp;
-    e = cudaFuncSetAttribute(bw_p_kernel<Tin>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = p.gate == GDR_GATE_NONE
+            ? run_wy<Tin, 0>(p, b, Tb, Pb, s)
+            : p.gate == GDR_GATE_SCALAR ? run_wy<Tin, 1>(p, b, Tb, Pb, s)
+                                        : run_wy<Tin, 2>(p, b, Tb, Pb, s);
     if (e != cudaSuccess) return e;
-    bw_p_kernel<Tin><<<dim3(p.max_chunks, p.H), kNT, smem, s>>>(
-        q, k, b.g, Pb, b.table, b.nchunks, p.H, p.dk, gdim);
   }
   float *Cm = reinterpret_cast<float *>(ws + l.Cm);
   float *Dm = reinterpret_cast<float *>(ws + l.Dm);
@@ -964,7 +1108,7 @@ cudaError_t run_typed(const Problem &p, const BackwardIO &io, char *ws,
                                                b.seq_first, p.H, p.dk, p.dv);
   }
   if (p.max_chunks > 0) {
-    const int vp = kVH + 1;
+    const int vp = kVH + 4;
     const int smem = (int)sizeof(float) *
                      (2 * kBC * kP + kBC * kCP + 2 * 128 * vp + kBC * vp +
                       p.dk);

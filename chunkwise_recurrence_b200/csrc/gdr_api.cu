@@ -846,10 +846,9 @@ extern "C" gdr_status gdr_backward(
   const void *grads[] = {dq, dk, dv, d_log_alpha, d_beta, d_initial_state};
   for (const void *ptr : grads)
     if (ptr && !aligned16(ptr)) return GDR_ERR_INVALID_ARGUMENT;
-  // AUTO takes the reverse token recurrence, which is the faster of the two
-  // on every measured shape so far; STAGED names the chunked backward
-  const bool chunked = o.algo == GDR_ALGO_STAGED &&
-                       gdr::backward_chunked_applies(p);
+  // AUTO and STAGED: the chunked backward (the faster of the two on every
+  // measured shape); RECURRENT: the reverse token recurrence
+  const bool chunked = !recurrent && gdr::backward_chunked_applies(p);
   long long total_win = 0;
   const size_t bytes = chunked ? gdr::backward_chunked_bytes(p)
                                : gdr::backward_scratch_bytes(p, &total_win);

@@ -58,10 +58,9 @@ struct StagedBufs {
   float *g, *W, *U, *Vn, *Sbuf;
 };
 StagedBufs staged_bufs(const Problem &p, void *workspace);
-// The chunk table, g, W and U (and T [max_chunks][H][C][C] into Tout when
-// not nullptr) of every (chunk, head); no state pass, no output.
-cudaError_t staged_wy_run(const Problem &p, void *workspace, float *Tout,
-                          cudaStream_t s);
+// The staged path's chunk table and in-chunk cumulative log-decays g only.
+cudaError_t staged_chunks_run(const Problem &p, void *workspace,
+                              cudaStream_t s);
 
 // Fused tensor-core path.
 bool fused_tc_applies(const Problem &p);

@@ -127,7 +127,7 @@ __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
                           const float *__restrict__ write,
                           const float *__restrict__ wkey,
                           const float *__restrict__ g, float *__restrict__ W,
-                          float *__restrict__ U, float *__restrict__ Tout,
+                          float *__restrict__ U,
                           const ChunkInfo *__restrict__ table,
                           const int *__restrict__ nchunks, int H, int dk,
                           int dv, int C, int gdim) {
@@ -213,15 +213,6 @@ __global__ void wy_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
     __syncthreads();
   }
   if (L <= 1) __syncthreads();   // the X and Vs writes before their reads
-  // T itself, [C][C] per (chunk, head) (rows and columns past L zero), for
-  // the backward pass
-  if (Tout) {
-    float *Tg = Tout + ((size_t)j * H + h) * C * C;
-    for (int idx = tid; idx < C * C; idx += nt) {
-      const int r = idx / C, i = idx % C;
-      Tg[idx] = (r < L && i < L) ? Ts[r * (C + 1) + i] : 0.f;
-    }
-  }
 
   // W = T X,  U = T Vs
   for (int idx = tid; idx < L * dk; idx += nt) {
@@ -483,9 +474,8 @@ cudaError_t run_typed(const Problem &p, char *ws, cudaStream_t s) {
         (int)wy_smem);
     if (e != cudaSuccess) return e;
     wy_kernel<Tin><<<grid, 256, wy_smem, s>>>(k, v, p.beta, p.erase, p.write,
-                                             p.wkey, g, W, U, nullptr, table,
-                                             nchunks, p.H, p.dk, p.dv, C,
-                                             gdim);
+                                             p.wkey, g, W, U, table, nchunks,
+                                             p.H, p.dk, p.dv, C, gdim);
   }
   const int DVT = p.dv < 64 ? p.dv : 64;
   const size_t st_smem =
@@ -515,46 +505,6 @@ cudaError_t run_typed(const Problem &p, char *ws, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-// The per-chunk part of the staged path the backward pass reuses: the chunk
-// table, the in-chunk cumulative log-decays, and W, U (and T) of every
-// (chunk, head).  The state pass and the output are left to the caller.
-template <typename Tin>
-cudaError_t run_wy_typed(const Problem &p, char *ws, float *Tout,
-                         cudaStream_t s) {
-  const StagedLayout L = layout(p);
-  const int gdim = p.gate == GDR_GATE_NONE ? 0
-                   : p.gate == GDR_GATE_SCALAR ? 1
-                                               : p.dk;
-  const int gd = gdim == 0 ? 1 : gdim;
-  const int C = p.chunk;
-  ChunkInfo *table = reinterpret_cast<ChunkInfo *>(ws + L.table);
-  int *seq_first = reinterpret_cast<int *>(ws + L.seq_first);
-  int *nchunks = seq_first + p.nseq;
-  float *g = gdim ? reinterpret_cast<float *>(ws + L.g) : nullptr;
-  chunk_table_kernel<<<1, 32, 0, s>>>(p.cu, p.nseq, p.T, p.ntok, C, table,
-                                      seq_first);
-  if (p.max_chunks == 0) return cudaGetLastError();
-  const dim3 grid(p.max_chunks, p.H);
-  if (gdim)
-    cumsum_kernel<<<grid, 128, 0, s>>>(p.log_alpha, g, table, nchunks, p.H,
-                                       gdim);
-  const size_t dkp = (size_t)p.dk + 1;
-  const size_t wy_smem =
-      sizeof(float) * ((size_t)C * dkp + (size_t)C * gd +
-                       2 * (size_t)C * (C + 1) + C + (size_t)C * p.dv +
-                       ((p.erase || p.wkey) ? (size_t)C * dkp : 0));
-  cudaError_t e = cudaFuncSetAttribute(
-      wy_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-      (int)wy_smem);
-  if (e != cudaSuccess) return e;
-  wy_kernel<Tin><<<grid, 256, wy_smem, s>>>(
-      static_cast<const Tin *>(p.k), static_cast<const Tin *>(p.v), p.beta,
-      p.erase, p.write, p.wkey, g, reinterpret_cast<float *>(ws + L.W),
-      reinterpret_cast<float *>(ws + L.U), Tout, table, nchunks, p.H, p.dk,
-      p.dv, C, gdim);
-  return cudaGetLastError();
-}
-
 }  // namespace
 
 size_t staged_workspace_bytes(const Problem &p) { return layout(p).total; }
@@ -574,11 +524,18 @@ StagedBufs staged_bufs(const Problem &p, void *workspace) {
   return b;
 }
 
-cudaError_t staged_wy_run(const Problem &p, void *workspace, float *Tout,
-                          cudaStream_t s) {
-  char *ws = static_cast<char *>(workspace);
-  if (p.dtype == GDR_FP32) return run_wy_typed<float>(p, ws, Tout, s);
-  return run_wy_typed<__nv_bfloat16>(p, ws, Tout, s);
+cudaError_t staged_chunks_run(const Problem &p, void *workspace,
+                              cudaStream_t s) {
+  const StagedBufs b = staged_bufs(p, workspace);
+  const int gdim = p.gate == GDR_GATE_NONE ? 0
+                   : p.gate == GDR_GATE_SCALAR ? 1
+                                               : p.dk;
+  chunk_table_kernel<<<1, 32, 0, s>>>(p.cu, p.nseq, p.T, p.ntok, p.chunk,
+                                      b.table, b.seq_first);
+  if (gdim && p.max_chunks > 0)
+    cumsum_kernel<<<dim3(p.max_chunks, p.H), 128, 0, s>>>(
+        p.log_alpha, b.g, b.table, b.nchunks, p.H, gdim);
+  return cudaGetLastError();
 }
 
 cudaError_t staged_run(const Problem &p, void *workspace, cudaStream_t s) {

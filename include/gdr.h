@@ -447,19 +447,19 @@ GDR_API gdr_status gdr_decode_step_fg2(const void *q, const void *k,
  * dL/d final_state, it writes dL/dq, dL/dk, dL/dv, dL/d log_alpha,
  * dL/d beta and dL/d initial_state of the recurrence above (the same
  * definition gdr_chunk_fwd evaluates, whichever algorithm ran it), all in
- * fp32.  Two algorithms (AUTO runs the recurrent one, the faster on every
- * shape measured so far):
- *  - STAGED: the chunked backward.  The gradients of the chunkwise
+ * fp32.  Two algorithms:
+ *  - AUTO or STAGED: the chunked backward (the faster of the two on every
+ *    shape measured).  The gradients of the chunkwise
  *    (WY) forward, taken product by product over chunks of 64 tokens: the
  *    staged path's per-chunk W, U and T, a forward scan over the chunk
  *    boundaries for the chunk-start states, a reverse scan for dL/dS at
  *    every chunk end, then every chunk's input gradients in parallel
- *    (register-blocked fp32 products on CUDA cores).  The update being
+ *    (mma.sync tensor-core products on fp32 operands split into a tf32
+ *    part and its remainder, accurate to about 2^-21).  The update being
  *    affine in the preceding memory ("DeltaTTT" page, §2 Background) is
  *    what makes the two scans exact.  Deterministic except for the order in
  *    which a chunk's per-channel shares of the decay gradient are added.
- *  - RECURRENT (and AUTO): the reverse token recurrence.  It runs the
- *    recurrence
+ *  - RECURRENT: the reverse token recurrence.  It runs the recurrence
  *    forward, checkpointing the state every 8 tokens in scratch (16 when dk
  *    or dv is 16), then the reverse token recurrence window by window.  For
  *    dk, dv >= 32 each (sequence, head) runs on dv/32 blocks of 32 value
