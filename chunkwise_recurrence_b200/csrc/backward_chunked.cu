@@ -340,6 +340,8 @@ template <typename Tin, int GATE>
 __global__ void __launch_bounds__(kNT)
     bw_wy_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                  const Tin *__restrict__ v, const float *__restrict__ beta,
+                 const float *__restrict__ erase,
+                 const float *__restrict__ write,
                  const float *__restrict__ g, float *__restrict__ Tout,
                  float *__restrict__ Pout, float *__restrict__ Wout,
                  float *__restrict__ Uout, const ChunkInfo *__restrict__ table,
@@ -375,18 +377,21 @@ __global__ void __launch_bounds__(kNT)
   }
   for (int idx = tid; idx < kBC * dk; idx += kNT) {
     const int t = idx / dk, c = idx % dk;
-    float kv = 0.f, qv = 0.f, d = 0.f;
+    float kv = 0.f, qv = 0.f, d = 0.f, rv = 0.f;
     if (t < L) {
       kv = ldf(k + row(t) * dk + c);
       qv = ldf(q + row(t) * dk + c);
+      rv = erase ? erase[row(t) * dk + c] * kv : kv;   // the read key
       if (GATE == 2 && fact) d = gt(t, c) - gt(ref, c);
     }
     const float up = __expf(d), dn = __expf(-d);
     Qu[t * kP + c] = qv * up;
-    Ku[t * kP + c] = kv * up;
+    Ku[t * kP + c] = rv * up;
     Kd[t * kP + c] = kv * dn;
   }
-  for (int t = tid; t < kBC; t += kNT) bs[t] = t < L ? beta[row(t)] : 0.f;
+  // beta, or 1 with the Gated DeltaNet-2 gates (0 past the sequence end)
+  for (int t = tid; t < kBC; t += kNT)
+    bs[t] = t < L ? (erase ? 1.f : beta[row(t)]) : 0.f;
   if (GATE == 1)
     for (int idx = tid; idx < kBC * kBC; idx += kNT) {
       const int r = idx / kBC, i = idx % kBC;
@@ -432,15 +437,24 @@ __global__ void __launch_bounds__(kNT)
   float *Tg = Tout + ((size_t)j * H + h) * kBC * kBC;
   for (int idx = tid; idx < kBC * kBC; idx += kNT)
     Tg[idx] = Ts[(idx / kBC) * kCP + idx % kBC];
-  // the W and U operands: beta k e^g over Qu, beta v over Ku
+  // the W and U operands: beta (read key) e^g over Qu, beta (target) over Ku
   for (int idx = tid; idx < kBC * dk; idx += kNT) {
     const int t = idx / dk, c = idx % dk;
-    Qu[t * kP + c] =
-        t < L ? bs[t] * ldf(k + row(t) * dk + c) * __expf(gt(t, c)) : 0.f;
+    float x = 0.f;
+    if (t < L) {
+      x = bs[t] * ldf(k + row(t) * dk + c) * __expf(gt(t, c));
+      if (erase) x *= erase[row(t) * dk + c];
+    }
+    Qu[t * kP + c] = x;
   }
   for (int idx = tid; idx < kBC * dv; idx += kNT) {
     const int t = idx / dv, c = idx % dv;
-    Ku[t * kP + c] = t < L ? bs[t] * ldf(v + row(t) * dv + c) : 0.f;
+    float x = 0.f;
+    if (t < L) {
+      x = bs[t] * ldf(v + row(t) * dv + c);
+      if (write) x *= write[row(t) * dv + c];
+    }
+    Ku[t * kP + c] = x;
   }
   __syncthreads();
   gemm_tcn(
@@ -691,6 +705,8 @@ __global__ void __launch_bounds__(kNT)
     bw_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                    const Tin *__restrict__ v, const Tin *__restrict__ dout,
                    const float *__restrict__ beta, const float *__restrict__ g,
+                   const float *__restrict__ erase,
+                   const float *__restrict__ write,
                    const float *__restrict__ Tbuf,
                    const float *__restrict__ Sbuf,
                    const float *__restrict__ Lam,
@@ -698,6 +714,7 @@ __global__ void __launch_bounds__(kNT)
                    const float *__restrict__ dVnb, float *__restrict__ dq,
                    float *__restrict__ dkg, float *__restrict__ dvg,
                    float *__restrict__ dbeta, float *__restrict__ dla,
+                   float *__restrict__ derase, float *__restrict__ dwrite,
                    const ChunkInfo *__restrict__ table,
                    const int *__restrict__ nchunks, int H, int dk, int dv) {
   const int j = blockIdx.x, h = blockIdx.y;
@@ -733,10 +750,11 @@ __global__ void __launch_bounds__(kNT)
     Ds[t * kP + c] = live ? dVnb[o] : 0.f;
     Vs[t * kP + c] = live ? Vnb[o] : 0.f;
     Os[t * kP + c] = live ? ldf(dout + o) : 0.f;
-    Ys[t * kP + c] = live ? ldf(v + o) : 0.f;
+    // Y starts from the target (v, or w . v with Gated DeltaNet-2's gates)
+    Ys[t * kP + c] = live ? ldf(v + o) * (write ? write[o] : 1.f) : 0.f;
   }
   for (int t = tid; t < 64; t += kNT) {
-    bs[t] = t < L ? beta[row(t)] : 0.f;
+    bs[t] = t < L ? (erase ? 1.f : beta[row(t)]) : 0.f;
     dbs[t] = 0.f;
     dgs[t] = 0.f;
   }
@@ -759,8 +777,14 @@ __global__ void __launch_bounds__(kNT)
     }
     for (int idx = tid; idx < kBC * kSl; idx += kNT) {
       const int t = idx / kSl, cc = idx % kSl;
-      Rs[t * kRS + cc] =
-          t < L ? ldf(k + row(t) * dk + c0 + cc) * __expf(gt(t, c0 + cc)) : 0.f;
+      // the read key times e^g
+      float x = 0.f;
+      if (t < L) {
+        const size_t o = row(t) * dk + c0 + cc;
+        x = ldf(k + o) * __expf(gt(t, c0 + cc));
+        if (erase) x *= erase[o];
+      }
+      Rs[t * kRS + cc] = x;
     }
     __syncthreads();
     // Y -= (K . e^g)[:, slice] S[slice, :]
@@ -797,12 +821,16 @@ __global__ void __launch_bounds__(kNT)
     for (int idx = tid; idx < L * kSl; idx += kNT) {
       const int t = idx / kSl, cc = idx % kSl, c = c0 + cc;
       const float gg = gt(t, c), e = __expf(gg), ec = __expf(gC[c] - gg);
-      const float qv = ldf(q + row(t) * dk + c), kv = ldf(k + row(t) * dk + c);
+      const size_t o = row(t) * dk + c;
+      const float qv = ldf(q + o), kv = ldf(k + o);
+      const float bv = erase ? erase[o] : 1.f;   // read key = bv kv
       const float x1 = X1[t * kSl + cc], x2 = X2[t * kSl + cc],
                   x3 = X3[t * kSl + cc];
-      dq[row(t) * dk + c] = x1 * e;
-      dkg[row(t) * dk + c] = -x2 * e + x3 * ec;
-      const float dgv = (x1 * qv - x2 * kv) * e - x3 * kv * ec;
+      // read-key gradient -x2 e^g, write-key gradient x3 e^{g_C - g}
+      dq[o] = x1 * e;
+      dkg[o] = -x2 * e * bv + x3 * ec;
+      if (erase) derase[o] = -x2 * e * kv;
+      const float dgv = (x1 * qv - x2 * bv * kv) * e - x3 * kv * ec;
       if (GATE == 2) dla[row(t) * dk + c] = dgv;
       if (GATE == 1) atomicAdd(&dgs[t], dgv);
       if (GATE != 0) atomicAdd(&dgC[c], x3 * kv * ec);
@@ -820,7 +848,11 @@ __global__ void __launch_bounds__(kNT)
   }
   for (int idx = tid; idx < L * dv; idx += kNT) {
     const int t = idx / dv, c = idx % dv;
-    dvg[row(t) * dv + c] = bs[t] * Zs[t * kP + c];
+    const size_t o = row(t) * dv + c;
+    // the target's gradient beta Z, through w . v with the gates
+    const float dt = bs[t] * Zs[t * kP + c];
+    dvg[o] = write ? write[o] * dt : dt;
+    if (write) dwrite[o] = ldf(v + o) * dt;
   }
   __syncthreads();
   float *dTs = sm + kBIG + 3 * kBC * kP;   // over Z (phase 2: then dA)
@@ -861,14 +893,15 @@ __global__ void __launch_bounds__(kNT)
   }
   for (int idx = tid; idx < kBC * dk; idx += kNT) {
     const int t = idx / dk, c = idx % dk;
-    float kv = 0.f, qv = 0.f, d = 0.f;
+    float kv = 0.f, qv = 0.f, d = 0.f, rv = 0.f;
     if (t < L) {
       kv = ldf(k + row(t) * dk + c);
       qv = ldf(q + row(t) * dk + c);
+      rv = erase ? erase[row(t) * dk + c] * kv : kv;   // the read key
       if (GATE == 2 && fact) d = gt(t, c) - gt(ref, c);
     }
     const float up = __expf(d), dn = __expf(-d);
-    Ku[t * kP + c] = kv * up;
+    Ku[t * kP + c] = rv * up;
     Kd[t * kP + c] = kv * dn;
     Qu[t * kP + c] = qv * up;
   }
@@ -931,9 +964,11 @@ __global__ void __launch_bounds__(kNT)
       const float drho = up * r1, dkap = dn * r2, dqP = up * r3, dkP = dn * r4;
       const size_t o = row(t) * dk + c;
       const float kv = ldf(k + o), qv = ldf(q + o);
+      const float bv = erase ? erase[o] : 1.f;   // read key = bv kv
       dq[o] += dqP;
-      dkg[o] += drho + dkap + dkP;
-      const float dgv = kv * (drho - dkap - dkP) + qv * dqP;
+      dkg[o] += bv * drho + dkap + dkP;
+      if (erase) derase[o] += kv * drho;
+      const float dgv = bv * kv * drho - kv * (dkap + dkP) + qv * dqP;
       if (GATE == 2) dla[o] += dgv;
       if (GATE == 1) atomicAdd(&dgs[t], dgv);
     };
@@ -963,10 +998,14 @@ __global__ void __launch_bounds__(kNT)
         if (i >= t) dkP += dPs[i * kCP + t] * Qu[i * kP + c] * e;
       }
       const size_t o = row(t) * dk + c;
-      const float kv = Ku[t * kP + c], qv = Qu[t * kP + c];
+      // (unfactored: Ku holds the read key, Kd the key, Qu the query)
+      const float rv = Ku[t * kP + c], kv = Kd[t * kP + c],
+                  qv = Qu[t * kP + c];
+      const float bv = erase ? erase[o] : 1.f;
       dq[o] += dqP;
-      dkg[o] += drho + dkap + dkP;
-      dla[o] += kv * (drho - dkap - dkP) + qv * dqP;
+      dkg[o] += bv * drho + dkap + dkP;
+      if (erase) derase[o] += kv * drho;
+      dla[o] += rv * drho - kv * (dkap + dkP) + qv * dqP;
     }
   }
   __syncthreads();
@@ -996,7 +1035,8 @@ __global__ void __launch_bounds__(kNT)
       }
     }
   }
-  for (int t = tid; t < L; t += kNT) dbeta[row(t)] = dbs[t];
+  if (dbeta)
+    for (int t = tid; t < L; t += kNT) dbeta[row(t)] = dbs[t];
 }
 
 // ---------------------------------------------------------------------------
@@ -1036,8 +1076,9 @@ cudaError_t run_grad(const Problem &p, const BackwardIO &io,
   bw_grad_kernel<Tin, GATE><<<dim3(p.max_chunks, p.H), kNT, smem, s>>>(
       static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k),
       static_cast<const Tin *>(p.v), static_cast<const Tin *>(io.dout),
-      p.beta, b.g, Tb, b.Sbuf, Lam, b.Vn, dVn, io.dq, io.dk, io.dv, io.dbeta,
-      io.dla, b.table, b.nchunks, p.H, p.dk, p.dv);
+      p.beta, b.g, p.erase, p.write, Tb, b.Sbuf, Lam, b.Vn, dVn, io.dq, io.dk,
+      io.dv, io.dbeta, io.dla, io.derase, io.dwrite, b.table, b.nchunks, p.H,
+      p.dk, p.dv);
   return cudaGetLastError();
 }
 
@@ -1052,8 +1093,8 @@ cudaError_t run_wy(const Problem &p, const StagedBufs &b, float *Tb, float *Pb,
   if (e != cudaSuccess) return e;
   bw_wy_kernel<Tin, GATE><<<dim3(p.max_chunks, p.H), kNT, smem, s>>>(
       static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k),
-      static_cast<const Tin *>(p.v), p.beta, b.g, Tb, Pb, b.W, b.U, b.table,
-      b.nchunks, p.H, p.dk, p.dv);
+      static_cast<const Tin *>(p.v), p.beta, p.erase, p.write, b.g, Tb, Pb,
+      b.W, b.U, b.table, b.nchunks, p.H, p.dk, p.dv);
   return cudaGetLastError();
 }
 

@@ -821,34 +821,56 @@ extern "C" gdr_status gdr_chunk_fwd_segmented(
   return st;
 }
 
-extern "C" gdr_status gdr_backward(
-    const void *q, const void *k, const void *v, const float *log_alpha,
-    const float *beta, const float *initial_state, const void *d_out,
-    const float *d_final_state, float *dq, float *dk, float *dv,
-    float *d_log_alpha, float *d_beta, float *d_initial_state, int B, int T,
-    int H, int dk_, int dv_, cudaStream_t stream, const gdr_opts *opts) {
+namespace {
+
+// gdr_backward and gdr_backward_gdn2: with erase != nullptr the Gated
+// DeltaNet-2 gates (erase, write) replace beta, and their gradients go to
+// d_erase, d_write (the chunked backward only).
+gdr_status backward_entry(const void *q, const void *k, const void *v,
+                          const float *log_alpha, const float *beta,
+                          const float *erase, const float *write,
+                          const float *initial_state, const void *d_out,
+                          const float *d_final_state, float *dq, float *dk,
+                          float *dv, float *d_log_alpha, float *d_beta,
+                          float *d_erase, float *d_write,
+                          float *d_initial_state, int B, int T, int H,
+                          int dk_, int dv_, cudaStream_t stream,
+                          const gdr_opts *opts) {
   const gdr_opts o = opts ? *opts : default_opts();
+  const bool gates = erase != nullptr || write != nullptr;
   if (o.algo == GDR_ALGO_FUSED_TC) return GDR_ERR_UNSUPPORTED;
   const bool recurrent = o.algo == GDR_ALGO_RECURRENT;
+  if (recurrent && gates) return GDR_ERR_UNSUPPORTED;
   gdr_opts ov = o;
   if (recurrent) ov.algo = GDR_ALGO_AUTO;
   Problem p;
   // the forward pass's checks, with d_out in the place of out and
   // d_final_state in the place of final_state (the chunked backward runs
-  // chunks of 64 tokens whatever the forward used)
-  gdr_status st = validate(q, k, v, log_alpha, beta, initial_state, d_out,
-                           d_final_state, B, T, H, dk_, dv_, 64, ov, &p);
+  // chunks of 64 tokens whatever the forward used); the erase gate stands in
+  // for beta with the gates
+  gdr_status st = validate(q, k, v, log_alpha, gates ? erase : beta,
+                           initial_state, d_out, d_final_state, B, T, H, dk_,
+                           dv_, 64, ov, &p);
   if (st != GDR_OK) return st;
   if (p.nseq == 0 || p.H == 0) return GDR_OK;
-  if (!dq || !dk || !dv || !d_beta) return GDR_ERR_INVALID_ARGUMENT;
+  if (!dq || !dk || !dv) return GDR_ERR_INVALID_ARGUMENT;
+  if (gates ? (!write || !d_erase || !d_write) : !d_beta)
+    return GDR_ERR_INVALID_ARGUMENT;
   if ((o.gate == GDR_GATE_NONE) != (d_log_alpha == nullptr))
     return GDR_ERR_INVALID_ARGUMENT;
-  const void *grads[] = {dq, dk, dv, d_log_alpha, d_beta, d_initial_state};
-  for (const void *ptr : grads)
+  const void *ptrs[] = {dq, dk, dv, d_log_alpha, d_beta, d_initial_state,
+                        write, d_erase, d_write};
+  for (const void *ptr : ptrs)
     if (ptr && !aligned16(ptr)) return GDR_ERR_INVALID_ARGUMENT;
   // AUTO and STAGED: the chunked backward (the faster of the two on every
   // measured shape); RECURRENT: the reverse token recurrence
   const bool chunked = !recurrent && gdr::backward_chunked_applies(p);
+  if (gates && !chunked) return GDR_ERR_UNSUPPORTED;
+  if (gates) {
+    p.beta = nullptr;
+    p.erase = erase;
+    p.write = write;
+  }
   long long total_win = 0;
   const size_t bytes = chunked ? gdr::backward_chunked_bytes(p)
                                : gdr::backward_scratch_bytes(p, &total_win);
@@ -875,14 +897,45 @@ extern "C" gdr_status gdr_backward(
   io.dk = dk;
   io.dv = dv;
   io.dla = d_log_alpha;
-  io.dbeta = d_beta;
+  io.dbeta = gates ? nullptr : d_beta;
   io.ds0 = d_initial_state;
+  io.derase = gates ? d_erase : nullptr;
+  io.dwrite = gates ? d_write : nullptr;
   cudaError_t e =
       chunked ? gdr::backward_chunked_run(p, io, ws, stream)
               : gdr::backward_run(p, io, static_cast<float *>(ws), total_win,
                                   stream);
   cudaError_t f = cudaFreeAsync(ws, stream);
   return (e == cudaSuccess && f == cudaSuccess) ? GDR_OK : GDR_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" gdr_status gdr_backward(
+    const void *q, const void *k, const void *v, const float *log_alpha,
+    const float *beta, const float *initial_state, const void *d_out,
+    const float *d_final_state, float *dq, float *dk, float *dv,
+    float *d_log_alpha, float *d_beta, float *d_initial_state, int B, int T,
+    int H, int dk_, int dv_, cudaStream_t stream, const gdr_opts *opts) {
+  return backward_entry(q, k, v, log_alpha, beta, nullptr, nullptr,
+                        initial_state, d_out, d_final_state, dq, dk, dv,
+                        d_log_alpha, d_beta, nullptr, nullptr,
+                        d_initial_state, B, T, H, dk_, dv_, stream, opts);
+}
+
+extern "C" gdr_status gdr_backward_gdn2(
+    const void *q, const void *k, const void *v, const float *log_alpha,
+    const float *erase_gate, const float *write_gate,
+    const float *initial_state, const void *d_out,
+    const float *d_final_state, float *dq, float *dk, float *dv,
+    float *d_log_alpha, float *d_erase, float *d_write,
+    float *d_initial_state, int B, int T, int H, int dk_, int dv_,
+    cudaStream_t stream, const gdr_opts *opts) {
+  if (!erase_gate || !write_gate) return GDR_ERR_INVALID_ARGUMENT;
+  return backward_entry(q, k, v, log_alpha, nullptr, erase_gate, write_gate,
+                        initial_state, d_out, d_final_state, dq, dk, dv,
+                        d_log_alpha, nullptr, d_erase, d_write,
+                        d_initial_state, B, T, H, dk_, dv_, stream, opts);
 }
 
 extern "C" gdr_status gdr_device_error(cudaStream_t stream, int clear) {

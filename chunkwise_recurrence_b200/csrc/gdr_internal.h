@@ -91,6 +91,9 @@ struct BackwardIO {
   float *dla;            // fp32, layout of log_alpha (nullptr for no gate)
   float *dbeta;          // fp32 [ntok][H]
   float *ds0;            // fp32 [N][H][dk][dv], or nullptr
+  // Gated DeltaNet-2 gates' gradients (chunked backward; the gates are the
+  // Problem's erase / write): layouts of k and v, or nullptr
+  float *derase = nullptr, *dwrite = nullptr;
 };
 // Chunked backward pass (csrc/backward_chunked.cu): the gradients of the
 // chunked forward product by product, fp32, chunk-parallel except for one

@@ -497,6 +497,33 @@ GDR_API gdr_status gdr_backward(const void *q, const void *k, const void *v,
                                 cudaStream_t stream, const gdr_opts *opts);
 
 /*
+ * gdr_backward_gdn2 -- gdr_backward for gdr_chunk_fwd_gdn2: the gradients of
+ * the forward pass with Gated DeltaNet-2's erase and write gates, the gates'
+ * own included (the gate-aware backward the Gated DeltaNet-2 abstract,
+ * comparative-study page 2607.07953, pairs with its chunkwise algorithm).
+ *
+ * The chunked backward of gdr_backward with the read key b . k (erase gate b)
+ * on the row side of A and in W, the write key k in the state update and in
+ * P, and the target w . v (write gate w) in U; beta is 1.  Gradients, fp32,
+ * 16-byte aligned, written:
+ *   dq, dk [B][T][H][dk];  dv [B][T][H][dv];  d_log_alpha (layout of
+ *   log_alpha; NULL iff gate is NONE);  d_erase (layout of k) and d_write
+ *   (layout of v), required;  d_initial_state [N][H][dk][dv] or NULL.
+ * Inputs as for gdr_chunk_fwd_gdn2 (erase_gate, write_gate required) plus
+ * d_out and d_final_state as for gdr_backward.  opts->algo AUTO or STAGED;
+ * RECURRENT and FUSED_TC return GDR_ERR_UNSUPPORTED.  Scratch and status
+ * codes as for gdr_backward's chunked algorithm.
+ */
+GDR_API gdr_status gdr_backward_gdn2(
+    const void *q, const void *k, const void *v, const float *log_alpha,
+    const float *erase_gate, const float *write_gate,
+    const float *initial_state, const void *d_out,
+    const float *d_final_state, float *dq, float *dk, float *dv,
+    float *d_log_alpha, float *d_erase, float *d_write,
+    float *d_initial_state, int B, int T, int H, int dk_, int dv_,
+    cudaStream_t stream, const gdr_opts *opts);
+
+/*
  * gdr_efla_beta -- exact-flow step size (EFLA) for the delta rule.
  *
  * The delta rule's update is one explicit Euler step of length beta of the

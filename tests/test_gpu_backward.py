@@ -119,3 +119,82 @@ def test_backward_headline_shape_sampled():
     for algo in ("staged", "recurrent"):
         errs = _check(w, algo=algo)
         assert max(errs.values()) <= TOL
+
+
+# ---------------------------------------------------------------------------
+# gdr_backward_gdn2: the gate-aware backward of the Gated DeltaNet-2 forward,
+# against fp64 autograd through oracle.gdn2_fwd's token loop
+# (oracle.gdn2_grads, pinned by central differences).
+
+def _check_gdn2(w, seed=0, with_final=True):
+    from chunkwise_recurrence_b200.inputs import gdn2_gates
+    inp = generate(w, seed=seed)
+    erase, write = gdn2_gates(inp, seed=seed)
+    g = torch.Generator().manual_seed(seed + 200)
+    dO = torch.randn(inp.v.shape, generator=g).to(inp.v.dtype)
+    dS = (torch.randn(inp.nseq, w.H, w.dk, w.dv, generator=g) * 0.1
+          if with_final else None)
+    c = lambda t: None if t is None else t.cuda()  # noqa: E731
+    res = gdr.backward_gdn2(c(inp.q), c(inp.k), c(inp.v), c(erase),
+                            c(write), c(inp.log_alpha), c(inp.s0), c(dO),
+                            c(dS), gate=w.gate, cu_seqlens=c(inp.cu_seqlens))
+    torch.cuda.synchronize()
+    f = inp.f64()
+    ref = oracle.gdn2_grads(f["q"], f["k"], f["v"], erase.double().numpy(),
+                            write.double().numpy(), f["log_alpha"],
+                            gate=w.gate, initial_state=f["initial_state"],
+                            d_out=dO.double().numpy(),
+                            d_final_state=None if dS is None else dS.numpy(),
+                            cu_seqlens=f["cu_seqlens"])
+    errs = {}
+    for key in ("dq", "dk", "dv", "derase", "dwrite", "dlog_alpha"):
+        if ref[key] is None:
+            continue
+        errs[key] = rel_err(res[key].cpu().numpy(), ref[key])
+    if ref["dinitial_state"] is not None:
+        errs["ds0"] = rel_err(res["dinitial_state"].cpu().numpy(),
+                              ref["dinitial_state"])
+    for key, e in errs.items():
+        assert e <= TOL, (key, e, errs)
+    return errs
+
+
+@pytest.mark.parametrize("gate", ["none", "scalar", "channel"])
+@pytest.mark.parametrize("dtype,dk,dv", [("bf16", 128, 128), ("fp32", 32, 64)])
+def test_backward_gdn2_matches_autograd(gate, dtype, dk, dv):
+    w = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(
+        B=2, T=2 * 64 + 29, H=2, dk=dk, dv=dv, dtype=dtype, gate=gate,
+        init_state=True)
+    _check_gdn2(w, seed=7)
+
+
+def test_backward_gdn2_varlen_and_strong_decay():
+    w = WORKLOADS["gdn_varlen8_h16_d128_bf16"].with_(
+        varlen_nseq=4, varlen_lo=1, varlen_hi=200, H=2, gate="channel")
+    _check_gdn2(w, seed=8, with_final=False)
+    w2 = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(
+        B=1, T=64 + 40, H=1, decay_lo=3.0, decay_hi=3.0)
+    _check_gdn2(w2, seed=9)
+
+
+def test_backward_gdn2_with_gates_equal_to_beta_is_the_delta_rule():
+    """b = w = beta on every channel: the Gated DeltaNet-2 gradients are the
+    delta rule's, with dbeta the sum of the two gates' gradients over their
+    channels."""
+    w = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(B=2, T=100, H=2,
+                                                       dtype="fp32")
+    inp = generate(w, seed=10)
+    erase = inp.beta[..., None].expand(inp.k.shape).contiguous()
+    write = inp.beta[..., None].expand(inp.v.shape).contiguous()
+    g = torch.Generator().manual_seed(11)
+    dO = torch.randn(inp.v.shape, generator=g)
+    c = lambda t: None if t is None else t.cuda()  # noqa: E731
+    r2 = gdr.backward_gdn2(c(inp.q), c(inp.k), c(inp.v), c(erase), c(write),
+                           c(inp.log_alpha), c(inp.s0), c(dO), gate=w.gate)
+    r1 = gdr.backward(c(inp.q), c(inp.k), c(inp.v), c(inp.beta),
+                      c(inp.log_alpha), c(inp.s0), c(dO), gate=w.gate)
+    torch.cuda.synchronize()
+    for key in ("dq", "dk", "dv", "dlog_alpha", "dinitial_state"):
+        assert rel_err(r2[key].cpu().numpy(), r1[key].cpu().numpy()) <= 1e-4
+    db = (r2["derase"].sum(-1) + r2["dwrite"].sum(-1)).cpu().numpy()
+    assert rel_err(db, r1["dbeta"].cpu().numpy()) <= 1e-4
