@@ -781,10 +781,21 @@ def run_backward(args, w):
     stream = torch.cuda.current_stream(dev)
 
     # --algo auto / staged: the chunked backward (gdr_backward's AUTO);
-    # recurrent: the reverse token recurrence
+    # recurrent: the reverse token recurrence.  --gdn2: gdr_backward_gdn2
+    # with Gated DeltaNet-2's erase and write gates (chunked only)
     algo = "recurrent" if args.algo == "recurrent" else "auto"
+    g2 = args.gdn2
+    if g2:
+        if algo == "recurrent":
+            raise SystemExit("--gdn2 --backward runs the chunked backward")
+        from chunkwise_recurrence_b200.inputs import gdn2_gates
+        er, wr = (t.to(dev) for t in gdn2_gates(inp, seed=args.seed))
 
     def step():
+        if g2:
+            return gdr.backward_gdn2(q, k, v, er, wr, la, s0, dO, dS,
+                                     gate=w.gate, cu_seqlens=cu,
+                                     stream=stream)
         return gdr.backward(q, k, v, b, la, s0, dO, dS, gate=w.gate,
                             cu_seqlens=cu, stream=stream, algo=algo)
 
@@ -808,6 +819,8 @@ def run_backward(args, w):
     # gradients (fp32) written once, states in and out
     by = ntok * H * (esz * (2 * dk + 2 * dv) + 4 + la_b +
                      4 * (2 * dk + dv) + 4 + la_b)
+    if g2:   # the gates read and their gradients written, in place of beta's
+        by += ntok * H * (2 * 4 * (dk + dv) - 8)
     by += inp.nseq * H * dk * dv * 4 * (2 + (1 if inp.s0 is not None else 0))
     gbs = by / (statistics.mean(per_step) / 1e3) / 1e9
     cols = dk >= 32 and dv >= 32   # the column-split kernel + its reduction
@@ -829,7 +842,8 @@ def run_backward(args, w):
         # chunk table, cumsum (with a gate), WY, prep, two scans, V_new,
         # gradients
         launches = 7 + (0 if w.gate == "none" else 1)
-        algo_name = "chunked (64-token chunks, fp32)"
+        algo_name = "chunked (64-token chunks, fp32)" + (
+            ", Gated DeltaNet-2 gates" if g2 else "")
     tflops = flops / (statistics.mean(per_step) / 1e3) / 1e12
     line = {
         "metric": BACKWARD_METRIC, "value": ntok / (ms / 1e3),

@@ -476,10 +476,10 @@ GDR_API gdr_status gdr_decode_step_fg2(const void *q, const void *k,
  *   dq, dk         [B][T][H][dk];   dv [B][T][H][dv];   d_beta [B][T][H];
  *   d_log_alpha    the layout of log_alpha; NULL iff gate is NONE;
  *   d_initial_state [N][H][dk][dv], or NULL to skip.
- * Scratch, chunked: the staged path's (about (2 dk + 2 dv) ntok H floats
- * plus one state per chunk and head), T and P of every chunk (2 * 64 * 64
- * floats per chunk and head), one more state per chunk and head, and
- * ntok * H * dv floats.  Recurrent (dk, dv >= 32): (ntok/8 + N) * H + 8 * N
+ * Scratch, chunked, in floats: (1 + dk + 3 dv) ntok H (g, W, U, V_new,
+ * dV_new) plus, per chunk of 64 tokens and head, 2 * 64 * 64 (T, P),
+ * 4 dk dv (the chunk-start state, dL/dS at the chunk end, Dm, Bm) and
+ * dk * dk (the chunk's state map): about 4 GB at B8 H16 T4096 d128.  Recurrent (dk, dv >= 32): (ntok/8 + N) * H + 8 * N
  * * H states of dk*dv floats, plus the row-sum shares, 2 * (dv/32) * ntok *
  * H * dk floats (3 * for the channel gate); for dk or dv = 16: (ntok/16 +
  * N) * H + 16 * N * H states.  Allocated stream-ordered on `stream` from the library's per-device memory
