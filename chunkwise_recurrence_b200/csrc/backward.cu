@@ -30,8 +30,9 @@
 // column-split kernel further down runs the same three sweeps on dv / 32
 // CTAs per (sequence, head).  Both evaluate every token's rank-one products
 // on CUDA cores (about 29 dk dv flops per token and head over the three
-// sweeps), so they are bound by fp32 issue, not by HBM; a chunked
-// tensor-core backward is the next step.
+// sweeps), so they are bound by fp32 issue, not by HBM.  gdr_backward runs
+// them as its RECURRENT algorithm; the chunked backward
+// (backward_chunked.cu) is the default.
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>

@@ -694,7 +694,8 @@ constexpr int kBIG = kTS + kBC * kCP;
 constexpr int kSLo = kBIG + 5 * kBC * kP;
 constexpr int kXT = kSLo + 2 * kSl * kP + kBC * kRS;
 constexpr int kSM = kXT + 3 * kBC * kSl;
-constexpr int kSmall = 64 * 3 + 128 * 2 + 16;
+constexpr int kSmall = 64 * 3 + 128 * 3 + 16;
+static_assert(kBC * kSl <= 2 * kNT, "two slice elements per thread");
 constexpr int kGradSmemFloats = kSM + kSmall;
 static_assert(kBIG + 3 * kBC * kP + 3 * kBC * kCP <= kSLo, "phase-2 tiles");
 static_assert(kGradSmemFloats * 4 <= 232448, "shared memory");
@@ -729,7 +730,7 @@ __global__ void __launch_bounds__(kNT)
   float *Ss = sm + kSLo, *Ls = Ss + kSl * kP, *Rs = Ls + kSl * kP;
   float *X1 = sm + kXT, *X2 = X1 + kBC * kSl, *X3 = X2 + kBC * kSl;
   float *bs = sm + kSM, *dbs = bs + 64, *dgs = dbs + 64, *dgC = dgs + 64,
-        *gC = dgC + 128, *red = gC + 128;
+        *gC = dgC + 128, *gR = gC + 128, *red = gR + 128;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t base = (size_t)ci.tok0 * H + h;   // row of token 0
   auto row = [&](int t) { return base + (size_t)t * H; };
@@ -775,6 +776,23 @@ __global__ void __launch_bounds__(kNT)
       Ss[cc * kP + c] = Sg[(size_t)(c0 + cc) * dv + c];
       Ls[cc * kP + c] = Lg[(size_t)(c0 + cc) * dv + c];
     }
+    // the elementwise pass's inputs (two elements per thread), fetched
+    // before the products so that their latency hides behind them
+    float pg[2], pq[2], pk[2], pb[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int idx = tid + u * kNT;
+      pg[u] = pq[u] = pk[u] = 0.f;
+      pb[u] = 1.f;
+      if (idx < L * kSl) {
+        const int t = idx / kSl, c = c0 + idx % kSl;
+        const size_t o = row(t) * dk + c;
+        pg[u] = gt(t, c);
+        pq[u] = ldf(q + o);
+        pk[u] = ldf(k + o);
+        if (erase) pb[u] = erase[o];
+      }
+    }
     for (int idx = tid; idx < kBC * kSl; idx += kNT) {
       const int t = idx / kSl, cc = idx % kSl;
       // the read key times e^g
@@ -818,12 +836,15 @@ __global__ void __launch_bounds__(kNT)
     // elementwise: dq = X1 e^g; dk = -X2 e^g + X3 e^{g_C - g}; the decay
     // gradient of the factors e^g (on q and on the read key) and
     // e^{g_C - g} (on the update key)
-    for (int idx = tid; idx < L * kSl; idx += kNT) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int idx = tid + u * kNT;
+      if (idx >= L * kSl) continue;
       const int t = idx / kSl, cc = idx % kSl, c = c0 + cc;
-      const float gg = gt(t, c), e = __expf(gg), ec = __expf(gC[c] - gg);
+      const float gg = pg[u], e = __expf(gg), ec = __expf(gC[c] - gg);
       const size_t o = row(t) * dk + c;
-      const float qv = ldf(q + o), kv = ldf(k + o);
-      const float bv = erase ? erase[o] : 1.f;   // read key = bv kv
+      const float qv = pq[u], kv = pk[u];
+      const float bv = pb[u];   // read key = bv kv
       const float x1 = X1[t * kSl + cc], x2 = X2[t * kSl + cc],
                   x3 = X3[t * kSl + cc];
       // read-key gradient -x2 e^g, write-key gradient x3 e^{g_C - g}
@@ -884,12 +905,13 @@ __global__ void __launch_bounds__(kNT)
   const int ref = (L - 1) / 2;
   bool fact = true;
   if (GATE == 2) {
+    for (int c = tid; c < dk; c += kNT) gR[c] = gt(ref, c);
     float spread = 0.f;
     for (int idx = tid; idx < L * dk; idx += kNT) {
       const int t = idx / dk, c = idx % dk;
       spread = fmaxf(spread, fabsf(gt(t, c) - gt(ref, c)));
     }
-    fact = block_max(spread, red) <= kFactRange;
+    fact = block_max(spread, red) <= kFactRange;   // (its barriers publish gR)
   }
   for (int idx = tid; idx < kBC * dk; idx += kNT) {
     const int t = idx / dk, c = idx % dk;
@@ -959,16 +981,17 @@ __global__ void __launch_bounds__(kNT)
   if (GATE != 2 || fact) {
     auto pair_out = [&](int t, int c, float r1, float r2, float r3, float r4) {
       if (t >= L) return;
-      const float d = (GATE == 2) ? gt(t, c) - gt(ref, c) : 0.f;
+      const float d = (GATE == 2) ? gt(t, c) - gR[c] : 0.f;
       const float up = __expf(d), dn = __expf(-d);
       const float drho = up * r1, dkap = dn * r2, dqP = up * r3, dkP = dn * r4;
       const size_t o = row(t) * dk + c;
-      const float kv = ldf(k + o), qv = ldf(q + o);
-      const float bv = erase ? erase[o] : 1.f;   // read key = bv kv
+      // the key, query and read key back from their rescaled tiles
+      const float kv = Kd[t * kP + c] * up, qv = Qu[t * kP + c] * dn,
+                  rv = Ku[t * kP + c] * dn;
       dq[o] += dqP;
-      dkg[o] += bv * drho + dkap + dkP;
+      dkg[o] += (erase ? erase[o] : 1.f) * drho + dkap + dkP;
       if (erase) derase[o] += kv * drho;
-      const float dgv = bv * kv * drho - kv * (dkap + dkP) + qv * dqP;
+      const float dgv = rv * drho - kv * (dkap + dkP) + qv * dqP;
       if (GATE == 2) dla[o] += dgv;
       if (GATE == 1) atomicAdd(&dgs[t], dgv);
     };

@@ -34,13 +34,15 @@ struct Problem {
   gdr_dtype dtype;
   gdr_gate gate;
   int max_chunks;     // upper bound on the number of chunks over all sequences
-  // Gated DeltaNet-2 gates (staged path only; nullptr otherwise): the
-  // per-key-channel erase gate [ntok][H][dk] and per-value-channel write
-  // gate [ntok][H][dv] that replace beta
+  // Gated DeltaNet-2 gates (staged path, the fused channel-gate kernel, the
+  // chunked backward; nullptr otherwise): the per-key-channel erase gate
+  // [ntok][H][dk] and per-value-channel write gate [ntok][H][dv] that
+  // replace beta
   const float *erase = nullptr, *write = nullptr;
-  // FG^2-GDN's per-key-channel rate [ntok][H][dk] (staged path and decode
-  // only; nullptr otherwise): the write key of token t is wkey_t . k_t and
-  // the read key k_t; `write` (or nullptr for ones) then scales the target
+  // FG^2-GDN's per-key-channel rate [ntok][H][dk] (staged path, the fused
+  // channel-gate kernel; nullptr otherwise): the write key of token t is
+  // wkey_t . k_t and the read key k_t; `write` (or nullptr for ones) then
+  // scales the target
   const float *wkey = nullptr;
 };
 
