@@ -916,12 +916,12 @@ def run_gdn2(args, w, kind="gdn2"):
     sT = torch.empty(inp.nseq, w.H, w.dk, w.dv, dtype=torch.float32,
                      device=dev)
     stream = torch.cuda.current_stream(dev)
-    # the fused kernel takes these gates with the channel-wise decay (bf16,
-    # d = 128, C = 64); every other shape runs the staged path
+    # the fused kernel takes these gates for bf16, d = 128, C = 64 (a scalar
+    # or absent decay as the channel-wise one with all channels equal);
+    # every other shape runs the staged path
     algo_used = args.algo
     if algo_used == "auto":
-        algo_used = ("fused_tc" if (w.gate == "channel" and
-                                    w.dtype == "bf16" and w.dk == 128 and
+        algo_used = ("fused_tc" if (w.dtype == "bf16" and w.dk == 128 and
                                     w.dv == 128 and w.chunk == 64 and
                                     gdr_fused_available())
                      else "staged")

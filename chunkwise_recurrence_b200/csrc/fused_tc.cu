@@ -1506,17 +1506,49 @@ cudaError_t launch(const Problem &pr, const float *gk, const float *gv,
   return cudaGetLastError();
 }
 
+// The per-channel gate variants run on the channel-gate kernel; a scalar or
+// absent decay is handed to it as the channel-wise decay with every channel
+// equal (log-decays expanded into scratch, [ntok][H][128] fp32).
+__global__ void expand_log_decay_kernel(const float *__restrict__ la,
+                                        float *__restrict__ out, long long n4) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const long long row = i / (kD / 4);   // (token, head)
+  const float x = la ? la[row] : 0.f;
+  reinterpret_cast<float4 *>(out)[i] = make_float4(x, x, x, x);
+}
+
+bool variant_needs_expand(const Problem &p) {
+  return (p.erase || p.write || p.wkey) && p.gate != GDR_GATE_CHANNEL;
+}
+
 }  // namespace
 
 bool fused_tc_applies(const Problem &p) {
-  // the per-channel gate variants run with the channel-wise decay only
-  const bool variant = p.erase || p.write || p.wkey;
   return p.dtype == GDR_BF16 && p.dk == kD && p.dv == kD && p.chunk == kC &&
-         (long long)p.nseq * p.H < (1ll << 31) &&
-         (!variant || p.gate == GDR_GATE_CHANNEL);
+         (long long)p.nseq * p.H < (1ll << 31);
 }
 
-cudaError_t fused_tc_run(const Problem &p, cudaStream_t s) {
+size_t fused_tc_scratch_bytes(const Problem &p) {
+  return variant_needs_expand(p) ? (size_t)p.ntok * p.H * kD * sizeof(float)
+                                 : 0;
+}
+
+cudaError_t fused_tc_run(const Problem &p, void *scratch, cudaStream_t s) {
+  if (variant_needs_expand(p)) {
+    if (!scratch) return cudaErrorInvalidValue;
+    float *la = static_cast<float *>(scratch);
+    const long long n4 = (long long)p.ntok * p.H * (kD / 4);
+    if (n4 > 0) {
+      const int bs = 256;
+      expand_log_decay_kernel<<<(unsigned)((n4 + bs - 1) / bs), bs, 0, s>>>(
+          p.gate == GDR_GATE_SCALAR ? p.log_alpha : nullptr, la, n4);
+    }
+    Problem pc = p;
+    pc.gate = GDR_GATE_CHANNEL;
+    pc.log_alpha = la;
+    return fused_tc_run(pc, nullptr, s);
+  }
   if (p.erase) return launch<2, 1>(p, p.erase, p.write, s);
   if (p.wkey) return launch<2, 2>(p, p.wkey, p.write, s);
   switch (p.gate) {

@@ -121,13 +121,20 @@ gdr_status scratch_alloc(void **ptr, size_t bytes, cudaStream_t s) {
 
 gdr_status run(const Problem &p, gdr_algo algo, cudaStream_t stream) {
   if (p.nseq == 0 || p.H == 0) return GDR_OK;
-  // (the Gated DeltaNet-2 gates and FG^2-GDN's rate run on the fused path
-  // with the channel-wise decay only: fused_tc_applies)
   const bool tc = gdr::fused_tc_applies(p);
   if (algo == GDR_ALGO_FUSED_TC && !tc) return GDR_ERR_UNSUPPORTED;
   if (tc && algo != GDR_ALGO_STAGED) {
-    cudaError_t e = gdr::fused_tc_run(p, stream);
-    return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+    // (the gate variants with a scalar or no decay take their log-decays
+    // expanded per channel, in scratch)
+    const size_t bytes = gdr::fused_tc_scratch_bytes(p);
+    void *ws = nullptr;
+    if (bytes) {
+      gdr_status st = scratch_alloc(&ws, bytes, stream);
+      if (st != GDR_OK) return st;
+    }
+    cudaError_t e = gdr::fused_tc_run(p, ws, stream);
+    cudaError_t f = ws ? cudaFreeAsync(ws, stream) : cudaSuccess;
+    return (e == cudaSuccess && f == cudaSuccess) ? GDR_OK : GDR_ERR_CUDA;
   }
   void *ws = nullptr;
   gdr_status st = scratch_alloc(&ws, gdr::staged_workspace_bytes(p), stream);

@@ -66,7 +66,10 @@ cudaError_t staged_chunks_run(const Problem &p, void *workspace,
 
 // Fused tensor-core path.
 bool fused_tc_applies(const Problem &p);
-cudaError_t fused_tc_run(const Problem &p, cudaStream_t s);
+// scratch fused_tc_run needs (bytes; 0 for most problems: the gate variants
+// with a scalar or no decay take their log-decays expanded per channel)
+size_t fused_tc_scratch_bytes(const Problem &p);
+cudaError_t fused_tc_run(const Problem &p, void *scratch, cudaStream_t s);
 // Reads (and optionally clears) the fused kernel's sticky device error word.
 cudaError_t fused_tc_read_error(unsigned *word, bool clear);
 

@@ -214,13 +214,14 @@ GDR_API gdr_status gdr_chunk_fwd_host(const void *q, const void *k, const void *
  *   write_gate  [B][T][H][dv] fp32 (device, 16-byte aligned), required;
  * (packed layouts with cu_seqlens as for gdr_chunk_fwd).  The decay form is
  * opts->gate (NONE, SCALAR or CHANNEL) as before.  Paths as for
- * gdr_chunk_fwd, except that the fused tensor-core kernel takes these gates
- * with the channel-wise decay (CHANNEL, bf16, dk = dv = 128, chunk = 64)
- * only: AUTO runs it there and the staged path (fp32 CUDA-core arithmetic)
- * everywhere else; FUSED_TC on another decay form returns
- * GDR_ERR_UNSUPPORTED.  On the fused path b . k and w . v are formed in
- * fp32 and rounded once to the fp16 operands.  Status codes as for
- * gdr_chunk_fwd (GDR_ERR_RANGE from the fused path as there).
+ * gdr_chunk_fwd (fused tensor-core kernel for bf16, dk = dv = 128,
+ * chunk = 64; the staged path otherwise).  The fused kernel runs these gates
+ * on its channel-wise decay: a scalar or absent decay is expanded into
+ * scratch as the channel-wise decay with every channel equal (ntok * H * 128
+ * floats, from `stream`, GDR_ERR_OUT_OF_MEMORY on failure).  On the fused
+ * path b . k and w . v are formed in fp32 and rounded once to the fp16
+ * operands.  Status codes as for gdr_chunk_fwd (GDR_ERR_RANGE from the fused
+ * path as for its channel gate).
  */
 GDR_API gdr_status gdr_chunk_fwd_gdn2(const void *q, const void *k,
                                       const void *v, const float *log_alpha,
@@ -255,10 +256,10 @@ GDR_API gdr_status gdr_chunk_fwd_gdn2(const void *q, const void *k,
  *           FG^2-GDN (c = 1): FG^2-GDN+'s per-value-channel scaling;
  * (packed layouts with cu_seqlens as for gdr_chunk_fwd).  The decay form is
  * opts->gate (NONE, SCALAR or CHANNEL).  Paths as for gdr_chunk_fwd_gdn2:
- * the fused tensor-core kernel with the channel-wise decay (bf16,
- * dk = dv = 128, chunk = 64), where it forms beta_k . k and c . v in fp32
- * and rounds them once to its fp16 operands; the staged path otherwise.
- * Status codes as for gdr_chunk_fwd.
+ * the fused tensor-core kernel for bf16, dk = dv = 128, chunk = 64 (any
+ * decay form, expanded as there), where it forms beta_k . k and c . v in
+ * fp32 and rounds them once to its fp16 operands; the staged path
+ * otherwise.  Status codes as for gdr_chunk_fwd.
  */
 GDR_API gdr_status gdr_chunk_fwd_fg2(const void *q, const void *k,
                                      const void *v, const float *log_alpha,

@@ -268,11 +268,9 @@ def test_gdn2_rejects_bad_arguments(lib):
     assert c(wr=None) == INVALID
     assert c(wr=A + 4) == INVALID         # 16-byte alignment
     assert c(la=None) == INVALID          # a decay gate needs log_alpha
-    # the fused path takes these gates with the channel-wise decay only
-    # (rejected before any CUDA call; the channel-gate case would launch,
-    # so it is not called with these placeholder addresses)
-    assert c(algo=2, gate=1) == UNSUPPORTED
-    assert c(algo=2, gate=0, la=None) == UNSUPPORTED
+    # the fused path takes bf16 only (rejected before any CUDA call; the
+    # cases it takes would launch, so they are not called with these
+    # placeholder addresses)
     assert c(algo=2, dtype=1) == UNSUPPORTED
     assert c(dk=48) == UNSUPPORTED
     assert c(q=None, k=None, v=None, la=None, er=None, wr=None, out=None,
@@ -296,11 +294,9 @@ def test_fg2_rejects_bad_arguments(lib):
     assert c(bk=A + 4) == INVALID         # 16-byte alignment
     assert c(bv=A + 8) == INVALID
     assert c(la=None) == INVALID          # a decay gate needs log_alpha
-    # the fused path takes the rate with the channel-wise decay only
-    # (rejected before any CUDA call; the channel-gate case would launch)
-    assert c(algo=2, gate=1) == UNSUPPORTED
-    assert c(algo=2, gate=1, bv=A) == UNSUPPORTED
+    # the fused path takes bf16 only (rejected before any CUDA call)
     assert c(algo=2, dtype=1) == UNSUPPORTED
+    assert c(algo=2, dtype=1, bv=A) == UNSUPPORTED
     assert c(dk=48) == UNSUPPORTED
     assert c(q=None, k=None, v=None, la=None, bk=None, out=None, gate=0,
              B=0) == OK

@@ -104,14 +104,23 @@ def test_fg2_with_a_uniform_rate_is_the_delta_rule():
     assert rel_err(o2.cpu().numpy(), o1.cpu().numpy()) <= 1e-5
 
 
-def test_fg2_fused_algo_needs_the_channel_decay():
-    w = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=1, T=64, H=1)
+@pytest.mark.parametrize("gate", ["scalar", "none"])
+def test_fg2_fused_with_a_scalar_or_no_decay(gate):
+    """The fused kernel takes the rate with a scalar or absent decay as the
+    channel-wise decay with every channel equal."""
+    w = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=2, T=2 * 64 + 19, H=2,
+                                                       gate=gate)
     inp = generate(w, seed=55)
-    beta_k, _ = fg2_gates(inp, seed=55)
-    with pytest.raises(gdr.GdrError):
-        gdr.chunk_fwd_fg2(_dev(inp.q), _dev(inp.k), _dev(inp.v),
-                          _dev(beta_k), None, _dev(inp.log_alpha),
-                          algo="fused_tc", gate=w.gate)
+    beta_k, beta_v = fg2_gates(inp, seed=55)
+    o, s = gdr.chunk_fwd_fg2(_dev(inp.q), _dev(inp.k), _dev(inp.v),
+                             _dev(beta_k), _dev(beta_v), _dev(inp.log_alpha),
+                             _dev(inp.s0), algo="fused_tc", gate=w.gate)
+    torch.cuda.synchronize()
+    assert gdr.device_error() == 0
+    ro, rs = oracle.fg2_fwd(_f(inp.q), _f(inp.k), _f(inp.v), _f(beta_k),
+                            _f(beta_v), _f(inp.log_alpha), gate, _f(inp.s0))
+    assert out_err(o.float().cpu().numpy(), ro, "bf16") <= TOL["bf16"]
+    assert rel_err(s.cpu().numpy(), rs) <= TOL["bf16"]
 
 
 # ---------------------------------------------------------------------------

@@ -86,14 +86,24 @@ def test_gdn2_with_gates_equal_to_beta_is_the_delta_rule():
     assert rel_err(o2.cpu().numpy(), o1.cpu().numpy()) <= 1e-5
 
 
-def test_gdn2_fused_algo_needs_the_channel_decay():
-    w = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=1, T=64, H=1)
+@pytest.mark.parametrize("gate", ["scalar", "none"])
+def test_gdn2_fused_with_a_scalar_or_no_decay(gate):
+    """The fused kernel takes the gates with a scalar or absent decay as the
+    channel-wise decay with every channel equal."""
+    w = WORKLOADS["gdn_b8_h16_t4096_d128_bf16"].with_(B=2, T=2 * 64 + 19, H=2,
+                                                       gate=gate)
     inp = generate(w, seed=44)
     erase, write = gdn2_gates(inp, seed=44)
-    with pytest.raises(gdr.GdrError):
-        gdr.chunk_fwd_gdn2(_dev(inp.q), _dev(inp.k), _dev(inp.v), _dev(erase),
-                           _dev(write), _dev(inp.log_alpha), algo="fused_tc",
-                           gate=w.gate)
+    o, s = gdr.chunk_fwd_gdn2(_dev(inp.q), _dev(inp.k), _dev(inp.v),
+                              _dev(erase), _dev(write), _dev(inp.log_alpha),
+                              _dev(inp.s0), algo="fused_tc", gate=w.gate)
+    torch.cuda.synchronize()
+    assert gdr.device_error() == 0
+    f = lambda t: None if t is None else t.double().numpy()  # noqa: E731
+    ro, rs = oracle.gdn2_fwd(f(inp.q), f(inp.k), f(inp.v), f(erase), f(write),
+                             f(inp.log_alpha), gate, f(inp.s0))
+    assert out_err(o.float().cpu().numpy(), ro, "bf16") <= TOL["bf16"]
+    assert rel_err(s.cpu().numpy(), rs) <= TOL["bf16"]
 
 
 # ---------------------------------------------------------------------------
