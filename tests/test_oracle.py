@@ -867,6 +867,76 @@ def test_gdn2_gradients_match_finite_differences():
         np.testing.assert_allclose(g["final_state"], sT, atol=1e-13)
 
 
+@pytest.mark.parametrize("plus", [False, True])
+def test_fg2_gradients_match_finite_differences(plus):
+    """The FG^2-GDN autograd gradients (oracle.fg2_grads, a PyTorch token
+    loop) agree with central differences of the numpy loop's loss
+    (oracle.fg2_fwd), element by element, for every input -- the key-side
+    rate and, for FG^2-GDN+, the value scaling included -- and every gate
+    kind."""
+    rng = np.random.default_rng(51 + plus)
+    for gate in ("none", "scalar", "channel"):
+        c = _rand_case(rng, B=1, T=5, H=1, dk=3, dv=2, gate=gate)
+        case = dict(q=c["q"], k=c["k"], v=c["v"],
+                    beta_k=rng.uniform(0.1, 0.9, size=(1, 5, 1, 3)),
+                    beta_v=(rng.uniform(0.1, 1.5, size=(1, 5, 1, 2))
+                            if plus else None),
+                    log_alpha=c["log_alpha"], initial_state=c["initial_state"])
+        dO = rng.standard_normal(c["v"].shape)
+        dS = rng.standard_normal((1, 1, 3, 2))
+        g = oracle.fg2_grads(**case, gate=gate, d_out=dO, d_final_state=dS)
+
+        def loss(x):
+            o, sT = oracle.fg2_fwd(x["q"], x["k"], x["v"], x["beta_k"],
+                                   x["beta_v"], x["log_alpha"], gate,
+                                   x["initial_state"])
+            return float((o * dO).sum() + (sT * dS).sum())
+
+        names = ["q", "k", "v", "beta_k", "initial_state"]
+        if plus:
+            names.append("beta_v")
+        if gate != "none":
+            names.append("log_alpha")
+        eps = 1e-6
+        for key in names:
+            x = case[key]
+            fd = np.zeros_like(x)
+            for i in np.ndindex(x.shape):
+                xp, xm = x.copy(), x.copy()
+                xp[i] += eps
+                xm[i] -= eps
+                fd[i] = (loss({**case, key: xp}) - loss({**case, key: xm})) / (
+                    2 * eps)
+            np.testing.assert_allclose(g["d" + key], fd, atol=2e-7, rtol=1e-6,
+                                       err_msg=f"{gate} {key}")
+        if not plus:
+            assert g["dbeta_v"] is None
+        o, sT = oracle.fg2_fwd(case["q"], case["k"], case["v"],
+                               case["beta_k"], case["beta_v"],
+                               case["log_alpha"], gate, case["initial_state"])
+        np.testing.assert_allclose(g["out"], o, atol=1e-13)
+        np.testing.assert_allclose(g["final_state"], sT, atol=1e-13)
+
+
+def test_fg2_gradients_reduce_to_the_delta_rule():
+    """A key-side rate of beta on every channel (no value scaling) is the
+    delta rule: the gradients equal oracle.gdr_grads', with dbeta the rate's
+    gradient summed over its channels."""
+    rng = np.random.default_rng(53)
+    c = _rand_case(rng, B=1, T=6, H=2, dk=3, dv=2, gate="channel")
+    dO = rng.standard_normal(c["v"].shape)
+    g1 = oracle.gdr_grads(c["q"], c["k"], c["v"], c["beta"], c["log_alpha"],
+                          gate="channel", initial_state=c["initial_state"],
+                          d_out=dO)
+    bk = np.repeat(c["beta"][..., None], 3, axis=-1)
+    g2 = oracle.fg2_grads(c["q"], c["k"], c["v"], bk, None, c["log_alpha"],
+                          gate="channel", initial_state=c["initial_state"],
+                          d_out=dO)
+    for key in ("dq", "dk", "dv", "dlog_alpha", "dinitial_state"):
+        np.testing.assert_allclose(g2[key], g1[key], atol=1e-12)
+    np.testing.assert_allclose(g2["dbeta_k"].sum(-1), g1["dbeta"], atol=1e-12)
+
+
 def test_gdn2_gradients_reduce_to_the_delta_rule():
     """Both gates equal to beta_t on every channel: the Gated DeltaNet-2
     gradients of q, k, v, log-alpha and the initial state are the delta
