@@ -17,7 +17,7 @@ import torch
 __all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_noalloc",
            "chunk_fwd_segmented", "chunk_fwd_gdn2", "chunk_fwd_fg2",
            "decode_step", "decode_step_gdn2", "decode_step_fg2",
-           "efla_beta", "backward", "backward_gdn2",
+           "efla_beta", "backward", "backward_gdn2", "backward_fg2",
            "device_error", "status_string",
            "algo_applies", "fused_tc_available",
            "GdrError", "load_library", "LIB_PATH", "GATES", "ALGOS",
@@ -38,7 +38,8 @@ EXPORTED_SYMBOLS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_device_error",
                     "gdr_efla_beta", "gdr_backward",
                     "gdr_chunk_fwd_segmented", "gdr_chunk_fwd_gdn2",
                     "gdr_decode_step_gdn2", "gdr_chunk_fwd_fg2",
-                    "gdr_decode_step_fg2", "gdr_backward_gdn2")
+                    "gdr_decode_step_fg2", "gdr_backward_gdn2",
+                    "gdr_backward_fg2")
 # size of the static scratch array behind gdr_chunk_fwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -95,10 +96,11 @@ def load_library(path: str = LIB_PATH):
     lib.gdr_backward.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, fp, fp, fp,
                                  fp, fp, fp, i, i, i, i, i, vp,
                                  ctypes.POINTER(_Opts)]
-    lib.gdr_backward_gdn2.restype = ctypes.c_int
-    lib.gdr_backward_gdn2.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, fp,
-                                      fp, fp, fp, fp, fp, fp, i, i, i, i, i,
-                                      vp, ctypes.POINTER(_Opts)]
+    for name in ("gdr_backward_gdn2", "gdr_backward_fg2"):
+        f = getattr(lib, name)
+        f.restype = ctypes.c_int
+        f.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, fp, fp, fp, fp, fp,
+                      fp, fp, i, i, i, i, i, vp, ctypes.POINTER(_Opts)]
     lib.gdr_efla_beta.restype = ctypes.c_int
     lib.gdr_efla_beta.argtypes = [vp, fp, fp, i, i, i, i, vp]
     lib.gdr_device_error.restype = ctypes.c_int
@@ -483,6 +485,42 @@ def backward_gdn2(q, k, v, erase_gate, write_gate, log_alpha, initial_state,
         raise GdrError(rc, "gdr_backward_gdn2")
     return dict(dq=gq, dk=gk, dv=gv, derase=ge, dwrite=gw, dlog_alpha=gla,
                 dinitial_state=gs0)
+
+
+def backward_fg2(q, k, v, beta_k, beta_v, log_alpha, initial_state, d_out,
+                 d_final_state=None, *, gate: str | None = None,
+                 cu_seqlens=None, need_initial_state_grad: bool = True,
+                 algo: str = "auto", stream=None):
+    """Run ``gdr_backward_fg2``: gradients of ``chunk_fwd_fg2``'s outputs
+    (same inputs; ``beta_v`` None for FG^2-GDN) given dL/d out and,
+    optionally, dL/d final_state.  Returns a dict of fp32 CUDA tensors dq,
+    dk, dv, dbeta_k, dbeta_v (None without beta_v), dlog_alpha (None without
+    a gate) and dinitial_state (None unless requested)."""
+    lib = load_library()
+    B, T, H, dk, dv, nseq = _shapes(q, v, cu_seqlens)
+    g = _gate_of(log_alpha, gate)
+    f32 = lambda t: torch.empty(t.shape, dtype=torch.float32,  # noqa: E731
+                                device=q.device)
+    gq, gk, gv, gbk = f32(q), f32(k), f32(v), f32(beta_k)
+    gbv = None if beta_v is None else f32(beta_v)
+    gla = None if log_alpha is None else f32(log_alpha)
+    gs0 = (torch.empty(nseq, H, dk, dv, dtype=torch.float32, device=q.device)
+           if need_initial_state_grad else None)
+    opts = _Opts(DTYPES[q.dtype], GATES[g],
+                 None if cu_seqlens is None else cu_seqlens.data_ptr(),
+                 nseq if cu_seqlens is not None else 0, ALGOS[algo])
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    rc = lib.gdr_backward_fg2(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta_k),
+        _ptr(beta_v), _ptr(initial_state), _ptr(d_out), _ptr(d_final_state),
+        _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gla), _ptr(gbk), _ptr(gbv),
+        _ptr(gs0), B, T, H, dk, dv, ctypes.c_void_p(stream.cuda_stream),
+        ctypes.byref(opts))
+    if rc != 0:
+        raise GdrError(rc, "gdr_backward_fg2")
+    return dict(dq=gq, dk=gk, dv=gv, dbeta_k=gbk, dbeta_v=gbv,
+                dlog_alpha=gla, dinitial_state=gs0)
 
 
 def efla_beta(k, beta, *, out=None, stream=None):

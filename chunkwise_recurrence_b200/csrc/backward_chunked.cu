@@ -342,6 +342,7 @@ __global__ void __launch_bounds__(kNT)
                  const Tin *__restrict__ v, const float *__restrict__ beta,
                  const float *__restrict__ erase,
                  const float *__restrict__ write,
+                 const float *__restrict__ wkey,
                  const float *__restrict__ g, float *__restrict__ Tout,
                  float *__restrict__ Pout, float *__restrict__ Wout,
                  float *__restrict__ Uout, const ChunkInfo *__restrict__ table,
@@ -382,6 +383,7 @@ __global__ void __launch_bounds__(kNT)
       kv = ldf(k + row(t) * dk + c);
       qv = ldf(q + row(t) * dk + c);
       rv = erase ? erase[row(t) * dk + c] * kv : kv;   // the read key
+      if (wkey) kv *= wkey[row(t) * dk + c];            // the write key
       if (GATE == 2 && fact) d = gt(t, c) - gt(ref, c);
     }
     const float up = __expf(d), dn = __expf(-d);
@@ -389,9 +391,9 @@ __global__ void __launch_bounds__(kNT)
     Ku[t * kP + c] = rv * up;
     Kd[t * kP + c] = kv * dn;
   }
-  // beta, or 1 with the Gated DeltaNet-2 gates (0 past the sequence end)
+  // beta, or 1 with the gate variants (0 past the sequence end)
   for (int t = tid; t < kBC; t += kNT)
-    bs[t] = t < L ? (erase ? 1.f : beta[row(t)]) : 0.f;
+    bs[t] = t < L ? ((erase || wkey) ? 1.f : beta[row(t)]) : 0.f;
   if (GATE == 1)
     for (int idx = tid; idx < kBC * kBC; idx += kNT) {
       const int r = idx / kBC, i = idx % kBC;
@@ -480,7 +482,8 @@ __global__ void __launch_bounds__(kNT)
 template <typename Tin>
 __global__ void __launch_bounds__(kNT)
     bw_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
-                   const Tin *__restrict__ dout, const float *__restrict__ g,
+                   const Tin *__restrict__ dout, const float *__restrict__ wkey,
+                   const float *__restrict__ g,
                    const float *__restrict__ W, const float *__restrict__ U,
                    const float *__restrict__ Pbuf, float *__restrict__ Cm,
                    float *__restrict__ Dm, float *__restrict__ Bm,
@@ -509,7 +512,9 @@ __global__ void __launch_bounds__(kNT)
     const bool live = r < L;
     const float gr = live ? gv(g, gdim, row, c) : 0.f;
     Ws[r * kP + c] = live ? W[row * dk + c] : 0.f;
-    Ks[r * kP + c] = live ? ldf(k + row * dk + c) * __expf(gl[c] - gr) : 0.f;
+    Ks[r * kP + c] = live ? ldf(k + row * dk + c) * __expf(gl[c] - gr) *
+                                (wkey ? wkey[row * dk + c] : 1.f)
+                          : 0.f;
     Qs[r * kP + c] = live ? ldf(q + row * dk + c) * __expf(gr) : 0.f;
   }
   for (int idx = tid; idx < kBC * dv; idx += kNT) {
@@ -610,6 +615,7 @@ constexpr int kVH = 64;
 template <typename Tin>
 __global__ void __launch_bounds__(kNT)
     bw_vn_kernel(const Tin *__restrict__ k, const Tin *__restrict__ dout,
+                 const float *__restrict__ wkey,
                  const float *__restrict__ g, const float *__restrict__ W,
                  const float *__restrict__ U, const float *__restrict__ Pbuf,
                  const float *__restrict__ Sbuf,
@@ -641,7 +647,8 @@ __global__ void __launch_bounds__(kNT)
     const bool live = r < L;
     Ws[r * kP + c] = live ? W[row * dk + c] : 0.f;
     Ks[r * kP + c] = live ? ldf(k + row * dk + c) *
-                                __expf(gl[c] - gv(g, gdim, row, c))
+                                __expf(gl[c] - gv(g, gdim, row, c)) *
+                                (wkey ? wkey[row * dk + c] : 1.f)
                           : 0.f;
   }
   const float *Pg = Pbuf + ((size_t)j * H + h) * kBC * kBC;
@@ -708,6 +715,7 @@ __global__ void __launch_bounds__(kNT)
                    const float *__restrict__ beta, const float *__restrict__ g,
                    const float *__restrict__ erase,
                    const float *__restrict__ write,
+                   const float *__restrict__ wkey,
                    const float *__restrict__ Tbuf,
                    const float *__restrict__ Sbuf,
                    const float *__restrict__ Lam,
@@ -716,6 +724,7 @@ __global__ void __launch_bounds__(kNT)
                    float *__restrict__ dkg, float *__restrict__ dvg,
                    float *__restrict__ dbeta, float *__restrict__ dla,
                    float *__restrict__ derase, float *__restrict__ dwrite,
+                   float *__restrict__ dwkey,
                    const ChunkInfo *__restrict__ table,
                    const int *__restrict__ nchunks, int H, int dk, int dv) {
   const int j = blockIdx.x, h = blockIdx.y;
@@ -755,7 +764,7 @@ __global__ void __launch_bounds__(kNT)
     Ys[t * kP + c] = live ? ldf(v + o) * (write ? write[o] : 1.f) : 0.f;
   }
   for (int t = tid; t < 64; t += kNT) {
-    bs[t] = t < L ? (erase ? 1.f : beta[row(t)]) : 0.f;
+    bs[t] = t < L ? ((erase || wkey) ? 1.f : beta[row(t)]) : 0.f;
     dbs[t] = 0.f;
     dgs[t] = 0.f;
   }
@@ -778,12 +787,12 @@ __global__ void __launch_bounds__(kNT)
     }
     // the elementwise pass's inputs (two elements per thread), fetched
     // before the products so that their latency hides behind them
-    float pg[2], pq[2], pk[2], pb[2];
+    float pg[2], pq[2], pk[2], pb[2], pa[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int idx = tid + u * kNT;
       pg[u] = pq[u] = pk[u] = 0.f;
-      pb[u] = 1.f;
+      pb[u] = pa[u] = 1.f;
       if (idx < L * kSl) {
         const int t = idx / kSl, c = c0 + idx % kSl;
         const size_t o = row(t) * dk + c;
@@ -791,6 +800,7 @@ __global__ void __launch_bounds__(kNT)
         pq[u] = ldf(q + o);
         pk[u] = ldf(k + o);
         if (erase) pb[u] = erase[o];
+        if (wkey) pa[u] = wkey[o];
       }
     }
     for (int idx = tid; idx < kBC * kSl; idx += kNT) {
@@ -844,17 +854,18 @@ __global__ void __launch_bounds__(kNT)
       const float gg = pg[u], e = __expf(gg), ec = __expf(gC[c] - gg);
       const size_t o = row(t) * dk + c;
       const float qv = pq[u], kv = pk[u];
-      const float bv = pb[u];   // read key = bv kv
+      const float bv = pb[u], av = pa[u];   // read key bv kv, write key av kv
       const float x1 = X1[t * kSl + cc], x2 = X2[t * kSl + cc],
                   x3 = X3[t * kSl + cc];
       // read-key gradient -x2 e^g, write-key gradient x3 e^{g_C - g}
       dq[o] = x1 * e;
-      dkg[o] = -x2 * e * bv + x3 * ec;
+      dkg[o] = -x2 * e * bv + av * x3 * ec;
       if (erase) derase[o] = -x2 * e * kv;
-      const float dgv = (x1 * qv - x2 * bv * kv) * e - x3 * kv * ec;
+      if (wkey) dwkey[o] = kv * x3 * ec;
+      const float dgv = (x1 * qv - x2 * bv * kv) * e - x3 * av * kv * ec;
       if (GATE == 2) dla[row(t) * dk + c] = dgv;
       if (GATE == 1) atomicAdd(&dgs[t], dgv);
-      if (GATE != 0) atomicAdd(&dgC[c], x3 * kv * ec);
+      if (GATE != 0) atomicAdd(&dgC[c], x3 * av * kv * ec);
     }
     __syncthreads();
   }
@@ -920,6 +931,7 @@ __global__ void __launch_bounds__(kNT)
       kv = ldf(k + row(t) * dk + c);
       qv = ldf(q + row(t) * dk + c);
       rv = erase ? erase[row(t) * dk + c] * kv : kv;   // the read key
+      if (wkey) kv *= wkey[row(t) * dk + c];            // the write key
       if (GATE == 2 && fact) d = gt(t, c) - gt(ref, c);
     }
     const float up = __expf(d), dn = __expf(-d);
@@ -985,12 +997,16 @@ __global__ void __launch_bounds__(kNT)
       const float up = __expf(d), dn = __expf(-d);
       const float drho = up * r1, dkap = dn * r2, dqP = up * r3, dkP = dn * r4;
       const size_t o = row(t) * dk + c;
-      // the key, query and read key back from their rescaled tiles
+      // the write key, query and read key back from their rescaled tiles
+      // (the raw key is the write key with the erase gate, the read key
+      // with FG^2-GDN's rate)
       const float kv = Kd[t * kP + c] * up, qv = Qu[t * kP + c] * dn,
                   rv = Ku[t * kP + c] * dn;
       dq[o] += dqP;
-      dkg[o] += (erase ? erase[o] : 1.f) * drho + dkap + dkP;
+      dkg[o] += (erase ? erase[o] : 1.f) * drho +
+                (wkey ? wkey[o] : 1.f) * (dkap + dkP);
       if (erase) derase[o] += kv * drho;
+      if (wkey) dwkey[o] += rv * (dkap + dkP);
       const float dgv = rv * drho - kv * (dkap + dkP) + qv * dqP;
       if (GATE == 2) dla[o] += dgv;
       if (GATE == 1) atomicAdd(&dgs[t], dgv);
@@ -1021,13 +1037,14 @@ __global__ void __launch_bounds__(kNT)
         if (i >= t) dkP += dPs[i * kCP + t] * Qu[i * kP + c] * e;
       }
       const size_t o = row(t) * dk + c;
-      // (unfactored: Ku holds the read key, Kd the key, Qu the query)
+      // (unfactored: Ku holds the read key, Kd the write key, Qu the query)
       const float rv = Ku[t * kP + c], kv = Kd[t * kP + c],
                   qv = Qu[t * kP + c];
-      const float bv = erase ? erase[o] : 1.f;
       dq[o] += dqP;
-      dkg[o] += bv * drho + dkap + dkP;
+      dkg[o] += (erase ? erase[o] : 1.f) * drho +
+                (wkey ? wkey[o] : 1.f) * (dkap + dkP);
       if (erase) derase[o] += kv * drho;
+      if (wkey) dwkey[o] += rv * (dkap + dkP);
       dla[o] += rv * drho - kv * (dkap + dkP) + qv * dqP;
     }
   }
@@ -1099,9 +1116,9 @@ cudaError_t run_grad(const Problem &p, const BackwardIO &io,
   bw_grad_kernel<Tin, GATE><<<dim3(p.max_chunks, p.H), kNT, smem, s>>>(
       static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k),
       static_cast<const Tin *>(p.v), static_cast<const Tin *>(io.dout),
-      p.beta, b.g, p.erase, p.write, Tb, b.Sbuf, Lam, b.Vn, dVn, io.dq, io.dk,
-      io.dv, io.dbeta, io.dla, io.derase, io.dwrite, b.table, b.nchunks, p.H,
-      p.dk, p.dv);
+      p.beta, b.g, p.erase, p.write, p.wkey, Tb, b.Sbuf, Lam, b.Vn, dVn,
+      io.dq, io.dk, io.dv, io.dbeta, io.dla, io.derase, io.dwrite, io.dwkey,
+      b.table, b.nchunks, p.H, p.dk, p.dv);
   return cudaGetLastError();
 }
 
@@ -1116,8 +1133,8 @@ cudaError_t run_wy(const Problem &p, const StagedBufs &b, float *Tb, float *Pb,
   if (e != cudaSuccess) return e;
   bw_wy_kernel<Tin, GATE><<<dim3(p.max_chunks, p.H), kNT, smem, s>>>(
       static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k),
-      static_cast<const Tin *>(p.v), p.beta, p.erase, p.write, b.g, Tb, Pb,
-      b.W, b.U, b.table, b.nchunks, p.H, p.dk, p.dv);
+      static_cast<const Tin *>(p.v), p.beta, p.erase, p.write, p.wkey, b.g,
+      Tb, Pb, b.W, b.U, b.table, b.nchunks, p.H, p.dk, p.dv);
   return cudaGetLastError();
 }
 
@@ -1154,8 +1171,8 @@ cudaError_t run_typed(const Problem &p, const BackwardIO &io, char *ws,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     bw_prep_kernel<Tin><<<dim3(p.max_chunks, p.H), kNT, smem, s>>>(
-        q, k, dout, b.g, b.W, b.U, Pb, Cm, Dm, Bm, b.table, b.nchunks, p.H,
-        p.dk, p.dv, gdim);
+        q, k, dout, p.wkey, b.g, b.W, b.U, Pb, Cm, Dm, Bm, b.table,
+        b.nchunks, p.H, p.dk, p.dv, gdim);
   }
   {
     const int smem = (int)sizeof(float) * 3 * 128 * kP;
@@ -1181,7 +1198,7 @@ cudaError_t run_typed(const Problem &p, const BackwardIO &io, char *ws,
     if (e != cudaSuccess) return e;
     const int dvh = p.dv < kVH ? p.dv : kVH;
     bw_vn_kernel<Tin><<<dim3(p.max_chunks, p.H, p.dv / dvh), kNT, smem, s>>>(
-        k, dout, b.g, b.W, b.U, Pb, b.Sbuf, Lam, b.Vn, dVn, b.table,
+        k, dout, p.wkey, b.g, b.W, b.U, Pb, b.Sbuf, Lam, b.Vn, dVn, b.table,
         b.nchunks, p.H, p.dk, p.dv, gdim);
   }
   if (p.max_chunks == 0) return cudaGetLastError();

@@ -830,21 +830,23 @@ extern "C" gdr_status gdr_chunk_fwd_segmented(
 
 namespace {
 
-// gdr_backward and gdr_backward_gdn2: with erase != nullptr the Gated
-// DeltaNet-2 gates (erase, write) replace beta, and their gradients go to
-// d_erase, d_write (the chunked backward only).
+// gdr_backward, gdr_backward_gdn2 and gdr_backward_fg2: with erase the
+// Gated DeltaNet-2 gates (erase, write) replace beta, with wkey FG^2-GDN's
+// rate (and, when write is given, FG^2-GDN+'s value scaling); their
+// gradients go to d_erase / d_wkey and d_write (the chunked backward only).
 gdr_status backward_entry(const void *q, const void *k, const void *v,
                           const float *log_alpha, const float *beta,
                           const float *erase, const float *write,
-                          const float *initial_state, const void *d_out,
-                          const float *d_final_state, float *dq, float *dk,
-                          float *dv, float *d_log_alpha, float *d_beta,
-                          float *d_erase, float *d_write,
-                          float *d_initial_state, int B, int T, int H,
-                          int dk_, int dv_, cudaStream_t stream,
+                          const float *wkey, const float *initial_state,
+                          const void *d_out, const float *d_final_state,
+                          float *dq, float *dk, float *dv, float *d_log_alpha,
+                          float *d_beta, float *d_erase, float *d_write,
+                          float *d_wkey, float *d_initial_state, int B, int T,
+                          int H, int dk_, int dv_, cudaStream_t stream,
                           const gdr_opts *opts) {
   const gdr_opts o = opts ? *opts : default_opts();
-  const bool gates = erase != nullptr || write != nullptr;
+  const bool gates = erase != nullptr || wkey != nullptr;
+  const float *key_gate = erase ? erase : wkey;
   if (o.algo == GDR_ALGO_FUSED_TC) return GDR_ERR_UNSUPPORTED;
   const bool recurrent = o.algo == GDR_ALGO_RECURRENT;
   if (recurrent && gates) return GDR_ERR_UNSUPPORTED;
@@ -855,18 +857,21 @@ gdr_status backward_entry(const void *q, const void *k, const void *v,
   // d_final_state in the place of final_state (the chunked backward runs
   // chunks of 64 tokens whatever the forward used); the erase gate stands in
   // for beta with the gates
-  gdr_status st = validate(q, k, v, log_alpha, gates ? erase : beta,
+  gdr_status st = validate(q, k, v, log_alpha, gates ? key_gate : beta,
                            initial_state, d_out, d_final_state, B, T, H, dk_,
                            dv_, 64, ov, &p);
   if (st != GDR_OK) return st;
   if (p.nseq == 0 || p.H == 0) return GDR_OK;
   if (!dq || !dk || !dv) return GDR_ERR_INVALID_ARGUMENT;
-  if (gates ? (!write || !d_erase || !d_write) : !d_beta)
+  if (!gates && !d_beta) return GDR_ERR_INVALID_ARGUMENT;
+  if (erase && (!write || !d_erase || !d_write))
+    return GDR_ERR_INVALID_ARGUMENT;
+  if (wkey && (!d_wkey || (write != nullptr) != (d_write != nullptr)))
     return GDR_ERR_INVALID_ARGUMENT;
   if ((o.gate == GDR_GATE_NONE) != (d_log_alpha == nullptr))
     return GDR_ERR_INVALID_ARGUMENT;
   const void *ptrs[] = {dq, dk, dv, d_log_alpha, d_beta, d_initial_state,
-                        write, d_erase, d_write};
+                        write, d_erase, d_write, d_wkey};
   for (const void *ptr : ptrs)
     if (ptr && !aligned16(ptr)) return GDR_ERR_INVALID_ARGUMENT;
   // AUTO and STAGED: the chunked backward (the faster of the two on every
@@ -877,6 +882,7 @@ gdr_status backward_entry(const void *q, const void *k, const void *v,
     p.beta = nullptr;
     p.erase = erase;
     p.write = write;
+    p.wkey = wkey;
   }
   long long total_win = 0;
   const size_t bytes = chunked ? gdr::backward_chunked_bytes(p)
@@ -906,8 +912,9 @@ gdr_status backward_entry(const void *q, const void *k, const void *v,
   io.dla = d_log_alpha;
   io.dbeta = gates ? nullptr : d_beta;
   io.ds0 = d_initial_state;
-  io.derase = gates ? d_erase : nullptr;
-  io.dwrite = gates ? d_write : nullptr;
+  io.derase = erase ? d_erase : nullptr;
+  io.dwrite = write ? d_write : nullptr;
+  io.dwkey = wkey ? d_wkey : nullptr;
   cudaError_t e =
       chunked ? gdr::backward_chunked_run(p, io, ws, stream)
               : gdr::backward_run(p, io, static_cast<float *>(ws), total_win,
@@ -924,9 +931,9 @@ extern "C" gdr_status gdr_backward(
     const float *d_final_state, float *dq, float *dk, float *dv,
     float *d_log_alpha, float *d_beta, float *d_initial_state, int B, int T,
     int H, int dk_, int dv_, cudaStream_t stream, const gdr_opts *opts) {
-  return backward_entry(q, k, v, log_alpha, beta, nullptr, nullptr,
+  return backward_entry(q, k, v, log_alpha, beta, nullptr, nullptr, nullptr,
                         initial_state, d_out, d_final_state, dq, dk, dv,
-                        d_log_alpha, d_beta, nullptr, nullptr,
+                        d_log_alpha, d_beta, nullptr, nullptr, nullptr,
                         d_initial_state, B, T, H, dk_, dv_, stream, opts);
 }
 
@@ -940,8 +947,22 @@ extern "C" gdr_status gdr_backward_gdn2(
     cudaStream_t stream, const gdr_opts *opts) {
   if (!erase_gate || !write_gate) return GDR_ERR_INVALID_ARGUMENT;
   return backward_entry(q, k, v, log_alpha, nullptr, erase_gate, write_gate,
+                        nullptr, initial_state, d_out, d_final_state, dq, dk,
+                        dv, d_log_alpha, nullptr, d_erase, d_write, nullptr,
+                        d_initial_state, B, T, H, dk_, dv_, stream, opts);
+}
+
+extern "C" gdr_status gdr_backward_fg2(
+    const void *q, const void *k, const void *v, const float *log_alpha,
+    const float *beta_k, const float *beta_v, const float *initial_state,
+    const void *d_out, const float *d_final_state, float *dq, float *dk,
+    float *dv, float *d_log_alpha, float *d_beta_k, float *d_beta_v,
+    float *d_initial_state, int B, int T, int H, int dk_, int dv_,
+    cudaStream_t stream, const gdr_opts *opts) {
+  if (!beta_k) return GDR_ERR_INVALID_ARGUMENT;
+  return backward_entry(q, k, v, log_alpha, nullptr, nullptr, beta_v, beta_k,
                         initial_state, d_out, d_final_state, dq, dk, dv,
-                        d_log_alpha, nullptr, d_erase, d_write,
+                        d_log_alpha, nullptr, nullptr, d_beta_v, d_beta_k,
                         d_initial_state, B, T, H, dk_, dv_, stream, opts);
 }
 

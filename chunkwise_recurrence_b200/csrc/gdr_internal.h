@@ -99,6 +99,8 @@ struct BackwardIO {
   // Gated DeltaNet-2 gates' gradients (chunked backward; the gates are the
   // Problem's erase / write): layouts of k and v, or nullptr
   float *derase = nullptr, *dwrite = nullptr;
+  // FG^2-GDN's rate gradient (the Problem's wkey): layout of k, or nullptr
+  float *dwkey = nullptr;
 };
 // Chunked backward pass (csrc/backward_chunked.cu): the gradients of the
 // chunked forward product by product, fp32, chunk-parallel except for one

@@ -525,6 +525,30 @@ GDR_API gdr_status gdr_backward_gdn2(
     cudaStream_t stream, const gdr_opts *opts);
 
 /*
+ * gdr_backward_fg2 -- gdr_backward for gdr_chunk_fwd_fg2: the gradients of
+ * the forward pass with FG^2-GDN's per-key-channel rate (and FG^2-GDN+'s
+ * value scaling), the rate's and the scaling's own included.
+ *
+ * The chunked backward with the write key beta_k . k (rate beta_k) in the
+ * state update, in P and on the column side of A, the read key k on A's row
+ * side and in W, and the target c . v (c = beta_v, or 1) in U; beta is 1.
+ * Gradients, fp32, 16-byte aligned, written: dq, dk, dv, d_log_alpha (NULL
+ * iff gate is NONE), d_beta_k (layout of k, required), d_beta_v (layout of
+ * v; required iff beta_v is given, else NULL), d_initial_state (or NULL).
+ * Inputs as for gdr_chunk_fwd_fg2 plus d_out and d_final_state as for
+ * gdr_backward.  opts->algo AUTO or STAGED; RECURRENT and FUSED_TC return
+ * GDR_ERR_UNSUPPORTED.  Scratch and status codes as for gdr_backward's
+ * chunked algorithm.
+ */
+GDR_API gdr_status gdr_backward_fg2(
+    const void *q, const void *k, const void *v, const float *log_alpha,
+    const float *beta_k, const float *beta_v, const float *initial_state,
+    const void *d_out, const float *d_final_state, float *dq, float *dk,
+    float *dv, float *d_log_alpha, float *d_beta_k, float *d_beta_v,
+    float *d_initial_state, int B, int T, int H, int dk_, int dv_,
+    cudaStream_t stream, const gdr_opts *opts);
+
+/*
  * gdr_efla_beta -- exact-flow step size (EFLA) for the delta rule.
  *
  * The delta rule's update is one explicit Euler step of length beta of the

@@ -230,6 +230,32 @@ def test_backward_gdn2_rejects_bad_arguments(lib):
              dv=None, dla=None, gate=0, B=0) == OK
 
 
+def test_backward_fg2_rejects_bad_arguments(lib):
+    def c(**kw):
+        a = dict(q=A, k=A, v=A, la=A, bk=A, bv=None, s0=None, dout=A,
+                 dsT=None, dq=A, dk=A, dv=A, dla=A, dbk=A, dbv=None, ds0=None,
+                 B=1, T=32, H=1, dk_=64, dv_=64, gate=2, dtype=0, algo=0)
+        a.update(kw)
+        opts = gdr._Opts(a["dtype"], a["gate"], None, 0, a["algo"])
+        return lib.gdr_backward_fg2(
+            a["q"], a["k"], a["v"], a["la"], a["bk"], a["bv"], a["s0"],
+            a["dout"], a["dsT"], a["dq"], a["dk"], a["dv"], a["dla"],
+            a["dbk"], a["dbv"], a["ds0"], a["B"], a["T"], a["H"], a["dk_"],
+            a["dv_"], None, ctypes.byref(opts))
+    # every case is rejected on the host, before any CUDA call
+    assert c(bk=None) == INVALID          # the rate is required
+    assert c(dbk=None) == INVALID         # and its gradient
+    assert c(bv=A) == INVALID             # a value scaling needs its gradient
+    assert c(dbv=A) == INVALID            # ... and its gradient needs it
+    assert c(dbk=A + 4) == INVALID        # misaligned
+    assert c(dla=None) == INVALID
+    assert c(algo=3) == UNSUPPORTED       # no token recurrence with gates
+    assert c(algo=2) == UNSUPPORTED
+    assert c(dk_=48) == UNSUPPORTED
+    assert c(q=None, k=None, v=None, la=None, dout=None, dq=None, dk=None,
+             dv=None, dla=None, gate=0, B=0) == OK
+
+
 def test_segmented_rejects_bad_arguments(lib):
     def c(segments=4, **kw):
         args = dict(q=A, k=A, v=A, la=A, beta=A, s0=None, out=A, sT=None, B=1,

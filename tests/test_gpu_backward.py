@@ -198,3 +198,63 @@ def test_backward_gdn2_with_gates_equal_to_beta_is_the_delta_rule():
         assert rel_err(r2[key].cpu().numpy(), r1[key].cpu().numpy()) <= 1e-4
     db = (r2["derase"].sum(-1) + r2["dwrite"].sum(-1)).cpu().numpy()
     assert rel_err(db, r1["dbeta"].cpu().numpy()) <= 1e-4
+
+
+# ---------------------------------------------------------------------------
+# gdr_backward_fg2: FG^2-GDN's rate (and FG^2-GDN+'s value scaling) through
+# the chunked backward, against fp64 autograd through oracle.fg2_fwd's token
+# loop (oracle.fg2_grads, pinned by central differences).
+
+def _check_fg2(w, seed=0, plus=True, with_final=True):
+    from chunkwise_recurrence_b200.inputs import fg2_gates
+    inp = generate(w, seed=seed)
+    bk, bv = fg2_gates(inp, seed=seed)
+    if not plus:
+        bv = None
+    g = torch.Generator().manual_seed(seed + 300)
+    dO = torch.randn(inp.v.shape, generator=g).to(inp.v.dtype)
+    dS = (torch.randn(inp.nseq, w.H, w.dk, w.dv, generator=g) * 0.1
+          if with_final else None)
+    c = lambda t: None if t is None else t.cuda()  # noqa: E731
+    res = gdr.backward_fg2(c(inp.q), c(inp.k), c(inp.v), c(bk), c(bv),
+                           c(inp.log_alpha), c(inp.s0), c(dO), c(dS),
+                           gate=w.gate, cu_seqlens=c(inp.cu_seqlens))
+    torch.cuda.synchronize()
+    f = inp.f64()
+    ref = oracle.fg2_grads(f["q"], f["k"], f["v"], bk.double().numpy(),
+                           None if bv is None else bv.double().numpy(),
+                           f["log_alpha"], gate=w.gate,
+                           initial_state=f["initial_state"],
+                           d_out=dO.double().numpy(),
+                           d_final_state=None if dS is None else dS.numpy(),
+                           cu_seqlens=f["cu_seqlens"])
+    errs = {}
+    for key in ("dq", "dk", "dv", "dbeta_k", "dbeta_v", "dlog_alpha"):
+        if ref[key] is None:
+            assert res[key] is None or key == "dlog_alpha"
+            continue
+        errs[key] = rel_err(res[key].cpu().numpy(), ref[key])
+    if ref["dinitial_state"] is not None:
+        errs["ds0"] = rel_err(res["dinitial_state"].cpu().numpy(),
+                              ref["dinitial_state"])
+    for key, e in errs.items():
+        assert e <= TOL, (key, e, errs)
+    return errs
+
+
+@pytest.mark.parametrize("plus", [False, True])
+@pytest.mark.parametrize("gate", ["none", "scalar", "channel"])
+def test_backward_fg2_matches_autograd(gate, plus):
+    w = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(
+        B=2, T=2 * 64 + 29, H=2, gate=gate, init_state=True)
+    _check_fg2(w, seed=12, plus=plus)
+
+
+def test_backward_fg2_varlen_fp32_and_strong_decay():
+    w = WORKLOADS["gdn_varlen8_h16_d128_bf16"].with_(
+        varlen_nseq=4, varlen_lo=1, varlen_hi=200, H=2, gate="channel",
+        dtype="fp32", dk=64, dv=32)
+    _check_fg2(w, seed=13, with_final=False)
+    w2 = WORKLOADS["kda_b4_h16_t4096_d128_bf16"].with_(
+        B=1, T=64 + 40, H=1, decay_lo=3.0, decay_hi=3.0)
+    _check_fg2(w2, seed=14)
