@@ -566,6 +566,7 @@ def run_ours(args, w):
         "gpu_launches": launches_per_step(algo_used, w, args.segments) *
         args.steps,
         "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
+        "ms_per_step_median": statistics.median(per_step),
     }
     if rank == 0:
         line["parity"] = sampled_parity(inp, out, sT)
@@ -714,6 +715,7 @@ def run_decode(args):
                 + ", token inputs from pinned host memory, state resident"},
         "gpu_launches": args.steps,
         "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
+        "ms_per_step_median": statistics.median(per_step),
     }
     if not args.no_cpu_baseline:
         import oracle
@@ -865,6 +867,7 @@ def run_backward(args, w):
         "clocks": clk,
         "gpu_launches": args.steps * launches,
         "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
+        "ms_per_step_median": statistics.median(per_step),
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -1008,6 +1011,7 @@ def run_gdn2(args, w, kind="gdn2"):
                          "memory and results back each step"},
         "gpu_launches": launches_per_step(algo_used, w) * args.steps,
         "ms_per_step_min": min(per_step), "ms_per_step_max": max(per_step),
+        "ms_per_step_median": statistics.median(per_step),
     }
     if not args.no_cpu_baseline:
         import oracle
