@@ -165,5 +165,6 @@ def decode_step(q, k, v, beta, log_alpha=None, gate="scalar", state=None,
 from .chunkwise_ref import chunkwise_ref  # noqa: E402  (re-export)
 from .efla_ref import efla_fwd  # noqa: E402  (re-export)
 from .gdn2_ref import gdn2_fwd  # noqa: E402  (re-export)
-from .grad_ref import fg2_grads, gdn2_grads, gdr_grads  # noqa: E402
+from .grad_ref import (efla_grads, fg2_grads, gdn2_grads,  # noqa: E402
+                       gdr_grads)
 from .fg2_ref import fg2_fwd  # noqa: E402  (re-export)

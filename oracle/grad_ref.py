@@ -12,7 +12,9 @@ only (one autograd node per token operation).
 ``gdn2_grads`` does the same for Gated DeltaNet-2's separate gates (the
 update of oracle/gdn2_ref.py: read key b_t . k_t, target w_t . v_t, no beta;
 Gated DeltaNet-2 abstract on the comparative-study page 2607.07953, which
-credits the model with a gate-aware backward pass), and ``fg2_grads`` for
+credits the model with a gate-aware backward pass), ``efla_grads`` for the
+EFLA recurrence (the exact-flow step size formed inside the graph), and
+``fg2_grads`` for
 FG^2-GDN's per-key-channel rate and FG^2-GDN+'s value scaling (the update of
 oracle/fg2_ref.py: write key beta_k . k_t, read key k_t, target
 c_t . v_t).
@@ -75,6 +77,50 @@ def gdn2_grads(q, k, v, erase, write, log_alpha=None, gate="channel",
     final_state (dbeta is None)."""
     return _grads(q, k, v, None, erase, write, log_alpha, gate,
                   initial_state, d_out, d_final_state, cu_seqlens)
+
+
+def efla_grads(q, k, v, beta, log_alpha=None, gate="scalar",
+               initial_state=None, d_out=None, d_final_state=None):
+    """Gradients of sum(out * d_out) + sum(final * d_final_state) through the
+    EFLA recurrence: the delta rule with the exact-flow step size
+    beta' = (1 - e^{-beta |k|^2}) / |k|^2 ("Delta-Rule Linear Attention"
+    topic page, EFLA card), beta' formed inside the autograd graph so that
+    dbeta and dk carry its chain rule.  Fixed-length batches; returns the
+    same keys as gdr_grads."""
+    t64 = lambda a: None if a is None else torch.tensor(  # noqa: E731
+        np.asarray(a, np.float64), requires_grad=True)
+    Bq, T = np.shape(q)[:2]
+    cu = [i * T for i in range(Bq + 1)]
+    flat = lambda a: None if a is None else a.reshape(  # noqa: E731
+        (-1,) + tuple(a.shape[2:]))
+    tq, tk, tv, tb = t64(q), t64(k), t64(v), t64(beta)
+    tla = t64(log_alpha) if gate != "none" else None
+    ts0 = t64(initial_state)
+    s = (tk * tk).sum(-1)
+    bprime = -torch.expm1(-tb * s) / s
+    outs, final = _loop(flat(tq), flat(tk), flat(tv), flat(bprime), flat(tla),
+                        gate, ts0, cu)
+    H, dv = np.shape(v)[2], np.shape(v)[3]
+    loss = torch.zeros((), dtype=torch.float64)
+    dO = None if d_out is None else torch.tensor(
+        np.asarray(d_out, np.float64)).reshape(Bq * T, H, dv)
+    out = torch.zeros(Bq * T, H, dv, dtype=torch.float64)
+    for (t, h), o in outs:
+        if dO is not None:
+            loss = loss + (o * dO[t, h]).sum()
+        out[t, h] = o.detach()
+    if d_final_state is not None:
+        loss = loss + (final * torch.tensor(
+            np.asarray(d_final_state, np.float64))).sum()
+    leaves = [x for x in (tq, tk, tv, tb, tla, ts0) if x is not None]
+    grads = torch.autograd.grad(loss, leaves, allow_unused=True)
+    gm = dict(zip([id(x) for x in leaves], grads))
+    g = lambda x: None if x is None else (  # noqa: E731
+        np.zeros(x.shape) if gm[id(x)] is None else gm[id(x)].numpy())
+    return dict(dq=g(tq), dk=g(tk), dv=g(tv), dbeta=g(tb),
+                dlog_alpha=g(tla), dinitial_state=g(ts0),
+                out=out.reshape(np.shape(v)).numpy(),
+                final_state=final.detach().numpy())
 
 
 def fg2_grads(q, k, v, beta_k, beta_v=None, log_alpha=None, gate="channel",

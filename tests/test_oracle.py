@@ -937,6 +937,43 @@ def test_fg2_gradients_reduce_to_the_delta_rule():
     np.testing.assert_allclose(g2["dbeta_k"].sum(-1), g1["dbeta"], atol=1e-12)
 
 
+def test_efla_gradients_match_finite_differences():
+    """The EFLA autograd gradients (oracle.efla_grads) agree with central
+    differences of the EFLA matrix-exponential flow's loss (oracle.efla_fwd),
+    element by element, for every input and gate -- unnormalised keys, so
+    the step size's dependence on |k| is exercised."""
+    rng = np.random.default_rng(61)
+    for gate in ("none", "scalar", "channel"):
+        c = _rand_case(rng, B=1, T=4, H=1, dk=3, dv=2, gate=gate)
+        case = dict(q=c["q"], k=c["k"] * rng.uniform(0.5, 2.0, (1, 4, 1, 1)),
+                    v=c["v"], beta=c["beta"], log_alpha=c["log_alpha"],
+                    initial_state=c["initial_state"])
+        dO = rng.standard_normal(c["v"].shape)
+        dS = rng.standard_normal((1, 1, 3, 2))
+        g = oracle.efla_grads(**case, gate=gate, d_out=dO, d_final_state=dS)
+
+        def loss(x):
+            o, sT = oracle.efla_fwd(x["q"], x["k"], x["v"], x["beta"],
+                                    x["log_alpha"], gate, x["initial_state"])
+            return float((o * dO).sum() + (sT * dS).sum())
+
+        names = ["q", "k", "v", "beta", "initial_state"]
+        if gate != "none":
+            names.append("log_alpha")
+        eps = 1e-6
+        for key in names:
+            x = case[key]
+            fd = np.zeros_like(x)
+            for i in np.ndindex(x.shape):
+                xp, xm = x.copy(), x.copy()
+                xp[i] += eps
+                xm[i] -= eps
+                fd[i] = (loss({**case, key: xp}) - loss({**case, key: xm})) / (
+                    2 * eps)
+            np.testing.assert_allclose(g["d" + key], fd, atol=1e-6, rtol=1e-5,
+                                       err_msg=f"{gate} {key}")
+
+
 def test_gdn2_gradients_reduce_to_the_delta_rule():
     """Both gates equal to beta_t on every channel: the Gated DeltaNet-2
     gradients of q, k, v, log-alpha and the initial state are the delta
