@@ -17,7 +17,8 @@ import torch
 __all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_noalloc",
            "chunk_fwd_segmented", "chunk_fwd_gdn2", "chunk_fwd_fg2",
            "decode_step", "decode_step_gdn2", "decode_step_fg2",
-           "efla_beta", "backward", "backward_gdn2", "backward_fg2",
+           "efla_beta", "efla_beta_backward", "backward", "backward_gdn2",
+           "backward_fg2",
            "device_error", "status_string",
            "algo_applies", "fused_tc_available",
            "GdrError", "load_library", "LIB_PATH", "GATES", "ALGOS",
@@ -39,7 +40,7 @@ EXPORTED_SYMBOLS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_device_error",
                     "gdr_chunk_fwd_segmented", "gdr_chunk_fwd_gdn2",
                     "gdr_decode_step_gdn2", "gdr_chunk_fwd_fg2",
                     "gdr_decode_step_fg2", "gdr_backward_gdn2",
-                    "gdr_backward_fg2")
+                    "gdr_backward_fg2", "gdr_efla_beta_backward")
 # size of the static scratch array behind gdr_chunk_fwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -103,6 +104,8 @@ def load_library(path: str = LIB_PATH):
                       fp, fp, i, i, i, i, i, vp, ctypes.POINTER(_Opts)]
     lib.gdr_efla_beta.restype = ctypes.c_int
     lib.gdr_efla_beta.argtypes = [vp, fp, fp, i, i, i, i, vp]
+    lib.gdr_efla_beta_backward.restype = ctypes.c_int
+    lib.gdr_efla_beta_backward.argtypes = [vp, fp, fp, fp, fp, i, i, i, i, vp]
     lib.gdr_device_error.restype = ctypes.c_int
     lib.gdr_device_error.argtypes = [vp, i]
     lib.gdr_algo_applies.restype = ctypes.c_int
@@ -542,6 +545,28 @@ def efla_beta(k, beta, *, out=None, stream=None):
     if rc != 0:
         raise GdrError(rc, "gdr_efla_beta")
     return out
+
+
+def efla_beta_backward(k, beta, d_beta_prime, dk, *, d_beta=None,
+                       stream=None):
+    """Run ``gdr_efla_beta_backward``: the chain rule through ``efla_beta``.
+    Returns d beta [..., H] (fp32) and adds d beta' (d beta' / d |k|^2) 2 k
+    into ``dk`` (fp32, the layout of k, e.g. ``backward``'s dk)."""
+    lib = load_library()
+    dkd = k.shape[-1]
+    H = k.shape[-2]
+    ntok = k.numel() // (H * dkd)
+    if d_beta is None:
+        d_beta = torch.empty_like(beta)
+    if stream is None:
+        stream = torch.cuda.current_stream(k.device)
+    rc = lib.gdr_efla_beta_backward(_ptr(k), _ptr(beta), _ptr(d_beta_prime),
+                                    _ptr(d_beta), _ptr(dk), ntok, H, dkd,
+                                    DTYPES[k.dtype],
+                                    ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise GdrError(rc, "gdr_efla_beta_backward")
+    return d_beta
 
 
 def device_error(stream=None, clear: bool = True) -> int:

@@ -571,6 +571,26 @@ GDR_API gdr_status gdr_efla_beta(const void *k, const float *beta,
                                  gdr_dtype dtype, cudaStream_t stream);
 
 /*
+ * gdr_efla_beta_backward -- the chain rule through gdr_efla_beta, for the
+ * EFLA backward pass: run gdr_backward with beta' (its d_beta is then
+ * d beta'), then this, which writes
+ *   d_beta[row] = d_beta_prime[row] e^{-beta s}        (s = |k_row|^2)
+ * and ADDS  d_beta_prime[row] (d beta' / d s) 2 k_row  to dk (fp32, the
+ * layout of k, typically gdr_backward's dk), with
+ * d beta' / d s = (beta s e^{-beta s} + e^{-beta s} - 1) / s^2 (its Taylor
+ * series for small beta s, limit -beta^2 / 2).
+ *
+ * k [ntok][H][dk] in `dtype`; beta, d_beta_prime, d_beta [ntok][H] fp32; all
+ * device, 16-byte aligned.  dk in {16, 32, 64, 128}.  Status codes as for
+ * gdr_efla_beta.
+ */
+GDR_API gdr_status gdr_efla_beta_backward(const void *k, const float *beta,
+                                          const float *d_beta_prime,
+                                          float *d_beta, float *dk, int ntok,
+                                          int H, int dk_, gdr_dtype dtype,
+                                          cudaStream_t stream);
+
+/*
  * gdr_device_error -- synchronise `stream`, then read (and clear if `clear`)
  * the library's sticky device-side error word for the current device.
  * Returns GDR_OK if no kernel has reported an error, GDR_ERR_TIMEOUT if a

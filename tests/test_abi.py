@@ -164,6 +164,19 @@ def test_decode_step_rejects_bad_arguments(lib):
              gate=0, H=0) == OK
 
 
+def test_efla_beta_backward_rejects_bad_arguments(lib):
+    f = lambda k=A, b=A, g=A + 4096, db=A + 8192, dk=A + 16384, ntok=8, H=2, \
+        d=64, dt=0: lib.gdr_efla_beta_backward(k, b, g, db, dk, ntok, H, d,
+                                                dt, None)  # noqa: E731
+    assert f(k=None) == INVALID
+    assert f(g=None) == INVALID
+    assert f(dk=A + 4) == INVALID        # misaligned
+    assert f(dt=3) == INVALID
+    assert f(ntok=-1) == INVALID
+    assert f(d=48) == UNSUPPORTED
+    assert f(k=None, b=None, g=None, db=None, dk=None, ntok=0) == OK
+
+
 def test_efla_beta_rejects_bad_arguments(lib):
     f = lambda k=A, b=A, o=A + 4096, ntok=8, H=2, dk=64, dt=0: \
         lib.gdr_efla_beta(k, b, o, ntok, H, dk, dt, None)  # noqa: E731
