@@ -34,7 +34,7 @@
 //                    and dV_new from those states;
 //   bw_grad_kernel   per (chunk, head), in parallel: every input gradient of
 //                    the chunk from S, Lambda, V_new and dV_new.
-// The products are register-blocked over shared-memory tiles (gemm_tile).
+// The products run on the tensor cores over shared-memory tiles (gemm_tc).
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -65,51 +65,9 @@ __device__ __forceinline__ float ldf(const __nv_bfloat16 *p) {
   return __bfloat162float(*p);
 }
 
-// acc(m, n) = sum_{k < K} A(m, k) B(k, n) for the M x N output, N a multiple
-// of TN: the threads form a GM x GN grid (GN = N / TN, GM = kNT / GN), thread
-// (r, c) owns rows r + GM i (i < TM) and columns c + GN j (j < TN), in passes
-// of GM TM rows; out(m, n, value) receives each finished element.  A, B, out
-// are callables, so operands may be transposed, scaled or masked in place.
-template <int TM, int TN, class FA, class FB, class FO>
-__device__ __forceinline__ void gemm_tile(int M, int N, int K, FA A, FB B,
-                                          FO out) {
-  const int GN = N / TN, GM = kNT / GN;
-  const int tr = threadIdx.x / GN, tc = threadIdx.x % GN;
-  if (tr >= GM) return;
-  for (int mb = 0; mb < M; mb += GM * TM) {
-    float acc[TM][TN];
-#pragma unroll
-    for (int i = 0; i < TM; ++i)
-#pragma unroll
-      for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
-    int mr[TM];
-#pragma unroll
-    for (int i = 0; i < TM; ++i) mr[i] = min(mb + tr + GM * i, M - 1);
-    for (int k = 0; k < K; ++k) {
-      float a[TM], b[TN];
-#pragma unroll
-      for (int i = 0; i < TM; ++i) a[i] = A(mr[i], k);
-#pragma unroll
-      for (int j = 0; j < TN; ++j) b[j] = B(k, tc + GN * j);
-#pragma unroll
-      for (int i = 0; i < TM; ++i)
-#pragma unroll
-        for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-#pragma unroll
-    for (int i = 0; i < TM; ++i) {
-      const int m = mb + tr + GM * i;
-      if (m < M) {
-#pragma unroll
-        for (int j = 0; j < TN; ++j) out(m, tc + GN * j, acc[i][j]);
-      }
-    }
-  }
-}
-
-// ---- the same products on the tensor cores: mma.sync m16n8k8 tf32 with
-// each fp32 operand split into a tf32 high part and the (tf32-truncated)
-// remainder, C += A_hi B_lo + A_lo B_hi + A_hi B_hi.  The dropped
+// ---- products on the tensor cores: mma.sync m16n8k8 tf32 with each fp32
+// operand split into a tf32 high part and the (tf32-truncated) remainder,
+// C += A_hi B_lo + A_lo B_hi + A_hi B_hi.  The dropped
 // A_lo B_lo and the truncation of the remainders leave a relative error near
 // 2^-21 per product, fp32-like; one tf32 product alone would leave 2^-11.
 __device__ __forceinline__ void tf32_split(float x, uint32_t &hi,
