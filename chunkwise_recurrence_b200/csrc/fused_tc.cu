@@ -571,6 +571,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint64_t base = st_mn(m);
         const uint32_t accv = tmem + ACC_V + (m & 1) * 64;
+        // W first: its commit (W done) lets the prep warps start P5 while
+        // the U products still run.  X, which accumulates onto U, is issued
+        // later by this thread, and one thread's MMAs complete in order.
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_f16kind(tmem + ACC_W, dadd(base, ks * 2048), dadd(d_tpw, ks * 32),
+                      kIdUW, ks > 0);
+        mma_commit(&bar[B_WDONE]);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           mma_f16kind(accv, dadd(d_vt, ks * 2048), dadd(d_tpb, ks * 32), kIdUW,
@@ -581,11 +589,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_f16kind(accv, dadd(d_vt, ks * 2048), dadd(d_tplo, ks * 32),
                         kIdUW, 1);
         }
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_f16kind(tmem + ACC_W, dadd(base, ks * 2048), dadd(d_tpw, ks * 32),
-                      kIdUW, ks > 0);
-        mma_commit(&bar[B_WDONE]);
         mma_commit(&bar[B_VFREE]);
         return true;
       };
@@ -1330,12 +1333,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bar[B_TREADY]);
       // P1 of the next chunk while U and W run
       if (m + 1 < NC) p1(m + 1);
-      // ---- P5: -W^T operand; Q e^g and K e^{g_C - g} in place (fp16)
+      // Q e^g (fp16, in place) while U and W run: K K^T of this chunk has
+      // read the raw tile (P3 waited for it)
+      if (GATE != 2) {
+        constexpr int kIq = kC * 16 / kPrep;   // 4
+        uint4 xq[kIq];
+        float eq[kIq];
+        uint32_t offq[kIq];
+#pragma unroll
+        for (int u = 0; u < kIq; ++u) {
+          const int idx = pt + u * kPrep;
+          const int r = idx >> 4, cc = idx & 15;
+          offq[u] = (cc >> 3) * 16384 + 8192 + sw128_chunk(r, cc & 7);
+          eq[u] = (GATE == 1) ? F[F_EG * 64 + r] : 1.f;
+          xq[u] = *reinterpret_cast<const uint4 *>(stg + offq[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kIq; ++u) {
+          uint32_t *wq = reinterpret_cast<uint32_t *>(&xq[u]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float a0, a1;
+            unpack_bf16(wq[e], a0, a1);
+            wq[e] = pack_f16(a0 * eq[u], a1 * eq[u]);
+          }
+          *reinterpret_cast<uint4 *>(stg + offq[u]) = xq[u];
+        }
+      }
+      // ---- P5: -W^T operand; K e^{g_C - g} in place (fp16).  The tensor-
+      // memory load of W is in flight while K is converted: v is read only
+      // after the load's wait.
       if (!group_all(wait_bar(cx, B_WDONE, m & 1), 2, kPrep)) break;
       tc_fence_after();
       {
         const int c0 = hf * 32;
         tmem_ld32(trow + ACC_W + c0, v);
+        if (GATE != 2) {
+          // K e^{g_C - g}, fp16 in place: all four 16-byte chunks of a thread
+          // are loaded before any is stored
+          constexpr int kIt = kC * 16 / kPrep;   // 4
+          uint4 xk[kIt];
+          float ek[kIt];
+          uint32_t off[kIt];
+#pragma unroll
+          for (int u = 0; u < kIt; ++u) {
+            const int idx = pt + u * kPrep;
+            const int r = idx >> 4, cc = idx & 15;
+            off[u] = (cc >> 3) * 16384 + sw128_chunk(r, cc & 7);
+            ek[u] = (GATE == 1) ? F[F_EK * 64 + r] : 1.f;
+            xk[u] = *reinterpret_cast<const uint4 *>(stg + off[u]);
+          }
+#pragma unroll
+          for (int u = 0; u < kIt; ++u) {
+            uint32_t *wk = reinterpret_cast<uint32_t *>(&xk[u]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float a0, a1;
+              unpack_bf16(wk[e], a0, a1);
+              wk[e] = pack_f16(a0 * ek[u], a1 * ek[u]);
+            }
+            *reinterpret_cast<uint4 *>(stg + off[u]) = xk[u];
+          }
+        }
         tmem_wait_ld();
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch)
@@ -1344,40 +1403,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                      pack_f16(-v[8 * ch + 2], -v[8 * ch + 3]),
                      pack_f16(-v[8 * ch + 4], -v[8 * ch + 5]),
                      pack_f16(-v[8 * ch + 6], -v[8 * ch + 7]));
-      }
-      if (GATE != 2) {
-        // raw bf16 -> fp16: Q times e^g, K times e^{g_C - g}.  All eight
-        // 16-byte chunks of a thread are loaded before any is stored, so
-        // their shared-memory latencies overlap.
-        constexpr int kIt = kC * 16 / kPrep;   // 4
-        uint4 xq[kIt], xk[kIt];
-        float eq[kIt], ek[kIt];
-        uint32_t off[kIt];
-#pragma unroll
-        for (int u = 0; u < kIt; ++u) {
-          const int idx = pt + u * kPrep;
-          const int r = idx >> 4, cc = idx & 15;
-          off[u] = (cc >> 3) * 16384 + sw128_chunk(r, cc & 7);
-          eq[u] = (GATE == 1) ? F[F_EG * 64 + r] : 1.f;
-          ek[u] = (GATE == 1) ? F[F_EK * 64 + r] : 1.f;
-          xq[u] = *reinterpret_cast<const uint4 *>(stg + off[u] + 8192);
-          xk[u] = *reinterpret_cast<const uint4 *>(stg + off[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < kIt; ++u) {
-          uint32_t *wq = reinterpret_cast<uint32_t *>(&xq[u]);
-          uint32_t *wk = reinterpret_cast<uint32_t *>(&xk[u]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float a0, a1;
-            unpack_bf16(wq[e], a0, a1);
-            wq[e] = pack_f16(a0 * eq[u], a1 * eq[u]);
-            unpack_bf16(wk[e], a0, a1);
-            wk[e] = pack_f16(a0 * ek[u], a1 * ek[u]);
-          }
-          *reinterpret_cast<uint4 *>(stg + off[u] + 8192) = xq[u];
-          *reinterpret_cast<uint4 *>(stg + off[u]) = xk[u];
-        }
       }
       const bool kn16 =
           GATE == 2 && reinterpret_cast<const int *>(sm + Lay::TT_F16)[m & 1];
