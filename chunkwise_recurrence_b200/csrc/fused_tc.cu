@@ -104,7 +104,13 @@ struct Layout {
   // factor; a single bf16 factor there quadruples the final-state error),
   // and T diag(b e^g) for W as one tile (TPG).  Channel gate: T diag(b) in
   // fp16 (TPB) for both, against fp16 V and K e^g.
-  static constexpr uint32_t TP_BYTES = (GATE == 2) ? 8192 : 24576;
+  // Scalar / no gate: one set per chunk parity, so that chunk m+1's factors
+  // are written while U of chunk m may still read its own (W done of chunk
+  // m+1 is waited for later and covers U of chunk m, issued before it).  The
+  // channel gate has no room for a second set: its prep warps wait for V
+  // free (U done) instead.
+  static constexpr uint32_t TP_PAR = (GATE == 2) ? 0 : 24576;
+  static constexpr uint32_t TP_BYTES = (GATE == 2) ? 8192 : 2 * 24576;
   static constexpr uint32_t TPB = OFF_TP, TPG = OFF_TP + 8192,
                             TPB_LO = OFF_TP + 16384;
   static constexpr uint32_t KN = OFF_TP + TP_BYTES;
@@ -571,23 +577,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint64_t base = st_mn(m);
         const uint32_t accv = tmem + ACC_V + (m & 1) * 64;
+        const uint32_t tpo = (m & 1) * Lay::TP_PAR;   // T-factor set
         // W first: its commit (W done) lets the prep warps start P5 while
         // the U products still run.  X, which accumulates onto U, is issued
         // later by this thread, and one thread's MMAs complete in order.
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_f16kind(tmem + ACC_W, dadd(base, ks * 2048), dadd(d_tpw, ks * 32),
-                      kIdUW, ks > 0);
+          mma_f16kind(tmem + ACC_W, dadd(base, ks * 2048),
+                      dadd(d_tpw, tpo + ks * 32), kIdUW, ks > 0);
         mma_commit(&bar[B_WDONE]);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_f16kind(accv, dadd(d_vt, ks * 2048), dadd(d_tpb, ks * 32), kIdUW,
-                      ks > 0);
+          mma_f16kind(accv, dadd(d_vt, ks * 2048), dadd(d_tpb, tpo + ks * 32),
+                      kIdUW, ks > 0);
         if (GATE != 2) {
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_f16kind(accv, dadd(d_vt, ks * 2048), dadd(d_tplo, ks * 32),
-                        kIdUW, 1);
+            mma_f16kind(accv, dadd(d_vt, ks * 2048),
+                        dadd(d_tplo, tpo + ks * 32), kIdUW, 1);
         }
         mma_commit(&bar[B_VFREE]);
         return true;
@@ -1234,8 +1241,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_bar_sync(2, kPrep);
         // step 3
         if (b2 == 0) run(3, 0, 2, true, true, nt);           // T30
+      }
+      // Channel gate: its single T-factor tile is rewritten only once U of
+      // the previous chunk, its last reader, has completed (V free); U is
+      // issued after W, so W done does not imply it.  Scalar / no gate: the
+      // tiles alternate by chunk parity.
+      if (GATE == 2) {
+        if (!group_all(m == 0 || pt != 0 || wait_bar(cx, B_VFREE, (m - 1) & 1),
+                       2, kPrep))
+          break;
+      } else {
         named_bar_sync(2, kPrep);
       }
+      const uint32_t tpo = (m & 1) * Lay::TP_PAR;   // T-factor set
       // ---- T-factor operands: T diag(b e^g) (scalar / no gate) and
       // T diag(b), with T diag(b)'s bf16 residual tile (scalar / no gate).
       // Item (tile, row r, 16-byte chunk ch); consecutive threads take
@@ -1282,9 +1300,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               lw[e] = pack_bf16(b0 - h0, b1 - h1);
             }
             const uint32_t o = sw128_chunk(r, ch);
-            st_smem_v4(sm + Lay::TPG + o, gw[0], gw[1], gw[2], gw[3]);
-            st_smem_v4(sm + Lay::TPB + o, hw[0], hw[1], hw[2], hw[3]);
-            st_smem_v4(sm + Lay::TPB_LO + o, lw[0], lw[1], lw[2], lw[3]);
+            st_smem_v4(sm + Lay::TPG + tpo + o, gw[0], gw[1], gw[2], gw[3]);
+            st_smem_v4(sm + Lay::TPB + tpo + o, hw[0], hw[1], hw[2], hw[3]);
+            st_smem_v4(sm + Lay::TPB_LO + tpo + o, lw[0], lw[1], lw[2], lw[3]);
           }
         }
         constexpr int kTiles = 1;
@@ -1314,7 +1332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t hw[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) hw[e] = pk(t8[2 * e], t8[2 * e + 1]);
-          st_smem_v4(sm + (tb ? Lay::TPB : Lay::TPG) + sw128_chunk(r, ch),
+          st_smem_v4(sm + (tb ? Lay::TPB : Lay::TPG) + tpo + sw128_chunk(r, ch),
                      hw[0], hw[1], hw[2], hw[3]);
           if (GATE != 2 && tb) {
             uint32_t lw[4];
